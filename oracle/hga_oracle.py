@@ -1,0 +1,273 @@
+"""CPU oracle for the HGA hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, the smoke check and the benchmark's CPU-baseline leg may import
+this module.  The library (libhga and its Python binding) never calls it, and it
+shares no code with the CUDA path: it imports numpy and nothing else.
+
+It is a plain, slow, float64 restatement of what the pages describe, one step
+after the other, with no blocking, fusion or reordering.  Sources (the HGA
+pages, all about "Long-Context Fine-Tuning with Limited VRAM"):
+
+  [P2]  adnankhan.ai notes "Long-Context Fine-Tuning with Limited VRAM",
+        section "Raw Abstract / Excerpt" (bounded set of exact historical
+        tokens per query block; only the active segment is differentiable,
+        older KV is detached).
+  [P3a] seventnews "BMW如何通过重新设计注意力机制，在16 GB GPU上实现16K上下文",
+        section "HGA的不同之处" (what HGA does differently): 64-token blocks
+        with a compact summary each; queries score the summaries, the top-k
+        blocks are opened at the level of 8-token groups, and only the
+        selected groups' exact-token K/V enter attention; the router has no
+        learned weights and scores the existing projected keys; summaries are
+        never attention values.
+  [P3b] same page, same section, last paragraph: 2048-token segments, forward
+        and backward per segment, no gradient across segment boundaries, later
+        segments still attend to earlier exact tokens through routing.
+  [P5]  gist.science retelling, section "解决方案" (the solution): 64-token
+        block summary cards and an 8-token group summary cache.
+
+Readings adopted where the pages are silent (each one is the plainest reading
+the rest supports):
+
+  R1  summary of a block / group = mean of its post-RoPE keys, per KV head;
+  R2  routing score of a candidate = mean, over the query block's 64 queries
+      and the G query heads sharing the KV head, of q.s/sqrt(d); by linearity
+      this equals qbar.s/sqrt(d) with qbar the mean query;
+  R3  candidates of query block j = every complete block strictly before the
+      query block's own block (history and earlier blocks of the segment);
+  R4  level 2 opens only the selected blocks: their groups compete for the
+      top-k group slots;
+  R5  ties go to the lower index (block index at level 1, global group index
+      at level 2); fewer candidates than k -> take all, pad with -1; the
+      selection is a set, reported in ascending order;
+  R6  attention of a query at global position p = softmax over the union of
+      the selected groups' tokens and its own block's tokens at positions <= p,
+      scale 1/sqrt(d), natural-log LSE;
+  R7  one selection per (batch, KV head, query block), shared by the G heads;
+  R8  under segment-wise backprop the history K/V are detached: history keys
+      give dQ only, keys of the active segment give dQ, dK and dV; no gradient
+      flows through the discrete routing or the summaries;
+  R9  near ties: when the k-th and (k+1)-th sorted scores of a level differ by
+      at most 1e-3 relative, the row is flagged; a flagged row's attention is
+      checked with the GPU's own selection.
+
+Parity pins (tests/test_oracle_pins.py): brute force of R2-R5 on tiny inputs,
+closed forms and hand-computed golden fixtures for R1, equality with dense
+causal attention (torch SDPA in float64, autograd for gradients) when top-k
+covers every candidate, equality with masked SDPA for general selections,
+finite differences, softmax rows summing to one, and the keyset bound.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+BLOCK = 64      # tokens per block                       [P3a], [P5]
+GROUP = 8       # tokens per group                       [P3a], [P5]
+QBLOCK = 64     # queries per query block (reading R1..R7 share this size)
+GROUPS_PER_BLOCK = BLOCK // GROUP
+TIE_REL = 1e-3
+
+
+# ----------------------------------------------------------------------------
+# step a1: summaries (R1)
+# ----------------------------------------------------------------------------
+
+def build_summaries(k: np.ndarray, t_begin: int, t_end: int):
+    """Group and block summaries of keys in [t_begin, t_end).
+
+    k: [B, Hkv, T, d] float64 post-RoPE keys.  Returns (gsum, bsum) with
+    gsum[b,h,i] = mean of the 8 keys of group t_begin/8 + i and
+    bsum[b,h,i] = mean of the 64 keys of block t_begin/64 + i.
+    """
+    assert t_begin % BLOCK == 0 and t_end % BLOCK == 0 and t_end <= k.shape[2]
+    B, H, _, d = k.shape
+    seg = k[:, :, t_begin:t_end, :]
+    n = t_end - t_begin
+    gsum = seg.reshape(B, H, n // GROUP, GROUP, d).mean(axis=3)
+    bsum = seg.reshape(B, H, n // BLOCK, BLOCK, d).mean(axis=3)
+    return gsum, bsum
+
+
+# ----------------------------------------------------------------------------
+# steps a2 + a3: two-level routing (R2..R5, R7, R9)
+# ----------------------------------------------------------------------------
+
+def _topk_lower_index(scores: np.ndarray, idx: np.ndarray, k: int):
+    """Order candidates by (-score, index); return (chosen indices, sorted scores)."""
+    order = np.lexsort((idx, -scores))
+    return idx[order[:k]], scores[order]
+
+
+def _near_tie(sorted_scores: np.ndarray, k: int) -> bool:
+    if k >= len(sorted_scores) or k == 0:
+        return False
+    a, b = sorted_scores[k - 1], sorted_scores[k]
+    return abs(a - b) <= TIE_REL * max(abs(a), abs(b))
+
+
+def route(q: np.ndarray, bsum: np.ndarray, gsum: np.ndarray, q_begin: int,
+          topk_blocks: int, topk_groups: int, n_kv_heads: int):
+    """Two-level weight-free routing of one segment's query blocks.
+
+    q: [B, Hq, S, d] float64 (the segment, first token at global q_begin).
+    bsum: [B, Hkv, >= J_max, d] block summaries by global block index.
+    gsum: [B, Hkv, >= 8 J_max, d] group summaries by global group index.
+    Returns sel_blk [B,Hkv,n_qb,k_b] int32, sel_grp [B,Hkv,n_qb,k_g] int32
+    (ascending, -1 padded) and near_tie [B,Hkv,n_qb] bool.
+    """
+    B, Hq, S, d = q.shape
+    G = Hq // n_kv_heads
+    n_qb = S // QBLOCK
+    sel_blk = np.full((B, n_kv_heads, n_qb, topk_blocks), -1, np.int32)
+    sel_grp = np.full((B, n_kv_heads, n_qb, topk_groups), -1, np.int32)
+    near_tie = np.zeros((B, n_kv_heads, n_qb), bool)
+    inv_sqrt_d = 1.0 / math.sqrt(d)
+    for b in range(B):
+        for h in range(n_kv_heads):
+            for j in range(n_qb):
+                own = (q_begin + QBLOCK * j) // BLOCK          # the query block's own block
+                qblk = q[b, h * G:(h + 1) * G, QBLOCK * j:QBLOCK * (j + 1), :]
+                qbar = qblk.reshape(-1, d).mean(axis=0)        # R2: mean over queries and heads
+                # level 1: candidates are the complete blocks before `own` (R3)
+                cand = np.arange(own)
+                s1 = (bsum[b, h, :own, :] @ qbar) * inv_sqrt_d
+                kb = min(topk_blocks, own)
+                blocks, s1_sorted = _topk_lower_index(s1, cand, kb)
+                blocks = np.sort(blocks)
+                # level 2: the groups of the selected blocks compete (R4)
+                groups = (blocks[:, None] * GROUPS_PER_BLOCK
+                          + np.arange(GROUPS_PER_BLOCK)[None, :]).reshape(-1)
+                s2 = (gsum[b, h, groups, :] @ qbar) * inv_sqrt_d
+                kg = min(topk_groups, len(groups))
+                chosen, s2_sorted = _topk_lower_index(s2, groups, kg)
+                chosen = np.sort(chosen)
+                sel_blk[b, h, j, :kb] = blocks
+                sel_grp[b, h, j, :kg] = chosen
+                near_tie[b, h, j] = _near_tie(s1_sorted, kb) or _near_tie(s2_sorted, kg)
+    return sel_blk, sel_grp, near_tie
+
+
+# ----------------------------------------------------------------------------
+# keysets (R6)
+# ----------------------------------------------------------------------------
+
+def routed_keys(sel_row: np.ndarray) -> np.ndarray:
+    """Token positions of the selected groups (ascending, padding dropped)."""
+    g = sel_row[sel_row >= 0].astype(np.int64)
+    return (g[:, None] * GROUP + np.arange(GROUP)[None, :]).reshape(-1)
+
+
+def keyset(q_begin: int, j: int, r: int, sel_row: np.ndarray) -> np.ndarray:
+    """All key positions attended by query r (0..63) of query block j."""
+    own0 = ((q_begin + QBLOCK * j) // BLOCK) * BLOCK
+    p = q_begin + QBLOCK * j + r
+    own = np.arange(own0, p + 1)
+    return np.concatenate([routed_keys(sel_row), own])
+
+
+def _block_keys(q_begin: int, j: int, sel_row: np.ndarray):
+    """Union of the query block's keys plus a [64, n] mask of which query sees which."""
+    own0 = ((q_begin + QBLOCK * j) // BLOCK) * BLOCK
+    routed = routed_keys(sel_row)
+    keys = np.concatenate([routed, own0 + np.arange(BLOCK)])
+    pos_q = q_begin + QBLOCK * j + np.arange(QBLOCK)
+    visible = np.ones((QBLOCK, len(keys)), bool)
+    visible[:, len(routed):] = keys[None, len(routed):] <= pos_q[:, None]
+    return keys, visible
+
+
+# ----------------------------------------------------------------------------
+# step a4: forward (R6, R7)
+# ----------------------------------------------------------------------------
+
+def attn_fwd(q, k, v, q_begin: int, sel_grp: np.ndarray, n_kv_heads: int):
+    """Exact-token attention of one segment over its selection.
+
+    q: [B,Hq,S,d], k/v: [B,Hkv,T,d] float64; sel_grp [B,Hkv,n_qb,k_g].
+    Returns o [B,Hq,S,d] and lse [B,Hq,S] (natural log).
+    """
+    B, Hq, S, d = q.shape
+    G = Hq // n_kv_heads
+    scale = 1.0 / math.sqrt(d)
+    o = np.zeros_like(q)
+    lse = np.zeros((B, Hq, S))
+    for b in range(B):
+        for h in range(n_kv_heads):
+            for j in range(S // QBLOCK):
+                keys, visible = _block_keys(q_begin, j, sel_grp[b, h, j])
+                kk, vv = k[b, h, keys, :], v[b, h, keys, :]
+                for hq in range(h * G, (h + 1) * G):
+                    rows = slice(QBLOCK * j, QBLOCK * (j + 1))
+                    s = (q[b, hq, rows, :] @ kk.T) * scale
+                    s = np.where(visible, s, -np.inf)
+                    m = s.max(axis=1, keepdims=True)
+                    p = np.exp(s - m)
+                    l = p.sum(axis=1, keepdims=True)
+                    o[b, hq, rows, :] = (p @ vv) / l
+                    lse[b, hq, rows] = (m + np.log(l))[:, 0]
+    return o, lse
+
+
+# ----------------------------------------------------------------------------
+# step a5: backward under segment-wise backprop (R8)
+# ----------------------------------------------------------------------------
+
+def attn_bwd(q, k, v, do, q_begin: int, sel_grp: np.ndarray, n_kv_heads: int):
+    """Gradients of sum(dO * O) for one segment.
+
+    Returns dq [B,Hq,S,d] and, for the active segment's keys only,
+    dk, dv [B,Hkv,S,d] (positions q_begin .. q_begin+S-1).  History keys are
+    detached, so their gradient is not produced.
+    """
+    B, Hq, S, d = q.shape
+    G = Hq // n_kv_heads
+    scale = 1.0 / math.sqrt(d)
+    T = k.shape[2]
+    dq = np.zeros_like(q)
+    dk_full = np.zeros((B, n_kv_heads, T, d))
+    dv_full = np.zeros((B, n_kv_heads, T, d))
+    for b in range(B):
+        for h in range(n_kv_heads):
+            for j in range(S // QBLOCK):
+                keys, visible = _block_keys(q_begin, j, sel_grp[b, h, j])
+                kk, vv = k[b, h, keys, :], v[b, h, keys, :]
+                for hq in range(h * G, (h + 1) * G):
+                    rows = slice(QBLOCK * j, QBLOCK * (j + 1))
+                    qq, dd = q[b, hq, rows, :], do[b, hq, rows, :]
+                    s = np.where(visible, (qq @ kk.T) * scale, -np.inf)
+                    m = s.max(axis=1, keepdims=True)
+                    p = np.exp(s - m)
+                    p = p / p.sum(axis=1, keepdims=True)       # softmax probabilities
+                    oo = p @ vv
+                    dp = dd @ vv.T
+                    D = (dd * oo).sum(axis=1, keepdims=True)
+                    ds = p * (dp - D)
+                    dq[b, hq, rows, :] = (ds @ kk) * scale
+                    np.add.at(dk_full[b, h], keys, (ds.T @ qq) * scale)
+                    np.add.at(dv_full[b, h], keys, p.T @ dd)
+    act = slice(q_begin, q_begin + S)
+    return dq, dk_full[:, :, act, :], dv_full[:, :, act, :]
+
+
+# ----------------------------------------------------------------------------
+# one segment of the segment-wise loop (a1 .. a5 in order)
+# ----------------------------------------------------------------------------
+
+def segment_step(q, k, v, do, q_begin: int, gsum, bsum, topk_blocks: int,
+                 topk_groups: int, n_kv_heads: int, backward: bool = True):
+    """Summarise the segment's keys into gsum/bsum (in place, global indices),
+    route, attend, and (optionally) backpropagate.  Returns a dict."""
+    S = q.shape[2]
+    g, bl = build_summaries(k, q_begin, q_begin + S)
+    gsum[:, :, q_begin // GROUP:(q_begin + S) // GROUP] = g
+    bsum[:, :, q_begin // BLOCK:(q_begin + S) // BLOCK] = bl
+    sel_blk, sel_grp, tie = route(q, bsum, gsum, q_begin, topk_blocks, topk_groups,
+                                  n_kv_heads)
+    o, lse = attn_fwd(q, k, v, q_begin, sel_grp, n_kv_heads)
+    out = dict(sel_blk=sel_blk, sel_grp=sel_grp, near_tie=tie, o=o, lse=lse)
+    if backward:
+        dq, dk, dv = attn_bwd(q, k, v, do, q_begin, sel_grp, n_kv_heads)
+        out.update(dq=dq, dk=dk, dv=dv)
+    return out

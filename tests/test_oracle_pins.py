@@ -1,0 +1,433 @@
+"""Pins of the CPU oracle against things other than itself (CPU only).
+
+Each check below ties one part of the oracle to a closed form, a brute-force
+enumeration of the definition, a hand-worked fixture, or a library routine
+(torch scaled_dot_product_attention / autograd in float64).  The last test
+plants mistakes in copies of oracle functions and checks that some pin fails.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from oracle import hga_oracle as ho
+from hierarchical_routed_sparse_hga_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+def tiny_case(seed=0, topk_blocks=2, topk_groups=5, ctx=384, seg=128, first_seg=2,
+              hq=4, hkv=2, d=16, batch=2):
+    w = synth.custom(batch=batch, n_q_heads=hq, n_kv_heads=hkv, head_dim=d, ctx_len=ctx,
+                     seg_len=seg, topk_blocks=topk_blocks, topk_groups=topk_groups,
+                     seed=seed, first_seg=first_seg)
+    k = synth.widen(synth.keys(w), "f32")
+    v = synth.widen(synth.values(w), "f32")
+    q_begin = w.segments()[0]
+    q = synth.widen(synth.queries(w, q_begin), "f32")
+    do = synth.widen(synth.douts(w, q_begin), "f32")
+    return w, q, k, v, do, q_begin
+
+
+def summaries_upto(k, t_end):
+    return oracle.build_summaries(k, 0, t_end)
+
+
+def brute_force_route(q, k, q_begin, topk_blocks, topk_groups, hkv):
+    """Literal definition: score = mean over (query, head, key) triples of q.k/sqrt(d)."""
+    B, Hq, S, d = q.shape
+    G = Hq // hkv
+    out_blk, out_grp = {}, {}
+    for b in range(B):
+        for h in range(hkv):
+            for j in range(S // 64):
+                own = (q_begin + 64 * j) // 64
+                qs = [q[b, hh, 64 * j + t] for hh in range(h * G, (h + 1) * G) for t in range(64)]
+
+                def score(positions):
+                    tot = 0.0
+                    for qq in qs:
+                        for p in positions:
+                            tot += float(np.dot(qq, k[b, h, p])) / math.sqrt(d)
+                    return tot / (len(qs) * len(positions))
+
+                blk_scores = [(score(range(64 * c, 64 * c + 64)), c) for c in range(own)]
+                blk_sorted = sorted(blk_scores, key=lambda sc: (-sc[0], sc[1]))
+                chosen = sorted(c for _, c in blk_sorted[:topk_blocks])
+                grp_scores = [(score(range(8 * g, 8 * g + 8)), g)
+                              for c in chosen for g in range(8 * c, 8 * c + 8)]
+                grp_sorted = sorted(grp_scores, key=lambda sc: (-sc[0], sc[1]))
+                out_blk[(b, h, j)] = chosen
+                out_grp[(b, h, j)] = sorted(g for _, g in grp_sorted[:topk_groups])
+    return out_blk, out_grp
+
+
+def keyset_mask(q_begin, S, T, sel_grp_bh):
+    """[S, T] bool: query row t sees key p (routed groups + own block causal)."""
+    mask = np.zeros((S, T), bool)
+    for t in range(S):
+        j = t // 64
+        for p in oracle.keyset(q_begin, j, t % 64, sel_grp_bh[j]):
+            mask[t, p] = True
+    return mask
+
+
+def sdpa_reference(q, k, v, do, q_begin, masks, hkv):
+    """float64 torch SDPA with explicit masks; gradients by autograd with the
+    history detached.  masks: [B, Hkv, S, T] bool.  Returns o, lse, dq, dk, dv."""
+    B, Hq, S, d = q.shape
+    G = Hq // hkv
+    T = q_begin + S
+    qt = torch.tensor(q, requires_grad=True)
+    k_hist = torch.tensor(k[:, :, :q_begin])
+    v_hist = torch.tensor(v[:, :, :q_begin])
+    k_act = torch.tensor(k[:, :, q_begin:T], requires_grad=True)
+    v_act = torch.tensor(v[:, :, q_begin:T], requires_grad=True)
+    kf = torch.cat([k_hist, k_act], dim=2).repeat_interleave(G, dim=1)
+    vf = torch.cat([v_hist, v_act], dim=2).repeat_interleave(G, dim=1)
+    m = torch.tensor(masks).repeat_interleave(G, dim=1)
+    o = F.scaled_dot_product_attention(qt, kf, vf, attn_mask=m)
+    (o * torch.tensor(do)).sum().backward()
+    s = (qt.detach() @ kf.transpose(-1, -2)) / math.sqrt(d)
+    lse = torch.logsumexp(s.masked_fill(~m, -math.inf), dim=-1)
+    return (o.detach().numpy(), lse.detach().numpy(), qt.grad.numpy(), k_act.grad.numpy(),
+            v_act.grad.numpy())
+
+
+def close(a, b, tol=1e-10):
+    return np.max(np.abs(np.asarray(a) - np.asarray(b))) <= tol * max(1.0, np.max(np.abs(b)))
+
+
+# ----------------------------------------------------------------------------
+# pins: summaries
+# ----------------------------------------------------------------------------
+
+def check_summaries_closed_form():
+    # K[t] = a + b*t per dimension: the mean of an arithmetic run is its midpoint
+    d, T = 3, 256
+    a, bb = np.array([1.0, -2.0, 0.5]), np.array([0.25, 1.0, -3.0])
+    k = (a[None, :] + bb[None, :] * np.arange(T)[:, None])[None, None]
+    g, bl = oracle.build_summaries(k, 64, 256)
+    for i in range(g.shape[2]):
+        first = 64 + 8 * i
+        assert close(g[0, 0, i], a + bb * (first + 3.5))
+    for i in range(bl.shape[2]):
+        first = 64 + 64 * i
+        assert close(bl[0, 0, i], a + bb * (first + 31.5))
+
+
+def test_summaries_closed_form():
+    check_summaries_closed_form()
+
+
+def test_block_summary_is_mean_of_its_groups():
+    _, q, k, v, do, q_begin = tiny_case()
+    g, bl = oracle.build_summaries(k, 0, k.shape[2])
+    B, H, nb, d = bl.shape
+    assert close(bl, g.reshape(B, H, nb, 8, d).mean(axis=3))
+
+
+# ----------------------------------------------------------------------------
+# pins: routing
+# ----------------------------------------------------------------------------
+
+def golden_inputs(fx, group_x, own_x=None):
+    x = np.array(fx[group_x], float)
+    if own_x is not None:
+        x[32:] = own_x
+    T = fx["q_begin"] + fx["seg_len"]
+    k = np.zeros((1, 1, T, 2))
+    k[0, 0, :, 0] = np.repeat(x, 8)
+    k[0, 0, :, 1] = fx["key_y"]
+    q = np.zeros((1, 1, fx["seg_len"], 2))
+    q[0, 0, :, :] = fx["query"]
+    return q, k
+
+
+def check_route_golden():
+    fx = json.load(open(os.path.join(GOLDEN, "route_attn_handworked.json")))
+    for case in fx["cases"]:
+        q, k = golden_inputs(fx, case["group_x"])
+        g, bl = summaries_upto(k, k.shape[2])
+        sb, sg, _ = oracle.route(q, bl, g, fx["q_begin"], case["topk_blocks"],
+                                 case["topk_groups"], 1)
+        assert list(sb[0, 0, 0]) == case["sel_blk"], case["name"]
+        if isinstance(case["sel_grp"], str):       # case D: everything selected
+            want = list(range(32)) + [-1] * 8
+        else:
+            want = case["sel_grp"]
+        assert list(sg[0, 0, 0]) == want, case["name"]
+
+
+def test_route_golden():
+    check_route_golden()
+
+
+def check_route_bruteforce(seed=0):
+    w, q, k, v, do, q_begin = tiny_case(seed=seed)
+    g, bl = summaries_upto(k, k.shape[2])
+    sb, sg, tie = oracle.route(q, bl, g, q_begin, w.topk_blocks, w.topk_groups, w.n_kv_heads)
+    bb, bg = brute_force_route(q, k, q_begin, w.topk_blocks, w.topk_groups, w.n_kv_heads)
+    n = 0
+    for key, blocks in bb.items():
+        if tie[key]:
+            continue
+        n += 1
+        assert [c for c in sb[key] if c >= 0] == blocks, key
+        assert [c for c in sg[key] if c >= 0] == bg[key], key
+    assert n >= len(bb) - 1
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_route_bruteforce(seed):
+    check_route_bruteforce(seed)
+
+
+def test_route_exact_ties_take_lower_index():
+    # every block identical -> every block ties; lowest indices win at both levels
+    d = 4
+    rng = np.random.default_rng(5)
+    one_block = rng.standard_normal((64, d))
+    k = np.tile(one_block, (6, 1))[None, None]
+    q = rng.standard_normal((1, 1, 64, d))
+    g, bl = summaries_upto(k, k.shape[2])
+    sb, sg, tie = oracle.route(q, bl, g, 320, 3, 5, 1)
+    assert list(sb[0, 0, 0]) == [0, 1, 2]
+    # groups inside a block differ, so level 2 keeps the same within-block
+    # ranking in every block; ties across blocks go to the lower block
+    order = np.argsort(-(one_block.reshape(8, 8, d).mean(axis=1) @ q[0, 0].mean(axis=0)),
+                       kind="stable")
+    want = sorted([int(order[0]), int(order[0]) + 8, int(order[0]) + 16,
+                   int(order[1]), int(order[1]) + 8])
+    assert list(sg[0, 0, 0]) == want
+    assert tie[0, 0, 0]
+
+
+def test_route_first_block_has_no_candidates():
+    w, q, k, v, do, _ = tiny_case(first_seg=0)
+    g, bl = summaries_upto(k, 128)
+    sb, sg, tie = oracle.route(q, bl, g, 0, 2, 5, w.n_kv_heads)
+    assert (sb[:, :, 0] == -1).all() and (sg[:, :, 0] == -1).all()
+    assert (sb[:, :, 1, 0] == 0).all() and (sb[:, :, 1, 1] == -1).all()
+
+
+def test_planted_target_ranks_first():
+    # statistical sanity check on the tiny fp32 workload (not an exactness test)
+    w = synth.workloads()["tiny_f32"]
+    k = synth.widen(synth.keys(w), w.dtype)
+    q_begin = w.segments()[0]
+    q = synth.widen(synth.queries(w, q_begin), w.dtype)
+    g, bl = summaries_upto(k, k.shape[2])
+    hits = 0
+    for j in range(w.seg_len // 64):
+        s = bl[0, 0, :(q_begin // 64 + j)] @ q[0, 0, 64 * j:64 * j + 64].mean(axis=0)
+        hits += int(np.argmax(s) == synth.targets(w, 0, 0, q_begin)[j])
+    assert hits == w.seg_len // 64
+
+
+# ----------------------------------------------------------------------------
+# pins: attention forward / backward
+# ----------------------------------------------------------------------------
+
+def check_attention_golden():
+    fx = json.load(open(os.path.join(GOLDEN, "route_attn_handworked.json")))
+    q, k = golden_inputs(fx, "group_x_case_A", own_x=0.0)
+    T = k.shape[2]
+    v = np.zeros((1, 1, T, 2))
+    grp = np.arange(T) // 8
+    v[0, 0, :, 0] = np.where(grp < 32, grp, 0)
+    v[0, 0, :, 1] = np.where(grp < 32, 0, 1)
+    g, bl = summaries_upto(k, T)
+    _, sg, _ = oracle.route(q, bl, g, fx["q_begin"], 2, 3, 1)
+    o, lse = oracle.attn_fwd(q, k, v, fx["q_begin"], sg, 1)
+    env = {"exp": math.exp, "log": math.log, "sqrt": math.sqrt}
+    for r in range(64):
+        env["r"] = r
+        assert abs(lse[0, 0, r] - eval(fx["lse_row_expr"], env)) < 1e-12
+        assert abs(o[0, 0, r, 0] - eval(fx["o_row_expr"][0], env)) < 1e-12
+        assert abs(o[0, 0, r, 1] - eval(fx["o_row_expr"][1], env)) < 1e-12
+
+
+def test_attention_golden():
+    check_attention_golden()
+
+
+def check_dense_equivalence(seed=1):
+    # top-k covering every candidate block and group -> dense causal attention
+    w, q, k, v, do, q_begin = tiny_case(seed=seed, topk_blocks=8, topk_groups=64)
+    T = q_begin + w.seg_len
+    g, bl = summaries_upto(k, T)
+    _, sg, _ = oracle.route(q, bl, g, q_begin, w.topk_blocks, w.topk_groups, w.n_kv_heads)
+    o, lse = oracle.attn_fwd(q, k, v, q_begin, sg, w.n_kv_heads)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, do, q_begin, sg, w.n_kv_heads)
+    pos_q = q_begin + np.arange(w.seg_len)
+    causal = np.arange(T)[None, :] <= pos_q[:, None]            # textbook causal mask
+    masks = np.broadcast_to(causal, (w.batch, w.n_kv_heads, w.seg_len, T))
+    ro, rlse, rdq, rdk, rdv = sdpa_reference(q, k[:, :, :T], v[:, :, :T], do, q_begin,
+                                             masks, w.n_kv_heads)
+    assert close(o, ro) and close(lse, rlse)
+    assert close(dq, rdq) and close(dk, rdk) and close(dv, rdv)
+
+
+def test_dense_equivalence_fwd_bwd():
+    check_dense_equivalence()
+
+
+def check_masked_sdpa(seed=2):
+    # general selection: the oracle equals SDPA with the keyset as its mask
+    w, q, k, v, do, q_begin = tiny_case(seed=seed)
+    T = q_begin + w.seg_len
+    g, bl = summaries_upto(k, T)
+    _, sg, _ = oracle.route(q, bl, g, q_begin, w.topk_blocks, w.topk_groups, w.n_kv_heads)
+    o, lse = oracle.attn_fwd(q, k, v, q_begin, sg, w.n_kv_heads)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, do, q_begin, sg, w.n_kv_heads)
+    masks = np.stack([np.stack([keyset_mask(q_begin, w.seg_len, T, sg[b, h])
+                                for h in range(w.n_kv_heads)]) for b in range(w.batch)])
+    ro, rlse, rdq, rdk, rdv = sdpa_reference(q, k[:, :, :T], v[:, :, :T], do, q_begin,
+                                             masks, w.n_kv_heads)
+    assert close(o, ro) and close(lse, rlse)
+    assert close(dq, rdq) and close(dk, rdk) and close(dv, rdv)
+
+
+def test_masked_sdpa_general_selection():
+    check_masked_sdpa()
+
+
+def check_finite_differences():
+    w, q, k, v, do, q_begin = tiny_case(seed=3, batch=1, hq=2, hkv=1, d=4, ctx=192, seg=128,
+                                        first_seg=0, topk_blocks=1, topk_groups=3)
+    # first_seg=0: segment [0,128) is active; second segment [128,192) unused
+    q_begin = 0
+    T = 128
+    k = k.copy()
+    g, bl = summaries_upto(k, T)
+    _, sg, _ = oracle.route(q, bl, g, q_begin, 1, 3, 1)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, do, q_begin, sg, 1)
+
+    def loss(qq, kk, vv):
+        o, _ = oracle.attn_fwd(qq, kk, vv, q_begin, sg, 1)
+        return float((o * do).sum())
+
+    rng = np.random.default_rng(0)
+    eps = 1e-6
+    for name, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(6):
+            idx = tuple(int(rng.integers(0, n)) for n in grad.shape)
+            plus, minus = arr.copy(), arr.copy()
+            plus[idx] += eps
+            minus[idx] -= eps
+            args_p = {"q": (plus, k, v), "k": (q, plus, v), "v": (q, k, plus)}[name]
+            args_m = {"q": (minus, k, v), "k": (q, minus, v), "v": (q, k, minus)}[name]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - grad[idx]) < 1e-6 * max(1.0, abs(fd)), (name, idx)
+
+
+def test_finite_differences():
+    check_finite_differences()
+
+
+def test_rows_sum_to_one_and_keyset_bound():
+    w, q, k, v, do, q_begin = tiny_case(seed=4)
+    T = q_begin + w.seg_len
+    g, bl = summaries_upto(k, T)
+    _, sg, _ = oracle.route(q, bl, g, q_begin, w.topk_blocks, w.topk_groups, w.n_kv_heads)
+    o, lse = oracle.attn_fwd(q, k, v, q_begin, sg, w.n_kv_heads)
+    G = w.group_heads
+    for b in range(w.batch):
+        for hq in range(w.n_q_heads):
+            h = hq // G
+            for t in range(w.seg_len):
+                j, r = divmod(t, 64)
+                ks = oracle.keyset(q_begin, j, r, sg[b, h, j])
+                assert len(ks) <= 8 * w.topk_groups + 64
+                assert len(set(ks.tolist())) == len(ks)          # routed groups avoid own block
+                s = k[b, h, ks] @ q[b, hq, t] / math.sqrt(w.head_dim)
+                assert abs(np.exp(s - lse[b, hq, t]).sum() - 1.0) < 1e-12
+
+
+def test_history_gets_no_gradient_and_segments_chain():
+    # three segments over 384 tokens; dk/dv cover exactly the active slice
+    w, q, k, v, do, _ = tiny_case(first_seg=0, topk_blocks=2, topk_groups=6)
+    T = w.ctx_len
+    gsum = np.zeros((w.batch, w.n_kv_heads, T // 8, w.head_dim))
+    bsum = np.zeros((w.batch, w.n_kv_heads, T // 64, w.head_dim))
+    for q_begin in w.segments():
+        qq = synth.widen(synth.queries(w, q_begin), "f32")
+        dd = synth.widen(synth.douts(w, q_begin), "f32")
+        out = oracle.segment_step(qq, k, v, dd, q_begin, gsum, bsum, w.topk_blocks,
+                                  w.topk_groups, w.n_kv_heads)
+        assert out["dk"].shape == (w.batch, w.n_kv_heads, w.seg_len, w.head_dim)
+        # every routed group lies strictly before the query block's own block
+        for j in range(w.seg_len // 64):
+            own = (q_begin + 64 * j) // 64
+            sel = out["sel_grp"][:, :, j]
+            assert ((sel < 0) | (sel // 8 < own)).all()
+    g_all, b_all = oracle.build_summaries(k, 0, T)
+    assert close(gsum, g_all) and close(bsum, b_all)
+
+
+# ----------------------------------------------------------------------------
+# planted mistakes: each mutated oracle must fail at least one pin
+# ----------------------------------------------------------------------------
+
+def _mut_route_wrong_heads(q, bsum, gsum, q_begin, kb, kg, hkv):
+    # mean over the wrong GQA head group (next group)
+    B, Hq, S, d = q.shape
+    G = Hq // hkv
+    q2 = np.roll(q, -G, axis=1)
+    return ORIG["route"](q2, bsum, gsum, q_begin, kb, kg, hkv)
+
+
+def _mut_topk_higher_index(scores, idx, k):
+    order = np.lexsort((-idx, -scores))
+    return idx[order[:k]], scores[order]
+
+
+def _mut_block_keys_strict(q_begin, j, sel_row):
+    keys, visible = ORIG["_block_keys"](q_begin, j, sel_row)
+    n_routed = len(keys) - 64
+    visible = visible.copy()
+    visible[:, n_routed:] &= ~np.eye(64, dtype=bool)            # diagonal dropped
+    return keys, visible
+
+
+def _mut_summaries_sum(k, t_begin, t_end):
+    g, b = ORIG["build_summaries"](k, t_begin, t_end)
+    return g * 8, b                                               # group sum, not mean
+
+
+ORIG = {"route": ho.route, "_topk_lower_index": ho._topk_lower_index,
+        "_block_keys": ho._block_keys, "build_summaries": ho.build_summaries}
+
+ALL_PINS = [check_summaries_closed_form, check_route_golden, check_route_bruteforce,
+            check_attention_golden, check_dense_equivalence, check_masked_sdpa,
+            check_finite_differences]
+
+
+@pytest.mark.parametrize("target,mutant", [
+    ("route", _mut_route_wrong_heads),
+    ("_topk_lower_index", _mut_topk_higher_index),
+    ("_block_keys", _mut_block_keys_strict),
+    ("build_summaries", _mut_summaries_sum),
+])
+def test_pins_catch_planted_mistakes(monkeypatch, target, mutant):
+    monkeypatch.setattr(ho, target, mutant)
+    if hasattr(oracle, target):
+        monkeypatch.setattr(oracle, target, mutant)
+    failed = 0
+    for pin in ALL_PINS:
+        try:
+            pin()
+        except AssertionError:
+            failed += 1
+    assert failed >= 1, f"no pin caught the planted mistake in {target}"
