@@ -1,0 +1,561 @@
+#!/usr/bin/env python
+"""HGA attention fwd+bwd tokens/s per layer (Qwen3-8B attention shape).
+
+One step = one pass of the whole hot path over one sequence of the workload:
+for every segment, in order: summaries of the segment's keys, two-level
+routing, exact-token attention forward, and (for training workloads) the
+backward under segment-wise backprop.  The default workload is the 16384-token
+sequence processed as 8 segments of 2048 with forward and backward
+(32 query heads, 8 KV heads, d=128, bf16, top-16 blocks then top-64 groups).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hga|reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own sequence
+(different seed): the units shard with no data-path exchange ("weak" scaling);
+the only collective is the max over ranks of the timed duration.
+
+Timing: W untimed warm-up steps; then K steps, each bracketed by CUDA events on
+the launching stream, with a 512 MiB write between steps (outside the events)
+to flush the 126 MB L2; barrier + synchronize around the whole loop.
+Per-kernel durations come from libhga's own event brackets around each launch
+inside the same timed steps.
+"""
+
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HGA attn fwd+bwd tokens/s per layer (Qwen3-8B shape); % of TC/HBM roofline"
+DEFAULT_WORKLOAD = "qwen3_fwdbwd_16k"
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x FP32 lanes x FMA x max clock
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=30)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["hga", "reference"], default="hga")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--graph", action="store_true", help="replay each step as a CUDA graph")
+    p.add_argument("--simt", action="store_true", help="force the CUDA-core attention kernels")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-clocks", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm=d["hbm_gbs"], tc=d["bf16_tflops"], tc_sustained=d["bf16_tflops_sustained"],
+                    sm_max_mhz=d.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm=6650.0, tc=1590.0, tc_sustained=1400.0, sm_max_mhz=1965.0, source="fallback")
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (host logic; tested with gloo on CPU)
+# ----------------------------------------------------------------------------
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def rank_workload(w, rank: int):
+    """Each rank processes its own sequence: same shapes, seed offset by rank."""
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[device.index] if device is not None and device.type == "cuda"
+                     else None)
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id=None):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if bus_id:
+            cmd += ["-i", bus_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            r = [x.strip() for x in r]
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------
+# algorithmic work per kernel kind (the roofline numerators)
+# ----------------------------------------------------------------------------
+
+def segment_pairs(w, sel_grp, q_begin):
+    """(all attended (query row, key) pairs, pairs on active-segment keys)."""
+    import numpy as np
+    G, d = w.group_heads, w.head_dim
+    valid = sel_grp >= 0
+    routed = valid.sum(axis=-1) * 8                          # keys per (b, h, j)
+    active = (valid & (sel_grp * 8 >= q_begin)).sum(axis=-1) * 8
+    own = 64 * 65 // 2                                       # causal pairs of one block
+    rows = G * 64
+    all_pairs = int((routed * rows).sum() + own * G * routed.size)
+    act_pairs = int((active * rows).sum() + own * G * routed.size)
+    return all_pairs, act_pairs
+
+
+def kernel_work(name, w, sels):
+    """Algorithmic work of ALL launches of kernel `name` over one step.
+    Returns (amount, unit, bound): FLOP for contractions, bytes otherwise."""
+    d, S, B = w.head_dim, w.seg_len, w.batch
+    Hq, Hkv = w.n_q_heads, w.n_kv_heads
+    el = 2 if w.dtype == "bf16" else 4
+    n_qb = S // 64
+    tot = 0.0
+    for q_begin, sel in sels:
+        pairs, act = segment_pairs(w, sel, q_begin)
+        own0 = q_begin // 64
+        Js = [own0 + j for j in range(n_qb)]
+        kb = [min(w.topk_blocks, J) for J in Js]
+        if name.startswith("attn_fwd"):
+            tot += 4 * d * pairs
+        elif name.startswith("attn_bwd_dq"):
+            tot += 6 * d * pairs
+        elif name.startswith("attn_bwd_dkdv"):
+            tot += 8 * d * act
+        elif name == "summaries":
+            tot += B * Hkv * (S * d * el + (S // 8 + S // 64) * d * 4)
+        elif name == "route_qmean":
+            tot += B * (Hq * S * d * el + Hkv * n_qb * d * 4)
+        elif name == "route_block_score":
+            tot += B * Hkv * ((own0 + n_qb - 1) * d * 4 + n_qb * d * 4 + sum(Js) * 4)
+        elif name == "route_select":
+            tot += B * Hkv * sum(J * 4 + 8 * k * d * 4 + d * 4 + 4 * (w.topk_blocks + w.topk_groups)
+                                 for J, k in zip(Js, kb))
+    if name.startswith("attn"):
+        return tot, "FLOP", "alu" if name.endswith("simt") else "tensor"
+    return tot, "B", "hbm"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "hierarchical_routed_sparse_hga_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the
+    current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path))
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------
+# the GPU arm
+# ----------------------------------------------------------------------------
+
+class Runner:
+    def __init__(self, w, device, flags=0):
+        import torch
+        from hierarchical_routed_sparse_hga_b200 import HGA_BF16, HGA_F32, Config, HgaLayer
+        from hierarchical_routed_sparse_hga_b200 import synth
+        self.w, self.device = w, device
+        self.dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        cfg = Config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.topk_blocks,
+                     w.topk_groups, HGA_BF16 if w.dtype == "bf16" else HGA_F32, flags)
+
+        def dev(a):
+            return self.to_torch(a).to(device)
+
+        self.k_host = self.to_torch(synth.keys(w)).pin_memory()
+        self.v_host = self.to_torch(synth.values(w)).pin_memory()
+        self.layer = HgaLayer(cfg, w.ctx_len, w.seg_len, device=device,
+                              k=self.k_host.to(device), v=self.v_host.to(device))
+        self.segs = w.segments()
+        self.q_host = [self.to_torch(synth.queries(w, s)).pin_memory() for s in self.segs]
+        self.q = [t.to(device) for t in self.q_host]
+        if w.backward:
+            self.do_host = [self.to_torch(synth.douts(w, s)).pin_memory() for s in self.segs]
+            self.do = [t.to(device) for t in self.do_host]
+        self.history_end = self.segs[0]
+        if self.history_end:
+            # history before the first query-carrying segment: resident summaries
+            from hierarchical_routed_sparse_hga_b200 import hga_build_summaries
+            hga_build_summaries(self.layer.cfg, self.layer.k, w.ctx_len, 0, self.history_end,
+                                self.layer.gsum, self.layer.bsum)
+        torch.cuda.synchronize(device)
+
+    def to_torch(self, a):
+        import numpy as np
+        import torch
+        if self.w.dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+
+    def step(self, record_sel=None):
+        L = self.layer
+        for i, q_begin in enumerate(self.segs):
+            L.segment(self.q[i], q_begin, self.do[i] if self.w.backward else None)
+            if record_sel is not None:
+                record_sel.append((q_begin, L.sel_grp.cpu().numpy()))
+
+    def e2e_step(self, out_host):
+        """Host buffers in, host buffers out: H2D of the step's inputs, the step,
+        D2H of every segment's outputs (all on the current stream)."""
+        L = self.layer
+        L.k.copy_(self.k_host, non_blocking=True)
+        L.v.copy_(self.v_host, non_blocking=True)
+        for i, q_begin in enumerate(self.segs):
+            self.q[i].copy_(self.q_host[i], non_blocking=True)
+            if self.w.backward:
+                self.do[i].copy_(self.do_host[i], non_blocking=True)
+            L.segment(self.q[i], q_begin, self.do[i] if self.w.backward else None)
+            outs = (L.o, L.dq, L.dk, L.dv) if self.w.backward else (L.o,)
+            for dst, src in zip(out_host[i], outs):
+                dst.copy_(src, non_blocking=True)
+
+    def io_bytes(self):
+        nb = lambda t: t.numel() * t.element_size()  # noqa: E731
+        h2d = nb(self.k_host) + nb(self.v_host) + sum(nb(t) for t in self.q_host)
+        L = self.layer
+        outs = (L.o, L.dq, L.dk, L.dv) if self.w.backward else (L.o,)
+        if self.w.backward:
+            h2d += sum(nb(t) for t in self.do_host)
+        d2h = len(self.segs) * sum(nb(t) for t in outs)
+        return h2d, d2h
+
+
+def run_gpu(args, rank, world, local):
+    import numpy as np
+    import torch
+    from hierarchical_routed_sparse_hga_b200 import (HGA_FLAG_SIMT, hga_launch_count,
+                                                     hga_timing_collect, hga_timing_enable,
+                                                     hga_timing_reset, synth, timing_table)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=device)
+    w0 = synth.workloads()[args.workload]
+    w = rank_workload(w0, rank)
+    run = Runner(w, device, HGA_FLAG_SIMT if args.simt else 0)
+    tokens_per_step = w.batch * len(run.segs) * w.seg_len
+
+    sels = []
+    run.step(record_sel=sels)                       # first warm-up step records selections
+    for _ in range(max(args.warmup, 3) - 1):
+        run.step()
+    torch.cuda.synchronize(device)
+
+    per_step_launches = None
+    graph = None
+    n0 = hga_launch_count()
+    run.step()
+    torch.cuda.synchronize(device)
+    per_step_launches = hga_launch_count() - n0
+    slots = per_step_launches + 16
+    if args.graph:
+        hga_timing_enable(slots)
+        graph = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(device)
+        s.wait_stream(torch.cuda.current_stream(device))
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(graph, stream=s):
+                run.step()
+        torch.cuda.current_stream(device).wait_stream(s)
+        graph.replay()
+        torch.cuda.synchronize(device)
+        hga_timing_collect()
+    hga_timing_reset()
+
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    bus = None
+    try:
+        bus = torch.cuda.get_device_properties(device).pci_bus_id
+    except Exception:
+        pass
+    sampler = None if args.no_clocks else ClockSampler(bus)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    launches0 = hga_launch_count()
+    for i in range(args.steps):
+        flush.zero_()
+        if graph is None:
+            hga_timing_enable(slots)
+        starts[i].record()
+        if graph is not None:
+            graph.replay()
+        else:
+            run.step()
+        ends[i].record()
+        hga_timing_collect()
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    launches = hga_launch_count() - launches0
+    if graph is not None:
+        launches = per_step_launches * args.steps   # graph replays bypass the host counter
+    clocks = sampler.stop() if sampler else None
+    hga_timing_enable(0)
+
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(step_ms), world, device)
+    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+
+    # per-kernel table and the dominant kernel's roofline
+    table = timing_table()
+    kernels = {}
+    for name, (ms, n) in table.items():
+        kernels[name] = {"launches": n, "ms_total": round(ms, 4),
+                         "share": round(ms / max(sum(v[0] for v in table.values()), 1e-12), 4)}
+    dom = max(table, key=lambda k: table[k][0])
+    dom_ms, dom_n = table[dom]
+    work, unit, bound = kernel_work(dom, w, sels)
+    work_per_launch = work / (dom_n / args.steps)
+    pk = peaks()
+    avg_s = dom_ms / dom_n / 1e3
+    if bound == "tensor":
+        achieved = work_per_launch / avg_s / 1e12
+        peak, punit = pk["tc_sustained"], "TFLOP/s"
+        peak_note = f"bf16 dense, sustained ({pk['source']})"
+    elif bound == "alu":
+        achieved = work_per_launch / avg_s / 1e12
+        peak, punit = FP32_ALU_TFLOPS, "TFLOP/s"
+        peak_note = "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz"
+    else:
+        achieved = work_per_launch / avg_s / 1e9
+        peak, punit = pk["hbm"], "GB/s"
+        peak_note = f"HBM copy ({pk['source']})"
+    roofline = {"kernel": dom, "bound": bound, "achieved": round(achieved, 3),
+                "peak": peak, "unit": punit, "frac": round(achieved / peak, 4),
+                "traffic": measured_traffic(dom, args.workload),
+                "work_per_launch": work_per_launch, "work_unit": unit,
+                "avg_launch_us": round(avg_s * 1e6, 3), "peak_source": peak_note}
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        L = run.layer
+        outs = (L.o, L.dq, L.dk, L.dv) if w.backward else (L.o,)
+        out_host = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+                    for _ in run.segs]
+        run.e2e_step(out_host)
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world, device)
+        e0.record()
+        for _ in range(args.steps):
+            run.e2e_step(out_host)
+        e1.record()
+        torch.cuda.synchronize(device)
+        barrier(world, device)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+        h2d, d2h = run.io_bytes()
+        e2e = {"value": round(world * tokens_per_step * args.steps / (e_ms / 1e3), 1),
+               "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w0, budget_s=15.0)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": args.workload, "batch_per_gpu": w.batch,
+                       "seq_len": w.ctx_len, "seg_len": w.seg_len, "n_q_heads": w.n_q_heads,
+                       "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+                       "topk_blocks": w.topk_blocks, "topk_groups": w.topk_groups,
+                       "backward": w.backward, "parallelism": f"replicas{world}",
+                       "l2": "flushed between timed steps (512 MiB write, untimed)",
+                       "graph": bool(args.graph), "attention": "simt" if args.simt else "auto"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(launches), "clocks": clocks, "kernels": kernels,
+        }
+        print(json.dumps(line), flush=True)
+    if graph is not None:
+        del graph
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------
+# the CPU oracle (baseline and reference arm)
+# ----------------------------------------------------------------------------
+
+def oracle_sample(w, q_begin, kv_heads):
+    """Oracle work of one segment restricted to `kv_heads`: summaries of the
+    history and the segment, routing, forward and backward.  Returns tokens of
+    full-layer work it stands for (segment tokens x share of heads)."""
+    import numpy as np
+    import oracle
+    from hierarchical_routed_sparse_hga_b200 import synth
+    G = w.group_heads
+    qh = [h * G + g for h in kv_heads for g in range(G)]
+    k = synth.widen(synth.keys(w, kv_heads), w.dtype)
+    v = synth.widen(synth.values(w, kv_heads), w.dtype)
+    q = synth.widen(synth.queries(w, q_begin, qh), w.dtype)
+    do = synth.widen(synth.douts(w, q_begin, qh), w.dtype) if w.backward else None
+    T = q_begin + w.seg_len
+    t0 = time.perf_counter()
+    gsum = np.zeros((w.batch, len(kv_heads), w.ctx_len // 8, w.head_dim))
+    bsum = np.zeros((w.batch, len(kv_heads), w.ctx_len // 64, w.head_dim))
+    if q_begin:
+        g, b = oracle.build_summaries(k, 0, q_begin)
+        gsum[:, :, :q_begin // 8], bsum[:, :, :q_begin // 64] = g, b
+    oracle.segment_step(q, k, v, do, q_begin, gsum, bsum, w.topk_blocks, w.topk_groups,
+                        len(kv_heads), backward=w.backward)
+    dt = time.perf_counter() - t0
+    return w.batch * w.seg_len * len(kv_heads) / w.n_kv_heads, dt, T
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, budget_s=15.0):
+    """Oracle on a bounded sample: the last segment, KV heads taken one at a time
+    until about budget_s seconds of CPU work."""
+    q_begin = w.segments()[-1]
+    tokens, secs, heads = 0.0, 0.0, []
+    for h in range(w.n_kv_heads):
+        t, dt, _ = oracle_sample(w, q_begin, [h])
+        tokens += t
+        secs += dt
+        heads.append(h)
+        if secs >= budget_s:
+            break
+    return {"value": round(tokens / secs, 2), "unit": "tokens/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{args_workload_name(w)}: segment at q_begin={q_begin} "
+                      f"({'fwd+bwd' if w.backward else 'fwd'}, summaries+route+attention), "
+                      f"KV heads {heads} of {w.n_kv_heads} (their {w.group_heads} query heads "
+                      f"each); tokens counted as seg_len x heads/{w.n_kv_heads}; "
+                      f"{secs:.1f} s of float64 NumPy"}
+
+
+def args_workload_name(w):
+    return w.name
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from hierarchical_routed_sparse_hga_b200 import synth
+    w = synth.workloads()[args.workload]
+    q_begin = w.segments()[-1]
+    for i in range(args.warmup):
+        oracle_sample(w, q_begin, [i % w.n_kv_heads])
+    tokens, secs = 0.0, 0.0
+    for i in range(args.steps):
+        t, dt, _ = oracle_sample(w, q_begin, [i % w.n_kv_heads])
+        tokens += t
+        secs += dt
+    value = tokens / secs
+    sample = (f"{w.name}: per step the oracle on the segment at q_begin={q_begin}, one KV "
+              f"head (rotating) of {w.n_kv_heads}; tokens counted as seg_len/{w.n_kv_heads}")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "seq_len": w.ctx_len, "seg_len": w.seg_len},
+            "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s",
+                             "cores": blas_threads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_gpu(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

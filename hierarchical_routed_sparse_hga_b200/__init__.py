@@ -1,0 +1,22 @@
+"""B200-native HGA hot path: libhga (C ABI, sm_100a kernels) and its binding.
+
+    from hierarchical_routed_sparse_hga_b200 import Config, HgaLayer
+    from hierarchical_routed_sparse_hga_b200 import hga_route, hga_attn_fwd, ...
+
+The shared library is loaded on first use; build it with
+`python -m hierarchical_routed_sparse_hga_b200.build`.
+"""
+from ._lib import (EXPORTS, HGA_BF16, HGA_F32, HGA_FLAG_SIMT, Config, HgaError,  # noqa: F401
+                   hga_attn_bwd, hga_attn_bwd_workspace_size, hga_attn_fwd,
+                   hga_build_summaries, hga_get_device_status, hga_kernel_name,
+                   hga_launch_count, hga_route, hga_route_workspace_size, hga_status_string,
+                   hga_timing_collect, hga_timing_enable, hga_timing_get, hga_timing_reset,
+                   hga_version, load, timing_table)
+
+
+def __getattr__(name):
+    # HgaLayer needs torch; import it lazily so CPU-only tools stay light
+    if name == "HgaLayer":
+        from .runtime import HgaLayer
+        return HgaLayer
+    raise AttributeError(name)

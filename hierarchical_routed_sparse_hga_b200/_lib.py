@@ -1,0 +1,232 @@
+"""ctypes binding of libhga (argument marshalling only).
+
+Every function here has the name and argument order of the C entry point in
+include/hga.h.  Array arguments are CUDA torch tensors (contiguous) or raw
+device addresses (int); the stream defaults to torch's current stream.  Every
+step of the hot path runs in libhga's kernels: there is no other code path, and
+a missing library raises instead of falling back.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhga.so")
+
+HGA_OK, HGA_ERR_INVALID_ARG, HGA_ERR_UNSUPPORTED, HGA_ERR_CUDA, HGA_ERR_TIMEOUT, \
+    HGA_ERR_DEVICE_CHECK, HGA_ERR_WORKSPACE = range(7)
+HGA_F32, HGA_BF16 = 0, 1
+HGA_FLAG_SIMT = 1
+
+EXPORTS = ("hga_version", "hga_status_string", "hga_build_summaries",
+           "hga_route_workspace_size", "hga_route", "hga_attn_fwd",
+           "hga_attn_bwd_workspace_size", "hga_attn_bwd", "hga_get_device_status",
+           "hga_kernel_name", "hga_launch_count", "hga_timing_enable", "hga_timing_collect",
+           "hga_timing_get", "hga_timing_reset")
+HGA_K_COUNT = 10
+
+
+class HgaError(RuntimeError):
+    def __init__(self, fn: str, status: int, text: str):
+        super().__init__(f"{fn}: {text} (status {status})")
+        self.status = status
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("topk_blocks", ctypes.c_int32), ("topk_groups", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32),
+                ("scale", ctypes.c_float)]
+
+
+@dataclasses.dataclass
+class Config:
+    """Mirror of hga_config_t."""
+    batch: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    topk_blocks: int
+    topk_groups: int
+    dtype: int = HGA_BF16
+    flags: int = 0
+    scale: float | None = None
+
+    def c(self) -> _Config:
+        scale = self.scale if self.scale is not None else 1.0 / math.sqrt(self.head_dim)
+        return _Config(self.batch, self.n_q_heads, self.n_kv_heads, self.head_dim,
+                       self.topk_blocks, self.topk_groups, self.dtype, self.flags, scale)
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load the in-tree libhga.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libhga.so is not built at {LIB_PATH}; run "
+                          "`python -m hierarchical_routed_sparse_hga_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    CFG = ctypes.POINTER(_Config)
+    sig = {
+        "hga_version": (ctypes.c_char_p, []),
+        "hga_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "hga_build_summaries": (ctypes.c_int, [CFG, P, I64, I64, I64, P, P, P]),
+        "hga_route_workspace_size": (SZ, [CFG, I32, I64]),
+        "hga_route": (ctypes.c_int, [CFG, P, I64, I32, I64, P, P, P, P, P, SZ, P]),
+        "hga_attn_fwd": (ctypes.c_int, [CFG, P, P, P, I64, I64, I32, P, P, P, P]),
+        "hga_attn_bwd_workspace_size": (SZ, [CFG, I32]),
+        "hga_attn_bwd": (ctypes.c_int, [CFG, P, P, P, I64, I64, I32, P, P, P, P, P, P, P,
+                                        P, SZ, P]),
+        "hga_get_device_status": (ctypes.c_int, [P]),
+        "hga_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
+        "hga_launch_count": (ctypes.c_uint64, []),
+        "hga_timing_enable": (ctypes.c_int, [I32]),
+        "hga_timing_collect": (ctypes.c_int, []),
+        "hga_timing_get": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_double),
+                                          ctypes.POINTER(ctypes.c_uint64)]),
+        "hga_timing_reset": (None, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    _lib = lib
+    return lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if not x.is_cuda:
+        raise ValueError("libhga takes device tensors")
+    if not x.is_contiguous():
+        raise ValueError("libhga takes contiguous tensors")
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn: str, status: int):
+    if status != HGA_OK:
+        raise HgaError(fn, status, load().hga_status_string(status).decode())
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+# ----------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ----------------------------------------------------------------------------
+
+def hga_version() -> str:
+    return load().hga_version().decode()
+
+
+def hga_status_string(status: int) -> str:
+    return load().hga_status_string(status).decode()
+
+
+def hga_build_summaries(cfg: Config, k, ctx_cap, t_begin, t_end, gsum, bsum, stream=None):
+    c = cfg.c()
+    _check("hga_build_summaries", load().hga_build_summaries(
+        ctypes.byref(c), _ptr(k), ctx_cap, t_begin, t_end, _ptr(gsum), _ptr(bsum),
+        _stream(stream)))
+
+
+def hga_route_workspace_size(cfg: Config, s_len, q_begin) -> int:
+    c = cfg.c()
+    return int(load().hga_route_workspace_size(ctypes.byref(c), s_len, q_begin))
+
+
+def hga_route(cfg: Config, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp,
+              workspace, ws_bytes=None, stream=None):
+    c = cfg.c()
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check("hga_route", load().hga_route(
+        ctypes.byref(c), _ptr(q), q_begin, s_len, ctx_cap, _ptr(bsum), _ptr(gsum),
+        _ptr(sel_blk), _ptr(sel_grp), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def hga_attn_fwd(cfg: Config, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, stream=None):
+    c = cfg.c()
+    _check("hga_attn_fwd", load().hga_attn_fwd(
+        ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), ctx_cap, q_begin, s_len, _ptr(sel_grp),
+        _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def hga_attn_bwd_workspace_size(cfg: Config, s_len) -> int:
+    c = cfg.c()
+    return int(load().hga_attn_bwd_workspace_size(ctypes.byref(c), s_len))
+
+
+def hga_attn_bwd(cfg: Config, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk,
+                 dv, workspace, ws_bytes=None, stream=None):
+    c = cfg.c()
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check("hga_attn_bwd", load().hga_attn_bwd(
+        ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), ctx_cap, q_begin, s_len, _ptr(sel_grp),
+        _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes,
+        _stream(stream)))
+
+
+def hga_get_device_status(stream=None) -> int:
+    return int(load().hga_get_device_status(_stream(stream)))
+
+
+# ----------------------------------------------------------------------------
+# diagnostics
+# ----------------------------------------------------------------------------
+
+def hga_kernel_name(kind: int) -> str:
+    return load().hga_kernel_name(kind).decode()
+
+
+def hga_launch_count() -> int:
+    return int(load().hga_launch_count())
+
+
+def hga_timing_enable(slots: int):
+    _check("hga_timing_enable", load().hga_timing_enable(slots))
+
+
+def hga_timing_collect():
+    _check("hga_timing_collect", load().hga_timing_collect())
+
+
+def hga_timing_get(kind: int):
+    ms, n = ctypes.c_double(), ctypes.c_uint64()
+    _check("hga_timing_get", load().hga_timing_get(kind, ctypes.byref(ms), ctypes.byref(n)))
+    return ms.value, int(n.value)
+
+
+def hga_timing_reset():
+    load().hga_timing_reset()
+
+
+def timing_table() -> dict:
+    """{kernel name: (total ms, timed launches)} for every kind timed so far."""
+    out = {}
+    for kind in range(HGA_K_COUNT):
+        ms, n = hga_timing_get(kind)
+        if n:
+            out[hga_kernel_name(kind)] = (ms, n)
+    return out

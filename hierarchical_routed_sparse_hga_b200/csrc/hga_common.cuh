@@ -1,0 +1,198 @@
+// Shared device helpers for libhga (element loads, block-wide scans, the
+// per-device status word).  Everything here is compiled into one translation
+// unit (libhga.cu), so the status word needs no relocatable device code.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hga.h"
+
+namespace hga {
+
+constexpr int kBlock = HGA_BLOCK;
+constexpr int kGroup = HGA_GROUP;
+constexpr int kQBlock = HGA_QBLOCK;
+constexpr int kGroupsPerBlock = kBlock / kGroup;
+
+// Latched device-side status (first error wins); read by hga_get_device_status.
+__device__ int g_device_status = 0;
+
+__device__ __forceinline__ void latch_status(int code) {
+  atomicCAS(&g_device_status, 0, code);
+}
+
+// ---------------------------------------------------------------------------
+// element loads: 8 consecutive elements -> 8 floats (16 B for bf16, 32 B for f32)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* f) {
+  uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ void load8(const float* p, float* f) {
+  float4 a = reinterpret_cast<const float4*>(p)[0];
+  float4 b = reinterpret_cast<const float4*>(p)[1];
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_float(float x) { return x; }
+
+template <typename T> __device__ __forceinline__ T from_float(float x);
+template <> __device__ __forceinline__ float from_float<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ void store8(float* p, const float* f) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(f[0], f[1], f[2], f[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
+}
+
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float* f) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// ---------------------------------------------------------------------------
+// order-preserving float -> uint32 key (larger float -> larger key; -0 == +0)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7fffffffu) == 0u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// ---------------------------------------------------------------------------
+// block-wide, order-preserving enumeration of a predicate over [0, n):
+// calls f(i, rank) for each i with pred(i), rank = number of earlier i with
+// pred.  Each thread owns a contiguous chunk, so ranks follow index order.
+// Needs `scratch` of at least (blockDim.x/32 + 1) ints in shared memory.
+// Returns the total count (same value in every thread).
+// ---------------------------------------------------------------------------
+template <typename Pred, typename Fn>
+__device__ int block_enumerate(int n, Pred pred, Fn f, int* scratch) {
+  const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = nt >> 5;
+  const int chunk = (n + nt - 1) / nt;
+  const int lo = min(n, tid * chunk), hi = min(n, lo + chunk);
+  int cnt = 0;
+  for (int i = lo; i < hi; ++i) cnt += pred(i) ? 1 : 0;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int w = 0; w < nwarps; ++w) {
+      int v = scratch[w];
+      scratch[w] = run;
+      run += v;
+    }
+    scratch[nwarps] = run;
+  }
+  __syncthreads();
+  int rank = scratch[warp] + incl - cnt;
+  for (int i = lo; i < hi; ++i) {
+    if (pred(i)) f(i, rank++);
+  }
+  int total = scratch[nwarps];
+  __syncthreads();
+  return total;
+}
+
+// ---------------------------------------------------------------------------
+// block-wide top-k of n distinct-or-not uint32 keys held in shared memory:
+// sets sel[i] = 1 for the k largest keys, ties broken toward the lower index.
+// Radix select on 8-bit digits (MSB first) finds the k-th largest key T; keys
+// above T are taken, and among keys equal to T the lowest indices fill the
+// remaining slots.  Needs hist[256] and scratch (see block_enumerate).
+// ---------------------------------------------------------------------------
+__device__ void block_topk(const uint32_t* key, int n, int k, uint8_t* sel, int* hist,
+                           int* scratch) {
+  const int nt = blockDim.x, tid = threadIdx.x;
+  if (k >= n) {
+    for (int i = tid; i < n; i += nt) sel[i] = 1;
+    __syncthreads();
+    return;
+  }
+  __shared__ uint32_t s_prefix, s_mask;
+  __shared__ int s_remaining;
+  if (tid == 0) { s_prefix = 0u; s_mask = 0u; s_remaining = k; }
+  __syncthreads();
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = tid; i < 256; i += nt) hist[i] = 0;
+    __syncthreads();
+    const uint32_t prefix = s_prefix, mask = s_mask;
+    for (int i = tid; i < n; i += nt) {
+      uint32_t kk = key[i];
+      if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // lane l owns digits 255-8l .. 248-8l (descending); find the digit where
+      // the running count from the top first reaches `remaining`.
+      const int lane = tid;
+      int local = 0;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) local += hist[255 - 8 * lane - t];
+      int incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int remaining = s_remaining;
+      const int excl = incl - local;
+      const bool mine = excl < remaining && incl >= remaining;
+      const unsigned ball = __ballot_sync(0xffffffffu, mine);
+      const int owner = __ffs(ball) - 1;
+      if (lane == owner) {
+        int above = excl;
+        for (int t = 0; t < 8; ++t) {
+          const int dgt = 255 - 8 * lane - t;
+          const int c = hist[dgt];
+          if (above + c >= remaining) {
+            s_prefix = prefix | (uint32_t(dgt) << shift);
+            s_mask = mask | (255u << shift);
+            s_remaining = remaining - above;
+            break;
+          }
+          above += c;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  const uint32_t thr = s_prefix;
+  const int need_equal = s_remaining;  // how many keys equal to thr are taken
+  for (int i = tid; i < n; i += nt) sel[i] = key[i] > thr ? 1 : 0;
+  __syncthreads();
+  block_enumerate(
+      n, [&](int i) { return key[i] == thr; },
+      [&](int i, int rank) {
+        if (rank < need_equal) sel[i] = 1;
+      },
+      scratch);
+  __syncthreads();
+}
+
+}  // namespace hga

@@ -1,0 +1,337 @@
+// libhga: C ABI of the HGA hot path (declarations and contracts in hga.h).
+// Host side: argument checks, workspace carving, kernel selection and launch.
+// Nothing here allocates, frees or synchronises (except hga_get_device_status).
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "hga.h"
+#include "hga_common.cuh"
+#include "summaries.cuh"
+#include "route.cuh"
+#include "attn_simt.cuh"
+#include "trace.cuh"
+
+using namespace hga;
+
+namespace {
+
+constexpr int64_t kMaxSegment = 4096;  // s_len limit (64 query blocks)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+hga_status_t check_cfg(const hga_config_t* c) {
+  if (!c) return HGA_ERR_INVALID_ARG;
+  if (c->batch < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1) return HGA_ERR_INVALID_ARG;
+  if (c->n_q_heads % c->n_kv_heads != 0) return HGA_ERR_INVALID_ARG;
+  if (c->n_q_heads / c->n_kv_heads > 8) return HGA_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128) return HGA_ERR_UNSUPPORTED;
+  if (c->dtype != HGA_F32 && c->dtype != HGA_BF16) return HGA_ERR_UNSUPPORTED;
+  if (c->topk_blocks < 1 || c->topk_blocks > 64) return HGA_ERR_UNSUPPORTED;
+  if (c->topk_groups < 1 || c->topk_groups > 256) return HGA_ERR_UNSUPPORTED;
+  if (!(c->scale > 0.f) || c->scale != c->scale) return HGA_ERR_INVALID_ARG;
+  if (c->batch > 65535 || c->n_q_heads > 65535) return HGA_ERR_UNSUPPORTED;
+  return HGA_OK;
+}
+
+hga_status_t check_segment(int64_t ctx_cap, int64_t q_begin, int32_t s_len) {
+  if (ctx_cap <= 0 || ctx_cap % kBlock) return HGA_ERR_INVALID_ARG;
+  if (q_begin < 0 || q_begin % kBlock) return HGA_ERR_INVALID_ARG;
+  if (s_len <= 0 || s_len % kQBlock) return HGA_ERR_INVALID_ARG;
+  if (s_len > kMaxSegment) return HGA_ERR_UNSUPPORTED;
+  if (q_begin + s_len > ctx_cap) return HGA_ERR_INVALID_ARG;
+  return HGA_OK;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device).
+hga_status_t ensure_smem(const void* fn, size_t bytes) {
+  if (bytes <= 48 * 1024) return HGA_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HGA_ERR_CUDA;
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, size_t> done;
+  std::lock_guard<std::mutex> lock(mu);
+  auto key = std::make_pair(fn, dev);
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return HGA_OK;
+  int optin = 0;
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return HGA_ERR_CUDA;
+  if (bytes > size_t(optin)) return HGA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) !=
+      cudaSuccess)
+    return HGA_ERR_CUDA;
+  done[key] = bytes;
+  return HGA_OK;
+}
+
+// Calls body.template operator()<T, D>() for the configured element type and d.
+template <typename Body>
+hga_status_t dispatch(const hga_config_t* c, Body&& body) {
+  if (c->dtype == HGA_BF16) {
+    if (c->head_dim == 128) return body.template operator()<__nv_bfloat16, 128>();
+    return body.template operator()<__nv_bfloat16, 64>();
+  }
+  if (c->head_dim == 128) return body.template operator()<float, 128>();
+  return body.template operator()<float, 64>();
+}
+
+struct RouteCarve {
+  float* qbar;
+  float* scores;
+  int64_t jstride;
+  size_t bytes;
+};
+
+RouteCarve route_carve(const hga_config_t* c, int32_t s_len, int64_t q_begin, void* base) {
+  const int64_t n_qb = s_len / kQBlock;
+  const int64_t heads = int64_t(c->batch) * c->n_kv_heads;
+  RouteCarve r;
+  r.jstride = ((q_begin / kBlock + n_qb) + 3) & ~int64_t(3);
+  const size_t qbar_bytes = align256(size_t(heads * n_qb * c->head_dim) * 4);
+  const size_t score_bytes = align256(size_t(heads * n_qb * r.jstride) * 4);
+  r.qbar = static_cast<float*>(base);
+  r.scores = base ? reinterpret_cast<float*>(static_cast<char*>(base) + qbar_bytes) : nullptr;
+  r.bytes = qbar_bytes + score_bytes;
+  return r;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* hga_version(void) { return "libhga 0.1 (sm_100a)"; }
+
+const char* hga_status_string(hga_status_t s) {
+  switch (s) {
+    case HGA_OK: return "ok";
+    case HGA_ERR_INVALID_ARG: return "invalid argument";
+    case HGA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case HGA_ERR_CUDA: return "CUDA error";
+    case HGA_ERR_TIMEOUT: return "device wait timed out";
+    case HGA_ERR_DEVICE_CHECK: return "device-side index check failed";
+    case HGA_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+hga_status_t hga_build_summaries(const hga_config_t* cfg, const void* k, int64_t ctx_cap,
+                                 int64_t t_begin, int64_t t_end, float* gsum, float* bsum,
+                                 void* stream) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if (!k || !gsum || !bsum || !aligned16(k) || !aligned16(gsum) || !aligned16(bsum))
+    return HGA_ERR_INVALID_ARG;
+  if (ctx_cap <= 0 || ctx_cap % kBlock || t_begin < 0 || t_begin % kBlock || t_end % kBlock ||
+      t_end < t_begin || t_end > ctx_cap)
+    return HGA_ERR_INVALID_ARG;
+  if (t_end == t_begin) return HGA_OK;
+  const int64_t n_blk = (t_end - t_begin) / kBlock;
+  if (n_blk > 0x7fffffff) return HGA_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
+    dim3 grid(unsigned(n_blk), cfg->n_kv_heads, cfg->batch);
+    return traced_launch(HGA_K_SUMMARIES, s, [&] {
+      summaries_kernel<T, D><<<grid, D, 0, s>>>(static_cast<const T*>(k), ctx_cap,
+                                                t_begin / kBlock, cfg->n_kv_heads, gsum, bsum);
+    });
+  });
+}
+
+size_t hga_route_workspace_size(const hga_config_t* cfg, int32_t s_len, int64_t q_begin) {
+  if (check_cfg(cfg) != HGA_OK || s_len <= 0 || q_begin < 0) return 0;
+  return route_carve(cfg, s_len, q_begin, nullptr).bytes;
+}
+
+hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, int32_t s_len,
+                       int64_t ctx_cap, const float* bsum, const float* gsum, int32_t* sel_blk,
+                       int32_t* sel_grp, void* workspace, size_t ws_bytes, void* stream) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
+  if (!q || !bsum || !gsum || !sel_grp || !workspace) return HGA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(bsum) || !aligned16(gsum) || !aligned16(sel_grp) ||
+      !aligned16(workspace) || (sel_blk && !aligned16(sel_blk)))
+    return HGA_ERR_INVALID_ARG;
+  RouteCarve ws = route_carve(cfg, s_len, q_begin, workspace);
+  if (ws_bytes < ws.bytes) return HGA_ERR_WORKSPACE;
+  const int n_qb = s_len / kQBlock;
+  const int64_t own0 = q_begin / kBlock;
+  const int64_t j_max = own0 + n_qb - 1;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
+    dim3 g1(n_qb, cfg->n_kv_heads, cfg->batch);
+    hga_status_t e = traced_launch(HGA_K_QMEAN, s, [&] {
+      qmean_kernel<T, D><<<g1, kRouteThreads, 0, s>>>(static_cast<const T*>(q), cfg->n_q_heads,
+                                                      cfg->n_kv_heads, s_len, ws.qbar);
+    });
+    if (e != HGA_OK) return e;
+    if (j_max > 0) {
+      const size_t sm2 = size_t(n_qb * D + D * (kScoreChunk + 1)) * 4;
+      e = ensure_smem(reinterpret_cast<const void*>(&block_score_kernel<D>), sm2);
+      if (e != HGA_OK) return e;
+      dim3 g2(unsigned((j_max + kScoreChunk - 1) / kScoreChunk), cfg->n_kv_heads, cfg->batch);
+      e = traced_launch(HGA_K_BLOCK_SCORE, s, [&] {
+        block_score_kernel<D><<<g2, kRouteThreads, sm2, s>>>(ws.qbar, bsum, ctx_cap,
+                                                             cfg->n_kv_heads, n_qb, own0,
+                                                             ws.scores, ws.jstride);
+      });
+      if (e != HGA_OK) return e;
+    }
+    const size_t sm3 = select_layout(own0 + n_qb, cfg->topk_blocks, D).total;
+    e = ensure_smem(reinterpret_cast<const void*>(&select_kernel<D>), sm3);
+    if (e != HGA_OK) return e;
+    return traced_launch(HGA_K_SELECT, s, [&] {
+      select_kernel<D><<<g1, kRouteThreads, sm3, s>>>(ws.qbar, ws.scores, gsum, ctx_cap,
+                                                      cfg->n_kv_heads, n_qb, own0, ws.jstride,
+                                                      cfg->topk_blocks, cfg->topk_groups,
+                                                      sel_blk, sel_grp);
+    });
+  });
+}
+
+hga_status_t hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k, const void* v,
+                          int64_t ctx_cap, int64_t q_begin, int32_t s_len,
+                          const int32_t* sel_grp, void* o, float* lse, void* stream) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
+  if (!q || !k || !v || !sel_grp || !o || !lse) return HGA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(sel_grp) || !aligned16(o) ||
+      !aligned16(lse))
+    return HGA_ERR_INVALID_ARG;
+  const int n_qb = s_len / kQBlock;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
+    const size_t sm = size_t(simt_fwd_smem_floats<D>()) * 4;
+    hga_status_t e =
+        ensure_smem(reinterpret_cast<const void*>(&attn_fwd_simt_kernel<T, D>), sm);
+    if (e != HGA_OK) return e;
+    dim3 grid(n_qb, cfg->n_q_heads, cfg->batch);
+    return traced_launch(HGA_K_FWD_SIMT, s, [&] {
+      attn_fwd_simt_kernel<T, D><<<grid, kSimtFwdThreads, sm, s>>>(
+          static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), ctx_cap,
+          q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups, sel_grp,
+          cfg->scale, static_cast<T*>(o), lse);
+    });
+  });
+}
+
+size_t hga_attn_bwd_workspace_size(const hga_config_t* cfg, int32_t s_len) {
+  if (check_cfg(cfg) != HGA_OK || s_len <= 0) return 0;
+  return align256(size_t(cfg->batch) * cfg->n_q_heads * size_t(s_len) * 4);
+}
+
+hga_status_t hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k, const void* v,
+                          int64_t ctx_cap, int64_t q_begin, int32_t s_len,
+                          const int32_t* sel_grp, const void* o, const float* lse,
+                          const void* d_o, void* dq, void* dk, void* dv, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
+  const void* ptrs[] = {q, k, v, sel_grp, o, lse, d_o, dq, dk, dv, workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return HGA_ERR_INVALID_ARG;
+  if (ws_bytes < hga_attn_bwd_workspace_size(cfg, s_len)) return HGA_ERR_WORKSPACE;
+  const int n_qb = s_len / kQBlock;
+  float* dvec = static_cast<float*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
+    const size_t sm1 = size_t(simt_fwd_smem_floats<D>()) * 4;
+    hga_status_t e =
+        ensure_smem(reinterpret_cast<const void*>(&attn_bwd_dq_simt_kernel<T, D>), sm1);
+    if (e != HGA_OK) return e;
+    dim3 g1(n_qb, cfg->n_q_heads, cfg->batch);
+    e = traced_launch(HGA_K_BWD_DQ_SIMT, s, [&] {
+      attn_bwd_dq_simt_kernel<T, D><<<g1, kSimtFwdThreads, sm1, s>>>(
+          static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), ctx_cap,
+          q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups, sel_grp,
+          cfg->scale, static_cast<const T*>(o), lse, static_cast<const T*>(d_o),
+          static_cast<T*>(dq), dvec);
+    });
+    if (e != HGA_OK) return e;
+    const size_t sm2 = size_t(simt_kv_smem_floats<D>()) * 4;
+    e = ensure_smem(reinterpret_cast<const void*>(&attn_bwd_dkdv_simt_kernel<T, D>), sm2);
+    if (e != HGA_OK) return e;
+    dim3 g2(n_qb, cfg->n_kv_heads, cfg->batch);
+    return traced_launch(HGA_K_BWD_DKDV_SIMT, s, [&] {
+      attn_bwd_dkdv_simt_kernel<T, D><<<g2, kSimtKvThreads, sm2, s>>>(
+          static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), ctx_cap,
+          q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups, sel_grp,
+          cfg->scale, lse, static_cast<const T*>(d_o), dvec, static_cast<T*>(dk),
+          static_cast<T*>(dv));
+    });
+  });
+}
+
+hga_status_t hga_get_device_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return HGA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return HGA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return HGA_ERR_CUDA;
+  return static_cast<hga_status_t>(v);
+}
+
+const char* hga_kernel_name(int kind) {
+  static const char* names[HGA_K_COUNT] = {
+      "summaries",      "route_qmean",       "route_block_score",   "route_select",
+      "attn_fwd_simt",  "attn_bwd_dq_simt",  "attn_bwd_dkdv_simt",  "attn_fwd_tc",
+      "attn_bwd_dq_tc", "attn_bwd_dkdv_tc"};
+  return (kind >= 0 && kind < HGA_K_COUNT) ? names[kind] : "unknown";
+}
+
+uint64_t hga_launch_count(void) { return tracer().launches.load(); }
+
+hga_status_t hga_timing_enable(int32_t slots) {
+  Tracer& t = tracer();
+  std::lock_guard<std::mutex> lock(t.mu);
+  if (slots < 0) return HGA_ERR_INVALID_ARG;
+  while (t.slots.size() < size_t(slots)) {
+    TimingSlot ts;
+    if (cudaEventCreate(&ts.begin) != cudaSuccess || cudaEventCreate(&ts.end) != cudaSuccess)
+      return HGA_ERR_CUDA;
+    t.slots.push_back(ts);
+  }
+  t.on = slots > 0;
+  t.next = 0;
+  return HGA_OK;
+}
+
+hga_status_t hga_timing_collect(void) {
+  Tracer& t = tracer();
+  std::lock_guard<std::mutex> lock(t.mu);
+  for (size_t i = 0; i < t.next; ++i) {
+    TimingSlot& ts = t.slots[i];
+    if (cudaEventSynchronize(ts.end) != cudaSuccess) return HGA_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, ts.begin, ts.end) != cudaSuccess) return HGA_ERR_CUDA;
+    t.ms[ts.kind] += ms;
+    t.count[ts.kind] += 1;
+  }
+  return HGA_OK;
+}
+
+hga_status_t hga_timing_get(int kind, double* ms, uint64_t* launches) {
+  if (kind < 0 || kind >= HGA_K_COUNT || !ms || !launches) return HGA_ERR_INVALID_ARG;
+  Tracer& t = tracer();
+  std::lock_guard<std::mutex> lock(t.mu);
+  *ms = t.ms[kind];
+  *launches = t.count[kind];
+  return HGA_OK;
+}
+
+void hga_timing_reset(void) {
+  Tracer& t = tracer();
+  std::lock_guard<std::mutex> lock(t.mu);
+  for (int i = 0; i < HGA_K_COUNT; ++i) { t.ms[i] = 0.0; t.count[i] = 0; }
+}
+
+}  // extern "C"

@@ -1,0 +1,220 @@
+// Steps a2 + a3: two-level weight-free routing ("BMW如何通过重新设计注意力机制…",
+// section "HGA的不同之处": queries score the block summaries, the top-k blocks
+// are opened at 8-token-group level, the router uses no learned weights and
+// scores the existing projected keys).
+//
+// Three launches, all HBM/L2-bound:
+//   qmean_kernel        qbar[b,h,j] = mean of the 64 x G query rows of query
+//                       block j (reads Q once, coalesced 16-byte loads);
+//   block_score_kernel  S[b,h,j,c] = qbar[b,h,j] . bsum[b,h,c] for a 64-block
+//                       chunk of candidates and every query block of the
+//                       segment -- one read of each block summary per KV head
+//                       instead of one per query block;
+//   select_kernel       per (b,h,j): radix top-k over the J candidate scores,
+//                       gather the selected blocks' 8*kb group summaries,
+//                       score them, radix top-k again, write both selections in
+//                       ascending index order.
+// Scores are not multiplied by 1/sqrt(d): a positive factor does not change
+// the ranking.
+#pragma once
+
+#include "hga_common.cuh"
+
+namespace hga {
+
+constexpr int kRouteThreads = 256;
+constexpr int kScoreChunk = 64;  // candidate blocks per block_score CTA
+
+struct RouteWs {
+  float* qbar;     // [B, Hkv, n_qb, D]
+  float* scores;   // [B, Hkv, n_qb, jstride]
+  int64_t jstride;
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kRouteThreads)
+    qmean_kernel(const T* __restrict__ q, int n_q_heads, int n_kv_heads, int s_len,
+                 float* __restrict__ qbar) {
+  constexpr int CH = D / 8;
+  constexpr int RS = kRouteThreads / CH;  // row slots
+  __shared__ float part[RS][D];
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int G = n_q_heads / n_kv_heads;
+  const int rows = G * kQBlock;
+  const int ch = threadIdx.x % CH, rs = threadIdx.x / CH;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  for (int r = rs; r < rows; r += RS) {
+    const int hq = h * G + r / kQBlock, t = j * kQBlock + r % kQBlock;
+    float f[8];
+    load8(q + ((int64_t(b) * n_q_heads + hq) * s_len + t) * D + ch * 8, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += f[e];
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[rs][ch * 8 + e] = acc[e];
+  __syncthreads();
+  const int n_qb = s_len / kQBlock;
+  for (int e = threadIdx.x; e < D; e += kRouteThreads) {
+    float s = 0.f;
+    for (int r = 0; r < RS; ++r) s += part[r][e];
+    qbar[((int64_t(b) * n_kv_heads + h) * n_qb + j) * D + e] = s / float(rows);
+  }
+}
+
+// grid (ceil(j_max / 64), Hkv, B); dynamic smem: (n_qb*D + D*65) floats
+template <int D>
+__global__ void __launch_bounds__(kRouteThreads)
+    block_score_kernel(const float* __restrict__ qbar, const float* __restrict__ bsum,
+                       int64_t ctx_cap, int n_kv_heads, int n_qb, int64_t own0,
+                       float* __restrict__ scores, int64_t jstride) {
+  extern __shared__ float smem[];
+  float* qb = smem;                // [n_qb][D]
+  float* bsT = smem + n_qb * D;    // [D][65] transposed chunk (padded: no bank conflicts)
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int64_t head = int64_t(b) * n_kv_heads + h;
+  const int64_t c0 = int64_t(blockIdx.x) * kScoreChunk;
+  const int64_t j_max = own0 + n_qb - 1;  // candidates of the last query block
+  const float* qsrc = qbar + head * n_qb * D;
+  for (int i = threadIdx.x; i < n_qb * D; i += kRouteThreads) qb[i] = qsrc[i];
+  const float* bsrc = bsum + head * (ctx_cap / kBlock) * D;
+  for (int i = threadIdx.x; i < kScoreChunk * D; i += kRouteThreads) {
+    const int cl = i / D, e = i % D;
+    const int64_t c = c0 + cl;
+    bsT[e * (kScoreChunk + 1) + cl] = c < j_max ? bsrc[c * D + e] : 0.f;
+  }
+  __syncthreads();
+  const int cl = threadIdx.x % kScoreChunk;
+  const int jg = threadIdx.x / kScoreChunk;  // 4 query-block lanes
+  constexpr int JG = kRouteThreads / kScoreChunk;
+  const int64_t c = c0 + cl;
+  for (int j0 = jg; j0 < n_qb; j0 += 4 * JG) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int e = 0; e < D; ++e) {
+      const float bv = bsT[e * (kScoreChunk + 1) + cl];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + u * JG;
+        if (j < n_qb) acc[u] = fmaf(qb[j * D + e], bv, acc[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u * JG;
+      if (j < n_qb && c < own0 + j) scores[(head * n_qb + j) * jstride + c] = acc[u];
+    }
+  }
+}
+
+// Shared-memory layout of select_kernel (16-byte aligned sections).
+struct SelectLayout {
+  size_t qb, key1, key2, blocks, hist, scratch, sel1, sel2, total;
+};
+
+__host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
+
+__host__ __device__ inline SelectLayout select_layout(int64_t j_cap, int topk_blocks, int D) {
+  SelectLayout L;
+  size_t o = 0;
+  L.qb = o;      o = align16(o + size_t(D) * 4);
+  L.key1 = o;    o = align16(o + size_t(j_cap) * 4);
+  L.key2 = o;    o = align16(o + size_t(8) * topk_blocks * 4);
+  L.blocks = o;  o = align16(o + size_t(topk_blocks) * 4);
+  L.hist = o;    o = align16(o + 256 * 4);
+  L.scratch = o; o = align16(o + 16 * 4);
+  L.sel1 = o;    o = align16(o + size_t(j_cap));
+  L.sel2 = o;    o = align16(o + size_t(8) * topk_blocks);
+  L.total = o;
+  return L;
+}
+
+// grid (n_qb, Hkv, B); dynamic smem select_layout(...).total
+template <int D>
+__global__ void __launch_bounds__(kRouteThreads)
+    select_kernel(const float* __restrict__ qbar, const float* __restrict__ scores,
+                  const float* __restrict__ gsum, int64_t ctx_cap, int n_kv_heads, int n_qb,
+                  int64_t own0, int64_t jstride, int topk_blocks, int topk_groups,
+                  int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp) {
+  extern __shared__ __align__(16) unsigned char sm_raw[];
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int64_t head = int64_t(b) * n_kv_heads + h;
+  const int64_t J = own0 + j;                 // candidate blocks [0, J)
+  const int kb = int(J < topk_blocks ? J : topk_blocks);
+  const int64_t j_cap = own0 + n_qb;
+  const int n2 = 8 * kb;
+
+  const SelectLayout L = select_layout(j_cap, topk_blocks, D);
+  float* qb = reinterpret_cast<float*>(sm_raw + L.qb);
+  uint32_t* key1 = reinterpret_cast<uint32_t*>(sm_raw + L.key1);
+  uint32_t* key2 = reinterpret_cast<uint32_t*>(sm_raw + L.key2);
+  int* blocks = reinterpret_cast<int*>(sm_raw + L.blocks);
+  int* hist = reinterpret_cast<int*>(sm_raw + L.hist);
+  int* scratch = reinterpret_cast<int*>(sm_raw + L.scratch);
+  uint8_t* sel1 = sm_raw + L.sel1;
+  uint8_t* sel2 = sm_raw + L.sel2;
+
+  const float* srow = scores + (head * n_qb + j) * jstride;
+  for (int64_t i = threadIdx.x; i < J; i += kRouteThreads) key1[i] = ordered_key(srow[i]);
+  for (int i = threadIdx.x; i < D; i += kRouteThreads) qb[i] = qbar[(head * n_qb + j) * D + i];
+  __syncthreads();
+
+  // level 1
+  block_topk(key1, int(J), kb, sel1, hist, scratch);
+  block_enumerate(
+      int(J), [&](int i) { return sel1[i] != 0; }, [&](int i, int r) { blocks[r] = i; },
+      scratch);
+  int32_t* out_blk = sel_blk ? sel_blk + (head * n_qb + j) * topk_blocks : nullptr;
+  if (out_blk)
+    for (int i = threadIdx.x; i < topk_blocks; i += kRouteThreads)
+      out_blk[i] = i < kb ? blocks[i] : -1;
+
+  // level 2: score the 8 groups of every kept block (candidate p -> group
+  // blocks[p/8]*8 + p%8, which is ascending in p)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int NW = kRouteThreads / 32;
+  constexpr int V4 = D / 4;  // float4 per summary row
+  const float4* qb4 = reinterpret_cast<const float4*>(qb);
+  const float* gbase = gsum + head * (ctx_cap / kGroup) * D;
+  for (int p0 = warp * 4; p0 < n2; p0 += NW * 4) {
+    float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int p = p0 + u;
+      if (p < n2) {
+        const int64_t g = int64_t(blocks[p >> 3]) * kGroupsPerBlock + (p & 7);
+        const float4* row = reinterpret_cast<const float4*>(gbase + g * D);
+        for (int e = lane; e < V4; e += 32) {
+          const float4 x = row[e], y = qb4[e];
+          part[u] = fmaf(x.x, y.x, part[u]);
+          part[u] = fmaf(x.y, y.y, part[u]);
+          part[u] = fmaf(x.z, y.z, part[u]);
+          part[u] = fmaf(x.w, y.w, part[u]);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) part[u] += __shfl_xor_sync(0xffffffffu, part[u], o);
+    }
+    if (lane < 4 && p0 + lane < n2) {
+      float v = part[0];
+      if (lane == 1) v = part[1];
+      if (lane == 2) v = part[2];
+      if (lane == 3) v = part[3];
+      key2[p0 + lane] = ordered_key(v);
+    }
+  }
+  __syncthreads();
+  const int kg = n2 < topk_groups ? n2 : topk_groups;
+  block_topk(key2, n2, kg, sel2, hist, scratch);
+  int32_t* out_grp = sel_grp + (head * n_qb + j) * topk_groups;
+  block_enumerate(
+      n2, [&](int p) { return sel2[p] != 0; },
+      [&](int p, int r) { out_grp[r] = blocks[p >> 3] * kGroupsPerBlock + (p & 7); }, scratch);
+  for (int i = kg + threadIdx.x; i < topk_groups; i += kRouteThreads) out_grp[i] = -1;
+}
+
+}  // namespace hga

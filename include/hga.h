@@ -1,0 +1,233 @@
+/*
+ * libhga -- the data-parallel hot path of Hierarchical Global Attention (HGA)
+ * on NVIDIA B200 (sm_100a).  C ABI: plain pointers, sizes and a CUDA stream
+ * handle passed as void*.  No call allocates, frees or synchronises unless its
+ * comment says so; every call is asynchronous on the given stream.
+ *
+ * Method sources (the HGA pages, all on "Long-Context Fine-Tuning with Limited
+ * VRAM"):
+ *   [A] adnankhan.ai notes "Long-Context Fine-Tuning with Limited VRAM",
+ *       section "Raw Abstract / Excerpt": a bounded set of exact historical
+ *       tokens per query block; only the active segment stays differentiable,
+ *       older KV is detached.
+ *   [B] seventnews "BMW如何通过重新设计注意力机制，在16 GB GPU上实现16K上下文",
+ *       section "HGA的不同之处" (what HGA does differently): 64-token blocks
+ *       with one compact summary each kept on the GPU; queries score the
+ *       summaries and pick the top-k blocks; the blocks are opened at the level
+ *       of 8-token groups; only the selected groups' exact-token K/V enter the
+ *       attention; the router has no learned weights; summaries are never
+ *       attention values; 2048-token segments with forward and backward per
+ *       segment and no gradient across segment boundaries.
+ *   [C] gist.science retelling, section "解决方案" (the solution): block
+ *       summary cards and an 8-token group summary cache.
+ *
+ * Readings fixed here (the pages leave them open): a summary is the mean of
+ * the post-RoPE keys of its block/group per KV head; a query block is 64
+ * tokens; the routing score of a candidate is the mean over the query block's
+ * 64 queries and the G = n_q_heads/n_kv_heads heads sharing the KV head of
+ * q.s/sqrt(d); candidates of query block j are the complete blocks strictly
+ * before its own block; level 2 ranks only the groups of the selected blocks;
+ * ties go to the lower index; each query attends to the selected groups plus
+ * the causal part of its own block.
+ *
+ * Layouts (row-major, innermost last; element type = cfg->dtype unless noted):
+ *   K, V            [batch, n_kv_heads, ctx_cap, head_dim]   whole context;
+ *                   the active segment occupies tokens [q_begin, q_begin+s_len)
+ *   Q, O, dO, dQ    [batch, n_q_heads, s_len, head_dim]      active segment
+ *   dK, dV          [batch, n_kv_heads, s_len, head_dim]     active segment only
+ *   LSE             [batch, n_q_heads, s_len]                float32, natural log
+ *   gsum            [batch, n_kv_heads, ctx_cap/8,  head_dim] float32
+ *   bsum            [batch, n_kv_heads, ctx_cap/64, head_dim] float32
+ *   sel_blk         [batch, n_kv_heads, s_len/64, topk_blocks] int32
+ *   sel_grp         [batch, n_kv_heads, s_len/64, topk_groups] int32
+ *                   global group indices (token = 8*g + i), ascending, -1 padded
+ *
+ * Ownership: the caller allocates and owns every buffer (device memory for all
+ * arrays; the stream).  Pointers must be 16-byte aligned.  ctx_cap, q_begin,
+ * t_begin, t_end and s_len must be multiples of 64.
+ *
+ * Errors: host-side argument checks run before any launch and return
+ * HGA_ERR_INVALID_ARG / HGA_ERR_UNSUPPORTED / HGA_ERR_WORKSPACE with nothing
+ * launched.  A failed launch returns HGA_ERR_CUDA.  Kernels that detect a bad
+ * selection entry (a group outside [0, 8*own_block)) skip it and latch
+ * HGA_ERR_DEVICE_CHECK in a per-device status word; a bounded wait that gives
+ * up latches HGA_ERR_TIMEOUT.  hga_get_device_status() reads and clears it.
+ */
+#ifndef HGA_H
+#define HGA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define HGA_API __attribute__((visibility("default")))
+#else
+#define HGA_API
+#endif
+
+#define HGA_BLOCK 64   /* tokens per block  [B], [C] */
+#define HGA_GROUP 8    /* tokens per group  [B], [C] */
+#define HGA_QBLOCK 64  /* queries per query block */
+
+typedef enum {
+  HGA_OK = 0,
+  HGA_ERR_INVALID_ARG = 1,
+  HGA_ERR_UNSUPPORTED = 2,
+  HGA_ERR_CUDA = 3,
+  HGA_ERR_TIMEOUT = 4,
+  HGA_ERR_DEVICE_CHECK = 5,
+  HGA_ERR_WORKSPACE = 6
+} hga_status_t;
+
+typedef enum { HGA_F32 = 0, HGA_BF16 = 1 } hga_dtype_t;
+
+/* flags */
+#define HGA_FLAG_SIMT 1u  /* force the CUDA-core attention kernels (fp32 always uses them) */
+
+typedef struct {
+  int32_t batch;
+  int32_t n_q_heads;     /* multiple of n_kv_heads; G = n_q_heads / n_kv_heads <= 8 */
+  int32_t n_kv_heads;
+  int32_t head_dim;      /* 64 or 128 */
+  int32_t topk_blocks;   /* level-1 k, 1..64 */
+  int32_t topk_groups;   /* level-2 k, 1..256 */
+  int32_t dtype;         /* hga_dtype_t: HGA_F32 or HGA_BF16 */
+  uint32_t flags;        /* HGA_FLAG_* */
+  float scale;           /* softmax scale, normally 1/sqrt(head_dim) */
+} hga_config_t;
+
+/* Library version string. */
+HGA_API const char* hga_version(void);
+
+/* Human-readable name of a status code. */
+HGA_API const char* hga_status_string(hga_status_t status);
+
+/*
+ * Step a1 -- summaries [B], [C].  For tokens [t_begin, t_end) of K:
+ *   gsum[b,h,g] = mean of keys 8g .. 8g+7      (g = t_begin/8 .. t_end/8-1)
+ *   bsum[b,h,c] = mean of keys 64c .. 64c+63   (c = t_begin/64 .. t_end/64-1)
+ * accumulated in float32.  Rows outside the range are not touched, so calling
+ * it once per segment appends that segment's summaries.
+ */
+HGA_API hga_status_t hga_build_summaries(const hga_config_t* cfg, const void* k, int64_t ctx_cap,
+                                 int64_t t_begin, int64_t t_end, float* gsum, float* bsum,
+                                 void* stream);
+
+/* Bytes of device workspace hga_route needs for this segment. */
+HGA_API size_t hga_route_workspace_size(const hga_config_t* cfg, int32_t s_len, int64_t q_begin);
+
+/*
+ * Steps a2 + a3 -- two-level weight-free routing [B].  For every (b, KV head h,
+ * query block j) of the segment starting at global token q_begin:
+ *   qbar = mean of Q over the 64 tokens of block j and the G heads of h;
+ *   level 1: score_c = qbar . bsum[b,h,c] for c in [0, J), J = q_begin/64 + j,
+ *            keep the top min(topk_blocks, J) (ties: lower c);
+ *   level 2: score_g = qbar . gsum[b,h,g] for the 8 groups of each kept block,
+ *            keep the top min(topk_groups, 8*kept) (ties: lower g).
+ * Scores are ranked without the positive factor 1/sqrt(d) (order unchanged).
+ * Writes sel_grp and, if sel_blk is not NULL, sel_blk (ascending, -1 padded).
+ * bsum/gsum must hold every block/group before the segment's last block
+ * (call hga_build_summaries for the segment first).
+ * workspace: at least hga_route_workspace_size() bytes of device memory.
+ */
+HGA_API hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, int32_t s_len,
+                       int64_t ctx_cap, const float* bsum, const float* gsum,
+                       int32_t* sel_blk, int32_t* sel_grp, void* workspace, size_t ws_bytes,
+                       void* stream);
+
+/*
+ * Step a4 -- exact-token attention forward [A], [B].  Query t of head h'
+ * (KV head h'/G, query block j, global position p = q_begin + t) attends to
+ *   { 8g+i : g in sel_grp[b,h,j], i < 8 }  U  { own-block tokens at positions <= p }
+ * with softmax scale cfg->scale:  O = softmax(q K^T * scale) V,
+ * LSE = log(sum exp(q k * scale)).  K/V are read from the whole-context buffers.
+ */
+HGA_API hga_status_t hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k, const void* v,
+                          int64_t ctx_cap, int64_t q_begin, int32_t s_len,
+                          const int32_t* sel_grp, void* o, float* lse, void* stream);
+
+/* Bytes of device workspace hga_attn_bwd needs for this segment. */
+HGA_API size_t hga_attn_bwd_workspace_size(const hga_config_t* cfg, int32_t s_len);
+
+/*
+ * Step a5 -- backward under segment-wise backprop [A], [B].  Gradients of
+ * sum(dO * O) for the forward above, recomputed from the saved LSE:
+ *   D = rowsum(dO * O);  P = exp(q k * scale - LSE);  dS = P (dO v - D)
+ *   dQ = scale * sum_k dS k                               (every attended key)
+ *   dK = scale * sum dS q,  dV = sum P dO                 (active-segment keys only,
+ *        summed over the G heads and every query block that attends to them)
+ * History keys (positions < q_begin) are detached: no gradient is produced for
+ * them.  dq, dk, dv are written, not accumulated.  workspace: at least
+ * hga_attn_bwd_workspace_size() bytes of device memory.
+ */
+HGA_API hga_status_t hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k, const void* v,
+                          int64_t ctx_cap, int64_t q_begin, int32_t s_len,
+                          const int32_t* sel_grp, const void* o, const float* lse,
+                          const void* d_o, void* dq, void* dk, void* dv, void* workspace,
+                          size_t ws_bytes, void* stream);
+
+/*
+ * Reads and clears the calling device's latched device-side status
+ * (HGA_OK, HGA_ERR_DEVICE_CHECK or HGA_ERR_TIMEOUT).  Synchronises `stream`.
+ */
+HGA_API hga_status_t hga_get_device_status(void* stream);
+
+
+/* ------------------------------------------------------------------------
+ * Diagnostics: launch counting and per-kernel timing.
+ *
+ * Every kernel launch of the library increments a process-wide counter.
+ * When timing is enabled, each launch is bracketed by two CUDA events
+ * recorded on its stream (as external event nodes while the stream is being
+ * captured into a CUDA graph, so graph replays are timed too).  Events come
+ * from a pool created by hga_timing_enable (host-side event objects, no
+ * device memory); launches beyond the pool are not timed.
+ * ------------------------------------------------------------------------ */
+
+/* Kernel kinds reported by the timing facility. */
+typedef enum {
+  HGA_K_SUMMARIES = 0,
+  HGA_K_QMEAN = 1,
+  HGA_K_BLOCK_SCORE = 2,
+  HGA_K_SELECT = 3,
+  HGA_K_FWD_SIMT = 4,
+  HGA_K_BWD_DQ_SIMT = 5,
+  HGA_K_BWD_DKDV_SIMT = 6,
+  HGA_K_FWD_TC = 7,
+  HGA_K_BWD_DQ_TC = 8,
+  HGA_K_BWD_DKDV_TC = 9,
+  HGA_K_COUNT = 10
+} hga_kernel_kind_t;
+
+/* Name of a kernel kind ("attn_fwd_simt", ...). */
+HGA_API const char* hga_kernel_name(int kind);
+
+/* Number of kernels this library has launched in this process. */
+HGA_API uint64_t hga_launch_count(void);
+
+/* slots > 0: enable timing with a pool of `slots` event pairs (created on
+ * first use, reused afterwards); 0: disable.  Rewinds the pool cursor, so the
+ * next launches use slots 0, 1, ... again. */
+HGA_API hga_status_t hga_timing_enable(int32_t slots);
+
+/* Waits for the event pairs of the slots used since the last
+ * hga_timing_enable and adds their durations to the per-kind totals.  Eager
+ * use: enable, launch, collect.  Graph use: enable, capture (the captured
+ * launches keep their slots), then replay + collect as often as wanted. */
+HGA_API hga_status_t hga_timing_collect(void);
+
+/* Accumulated milliseconds and timed launches of one kernel kind. */
+HGA_API hga_status_t hga_timing_get(int kind, double* ms, uint64_t* launches);
+
+/* Zeroes the per-kind totals. */
+HGA_API void hga_timing_reset(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HGA_H */

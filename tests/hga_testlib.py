@@ -1,0 +1,137 @@
+"""Helpers shared by the parity tests: run the CUDA path through the C ABI on
+seeded synthetic inputs and run the oracle on the same inputs."""
+
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+from hierarchical_routed_sparse_hga_b200 import synth
+
+# tolerances: float32 path max-abs 1e-4; bf16 path 2e-2 of the tensor's max |oracle|
+F32_ABS = 1e-4
+BF16_REL = 2e-2
+LSE_ABS = 1e-4
+SUMMARY_REL = 1e-5
+
+
+def torch_dtype(w):
+    import torch
+    return torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+
+def to_device(arr, w, device="cuda"):
+    """Storage numpy array (uint16 bf16 bits or float32) -> CUDA tensor."""
+    import torch
+    if w.dtype == "bf16":
+        t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(np.ascontiguousarray(arr, dtype=np.float32))
+    return t.to(device)
+
+
+def to_f64(t):
+    import torch
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def config_of(w, flags=0):
+    from hierarchical_routed_sparse_hga_b200 import HGA_BF16, HGA_F32, Config
+    return Config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.topk_blocks,
+                  w.topk_groups, HGA_BF16 if w.dtype == "bf16" else HGA_F32, flags)
+
+
+def assert_close(gpu, ref, w, what, rel=None, abs_=None):
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
+    err = np.max(np.abs(gpu - ref)) if ref.size else 0.0
+    if abs_ is not None:
+        bound = abs_
+    elif rel is not None:
+        bound = rel * max(np.max(np.abs(ref)), 1e-30)
+    elif w.dtype == "f32":
+        bound = F32_ABS
+    else:
+        bound = BF16_REL * max(np.max(np.abs(ref)), 1e-30)
+    assert err <= bound, f"{what}: max err {err:.3e} > {bound:.3e}"
+    return err
+
+
+def check_selection(gpu_sel, ref_sel, tie, what):
+    """Indices bit-exact except on rows flagged as near ties."""
+    gpu_sel = np.asarray(gpu_sel)
+    mism = np.any(gpu_sel != ref_sel, axis=-1)
+    bad = mism & ~tie
+    assert not bad.any(), f"{what}: {int(bad.sum())} unflagged rows differ, first at " \
+                          f"{np.argwhere(bad)[0].tolist()}"
+    return int(mism.sum())
+
+
+class Segmenter:
+    """Runs a workload segment by segment on the GPU (HgaLayer) and, for the
+    segments asked for, on the oracle with the same inputs."""
+
+    def __init__(self, w, kv_heads=None, flags=0):
+        import torch
+        from hierarchical_routed_sparse_hga_b200 import HgaLayer
+        self.w = w
+        self.heads = list(range(w.n_kv_heads)) if kv_heads is None else list(kv_heads)
+        G = w.group_heads
+        self.q_heads = [h * G + g for h in self.heads for g in range(G)]
+        k_np, v_np = synth.keys(w), synth.values(w)
+        self.k64 = synth.widen(k_np[:, self.heads], w.dtype)
+        self.v64 = synth.widen(v_np[:, self.heads], w.dtype)
+        self.layer = HgaLayer(config_of(w, flags), w.ctx_len, w.seg_len,
+                              k=to_device(k_np, w), v=to_device(v_np, w))
+        # history before the first query-carrying segment is summarised up front
+        first = w.segments()[0]
+        if first:
+            from hierarchical_routed_sparse_hga_b200 import hga_build_summaries
+            hga_build_summaries(self.layer.cfg, self.layer.k, w.ctx_len, 0, first,
+                                self.layer.gsum, self.layer.bsum)
+        torch.cuda.synchronize()
+
+    def run_segment(self, q_begin, backward=None):
+        import torch
+        w = self.w
+        backward = w.backward if backward is None else backward
+        q_np = synth.queries(w, q_begin)
+        q = to_device(q_np, w)
+        d_o = to_device(synth.douts(w, q_begin), w) if backward else None
+        self.layer.segment(q, q_begin, d_o)
+        torch.cuda.synchronize()
+        L = self.layer
+        hs, qs = self.heads, self.q_heads
+        out = dict(q64=synth.widen(q_np[:, qs], w.dtype),
+                   sel_blk=L.sel_blk[:, hs].cpu().numpy(), sel_grp=L.sel_grp[:, hs].cpu().numpy(),
+                   o=to_f64(L.o[:, qs]), lse=to_f64(L.lse[:, qs]),
+                   gsum=to_f64(L.gsum[:, hs]), bsum=to_f64(L.bsum[:, hs]))
+        if backward:
+            out.update(do64=synth.widen(synth.douts(w, q_begin)[:, qs], w.dtype),
+                       dq=to_f64(L.dq[:, qs]), dk=to_f64(L.dk[:, hs]), dv=to_f64(L.dv[:, hs]))
+        return out
+
+
+def compare_segment(w, gpu, q_begin, n_kv, k64, v64, backward):
+    """Oracle on the same inputs (heads already sliced); asserts parity."""
+    T_end = q_begin + w.seg_len
+    g_ref, b_ref = oracle.build_summaries(k64, 0, T_end)
+    assert_close(gpu["gsum"][:, :, :T_end // 8], g_ref, w, "gsum", rel=SUMMARY_REL)
+    assert_close(gpu["bsum"][:, :, :T_end // 64], b_ref, w, "bsum", rel=SUMMARY_REL)
+    sb, sg, tie = oracle.route(gpu["q64"], b_ref, g_ref, q_begin, w.topk_blocks,
+                               w.topk_groups, n_kv)
+    check_selection(gpu["sel_blk"], sb, tie, "sel_blk")
+    check_selection(gpu["sel_grp"], sg, tie, "sel_grp")
+    # attention is checked on the GPU's selection (equal to the oracle's on
+    # every unflagged row, as just asserted)
+    o, lse = oracle.attn_fwd(gpu["q64"], k64, v64, q_begin, gpu["sel_grp"], n_kv)
+    assert_close(gpu["o"], o, w, "o")
+    assert_close(gpu["lse"], lse, w, "lse", abs_=LSE_ABS)
+    if backward:
+        dq, dk, dv = oracle.attn_bwd(gpu["q64"], k64, v64, gpu["do64"], q_begin,
+                                     gpu["sel_grp"], n_kv)
+        assert_close(gpu["dq"], dq, w, "dq")
+        assert_close(gpu["dk"], dk, w, "dk")
+        assert_close(gpu["dv"], dv, w, "dv")
+    return int(tie.sum())

@@ -1,0 +1,97 @@
+"""The C ABI library on the CPU: it loads, exports every declared entry point,
+and rejects bad arguments on the host before any launch (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import hierarchical_routed_sparse_hga_b200 as hga
+from hierarchical_routed_sparse_hga_b200 import _lib
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "include", "hga.h")
+
+
+def declared():
+    text = open(HEADER).read()
+    return set(re.findall(r"HGA_API\s+[\w\s\*]+?\b(hga_\w+)\s*\(", text))
+
+
+def test_header_declares_what_the_binding_names():
+    assert declared() == set(_lib.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(_lib.LIB_PATH)
+    for name in declared():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings():
+    assert "sm_100a" in hga.hga_version()
+    assert hga.hga_status_string(0) == "ok"
+    assert hga.hga_status_string(6) == "workspace too small"
+
+
+def cfg(**kw):
+    base = dict(batch=1, n_q_heads=32, n_kv_heads=8, head_dim=128, topk_blocks=16,
+                topk_groups=64)
+    base.update(kw)
+    return hga.Config(**base)
+
+
+FAKE = 0x10000  # aligned, never dereferenced: every call below fails its host check
+
+
+def status_of(fn, *args):
+    with pytest.raises(hga.HgaError) as e:
+        fn(*args)
+    return e.value.status
+
+
+def test_host_argument_checks():
+    c = cfg()
+    # null pointers
+    assert status_of(hga.hga_build_summaries, c, 0, 16384, 0, 2048, FAKE, FAKE, 0) == 1
+    # not a multiple of 64
+    assert status_of(hga.hga_build_summaries, c, FAKE, 16384, 32, 2048, FAKE, FAKE, 0) == 1
+    # misaligned pointer
+    assert status_of(hga.hga_attn_fwd, c, FAKE + 4, FAKE, FAKE, 16384, 0, 2048, FAKE, FAKE,
+                     FAKE, 0) == 1
+    # unsupported head dim / GQA ratio / k
+    assert status_of(hga.hga_attn_fwd, cfg(head_dim=96), FAKE, FAKE, FAKE, 16384, 0, 2048,
+                     FAKE, FAKE, FAKE, 0) == 2
+    assert status_of(hga.hga_attn_fwd, cfg(n_q_heads=80, n_kv_heads=8), FAKE, FAKE, FAKE,
+                     16384, 0, 2048, FAKE, FAKE, FAKE, 0) == 2
+    assert status_of(hga.hga_attn_fwd, cfg(topk_groups=0), FAKE, FAKE, FAKE, 16384, 0, 2048,
+                     FAKE, FAKE, FAKE, 0) == 2
+    # segment past the context
+    assert status_of(hga.hga_attn_fwd, c, FAKE, FAKE, FAKE, 16384, 15360, 2048, FAKE, FAKE,
+                     FAKE, 0) == 1
+    # segment too long
+    assert status_of(hga.hga_attn_fwd, c, FAKE, FAKE, FAKE, 16384, 0, 8192, FAKE, FAKE,
+                     FAKE, 0) == 2
+    # workspace too small
+    need = hga.hga_route_workspace_size(c, 2048, 14336)
+    assert status_of(hga.hga_route, c, FAKE, 14336, 2048, 16384, FAKE, FAKE, None, FAKE, FAKE,
+                     need - 256, 0) == 6
+    need = hga.hga_attn_bwd_workspace_size(c, 2048)
+    assert status_of(hga.hga_attn_bwd, c, FAKE, FAKE, FAKE, 16384, 14336, 2048, FAKE, FAKE,
+                     FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 4, 0) == 6
+
+
+def test_workspace_sizes():
+    c = cfg()
+    # qbar 8 heads x 32 blocks x 128 floats + scores 8 x 32 x 256 floats (256-B aligned)
+    assert hga.hga_route_workspace_size(c, 2048, 14336) == 8 * 32 * 128 * 4 + 8 * 32 * 256 * 4
+    assert hga.hga_attn_bwd_workspace_size(c, 2048) == 32 * 2048 * 4
+    assert hga.hga_route_workspace_size(cfg(head_dim=100), 2048, 0) == 0
+
+
+def test_diagnostics_without_gpu():
+    assert hga.hga_kernel_name(0) == "summaries"
+    assert hga.hga_kernel_name(99) == "unknown"
+    assert hga.hga_launch_count() >= 0
+    assert hga.timing_table() == {}

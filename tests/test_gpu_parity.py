@@ -1,0 +1,126 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Indices are compared bit-exactly except on rows the oracle flags as near ties
+(k-th and (k+1)-th scores within 1e-3 relative); attention there is checked on
+the GPU's own selection.  Values: float32 max-abs 1e-4; bf16 2e-2 of the
+tensor's max |oracle|; LSE 1e-4 absolute; summaries 1e-5 relative.
+"""
+
+import numpy as np
+import pytest
+
+from hierarchical_routed_sparse_hga_b200 import synth
+
+from hga_testlib import Segmenter, compare_segment
+
+pytestmark = pytest.mark.gpu
+
+WL = synth.workloads()
+
+
+def run_and_compare(w, segments=None, kv_heads=None, flags=0):
+    seg = Segmenter(w, kv_heads=kv_heads, flags=flags)
+    n_kv = len(seg.heads)
+    want = set(w.segments() if segments is None else segments)
+    flagged = 0
+    for q_begin in w.segments():
+        out = seg.run_segment(q_begin)
+        if q_begin in want:
+            flagged += compare_segment(w, out, q_begin, n_kv, seg.k64, seg.v64, w.backward)
+    return flagged
+
+
+def test_tiny_f32_fwd_bwd():
+    run_and_compare(WL["tiny_f32"])
+
+
+def test_qwen3_fwd_16k():
+    run_and_compare(WL["qwen3_fwd_16k"])
+
+
+def test_qwen3_fwdbwd_16k_all_segments():
+    # the benchmark's workload: 8 segments of 2048, fwd+bwd, every head
+    run_and_compare(WL["qwen3_fwdbwd_16k"])
+
+
+@pytest.mark.slow
+def test_qwen3_fwd_128k_sampled():
+    # 64 segments on the GPU; segments 0, 31 and 63 checked on two KV heads
+    w = WL["qwen3_fwd_128k"]
+    run_and_compare(w, segments=[0, 31 * 2048, 63 * 2048], kv_heads=[0, 5])
+
+
+@pytest.mark.parametrize("kw", [
+    # ragged: k_g not a multiple of 8, more k_b than candidates early on
+    dict(n_q_heads=4, n_kv_heads=1, head_dim=64, ctx_len=576, seg_len=192, topk_blocks=5,
+         topk_groups=13, dtype="bf16", first_seg=0),
+    # G = 1, d = 128, batch 2, float32
+    dict(batch=2, n_q_heads=2, n_kv_heads=2, head_dim=128, ctx_len=512, seg_len=256,
+         topk_blocks=2, topk_groups=9, dtype="f32", first_seg=0),
+    # G = 8, single query block segments, everything selected (dense)
+    dict(n_q_heads=8, n_kv_heads=1, head_dim=128, ctx_len=320, seg_len=64, topk_blocks=64,
+         topk_groups=256, dtype="bf16", first_seg=0),
+    # scaled + RoPE small shape, several segments with history
+    dict(batch=2, n_q_heads=8, n_kv_heads=2, head_dim=128, ctx_len=1024, seg_len=256,
+         topk_blocks=3, topk_groups=12, dtype="bf16", scaled=True, rope_base=1e6, first_seg=1),
+])
+def test_custom_shapes(kw):
+    w = synth.custom(seed=11, **kw)
+    run_and_compare(w)
+
+
+def test_simt_flag_matches_default_bf16():
+    import torch
+    from hierarchical_routed_sparse_hga_b200 import HGA_FLAG_SIMT
+    w = synth.custom(n_q_heads=4, n_kv_heads=1, head_dim=128, ctx_len=512, seg_len=256,
+                     topk_blocks=2, topk_groups=8, dtype="bf16", first_seg=1, seed=5)
+    outs = []
+    for flags in (0, HGA_FLAG_SIMT):
+        seg = Segmenter(w, flags=flags)
+        outs.append(seg.run_segment(256))
+    a, b = outs
+    assert (a["sel_grp"] == b["sel_grp"]).all()
+    for key in ("o", "dq", "dk", "dv"):
+        ref = np.max(np.abs(b[key]))
+        assert np.max(np.abs(a[key] - b[key])) <= 2e-2 * ref, key
+    torch.cuda.synchronize()
+
+
+def test_corrupt_selection_is_skipped_and_latched():
+    import torch
+    import oracle
+    from hierarchical_routed_sparse_hga_b200 import (HGA_ERR_DEVICE_CHECK, HGA_OK,
+                                                     hga_attn_fwd, hga_get_device_status)
+    from hga_testlib import assert_close, to_device
+    w = synth.custom(n_q_heads=4, n_kv_heads=1, head_dim=64, ctx_len=512, seg_len=128,
+                     topk_blocks=2, topk_groups=6, dtype="f32", first_seg=3, seed=3)
+    seg = Segmenter(w)
+    out = seg.run_segment(384, backward=False)
+    assert hga_get_device_status() == HGA_OK
+    L = seg.layer
+    bad = L.sel_grp.clone()
+    bad[0, 0, 0, 1] = 10_000          # beyond the query block's own block
+    bad[0, 0, 1, 0] = -7              # negative, not the -1 padding
+    q = to_device(synth.queries(w, 384), w)
+    hga_attn_fwd(L.cfg, q, L.k, L.v, w.ctx_len, 384, w.seg_len, bad, L.o, L.lse)
+    assert hga_get_device_status() == HGA_ERR_DEVICE_CHECK
+    assert hga_get_device_status() == HGA_OK          # reading clears it
+    # the output equals the oracle's with those two entries dropped
+    ref_sel = bad.cpu().numpy().copy()
+    ref_sel[0, 0, 0, 1] = -1
+    ref_sel[0, 0, 1, 0] = -1
+    o, lse = oracle.attn_fwd(out["q64"], seg.k64, seg.v64, 384, ref_sel, 1)
+    assert_close(L.o.double().cpu().numpy(), o, w, "o")
+    assert_close(L.lse.double().cpu().numpy(), lse, w, "lse", abs_=1e-4)
+
+
+def test_empty_summary_range_is_noop():
+    import torch
+    from hierarchical_routed_sparse_hga_b200 import hga_build_summaries
+    w = synth.custom(n_q_heads=1, n_kv_heads=1, head_dim=64, ctx_len=256, seg_len=64)
+    seg = Segmenter(w)
+    before = seg.layer.gsum.clone()
+    hga_build_summaries(seg.layer.cfg, seg.layer.k, 256, 128, 128, seg.layer.gsum,
+                        seg.layer.bsum)
+    torch.cuda.synchronize()
+    assert torch.equal(before, seg.layer.gsum)
