@@ -26,7 +26,8 @@ EXPORTS = ("hga_version", "hga_status_string", "hga_build_summaries",
            "hga_route_workspace_size", "hga_route", "hga_attn_fwd",
            "hga_attn_bwd_workspace_size", "hga_attn_bwd", "hga_get_device_status",
            "hga_kernel_name", "hga_launch_count", "hga_timing_enable", "hga_timing_collect",
-           "hga_timing_get", "hga_timing_reset")
+           "hga_timing_get", "hga_timing_reset", "hga_route_noalloc")
+HGA_NOALLOC_SCRATCH_BYTES = 4 << 20
 HGA_K_COUNT = 10
 
 
@@ -95,6 +96,7 @@ def load() -> ctypes.CDLL:
         "hga_timing_get": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_double),
                                           ctypes.POINTER(ctypes.c_uint64)]),
         "hga_timing_reset": (None, []),
+        "hga_route_noalloc": (ctypes.c_int, [CFG, P, I64, I32, I64, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -164,6 +166,16 @@ def hga_route(cfg: Config, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_
     _check("hga_route", load().hga_route(
         ctypes.byref(c), _ptr(q), q_begin, s_len, ctx_cap, _ptr(bsum), _ptr(gsum),
         _ptr(sel_blk), _ptr(sel_grp), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def hga_route_noalloc(cfg: Config, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp,
+                      stream=None):
+    """hga_route with the library's built-in scratch array instead of a
+    caller-provided workspace, for callers that cannot allocate device memory."""
+    c = cfg.c()
+    _check("hga_route_noalloc", load().hga_route_noalloc(
+        ctypes.byref(c), _ptr(q), q_begin, s_len, ctx_cap, _ptr(bsum), _ptr(gsum),
+        _ptr(sel_blk), _ptr(sel_grp), _stream(stream)))
 
 
 def hga_attn_fwd(cfg: Config, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, stream=None):

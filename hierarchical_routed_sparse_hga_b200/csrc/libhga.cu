@@ -103,6 +103,34 @@ RouteCarve route_carve(const hga_config_t* c, int32_t s_len, int64_t q_begin, vo
 
 }  // namespace
 
+// Scratch of hga_route_noalloc: a fixed device array, so that entry point
+// never allocates.  Host code must not pass `g_noalloc_scratch` itself to a
+// kernel (on the host it names a host-side stand-in); it passes the device
+// address that cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[HGA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (with that device current) and cached; nullptr on failure.
+void* noalloc_scratch() {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* hga_version(void) { return "libhga 0.1 (sm_100a)"; }
@@ -220,6 +248,21 @@ hga_status_t hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k,
           cfg->scale, static_cast<T*>(o), lse);
     });
   });
+}
+
+hga_status_t hga_route_noalloc(const hga_config_t* cfg, const void* q, int64_t q_begin,
+                               int32_t s_len, int64_t ctx_cap, const float* bsum,
+                               const float* gsum, int32_t* sel_blk, int32_t* sel_grp,
+                               void* stream) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
+  if (hga_route_workspace_size(cfg, s_len, q_begin) > HGA_NOALLOC_SCRATCH_BYTES)
+    return HGA_ERR_WORKSPACE;
+  void* scratch = noalloc_scratch();
+  if (!scratch) return HGA_ERR_CUDA;
+  return hga_route(cfg, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp, scratch,
+                   HGA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 size_t hga_attn_bwd_workspace_size(const hga_config_t* cfg, int32_t s_len) {

@@ -150,6 +150,36 @@ HGA_API hga_status_t hga_attn_fwd(const hga_config_t* cfg, const void* q, const 
                           int64_t ctx_cap, int64_t q_begin, int32_t s_len,
                           const int32_t* sel_grp, void* o, float* lse, void* stream);
 
+/*
+ * hga_route without a caller-provided workspace.  The paper has no
+ * counterpart: this is a library convenience for callers that cannot call
+ * cudaMalloc -- for example a plugin running inside a host runtime that owns
+ * every byte of device memory and hands its extensions no allocator, or code
+ * that must not allocate after start-up because cudaMalloc can synchronise
+ * the device and has unbounded latency.  Such callers still pass every input
+ * and output buffer; only the router's scratch (mean queries and block scores)
+ * comes from a fixed array inside the library.
+ *
+ * The array is HGA_NOALLOC_SCRATCH_BYTES (4 MiB) of device memory that every
+ * GPU which loads the library holds until the process exits.  A call whose
+ * hga_route_workspace_size() exceeds it returns HGA_ERR_WORKSPACE and
+ * launches nothing (for the Qwen3-8B shape -- 8 KV heads, d = 128, 2048-token
+ * segments, batch 1 -- contexts up to 253,952 tokens fit).
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it; make that first call before any stream
+ * capture.  Every call on a device shares the one array and it keeps the
+ * last call's contents; nothing in it needs to start at zero, because each
+ * call writes every scratch element before reading it.  Calls that can
+ * overlap on the GPU (different streams, or several host threads) race on
+ * the array: serialise them.  Results are identical to hga_route.
+ */
+#define HGA_NOALLOC_SCRATCH_BYTES (4u << 20)
+HGA_API hga_status_t hga_route_noalloc(const hga_config_t* cfg, const void* q, int64_t q_begin,
+                                       int32_t s_len, int64_t ctx_cap, const float* bsum,
+                                       const float* gsum, int32_t* sel_blk, int32_t* sel_grp,
+                                       void* stream);
+
 /* Bytes of device workspace hga_attn_bwd needs for this segment. */
 HGA_API size_t hga_attn_bwd_workspace_size(const hga_config_t* cfg, int32_t s_len);
 
