@@ -1,6 +1,7 @@
 // libhga: C ABI of the HGA hot path (declarations and contracts in hga.h).
 // Host side: argument checks, workspace carving, kernel selection and launch.
 // Nothing here allocates, frees or synchronises (except hga_get_device_status).
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -13,6 +14,7 @@
 #include "summaries.cuh"
 #include "route.cuh"
 #include "attn_simt.cuh"
+#include "attn_fwd_sm100.cuh"
 #include "trace.cuh"
 
 using namespace hga;
@@ -79,6 +81,72 @@ hga_status_t dispatch(const hga_config_t* c, Body&& body) {
   }
   if (c->head_dim == 128) return body.template operator()<float, 128>();
   return body.template operator()<float, 64>();
+}
+
+// ---- TMA tensor maps (driver entry point reached through the runtime) ----
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major [rows, 128] bf16 matrix, boxes of 64 columns (128 B, swizzled) x box_rows.
+bool make_map_bf16_d128(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {128 * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool use_tensor_cores(const hga_config_t* c, int64_t ctx_cap, int32_t s_len) {
+  const int G = c->n_q_heads / c->n_kv_heads;
+  if (c->flags & HGA_FLAG_SIMT) return false;
+  if (c->dtype != HGA_BF16 || c->head_dim != 128 || (G != 2 && G != 4)) return false;
+  // TMA row coordinates are 32-bit
+  if (int64_t(c->batch) * c->n_kv_heads * ctx_cap >= (int64_t(1) << 31)) return false;
+  if (int64_t(c->batch) * c->n_q_heads * s_len >= (int64_t(1) << 31)) return false;
+  return true;
+}
+
+template <int MT>
+hga_status_t launch_fwd_tc(const hga_config_t* cfg, const void* q, const void* k, const void* v,
+                           int64_t ctx_cap, int64_t q_begin, int32_t s_len,
+                           const int32_t* sel_grp, void* o, float* lse, cudaStream_t s) {
+  using L = fwdtc::Layout<MT>;
+  CUtensorMap tq, tk, tv;
+  const uint64_t q_rows = uint64_t(cfg->batch) * cfg->n_q_heads * s_len;
+  const uint64_t kv_rows = uint64_t(cfg->batch) * cfg->n_kv_heads * ctx_cap;
+  if (!make_map_bf16_d128(&tq, q, q_rows, 64) || !make_map_bf16_d128(&tk, k, kv_rows, 8) ||
+      !make_map_bf16_d128(&tv, v, kv_rows, 8))
+    return HGA_ERR_CUDA;
+  hga_status_t e = ensure_smem(reinterpret_cast<const void*>(&fwdtc::attn_fwd_tc_kernel<MT>),
+                               L::kDynSmem);
+  if (e != HGA_OK) return e;
+  dim3 grid(s_len / kQBlock, cfg->n_kv_heads, cfg->batch);
+  const float scale_log2 = cfg->scale * 1.4426950408889634f;
+  return traced_launch(HGA_K_FWD_TC, s, [&] {
+    fwdtc::attn_fwd_tc_kernel<MT><<<grid, L::kThreads, L::kDynSmem, s>>>(
+        tq, tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups,
+        sel_grp, scale_log2, static_cast<__nv_bfloat16*>(o), lse, cfg->flags);
+  });
 }
 
 struct RouteCarve {
@@ -235,6 +303,11 @@ hga_status_t hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k,
     return HGA_ERR_INVALID_ARG;
   const int n_qb = s_len / kQBlock;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (use_tensor_cores(cfg, ctx_cap, s_len)) {
+    if (cfg->n_q_heads / cfg->n_kv_heads == 4)
+      return launch_fwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, s);
+    return launch_fwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, s);
+  }
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
     const size_t sm = size_t(simt_fwd_smem_floats<D>()) * 4;
     hga_status_t e =

@@ -87,6 +87,14 @@ typedef enum { HGA_F32 = 0, HGA_BF16 = 1 } hga_dtype_t;
 
 /* flags */
 #define HGA_FLAG_SIMT 1u  /* force the CUDA-core attention kernels (fp32 always uses them) */
+/* Test only: the tensor-core forward kernel skips loading its first key tile,
+ * so its bounded wait runs out; the kernel latches HGA_ERR_TIMEOUT, drains
+ * what it started, frees its tensor memory and returns (outputs undefined). */
+#define HGA_FLAG_TEST_DROP_FIRST_TILE 0x80000000u
+
+/* Which attention kernels a call uses: the tensor-core (tcgen05) kernels for
+ * bf16, head_dim 128 and G in {2, 4} unless HGA_FLAG_SIMT is set; the
+ * CUDA-core kernels otherwise. */
 
 typedef struct {
   int32_t batch;

@@ -60,9 +60,15 @@ def test_qwen3_fwd_128k_sampled():
     # G = 8, single query block segments, everything selected (dense)
     dict(n_q_heads=8, n_kv_heads=1, head_dim=128, ctx_len=320, seg_len=64, topk_blocks=64,
          topk_groups=256, dtype="bf16", first_seg=0),
-    # scaled + RoPE small shape, several segments with history
+    # scaled + RoPE small shape, several segments with history (G = 4: 2 M tiles)
     dict(batch=2, n_q_heads=8, n_kv_heads=2, head_dim=128, ctx_len=1024, seg_len=256,
          topk_blocks=3, topk_groups=12, dtype="bf16", scaled=True, rope_base=1e6, first_seg=1),
+    # G = 2 (one M tile on the tensor-core path), k_g with a ragged last tile
+    dict(n_q_heads=4, n_kv_heads=2, head_dim=128, ctx_len=768, seg_len=256, topk_blocks=3,
+         topk_groups=20, dtype="bf16", first_seg=1),
+    # tensor-core path, every candidate selected, first segment has no history
+    dict(n_q_heads=4, n_kv_heads=1, head_dim=128, ctx_len=512, seg_len=128, topk_blocks=64,
+         topk_groups=256, dtype="bf16", first_seg=0),
 ])
 def test_custom_shapes(kw):
     w = synth.custom(seed=11, **kw)
@@ -124,3 +130,28 @@ def test_empty_summary_range_is_noop():
                         seg.layer.bsum)
     torch.cuda.synchronize()
     assert torch.equal(before, seg.layer.gsum)
+
+
+def test_bounded_wait_times_out_and_context_stays_usable():
+    # the forward kernel's test hook never loads its first key tile: the MMA
+    # warp's wait runs out (about a second), the kernel latches
+    # HGA_ERR_TIMEOUT, drains and returns; the next call works normally
+    import torch
+    from hierarchical_routed_sparse_hga_b200 import (HGA_ERR_TIMEOUT, HGA_OK, hga_attn_fwd,
+                                                     hga_get_device_status)
+    from hga_testlib import to_device
+    flag = 0x80000000
+    w = synth.custom(n_q_heads=4, n_kv_heads=1, head_dim=128, ctx_len=320, seg_len=64,
+                     topk_blocks=2, topk_groups=8, dtype="bf16", first_seg=4, seed=9)
+    seg = Segmenter(w)
+    good = seg.run_segment(256, backward=False)
+    L = seg.layer
+    q = to_device(synth.queries(w, 256), w)
+    cfg = L.cfg
+    cfg_bad = type(cfg)(**{**cfg.__dict__, "flags": flag})
+    hga_attn_fwd(cfg_bad, q, L.k, L.v, w.ctx_len, 256, w.seg_len, L.sel_grp, L.o, L.lse)
+    assert hga_get_device_status() == HGA_ERR_TIMEOUT
+    hga_attn_fwd(cfg, q, L.k, L.v, w.ctx_len, 256, w.seg_len, L.sel_grp, L.o, L.lse)
+    torch.cuda.synchronize()
+    assert hga_get_device_status() == HGA_OK
+    assert np.array_equal(L.o.double().cpu().numpy(), good["o"])
