@@ -15,6 +15,7 @@
 #include "route.cuh"
 #include "attn_simt.cuh"
 #include "attn_fwd_sm100.cuh"
+#include "attn_bwd_sm100.cuh"
 #include "trace.cuh"
 
 using namespace hga;
@@ -146,6 +147,43 @@ hga_status_t launch_fwd_tc(const hga_config_t* cfg, const void* q, const void* k
     fwdtc::attn_fwd_tc_kernel<MT><<<grid, L::kThreads, L::kDynSmem, s>>>(
         tq, tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups,
         sel_grp, scale_log2, static_cast<__nv_bfloat16*>(o), lse, cfg->flags);
+  });
+}
+
+template <int MT>
+hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k, const void* v,
+                           int64_t ctx_cap, int64_t q_begin, int32_t s_len,
+                           const int32_t* sel_grp, const void* o, const float* lse,
+                           const void* d_o, void* dq, void* dk, void* dv, float* dvec,
+                           cudaStream_t s) {
+  using LQ = bwdtc::DqLayout<MT>;
+  using LK = bwdtc::KvLayout<MT>;
+  CUtensorMap tq, tdo, tk, tv;
+  const uint64_t q_rows = uint64_t(cfg->batch) * cfg->n_q_heads * s_len;
+  const uint64_t kv_rows = uint64_t(cfg->batch) * cfg->n_kv_heads * ctx_cap;
+  if (!make_map_bf16_d128(&tq, q, q_rows, 64) || !make_map_bf16_d128(&tdo, d_o, q_rows, 64) ||
+      !make_map_bf16_d128(&tk, k, kv_rows, 8) || !make_map_bf16_d128(&tv, v, kv_rows, 8))
+    return HGA_ERR_CUDA;
+  hga_status_t e = ensure_smem(
+      reinterpret_cast<const void*>(&bwdtc::attn_bwd_dq_tc_kernel<MT>), LQ::kDynSmem);
+  if (e != HGA_OK) return e;
+  e = ensure_smem(reinterpret_cast<const void*>(&bwdtc::attn_bwd_dkdv_tc_kernel<MT>),
+                  LK::kDynSmem);
+  if (e != HGA_OK) return e;
+  dim3 grid(s_len / kQBlock, cfg->n_kv_heads, cfg->batch);
+  const float scale_log2 = cfg->scale * 1.4426950408889634f;
+  e = traced_launch(HGA_K_BWD_DQ_TC, s, [&] {
+    bwdtc::attn_bwd_dq_tc_kernel<MT><<<grid, LQ::kThreads, LQ::kDynSmem, s>>>(
+        tq, tdo, tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads,
+        cfg->topk_groups, sel_grp, cfg->scale, scale_log2, static_cast<const __nv_bfloat16*>(o),
+        static_cast<const __nv_bfloat16*>(d_o), lse, static_cast<__nv_bfloat16*>(dq), dvec);
+  });
+  if (e != HGA_OK) return e;
+  return traced_launch(HGA_K_BWD_DKDV_TC, s, [&] {
+    bwdtc::attn_bwd_dkdv_tc_kernel<MT><<<grid, LK::kThreads, LK::kDynSmem, s>>>(
+        tq, tdo, tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads,
+        cfg->topk_groups, sel_grp, cfg->scale, scale_log2, lse, dvec,
+        static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
   });
 }
 
@@ -358,6 +396,13 @@ hga_status_t hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k,
   const int n_qb = s_len / kQBlock;
   float* dvec = static_cast<float*>(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (use_tensor_cores(cfg, ctx_cap, s_len)) {
+    if (cfg->n_q_heads / cfg->n_kv_heads == 4)
+      return launch_bwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq,
+                              dk, dv, dvec, s);
+    return launch_bwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk,
+                            dv, dvec, s);
+  }
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
     const size_t sm1 = size_t(simt_fwd_smem_floats<D>()) * 4;
     hga_status_t e =
