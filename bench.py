@@ -56,6 +56,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--tier-sweep", action="store_true",
+                   help="host-tier sweep: top-k blocks {8,16,32} x context 1K..32K, batch 8")
     return p.parse_args()
 
 
@@ -110,12 +112,12 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, bus_id=None):
+    def __init__(self, gpu_id=None):
         self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                "-lms", "100"]
-        if bus_id:
-            cmd += ["-i", bus_id]
+        if gpu_id:
+            cmd += ["-i", gpu_id]
         try:
             self.proc = subprocess.Popen(cmd, stdout=self.file, stderr=subprocess.DEVNULL)
         except OSError:
@@ -168,9 +170,10 @@ def segment_pairs(w, sel_grp, q_begin):
     return all_pairs, act_pairs
 
 
-def kernel_work(name, w, sels):
+def kernel_work(name, w, sels, unique_groups=None):
     """Algorithmic work of ALL launches of kernel `name` over one step.
     Returns (amount, unit, bound): FLOP for contractions, bytes otherwise."""
+    unique_groups = unique_groups or {}
     d, S, B = w.head_dim, w.seg_len, w.batch
     Hq, Hkv = w.n_q_heads, w.n_kv_heads
     el = 2 if w.dtype == "bf16" else 4
@@ -196,8 +199,14 @@ def kernel_work(name, w, sels):
         elif name == "route_select":
             tot += B * Hkv * sum(J * 4 + 8 * k * d * 4 + d * 4 + 4 * (w.topk_blocks + w.topk_groups)
                                  for J, k in zip(Js, kb))
+        elif name == "tier_copy":
+            tot += 2 * 2 * unique_groups.get(q_begin, 0) * 8 * d * el   # read host + write HBM
+        elif name == "tier_dedup":
+            tot += B * Hkv * n_qb * w.topk_groups * 8
     if name.startswith("attn"):
         return tot, "FLOP", "alu" if name.endswith("simt") else "tensor"
+    if name == "tier_copy":
+        return tot / 2, "B", "pcie"          # bytes that cross PCIe (the host reads)
     return tot, "B", "hbm"
 
 
@@ -297,6 +306,122 @@ class Runner:
         return h2d, d2h
 
 
+class TierRunner:
+    """Host-tier workload: history K/V in pinned host memory, inputs drawn on
+    the device (synth.device_inputs).  One step = every segment: place the
+    segment's K/V in staging, summaries, route, tier gather over PCIe,
+    forward, backward, append of the segment's K/V to the host history."""
+
+    def __init__(self, w, device, flags=0):
+        import torch
+        from hierarchical_routed_sparse_hga_b200 import (HGA_BF16, HGA_F32, Config,
+                                                         HgaTieredLayer, synth)
+        self.w, self.device = w, device
+        cfg = Config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.topk_blocks,
+                     w.topk_groups, HGA_BF16 if w.dtype == "bf16" else HGA_F32, flags)
+        self.k, self.v, self.q, self.do = synth.device_inputs(w, device, w.backward)
+        self.layer = HgaTieredLayer(cfg, w.ctx_len, w.seg_len, device=device)
+        self.segs = w.segments()
+        torch.cuda.synchronize(device)
+
+    def step(self, record_sel=None):
+        L, S = self.layer, self.w.seg_len
+        for i, q_begin in enumerate(self.segs):
+            L.active_k().copy_(self.k[:, :, q_begin:q_begin + S])
+            L.active_v().copy_(self.v[:, :, q_begin:q_begin + S])
+            L.segment(self.q[i], q_begin, self.do[i] if self.w.backward else None)
+            if record_sel is not None:
+                record_sel.append((q_begin, L.sel_grp.cpu().numpy(),
+                                   int(L.n_unique.sum().item())))
+
+    def pcie_bytes(self, sels):
+        """Bytes over PCIe per step: gathered groups (K+V) and appended segments."""
+        w = self.w
+        el = 2 if w.dtype == "bf16" else 4
+        gathered = sum(u for _, _, u in sels) * 2 * 8 * w.head_dim * el
+        appended = len(self.segs) * 2 * w.batch * w.n_kv_heads * w.seg_len * w.head_dim * el
+        return gathered, appended
+
+
+def pcie_probe(device, nbytes=256 << 20, reps=5):
+    """Pinned host -> device copy bandwidth (GB/s), best of `reps`."""
+    import torch
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    best = 0.0
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        d.copy_(h, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize(device)
+        best = max(best, nbytes / (e0.elapsed_time(e1) / 1e3) / 1e9)
+    return best
+
+
+def dense_sdpa_tokens_per_s(w, device, reps=3):
+    """Dense causal attention (torch SDPA, bf16) fwd+bwd over the whole
+    context at the workload's shape: the in-run reference point."""
+    import torch
+    import torch.nn.functional as F
+    B, H, T, d = w.batch, w.n_q_heads, w.ctx_len, w.head_dim
+    q = torch.randn((B, H, T, d), device=device, dtype=torch.bfloat16, requires_grad=True)
+    k = torch.randn((B, w.n_kv_heads, T, d), device=device, dtype=torch.bfloat16,
+                    requires_grad=True)
+    v = torch.randn_like(k, requires_grad=True)
+    go = torch.randn((B, H, T, d), device=device, dtype=torch.bfloat16)
+
+    def run():
+        o = F.scaled_dot_product_attention(q, k, v, is_causal=True, enable_gqa=True)
+        o.backward(go)
+
+    run()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize(device)
+    return B * T * reps / (e0.elapsed_time(e1) / 1e3)
+
+
+def run_tier_sweep(args, device):
+    import torch
+    from hierarchical_routed_sparse_hga_b200 import synth
+    peak = pcie_probe(device)
+    for kb in (8, 16, 32):
+        for L in (1024, 2048, 4096, 8192, 16384, 32768):
+            w = synth.custom(f"tier_b8_L{L}_kb{kb}", batch=8, n_q_heads=32, n_kv_heads=8,
+                             head_dim=128, ctx_len=L, seg_len=min(2048, L), topk_blocks=kb,
+                             topk_groups=4 * kb, dtype="bf16", scaled=True, rope_base=1e6,
+                             seed=4)
+            run = TierRunner(w, device)
+            sels = []
+            run.step(record_sel=sels)
+            torch.cuda.synchronize(device)
+            steps = 2
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(steps):
+                run.step()
+            e1.record()
+            torch.cuda.synchronize(device)
+            ms = e0.elapsed_time(e1) / steps
+            gathered, appended = run.pcie_bytes(sels)
+            dense = dense_sdpa_tokens_per_s(w, device)
+            print(json.dumps({
+                "sweep": "tier", "context": L, "topk_blocks": kb, "topk_groups": 4 * kb,
+                "batch": 8, "seg_len": w.seg_len, "tokens_per_s": round(8 * L / (ms / 1e3), 1),
+                "ms_per_step": round(ms, 3), "pcie_gather_bytes": gathered,
+                "pcie_append_bytes": appended,
+                "pcie_gbs": round((gathered + appended) / (ms / 1e3) / 1e9, 2),
+                "pcie_probe_h2d_gbs": round(peak, 2),
+                "dense_sdpa_tokens_per_s": round(dense, 1)}), flush=True)
+            del run
+            torch.cuda.empty_cache()
+
+
 def run_gpu(args, rank, world, local):
     import numpy as np
     import torch
@@ -309,13 +434,19 @@ def run_gpu(args, rank, world, local):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=device)
+    if args.tier_sweep:
+        run_tier_sweep(args, device)
+        return
     w0 = synth.workloads()[args.workload]
     w = rank_workload(w0, rank)
-    run = Runner(w, device, HGA_FLAG_SIMT if args.simt else 0)
+    tiered = "tiered" in w.name
+    run = (TierRunner if tiered else Runner)(w, device, HGA_FLAG_SIMT if args.simt else 0)
     tokens_per_step = w.batch * len(run.segs) * w.seg_len
 
     sels = []
     run.step(record_sel=sels)                       # first warm-up step records selections
+    unique_groups = {rec[0]: rec[2] for rec in sels if len(rec) > 2}
+    sels = [(rec[0], rec[1]) for rec in sels]
     for _ in range(max(args.warmup, 3) - 1):
         run.step()
     torch.cuda.synchronize(device)
@@ -344,12 +475,12 @@ def run_gpu(args, rank, world, local):
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    bus = None
+    gpu_id = None
     try:
-        bus = torch.cuda.get_device_properties(device).pci_bus_id
+        gpu_id = f"GPU-{torch.cuda.get_device_properties(device).uuid}"
     except Exception:
         pass
-    sampler = None if args.no_clocks else ClockSampler(bus)
+    sampler = None if args.no_clocks else ClockSampler(gpu_id)
     barrier(world, device)
     torch.cuda.synchronize(device)
     launches0 = hga_launch_count()
@@ -384,7 +515,7 @@ def run_gpu(args, rank, world, local):
                          "share": round(ms / max(sum(v[0] for v in table.values()), 1e-12), 4)}
     dom = max(table, key=lambda k: table[k][0])
     dom_ms, dom_n = table[dom]
-    work, unit, bound = kernel_work(dom, w, sels)
+    work, unit, bound = kernel_work(dom, w, sels, unique_groups)
     work_per_launch = work / (dom_n / args.steps)
     pk = peaks()
     avg_s = dom_ms / dom_n / 1e3
@@ -396,6 +527,10 @@ def run_gpu(args, rank, world, local):
         achieved = work_per_launch / avg_s / 1e12
         peak, punit = FP32_ALU_TFLOPS, "TFLOP/s"
         peak_note = "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz"
+    elif bound == "pcie":
+        achieved = work_per_launch / avg_s / 1e9
+        peak, punit = round(pcie_probe(device), 2), "GB/s"
+        peak_note = "pinned host-to-device cudaMemcpyAsync probe, 256 MiB, best of 5"
     else:
         achieved = work_per_launch / avg_s / 1e9
         peak, punit = pk["hbm"], "GB/s"
@@ -408,7 +543,7 @@ def run_gpu(args, rank, world, local):
 
     # end to end through the public API with pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not tiered:
         L = run.layer
         outs = (L.o, L.dq, L.dk, L.dv) if w.backward else (L.o,)
         out_host = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]

@@ -10,7 +10,8 @@ from ._lib import (EXPORTS, HGA_BF16, HGA_ERR_CUDA, HGA_ERR_DEVICE_CHECK,  # noq
                    HGA_ERR_INVALID_ARG, HGA_ERR_TIMEOUT, HGA_ERR_UNSUPPORTED,
                    HGA_ERR_WORKSPACE, HGA_F32, HGA_FLAG_SIMT, HGA_OK, Config, HgaError,
                    hga_attn_bwd, hga_attn_bwd_workspace_size, hga_attn_fwd,
-                   hga_build_summaries, hga_get_device_status, hga_kernel_name,
+                   hga_build_summaries, hga_build_summaries_seg, hga_tier_append, hga_tier_gather,
+                   hga_tier_stage_rows, hga_tier_workspace_size, hga_get_device_status, hga_kernel_name,
                    hga_launch_count, hga_route, hga_route_noalloc,
                    hga_route_workspace_size, hga_status_string,
                    hga_timing_collect, hga_timing_enable, hga_timing_get, hga_timing_reset,
@@ -19,7 +20,7 @@ from ._lib import (EXPORTS, HGA_BF16, HGA_ERR_CUDA, HGA_ERR_DEVICE_CHECK,  # noq
 
 def __getattr__(name):
     # HgaLayer needs torch; import it lazily so CPU-only tools stay light
-    if name == "HgaLayer":
-        from .runtime import HgaLayer
-        return HgaLayer
+    if name in ("HgaLayer", "HgaTieredLayer"):
+        from . import runtime
+        return getattr(runtime, name)
     raise AttributeError(name)

@@ -26,9 +26,11 @@ EXPORTS = ("hga_version", "hga_status_string", "hga_build_summaries",
            "hga_route_workspace_size", "hga_route", "hga_attn_fwd",
            "hga_attn_bwd_workspace_size", "hga_attn_bwd", "hga_get_device_status",
            "hga_kernel_name", "hga_launch_count", "hga_timing_enable", "hga_timing_collect",
-           "hga_timing_get", "hga_timing_reset", "hga_route_noalloc")
+           "hga_timing_get", "hga_timing_reset", "hga_route_noalloc", "hga_build_summaries_seg",
+           "hga_tier_stage_rows", "hga_tier_workspace_size", "hga_tier_gather",
+           "hga_tier_append")
 HGA_NOALLOC_SCRATCH_BYTES = 4 << 20
-HGA_K_COUNT = 10
+HGA_K_COUNT = 12
 
 
 class HgaError(RuntimeError):
@@ -97,6 +99,12 @@ def load() -> ctypes.CDLL:
                                           ctypes.POINTER(ctypes.c_uint64)]),
         "hga_timing_reset": (None, []),
         "hga_route_noalloc": (ctypes.c_int, [CFG, P, I64, I32, I64, P, P, P, P, P]),
+        "hga_build_summaries_seg": (ctypes.c_int, [CFG, P, I64, I64, I64, I64, P, P, P]),
+        "hga_tier_stage_rows": (I64, [CFG, I64, I32]),
+        "hga_tier_workspace_size": (SZ, [CFG, I32, I64]),
+        "hga_tier_gather": (ctypes.c_int, [CFG, P, P, I64, I64, I32, P, P, P, I64, P, P, P, SZ,
+                                           P]),
+        "hga_tier_append": (ctypes.c_int, [CFG, P, P, I64, P, P, I64, I64, I32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -152,6 +160,52 @@ def hga_build_summaries(cfg: Config, k, ctx_cap, t_begin, t_end, gsum, bsum, str
     _check("hga_build_summaries", load().hga_build_summaries(
         ctypes.byref(c), _ptr(k), ctx_cap, t_begin, t_end, _ptr(gsum), _ptr(bsum),
         _stream(stream)))
+
+
+def hga_build_summaries_seg(cfg: Config, k_seg, seg_cap, t_begin, t_end, ctx_cap, gsum, bsum,
+                            stream=None):
+    c = cfg.c()
+    _check("hga_build_summaries_seg", load().hga_build_summaries_seg(
+        ctypes.byref(c), _ptr(k_seg), seg_cap, t_begin, t_end, ctx_cap, _ptr(gsum), _ptr(bsum),
+        _stream(stream)))
+
+
+def hga_tier_stage_rows(cfg: Config, q_begin, s_len) -> int:
+    c = cfg.c()
+    return int(load().hga_tier_stage_rows(ctypes.byref(c), q_begin, s_len))
+
+
+def hga_tier_workspace_size(cfg: Config, s_len, q_begin) -> int:
+    c = cfg.c()
+    return int(load().hga_tier_workspace_size(ctypes.byref(c), s_len, q_begin))
+
+
+def _host_ptr(x):
+    """Pinned host tensor (or raw address) for the tier's host-side arrays."""
+    if isinstance(x, int):
+        return x
+    if x.is_cuda or not x.is_pinned() or not x.is_contiguous():
+        raise ValueError("hga_tier_gather takes contiguous pinned host tensors for K/V")
+    return x.data_ptr()
+
+
+def hga_tier_gather(cfg: Config, k_host, v_host, ctx_cap, q_begin, s_len, sel_grp, k_stage,
+                    v_stage, stage_cap, sel_stage, n_unique, workspace, ws_bytes=None,
+                    stream=None):
+    c = cfg.c()
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check("hga_tier_gather", load().hga_tier_gather(
+        ctypes.byref(c), _host_ptr(k_host), _host_ptr(v_host), ctx_cap, q_begin, s_len,
+        _ptr(sel_grp), _ptr(k_stage), _ptr(v_stage), stage_cap, _ptr(sel_stage), _ptr(n_unique),
+        _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def hga_tier_append(cfg: Config, k_stage, v_stage, stage_cap, k_host, v_host, ctx_cap, q_begin,
+                    s_len, stream=None):
+    c = cfg.c()
+    _check("hga_tier_append", load().hga_tier_append(
+        ctypes.byref(c), _ptr(k_stage), _ptr(v_stage), stage_cap, _host_ptr(k_host),
+        _host_ptr(v_host), ctx_cap, q_begin, s_len, _stream(stream)))
 
 
 def hga_route_workspace_size(cfg: Config, s_len, q_begin) -> int:

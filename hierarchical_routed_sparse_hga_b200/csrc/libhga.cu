@@ -16,6 +16,7 @@
 #include "attn_simt.cuh"
 #include "attn_fwd_sm100.cuh"
 #include "attn_bwd_sm100.cuh"
+#include "tier.cuh"
 #include "trace.cuh"
 
 using namespace hga;
@@ -271,8 +272,33 @@ hga_status_t hga_build_summaries(const hga_config_t* cfg, const void* k, int64_t
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
     dim3 grid(unsigned(n_blk), cfg->n_kv_heads, cfg->batch);
     return traced_launch(HGA_K_SUMMARIES, s, [&] {
-      summaries_kernel<T, D><<<grid, D, 0, s>>>(static_cast<const T*>(k), ctx_cap,
-                                                t_begin / kBlock, cfg->n_kv_heads, gsum, bsum);
+      summaries_kernel<T, D><<<grid, D, 0, s>>>(static_cast<const T*>(k), ctx_cap, t_begin,
+                                                ctx_cap, t_begin / kBlock, cfg->n_kv_heads,
+                                                gsum, bsum);
+    });
+  });
+}
+
+hga_status_t hga_build_summaries_seg(const hga_config_t* cfg, const void* k_seg, int64_t seg_cap,
+                                     int64_t t_begin, int64_t t_end, int64_t ctx_cap,
+                                     float* gsum, float* bsum, void* stream) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if (!k_seg || !gsum || !bsum || !aligned16(k_seg) || !aligned16(gsum) || !aligned16(bsum))
+    return HGA_ERR_INVALID_ARG;
+  if (ctx_cap <= 0 || ctx_cap % kBlock || t_begin < 0 || t_begin % kBlock || t_end % kBlock ||
+      t_end < t_begin || t_end > ctx_cap || seg_cap < t_end - t_begin)
+    return HGA_ERR_INVALID_ARG;
+  if (t_end == t_begin) return HGA_OK;
+  const int64_t n_blk = (t_end - t_begin) / kBlock;
+  if (n_blk > 0x7fffffff) return HGA_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
+    dim3 grid(unsigned(n_blk), cfg->n_kv_heads, cfg->batch);
+    return traced_launch(HGA_K_SUMMARIES, s, [&] {
+      summaries_kernel<T, D><<<grid, D, 0, s>>>(static_cast<const T*>(k_seg), seg_cap, 0,
+                                                ctx_cap, t_begin / kBlock, cfg->n_kv_heads,
+                                                gsum, bsum);
     });
   });
 }
@@ -431,6 +457,114 @@ hga_status_t hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k,
   });
 }
 
+namespace {
+
+int64_t tier_slot_cap(const hga_config_t* cfg, int64_t q_begin, int32_t s_len) {
+  const int64_t by_sel = int64_t(s_len / kQBlock) * cfg->topk_groups;
+  const int64_t by_hist = q_begin / kGroup;
+  return by_sel < by_hist ? by_sel : by_hist;
+}
+
+// Device address of pinned, device-mapped host memory (nullptr otherwise).
+const void* mapped_host(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (a.type != cudaMemoryTypeHost || a.devicePointer == nullptr) return nullptr;
+  return a.devicePointer;
+}
+
+}  // namespace
+
+size_t hga_tier_workspace_size(const hga_config_t* cfg, int32_t s_len, int64_t q_begin) {
+  if (check_cfg(cfg) != HGA_OK || s_len <= 0 || q_begin < 0) return 0;
+  const int64_t heads = int64_t(cfg->batch) * cfg->n_kv_heads;
+  const int64_t cap = tier_slot_cap(cfg, q_begin, s_len);
+  return align256(size_t(heads) * 4) + align256(size_t(heads * (cap > 0 ? cap : 1)) * 4);
+}
+
+int64_t hga_tier_stage_rows(const hga_config_t* cfg, int64_t q_begin, int32_t s_len) {
+  if (check_cfg(cfg) != HGA_OK || s_len <= 0 || q_begin < 0) return 0;
+  const int64_t hist_rows = tier_slot_cap(cfg, q_begin, s_len) * kGroup;
+  return ((hist_rows + kBlock - 1) / kBlock) * kBlock + s_len;
+}
+
+hga_status_t hga_tier_gather(const hga_config_t* cfg, const void* k_host, const void* v_host,
+                             int64_t ctx_cap, int64_t q_begin, int32_t s_len,
+                             const int32_t* sel_grp, void* k_stage, void* v_stage,
+                             int64_t stage_cap, int32_t* sel_stage, int32_t* n_unique,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
+  const void* ptrs[] = {k_host, v_host, sel_grp, k_stage, v_stage, sel_stage, workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return HGA_ERR_INVALID_ARG;
+  if (stage_cap % kBlock || stage_cap < hga_tier_stage_rows(cfg, q_begin, s_len))
+    return HGA_ERR_INVALID_ARG;
+  if (ws_bytes < hga_tier_workspace_size(cfg, s_len, q_begin)) return HGA_ERR_WORKSPACE;
+  const void* kd = mapped_host(k_host);
+  const void* vd = mapped_host(v_host);
+  if (!kd || !vd) return HGA_ERR_INVALID_ARG;  // not pinned, device-mapped host memory
+  const int64_t heads = int64_t(cfg->batch) * cfg->n_kv_heads;
+  int32_t* counts = static_cast<int32_t*>(workspace);
+  int32_t* slots = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) +
+                                              align256(size_t(heads) * 4));
+  if (n_unique == nullptr) n_unique = counts;
+  const int64_t slot_cap = tier_slot_cap(cfg, q_begin, s_len) > 0
+                               ? tier_slot_cap(cfg, q_begin, s_len) : 1;
+  const int n_qb = s_len / kQBlock;
+  const int64_t n_words = (q_begin / kGroup + 31) / 32;
+  const size_t sm = size_t(n_words > 0 ? n_words : 1) * 8;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
+    hga_status_t e = ensure_smem(reinterpret_cast<const void*>(&tier_dedup_kernel<D>), sm);
+    if (e != HGA_OK) return e;
+    dim3 g1(cfg->n_kv_heads, cfg->batch);
+    e = traced_launch(HGA_K_TIER_DEDUP, s, [&] {
+      tier_dedup_kernel<D><<<g1, kTierThreads, sm, s>>>(sel_grp, cfg->n_kv_heads, n_qb,
+                                                        cfg->topk_groups, q_begin, stage_cap,
+                                                        s_len, sel_stage, slots, n_unique,
+                                                        slot_cap);
+    });
+    if (e != HGA_OK || q_begin == 0) return e;
+    const int per_cta = 8 * kTierCopyWarps;
+    dim3 g2(unsigned((slot_cap + per_cta - 1) / per_cta), cfg->n_kv_heads, cfg->batch);
+    return traced_launch(HGA_K_TIER_COPY, s, [&] {
+      tier_copy_kernel<T, D><<<g2, kTierCopyWarps * 32, 0, s>>>(
+          static_cast<const T*>(kd), static_cast<const T*>(vd), ctx_cap, cfg->n_kv_heads, slots,
+          n_unique, slot_cap, static_cast<T*>(k_stage), static_cast<T*>(v_stage), stage_cap);
+    });
+  });
+}
+
+hga_status_t hga_tier_append(const hga_config_t* cfg, const void* k_stage, const void* v_stage,
+                             int64_t stage_cap, void* k_host, void* v_host, int64_t ctx_cap,
+                             int64_t q_begin, int32_t s_len, void* stream) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
+  if (!k_stage || !v_stage || !k_host || !v_host || stage_cap < s_len || stage_cap % kBlock)
+    return HGA_ERR_INVALID_ARG;
+  if (!mapped_host(k_host) || !mapped_host(v_host)) return HGA_ERR_INVALID_ARG;
+  const size_t elt = cfg->dtype == HGA_BF16 ? 2 : 4;
+  const size_t row = size_t(cfg->head_dim) * elt;
+  const size_t heads = size_t(cfg->batch) * cfg->n_kv_heads;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const void* srcs[2] = {k_stage, v_stage};
+  void* dsts[2] = {k_host, v_host};
+  for (int i = 0; i < 2; ++i) {
+    const char* src = static_cast<const char*>(srcs[i]) + size_t(stage_cap - s_len) * row;
+    char* dst = static_cast<char*>(dsts[i]) + size_t(q_begin) * row;
+    if (cudaMemcpy2DAsync(dst, size_t(ctx_cap) * row, src, size_t(stage_cap) * row,
+                          size_t(s_len) * row, heads, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+      return HGA_ERR_CUDA;
+  }
+  return HGA_OK;
+}
+
 hga_status_t hga_get_device_status(void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return HGA_ERR_CUDA;
@@ -445,7 +579,7 @@ const char* hga_kernel_name(int kind) {
   static const char* names[HGA_K_COUNT] = {
       "summaries",      "route_qmean",       "route_block_score",   "route_select",
       "attn_fwd_simt",  "attn_bwd_dq_simt",  "attn_bwd_dkdv_simt",  "attn_fwd_tc",
-      "attn_bwd_dq_tc", "attn_bwd_dkdv_tc"};
+      "attn_bwd_dq_tc", "attn_bwd_dkdv_tc",  "tier_dedup",          "tier_copy"};
   return (kind >= 0 && kind < HGA_K_COUNT) ? names[kind] : "unknown";
 }
 

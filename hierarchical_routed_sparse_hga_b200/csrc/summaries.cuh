@@ -16,8 +16,13 @@
 
 namespace hga {
 
+// K rows of head (b, h): k + ((b * Hkv + h) * k_rows + row) * D, where block
+// blk0 + i starts at row k_first + 64 i (k_rows = ctx_cap, k_first = 64 blk0
+// for a whole-context buffer; k_rows = segment capacity, k_first = 0 for a
+// segment-local one).  Summaries are indexed by global group / block.
 template <typename T, int D>
-__global__ void __launch_bounds__(D) summaries_kernel(const T* __restrict__ k, int64_t ctx_cap,
+__global__ void __launch_bounds__(D) summaries_kernel(const T* __restrict__ k, int64_t k_rows,
+                                                      int64_t k_first, int64_t ctx_cap,
                                                       int64_t blk0, int n_kv_heads,
                                                       float* __restrict__ gsum,
                                                       float* __restrict__ bsum) {
@@ -27,7 +32,8 @@ __global__ void __launch_bounds__(D) summaries_kernel(const T* __restrict__ k, i
   const int h = blockIdx.y, b = blockIdx.z;
   const int gi = threadIdx.x / CH, ch = threadIdx.x % CH;
   const int64_t head = int64_t(b) * n_kv_heads + h;
-  const T* src = k + (head * ctx_cap + c * kBlock + gi * kGroup) * D + ch * 8;
+  const T* src =
+      k + (head * k_rows + k_first + int64_t(blockIdx.x) * kBlock + gi * kGroup) * D + ch * 8;
 
   float acc[8];
 #pragma unroll

@@ -78,3 +78,95 @@ class HgaLayer:
         self.forward(q, q_begin, stream)
         if d_o is not None:
             self.backward(q, d_o, q_begin, stream)
+
+
+class HgaTieredLayer:
+    """One layer with its history K/V in pinned host memory.
+
+    Summaries stay in HBM.  Per segment: summaries of the active keys (from the
+    staging buffer), routing, the host-tier gather of the selected history
+    groups into HBM staging (hga_tier_gather), attention forward/backward on
+    the staging buffer, and finally the append of the segment's K/V to the
+    host history.  The caller writes the active segment's K/V into
+    `active_k()` / `active_v()` before calling `segment`.
+    """
+
+    def __init__(self, cfg: Config, ctx_cap: int, seg_len: int, device="cuda",
+                 k_host=None, v_host=None):
+        self.cfg, self.ctx_cap, self.seg_len = cfg, ctx_cap, seg_len
+        self.device = torch.device(device)
+        dt = _TORCH_DTYPE[cfg.dtype]
+        B, Hq, Hkv, d = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
+        n_qb = seg_len // 64
+        shape = (B, Hkv, ctx_cap, d)
+        self.k_host = k_host if k_host is not None else torch.zeros(shape, dtype=dt).pin_memory()
+        self.v_host = v_host if v_host is not None else torch.zeros(shape, dtype=dt).pin_memory()
+        self.stage_cap = _lib.hga_tier_stage_rows(cfg, ctx_cap - seg_len, seg_len)
+        self.k_stage = torch.zeros((B, Hkv, self.stage_cap, d), dtype=dt, device=self.device)
+        self.v_stage = torch.zeros_like(self.k_stage)
+        self.gsum = torch.zeros((B, Hkv, ctx_cap // 8, d), dtype=torch.float32,
+                                device=self.device)
+        self.bsum = torch.zeros((B, Hkv, ctx_cap // 64, d), dtype=torch.float32,
+                                device=self.device)
+        dev = self.device
+        self.route_ws = torch.empty(max(_lib.hga_route_workspace_size(cfg, seg_len,
+                                                                      ctx_cap - seg_len), 256),
+                                    dtype=torch.uint8, device=dev)
+        self.bwd_ws = torch.empty(max(_lib.hga_attn_bwd_workspace_size(cfg, seg_len), 256),
+                                  dtype=torch.uint8, device=dev)
+        self.tier_ws = torch.empty(max(_lib.hga_tier_workspace_size(cfg, seg_len,
+                                                                    ctx_cap - seg_len), 256),
+                                   dtype=torch.uint8, device=dev)
+        self.sel_blk = torch.empty((B, Hkv, n_qb, cfg.topk_blocks), dtype=torch.int32, device=dev)
+        self.sel_grp = torch.empty((B, Hkv, n_qb, cfg.topk_groups), dtype=torch.int32, device=dev)
+        self.sel_stage = torch.empty_like(self.sel_grp)
+        self.n_unique = torch.zeros((B, Hkv), dtype=torch.int32, device=dev)
+        self.o = torch.empty((B, Hq, seg_len, d), dtype=dt, device=dev)
+        self.lse = torch.empty((B, Hq, seg_len), dtype=torch.float32, device=dev)
+        self.dq = torch.empty_like(self.o)
+        self.dk = torch.empty((B, Hkv, seg_len, d), dtype=dt, device=dev)
+        self.dv = torch.empty_like(self.dk)
+
+    @property
+    def q_begin_stage(self) -> int:
+        return self.stage_cap - self.seg_len
+
+    def active_k(self):
+        return self.k_stage[:, :, self.q_begin_stage:, :]
+
+    def active_v(self):
+        return self.v_stage[:, :, self.q_begin_stage:, :]
+
+    def _active_ptr(self, t):
+        return t.data_ptr() + self.q_begin_stage * t.shape[-1] * t.element_size()
+
+    def summarize(self, q_begin: int, stream=None):
+        _lib.hga_build_summaries_seg(self.cfg, self._active_ptr(self.k_stage), self.stage_cap,
+                                     q_begin, q_begin + self.seg_len, self.ctx_cap, self.gsum,
+                                     self.bsum, stream)
+
+    def gather(self, q_begin: int, stream=None):
+        _lib.hga_tier_gather(self.cfg, self.k_host, self.v_host, self.ctx_cap, q_begin,
+                             self.seg_len, self.sel_grp, self.k_stage, self.v_stage,
+                             self.stage_cap, self.sel_stage, self.n_unique, self.tier_ws,
+                             stream=stream)
+
+    def append_history(self, q_begin: int, stream=None):
+        """The segment's K/V join the host history (detached)."""
+        _lib.hga_tier_append(self.cfg, self.k_stage, self.v_stage, self.stage_cap, self.k_host,
+                             self.v_host, self.ctx_cap, q_begin, self.seg_len, stream)
+
+    def segment(self, q, q_begin: int, d_o=None, stream=None, append=True):
+        cfg, S, qs = self.cfg, self.seg_len, self.q_begin_stage
+        self.summarize(q_begin, stream)
+        _lib.hga_route(cfg, q, q_begin, S, self.ctx_cap, self.bsum, self.gsum, self.sel_blk,
+                       self.sel_grp, self.route_ws, stream=stream)
+        self.gather(q_begin, stream)
+        _lib.hga_attn_fwd(cfg, q, self.k_stage, self.v_stage, self.stage_cap, qs, S,
+                          self.sel_stage, self.o, self.lse, stream)
+        if d_o is not None:
+            _lib.hga_attn_bwd(cfg, q, self.k_stage, self.v_stage, self.stage_cap, qs, S,
+                              self.sel_stage, self.o, self.lse, d_o, self.dq, self.dk, self.dv,
+                              self.bwd_ws, stream=stream)
+        if append:
+            self.append_history(q_begin, stream)

@@ -244,3 +244,57 @@ def douts(w: Workload, seg_begin: int, q_heads=None) -> np.ndarray:
     hs = range(w.n_q_heads) if q_heads is None else q_heads
     return np.stack([np.stack([dout_head(w, b, hq, seg_begin) for hq in hs])
                      for b in range(w.batch)])
+
+
+# ----------------------------------------------------------------------------
+# the same recipe drawn on the device with torch (large performance sweeps)
+# ----------------------------------------------------------------------------
+
+def device_inputs(w: Workload, device, backward=True):
+    """K, V [B,Hkv,T,d] and per-segment Q, dO [B,Hq,S,d] drawn on `device`.
+
+    Same distributions and layout as the NumPy streams above (centroids per
+    block, 0.5 noise, planted target blocks, 1/sqrt(d) scaling and RoPE for
+    scaled workloads), drawn from torch's generator seeded with w.seed: the
+    values differ from the NumPy streams, so parity tests never use this; it
+    exists because drawing gigabytes of inputs with NumPy takes minutes.
+    """
+    import torch
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed)
+    B, Hkv, Hq, T, S, d = w.batch, w.n_kv_heads, w.n_q_heads, w.ctx_len, w.seg_len, w.head_dim
+    G = w.group_heads
+
+    def rope(x, pos0):
+        if w.rope_base is None:
+            return x
+        half = d // 2
+        inv = w.rope_base ** (-torch.arange(half, device=device, dtype=torch.float64) * 2.0 / d)
+        pos = pos0 + torch.arange(x.shape[-2], device=device, dtype=torch.float64)
+        ang = pos[:, None] * inv[None, :]
+        c, s = torch.cos(ang).float(), torch.sin(ang).float()
+        x1, x2 = x[..., :half], x[..., half:]
+        return torch.cat([x1 * c - x2 * s, x2 * c + x1 * s], dim=-1)
+
+    scale = w.scale if w.scaled else 1.0
+    cent = torch.randn((B, Hkv, T // BLOCK, d), generator=g, device=device)
+    k = cent.repeat_interleave(BLOCK, dim=2) + 0.5 * torch.randn((B, Hkv, T, d), generator=g,
+                                                                   device=device)
+    k = rope(k * scale, 0).to(dt)
+    v = torch.randn((B, Hkv, T, d), generator=g, device=device).to(dt)
+    qs, dos = [], []
+    n_qb = S // QBLOCK
+    for s0 in w.segments():
+        n_hist = s0 // BLOCK
+        if n_hist:
+            r = torch.randint(0, n_hist, (B, Hkv, n_qb), generator=g, device=device)
+        else:
+            r = (s0 // BLOCK + torch.arange(n_qb, device=device)).expand(B, Hkv, n_qb)
+        base = torch.gather(cent, 2, r[..., None].expand(B, Hkv, n_qb, d))
+        base = base.repeat_interleave(QBLOCK, dim=2).repeat_interleave(G, dim=1)
+        q = base + 0.5 * torch.randn((B, Hq, S, d), generator=g, device=device)
+        qs.append(rope(q * scale, s0).to(dt).contiguous())
+        if backward:
+            dos.append(torch.randn((B, Hq, S, d), generator=g, device=device).to(dt))
+    return k.contiguous(), v.contiguous(), qs, dos

@@ -125,6 +125,19 @@ HGA_API hga_status_t hga_build_summaries(const hga_config_t* cfg, const void* k,
                                  int64_t t_begin, int64_t t_end, float* gsum, float* bsum,
                                  void* stream);
 
+/*
+ * Step a1 for a segment held in its own buffer (used with the host tier,
+ * where the whole-context K is not on the device).  k_seg is
+ * [batch, n_kv_heads, seg_cap, head_dim] with token t_begin + i at row i;
+ * gsum/bsum are the whole-context summaries ([.., ctx_cap/8, ..] and
+ * [.., ctx_cap/64, ..]) and receive the rows of groups t_begin/8 .. t_end/8-1
+ * and blocks t_begin/64 .. t_end/64-1, exactly as hga_build_summaries would.
+ */
+HGA_API hga_status_t hga_build_summaries_seg(const hga_config_t* cfg, const void* k_seg,
+                                             int64_t seg_cap, int64_t t_begin, int64_t t_end,
+                                             int64_t ctx_cap, float* gsum, float* bsum,
+                                             void* stream);
+
 /* Bytes of device workspace hga_route needs for this segment. */
 HGA_API size_t hga_route_workspace_size(const hga_config_t* cfg, int32_t s_len, int64_t q_begin);
 
@@ -209,6 +222,47 @@ HGA_API hga_status_t hga_attn_bwd(const hga_config_t* cfg, const void* q, const 
                           size_t ws_bytes, void* stream);
 
 /*
+ * Step a7 -- the host tier [A] ("older KV is detached into RAM or NVMe, and
+ * HGA loads a bounded set of exact historical tokens for each query block").
+ * History K/V stay in pinned host memory (k_host, v_host: whole-context
+ * [batch, n_kv_heads, ctx_cap, head_dim], allocated with cudaHostAlloc or
+ * registered with cudaHostRegister, device-mapped; pageable memory is
+ * rejected with HGA_ERR_INVALID_ARG).  For the segment starting at q_begin,
+ * every history group (index < q_begin/8) that any query block of the segment
+ * selected in sel_grp is copied once, per (batch, KV head), in ascending
+ * order, into rows [8u, 8u+8) of the device staging buffers k_stage/v_stage
+ * ([batch, n_kv_heads, stage_cap, head_dim]); u is its slot.  sel_stage
+ * ([batch, n_kv_heads, s_len/64, topk_groups]) receives the selection in
+ * staging indices: a history group -> its slot; a group of the active segment
+ * g -> (stage_cap - s_len)/8 + g - q_begin/8; -1 stays -1.  The caller places
+ * the active segment's K/V at staging rows [stage_cap - s_len, stage_cap), so
+ * hga_attn_fwd / hga_attn_bwd with (k_stage, v_stage, stage_cap,
+ * q_begin' = stage_cap - s_len, sel_stage) compute exactly what they compute on
+ * the whole-context buffers.  n_unique ([batch, n_kv_heads] int32, optional)
+ * receives the number of groups copied per head: 4 KiB each for bf16, d=128.
+ * stage_cap must be a multiple of 64 and >= hga_tier_stage_rows().
+ */
+HGA_API int64_t hga_tier_stage_rows(const hga_config_t* cfg, int64_t q_begin, int32_t s_len);
+HGA_API size_t hga_tier_workspace_size(const hga_config_t* cfg, int32_t s_len, int64_t q_begin);
+HGA_API hga_status_t hga_tier_gather(const hga_config_t* cfg, const void* k_host,
+                                     const void* v_host, int64_t ctx_cap, int64_t q_begin,
+                                     int32_t s_len, const int32_t* sel_grp, void* k_stage,
+                                     void* v_stage, int64_t stage_cap, int32_t* sel_stage,
+                                     int32_t* n_unique, void* workspace, size_t ws_bytes,
+                                     void* stream);
+
+/*
+ * Step a6 for the host tier: the active segment's K/V (staging rows
+ * [stage_cap - s_len, stage_cap)) join the host history at rows
+ * [q_begin, q_begin + s_len) of k_host / v_host (pinned).  One strided
+ * device-to-host copy per tensor on `stream` (copy engine, asynchronous).
+ */
+HGA_API hga_status_t hga_tier_append(const hga_config_t* cfg, const void* k_stage,
+                                     const void* v_stage, int64_t stage_cap, void* k_host,
+                                     void* v_host, int64_t ctx_cap, int64_t q_begin,
+                                     int32_t s_len, void* stream);
+
+/*
  * Reads and clears the calling device's latched device-side status
  * (HGA_OK, HGA_ERR_DEVICE_CHECK or HGA_ERR_TIMEOUT).  Synchronises `stream`.
  */
@@ -238,7 +292,9 @@ typedef enum {
   HGA_K_FWD_TC = 7,
   HGA_K_BWD_DQ_TC = 8,
   HGA_K_BWD_DKDV_TC = 9,
-  HGA_K_COUNT = 10
+  HGA_K_TIER_DEDUP = 10,
+  HGA_K_TIER_COPY = 11,
+  HGA_K_COUNT = 12
 } hga_kernel_kind_t;
 
 /* Name of a kernel kind ("attn_fwd_simt", ...). */

@@ -252,6 +252,37 @@ def attn_bwd(q, k, v, do, q_begin: int, sel_grp: np.ndarray, n_kv_heads: int):
 
 
 # ----------------------------------------------------------------------------
+# step a7: host tier -- which history groups cross PCIe, and the selection in
+# staging indices (the adnankhan.ai notes, "Raw Abstract / Excerpt": older KV
+# is detached into RAM or NVMe; HGA loads a bounded set of exact historical
+# tokens per query block)
+# ----------------------------------------------------------------------------
+
+def tier_stage(sel_grp: np.ndarray, q_begin: int, s_len: int, stage_cap: int):
+    """Per (b, KV head): the distinct history groups (index < q_begin/8) any
+    query block of the segment selected, ascending -- these are copied once --
+    and the selection rewritten to staging indices: history group -> its rank
+    among them, active-segment group g -> (stage_cap - s_len)/8 + g - q_begin/8,
+    -1 -> -1.  Returns (list of per-(b,h) unique arrays, sel_stage)."""
+    B, H = sel_grp.shape[:2]
+    n_hist = q_begin // GROUP
+    act0 = (stage_cap - s_len) // GROUP
+    uniques = [[None] * H for _ in range(B)]
+    out = np.full_like(sel_grp, -1)
+    for b in range(B):
+        for h in range(H):
+            sel = sel_grp[b, h]
+            hist = np.unique(sel[(sel >= 0) & (sel < n_hist)])
+            uniques[b][h] = hist
+            rank = {int(g): i for i, g in enumerate(hist)}
+            for idx, g in np.ndenumerate(sel):
+                if g < 0:
+                    continue
+                out[b, h][idx] = rank[int(g)] if g < n_hist else act0 + (int(g) - n_hist)
+    return uniques, out
+
+
+# ----------------------------------------------------------------------------
 # one segment of the segment-wise loop (a1 .. a5 in order)
 # ----------------------------------------------------------------------------
 

@@ -431,3 +431,43 @@ def test_pins_catch_planted_mistakes(monkeypatch, target, mutant):
         except AssertionError:
             failed += 1
     assert failed >= 1, f"no pin caught the planted mistake in {target}"
+
+
+# ----------------------------------------------------------------------------
+# pins: host tier (dedup + remap)
+# ----------------------------------------------------------------------------
+
+def test_tier_stage_preserves_attention():
+    # staging the distinct selected history groups and remapping the selection
+    # must leave every output and gradient unchanged
+    w, q, k, v, do, q_begin = tiny_case(seed=6, topk_blocks=3, topk_groups=7)
+    S, T = w.seg_len, q_begin + w.seg_len
+    g, bl = summaries_upto(k, T)
+    _, sg, _ = oracle.route(q, bl, g, q_begin, w.topk_blocks, w.topk_groups, w.n_kv_heads)
+    n_qb = S // 64
+    stage_cap = ((min(n_qb * w.topk_groups, q_begin // 8) * 8 + 63) // 64) * 64 + S
+    uniq, sel_st = oracle.tier_stage(sg, q_begin, S, stage_cap)
+    ks = np.full((w.batch, w.n_kv_heads, stage_cap, w.head_dim), np.nan)
+    vs = np.full_like(ks, np.nan)
+    for b in range(w.batch):
+        for h in range(w.n_kv_heads):
+            u = uniq[b][h]
+            assert (np.diff(u) > 0).all() and (u < q_begin // 8).all()
+            rows = (u[:, None] * 8 + np.arange(8)[None, :]).reshape(-1)
+            ks[b, h, :len(rows)] = k[b, h, rows]
+            vs[b, h, :len(rows)] = v[b, h, rows]
+    ks[:, :, stage_cap - S:] = k[:, :, q_begin:T]
+    vs[:, :, stage_cap - S:] = v[:, :, q_begin:T]
+    o1, l1 = oracle.attn_fwd(q, k, v, q_begin, sg, w.n_kv_heads)
+    o2, l2 = oracle.attn_fwd(q, ks, vs, stage_cap - S, sel_st, w.n_kv_heads)
+    assert close(o1, o2, 1e-13) and close(l1, l2, 1e-13)
+    g1 = oracle.attn_bwd(q, k, v, do, q_begin, sg, w.n_kv_heads)
+    g2 = oracle.attn_bwd(q, ks, vs, do, stage_cap - S, sel_st, w.n_kv_heads)
+    for a, b_ in zip(g1, g2):
+        assert close(a, b_, 1e-13)
+    # every history group any query block selected is staged exactly once
+    for b in range(w.batch):
+        for h in range(w.n_kv_heads):
+            sel = sg[b, h]
+            want = sorted(set(int(x) for x in sel.ravel() if 0 <= x < q_begin // 8))
+            assert list(uniq[b][h]) == want
