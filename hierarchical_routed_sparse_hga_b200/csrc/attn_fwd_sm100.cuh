@@ -3,22 +3,31 @@
 // ("BMW如何通过重新设计注意力机制…", section "HGA的不同之处": only the selected
 // groups' exact K/V enter the attention; the summaries only steer selection).
 //
-// One CTA per (batch, KV head, query block).  The G query heads that share
-// the KV head share the selection, so the CTA stacks them into M = 64*G rows
-// (MT = G/2 tiles of 128 rows) and every gathered K/V tile feeds all of them.
+// One CTA per (batch, KV head, query block, set of 2*MT query heads): the G
+// query heads sharing a KV head share the selection, so up to four of them
+// are stacked into MT tiles of M = 128 rows and every gathered K/V tile feeds
+// all of them.
 //
-// Roles (warp-specialised, one CTA per SM: 192 KB of shared memory at MT=2):
-//   warp 0      TMA producer: Q once (64 x 64 boxes), then per key tile the
-//               8 selected groups of K and V as 8-row boxes (a group is a
-//               contiguous 2 KiB run of [B,Hkv,T,d]) into a 3-stage ring;
-//   warp 1      TMEM owner and MMA issuer: S = Q K^T into double-buffered TMEM
-//               (per M tile), then O += P V with P from shared memory;
-//   warps 4..   softmax, one warp group (4 warps = 128 TMEM lanes) per M
-//               tile, one thread per row: masks (padding slots, causal own
-//               block), online softmax in the log2 domain with lazy
-//               rescaling (O in TMEM is rescaled only when the running max
-//               grows by more than 2^8), P to shared memory (bf16, 128-byte
-//               swizzle), epilogue O / l and LSE.
+// Roles (128 + 128*MT threads, one CTA per SM):
+//   warps 0,2,3 producers: Q once by TMA (64 x 64 boxes); then per key tile
+//               the 8 selected groups of K and V (a group is a contiguous
+//               2 KiB run of [B,Hkv,T,d]) by 16-byte cp.async copies, 96
+//               threads x ~21 copies, written straight into the 128-byte-
+//               swizzled operand layout of a 4-stage ring -- far faster than
+//               8-row TMA boxes, whose per-box cost capped the gather at ~16 B
+//               per cycle per SM; the gather latency of one tile hides behind
+//               three others;
+//   warp 1      TMEM owner and MMA issuer.  It issues, as soon as each one's
+//               inputs are ready, S = Q K^T into double-buffered TMEM and
+//               O += P V with P read straight from TMEM (A operand in tensor
+//               memory) -- whichever is ready first, so a late K/V tile never
+//               holds back the PV of the tile before it;
+//   warps 4..   softmax, one warp group per M tile, one thread per row (TMEM
+//               lane): masks (padding slots, causal own block; skipped for
+//               full routed tiles), online softmax in the log2 domain with
+//               packed f32x2 arithmetic and lazy rescaling (O is rescaled only
+//               when the running max grows by more than 2^8), P written back as
+//               bf16 over its own S columns, epilogue O / l and LSE.
 // Every wait is bounded; a timeout latches HGA_ERR_TIMEOUT, raises a shared
 // abort flag, drains the copies and MMAs in flight and frees TMEM.
 #pragma once
@@ -35,7 +44,8 @@ namespace fwdtc {
 using namespace sm100;
 
 constexpr int kD = 128;
-constexpr int kStages = 3;
+constexpr int kStages = 4;
+constexpr int kProducers = 96;  // warps 0, 2, 3
 constexpr int kMaxTiles = 33;  // 256 groups / 8 + own block
 
 template <int MT>
@@ -43,22 +53,23 @@ struct Layout {
   static constexpr uint32_t kQ = 0;                                // [MT][2 halves][128][128 B]
   static constexpr uint32_t kKV = MT * 32768;                      // [stage][K 16 KB | V 16 KB]
   static constexpr uint32_t kStageBytes = 32768;
-  static constexpr uint32_t kP = kKV + kStages * kStageBytes;      // [MT][128][128 B]
-  static constexpr uint32_t kBytes = kP + MT * 16384;
+  static constexpr uint32_t kBytes = kKV + kStages * kStageBytes;
   static constexpr uint32_t kDynSmem = kBytes + 1024;              // + alignment slack
   static constexpr uint32_t kThreads = 128 + 128 * MT;
   static constexpr uint32_t kTmemCols = MT == 2 ? 512 : 256;
-  static constexpr uint32_t kColO = MT * 128;                      // S buffers first
+  static constexpr uint32_t colS(int m, int buf) { return (m * 2 + buf) * 64; }
+  static constexpr uint32_t colO(int m) { return MT * 128 + m * kD; }
 };
 
 struct Shared {
   uint64_t q_full;
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
+  // [M tile][tile & 1]: per-buffer barriers, so no waiter can ever fall two
+  // phases behind (that would need a tile whose S buffer is still in use)
   uint64_t s_full[2][2];
-  uint64_t s_free[2][2];
-  uint64_t p_full[2];
-  uint64_t pv_done[2];
+  uint64_t p_full[2][2];
+  uint64_t pv_done[2][2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
@@ -69,26 +80,27 @@ struct Shared {
 
 constexpr uint32_t kTestDropFirstTile = 0x80000000u;  // test hook, see hga.h
 
+// grid (n_qb * G / (2 MT), Hkv, B)
 template <int MT>
 __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
-                       const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, int64_t ctx_cap,
-                       int64_t q_begin, int s_len, int n_q_heads, int n_kv_heads,
+                       const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                       int64_t ctx_cap, int64_t q_begin, int s_len, int n_q_heads, int n_kv_heads,
                        int topk_groups, const int32_t* __restrict__ sel_grp, float scale_log2,
                        __nv_bfloat16* __restrict__ o, float* __restrict__ lse, uint32_t flags) {
   using L = Layout<MT>;
-  constexpr int G = 2 * MT;
   extern __shared__ uint8_t dsmem_raw[];
   __shared__ Shared sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sQ = smem_u32(smem + L::kQ);
   const uint32_t sKV = smem_u32(smem + L::kKV);
-  const uint32_t sP = smem_u32(smem + L::kP);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int G = n_q_heads / n_kv_heads, n_sets = G / (2 * MT);
+  const int j = blockIdx.x / n_sets, hs = blockIdx.x % n_sets;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int head0 = h * G + hs * 2 * MT;       // first query head of this CTA
   const int n_qb = s_len / kQBlock;
   const int64_t own_blk = (q_begin + int64_t(j) * kQBlock) / kBlock;
   volatile int* abort = &sh.abort;
@@ -97,17 +109,15 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
   if (tid == 0) {
     mbar_init(&sh.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sh.kv_full[s], 1);
+      mbar_init(&sh.kv_full[s], kProducers);
       mbar_init(&sh.kv_empty[s], 1);
     }
-    for (int m = 0; m < 2; ++m) {
+    for (int m = 0; m < 2; ++m)
       for (int u = 0; u < 2; ++u) {
         mbar_init(&sh.s_full[m][u], 1);
-        mbar_init(&sh.s_free[m][u], 128);
+        mbar_init(&sh.p_full[m][u], 128);
+        mbar_init(&sh.pv_done[m][u], 1);
       }
-      mbar_init(&sh.p_full[m], 128);
-      mbar_init(&sh.pv_done[m], 1);
-    }
     mbar_init(&sh.mma_done, 1);
     sh.abort = 0;
     fence_barrier_init();
@@ -152,180 +162,208 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
   const uint32_t tmem = sh.tmem_base;
   const int n_tiles = sh.n_tiles;
 
-  if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
+  if (warp == 0 || warp == 2 || warp == 3) {
+    // ---------------- producers ----------------
+    const int ptid = warp == 0 ? lane : 32 * (warp - 1) + lane;  // 0..95
+    if (tid == 0) {
       prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
       mbar_arrive_expect_tx(&sh.q_full, MT * 32768);
-      for (int g = 0; g < G; ++g) {
-        const int32_t row = int32_t((int64_t(b) * n_q_heads + h * G + g) * s_len + j * kQBlock);
+      for (int g = 0; g < 2 * MT; ++g) {
+        const int32_t row =
+            int32_t((int64_t(b) * n_q_heads + head0 + g) * s_len + j * kQBlock);
         for (int hf = 0; hf < 2; ++hf) {
           uint8_t* dst = smem + L::kQ + (g >> 1) * 32768 + hf * 16384 + (g & 1) * 8192;
           tma_load_2d(dst, &tm_q, &sh.q_full, hf * 64, row);
         }
       }
-      const int64_t kv_row0 = (int64_t(b) * n_kv_heads + h) * ctx_cap;
-      int issued = 0;
-      for (int t = 0; t < n_tiles; ++t) {
-        const int st = t % kStages;
-        if (t >= kStages && !mbar_wait(&sh.kv_empty[st], ((t / kStages) - 1) & 1, abort)) break;
-        if ((flags & kTestDropFirstTile) && t == 0) continue;  // test hook: never armed
-        mbar_arrive_expect_tx(&sh.kv_full[st], L::kStageBytes);
-        uint8_t* kdst = smem + L::kKV + st * L::kStageBytes;
-        for (int gi = 0; gi < 8; ++gi) {
-          const int32_t row = int32_t(kv_row0 + int64_t(sh.grp[t * 8 + gi]) * kGroup);
-          for (int hf = 0; hf < 2; ++hf) {
-            tma_load_2d(kdst + hf * 8192 + gi * 1024, &tm_k, &sh.kv_full[st], hf * 64, row);
-            tma_load_2d(kdst + 16384 + hf * 8192 + gi * 1024, &tm_v, &sh.kv_full[st], hf * 64,
-                        row);
-          }
-        }
-        issued = t + 1;
-      }
-      // drain: wait (bounded, independent of abort) for the copies in flight
-      int never = 0;
-      mbar_wait(&sh.q_full, 0, &never, 2000000000LL);
-      for (int t = issued - 1; t >= 0 && t >= issued - kStages; --t) {
-        if ((flags & kTestDropFirstTile) && t == 0) continue;
-        mbar_wait(&sh.kv_full[t % kStages], (t / kStages) & 1, &never, 2000000000LL);
-      }
     }
+    const __nv_bfloat16* kh = k + (int64_t(b) * n_kv_heads + h) * ctx_cap * kD;
+    const __nv_bfloat16* vh = v + (int64_t(b) * n_kv_heads + h) * ctx_cap * kD;
+    int issued = 0;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int st = t % kStages;
+      if (t >= kStages && !mbar_wait(&sh.kv_empty[st], ((t / kStages) - 1) & 1, abort)) break;
+      if ((flags & kTestDropFirstTile) && t == 0) continue;  // test hook: never arrives
+      const uint32_t kdst = sKV + st * L::kStageBytes;
+      // 2 tensors x 64 rows x 16 chunks of 16 B; a row's 16 chunks go to 16
+      // consecutive threads (coalesced 256-byte reads)
+      for (int c = ptid; c < 2048; c += kProducers) {
+        const int tensor = c >> 10, rc = c & 1023, r = rc >> 4, ch = rc & 15;
+        const int64_t row = int64_t(sh.grp[t * 8 + (r >> 3)]) * kGroup + (r & 7);
+        const __nv_bfloat16* src = (tensor ? vh : kh) + row * kD + ch * 8;
+        const uint32_t dst = kdst + tensor * 16384 + (ch >> 3) * 8192 + r * 128 +
+                             (((ch & 7) ^ (r & 7)) << 4);
+        cp_async16(dst, src);
+      }
+      cp_async_arrive(&sh.kv_full[st]);
+      issued = t + 1;
+    }
+    // drain: wait (bounded, independent of abort) for the copies in flight
+    int never = 0;
+    if (tid == 0) mbar_wait(&sh.q_full, 0, &never);
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    (void)issued;
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+    // ---------------- MMA issuer (event driven) ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kD, 0, 1);
       bool ok = mbar_wait(&sh.q_full, 0, abort);
       bool issued_any = false;
-      tc_fence_after();
-      for (int t = 0; ok && t <= n_tiles; ++t) {
-        if (t < n_tiles) {
-          const int st = t % kStages, buf = t & 1;
-          if (!mbar_wait(&sh.kv_full[st], (t / kStages) & 1, abort)) break;
-          for (int m = 0; m < MT && ok; ++m)
-            if (t >= 2) ok = mbar_wait(&sh.s_free[m][buf], ((t >> 1) - 1) & 1, abort);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t kbase = sKV + st * L::kStageBytes;
-          for (int m = 0; m < MT; ++m) {
-            const uint32_t d = tmem + (m * 2 + buf) * 64;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint64_t a =
-                  smem_desc_sw128(sQ + m * 32768 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(kbase + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024);
-              mma_bf16(d, a, bd, idesc_qk, k > 0);
-            }
-            mma_commit(&sh.s_full[m][buf]);
-          }
-          issued_any = true;
-        }
-        if (t >= 1) {
-          const int tt = t - 1, st = tt % kStages;
-          const uint32_t vbase = sKV + st * L::kStageBytes + 16384;
-          for (int m = 0; m < MT; ++m) {
-            if (!(ok = mbar_wait(&sh.p_full[m], tt & 1, abort))) break;
+      int next_qk = 0, next_pv = 0;  // next tile to issue S = QK^T for / O += PV for
+      long long t0 = clock64();
+      while (ok && next_pv < n_tiles) {
+        bool progressed = false;
+        // PV(next_pv) once every M tile's P is in TMEM
+        if (next_pv < next_qk) {
+          bool ready = true;
+          for (int m = 0; m < MT; ++m)
+            ready = ready && mbar_try_wait(&sh.p_full[m][next_pv & 1], (next_pv >> 1) & 1);
+          if (ready) {
+            const int tt = next_pv, st = tt % kStages;
+            const uint32_t vbase = sKV + st * L::kStageBytes + 16384;
             tc_fence_after();
-            const uint32_t d = tmem + L::kColO + m * kD;
+            for (int m = 0; m < MT; ++m) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t a = smem_desc_sw128(sP + m * 16384 + k * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(vbase + k * 2048, 8192, 1024);
-              mma_bf16(d, a, bd, idesc_pv, (tt > 0 || k > 0) ? 1u : 0u);
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t bd = smem_desc_sw128(vbase + k * 2048, 8192, 1024);
+                mma_bf16_tmem_a(tmem + L::colO(m), tmem + L::colS(m, tt & 1) + k * 8, bd,
+                                idesc_pv, (tt > 0 || k > 0) ? 1u : 0u);
+              }
+              mma_commit(&sh.pv_done[m][tt & 1]);
             }
-            mma_commit(&sh.pv_done[m]);
+            mma_commit(&sh.kv_empty[st]);
+            ++next_pv;
+            progressed = true;
           }
-          if (!ok) break;
-          mma_commit(&sh.kv_empty[st]);
+        }
+        // S(next_qk) once its K/V tile is in and its S buffer is free again:
+        // P(next_qk - 2) lives there until PV(next_qk - 2) has read it
+        if (!progressed && next_qk < n_tiles && next_qk < next_pv + 2) {
+          const int t = next_qk, st = t % kStages, buf = t & 1;
+          bool ready = mbar_try_wait(&sh.kv_full[st], (t / kStages) & 1);
+          for (int m = 0; m < MT && ready && t >= 2; ++m)
+            ready = mbar_try_wait(&sh.pv_done[m][buf], ((t - 2) >> 1) & 1);
+          if (ready) {
+            fence_proxy_async_smem();  // cp.async (generic proxy) data -> tensor-core reads
+            tc_fence_after();
+            const uint32_t kbase = sKV + st * L::kStageBytes;
+            for (int m = 0; m < MT; ++m) {
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const uint64_t a =
+                    smem_desc_sw128(sQ + m * 32768 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+                const uint64_t bd =
+                    smem_desc_sw128(kbase + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024);
+                mma_bf16(tmem + L::colS(m, buf), a, bd, idesc_qk, k > 0);
+              }
+              mma_commit(&sh.s_full[m][buf]);
+            }
+            ++next_qk;
+            issued_any = true;
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          t0 = clock64();
+        } else if (*abort) {
+          ok = false;
+        } else if (clock64() - t0 > 2000000000LL) {
+          latch_status(HGA_ERR_TIMEOUT);
+          *abort = 1;
+          ok = false;
         }
       }
       if (issued_any) {
         // every MMA this thread issued must finish before TMEM is freed
         int never = 0;
         mma_commit(&sh.mma_done);
-        mbar_wait(&sh.mma_done, 0, &never, 2000000000LL);
+        mbar_wait(&sh.mma_done, 0, &never);
       }
     }
   } else if (warp >= 4) {
     // ---------------- softmax / epilogue ----------------
-    const int m = (warp - 4) >> 2, wq = (warp - 4) & 3;
-    const int row = wq * 32 + lane;          // row inside the M tile = TMEM lane
-    const int grow = m * 128 + row;          // row inside the CTA: head g, token r
+    const int m = (warp - 4) >> 2, wq = warp & 3;
+    const int row = wq * 32 + lane;          // row in the M tile = TMEM lane
+    const int grow = m * 128 + row;          // row in the CTA: head, token
     const int g = grow >> 6, r = grow & 63;
     const uint32_t lane_addr = uint32_t(wq * 32) << 16;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    uint8_t* prow = smem + L::kP + m * 16384 + row * 128;
     for (int t = 0; t < n_tiles && ok; ++t) {
       const int buf = t & 1;
       if (!(ok = mbar_wait(&sh.s_full[m][buf], (t >> 1) & 1, abort))) break;
       tc_fence_after();
       float s[64];
-      tmem_ld32(tmem + lane_addr + (m * 2 + buf) * 64, s);
-      tmem_ld32(tmem + lane_addr + (m * 2 + buf) * 64 + 32, s + 32);
+      tmem_ld32(tmem + lane_addr + L::colS(m, buf), s);
+      tmem_ld32(tmem + lane_addr + L::colS(m, buf) + 32, s + 32);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&sh.s_free[m][buf]);
-
       const bool own = t == n_tiles - 1;
       const uint32_t mask = sh.tile_mask[t];
-      float tmax = -INFINITY;
+      if (own || mask != 0xffu) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const bool valid = ((mask >> (i >> 3)) & 1u) && (!own || i <= r);
-        s[i] = valid ? s[i] * scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, s[i]);
+        for (int i = 0; i < 64; ++i) {
+          const bool valid = ((mask >> (i >> 3)) & 1u) && (!own || i <= r);
+          if (!valid) s[i] = -INFINITY;
+        }
       }
-      if (t > 0 && !(ok = mbar_wait(&sh.pv_done[m], (t - 1) & 1, abort))) break;
-      tc_fence_after();
+      float m0 = fmax3(s[0], s[1], s[2]), m1 = fmax3(s[3], s[4], s[5]);
+#pragma unroll
+      for (int i = 6; i < 62; i += 4) {
+        m0 = fmax3(m0, s[i], s[i + 1]);
+        m1 = fmax3(m1, s[i + 2], s[i + 3]);
+      }
+      const float tmax = fmax3(m0, m1, fmaxf(s[62], s[63])) * scale_log2;
       if (t == 0) {
         m_run = tmax;
       } else if (tmax > m_run + 8.f) {
         // lazy rescale: only when the running max grows by more than 2^8
-        const float alpha = exp2f(m_run - tmax);
+        if (!(ok = mbar_wait(&sh.pv_done[m][(t - 1) & 1], ((t - 1) >> 1) & 1, abort))) break;
+        tc_fence_after();
+        const float alpha = ex2_approx(m_run - tmax);
         l_run *= alpha;
         for (int c = 0; c < kD; c += 32) {
           float ov[32];
-          tmem_ld32(tmem + lane_addr + L::kColO + m * kD + c, ov);
+          tmem_ld32(tmem + lane_addr + L::colO(m) + c, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-          tmem_st32(tmem + lane_addr + L::kColO + m * kD + c, ov);
+          tmem_st32(tmem + lane_addr + L::colO(m) + c, ov);
         }
         tmem_wait_st();
         m_run = tmax;
       }
-      float psum = 0.f;
+      // p = 2^(s c - m): one packed FMA per pair, then the exponential
+      const float2 c2 = make_float2(scale_log2, scale_log2);
+      const float2 nm = make_float2(-m_run, -m_run);
+      uint32_t pk[32];
+      float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float p0 = exp2f(s[8 * c + 2 * u] - m_run);
-          const float p1 = exp2f(s[8 * c + 2 * u + 1] - m_run);
-          psum += p0 + p1;
-          __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
-          w[u] = *reinterpret_cast<uint32_t*>(&pr);
-        }
-        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int i = 0; i < 32; ++i) {
+        float2 x = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), c2, nm);
+        x.x = ex2_approx(x.x);
+        x.y = ex2_approx(x.y);
+        acc = __fadd2_rn(acc, x);
+        pk[i] = pack_bf16x2(x.x, x.y);
       }
-      l_run += psum;
-      fence_proxy_async_smem();
+      l_run += acc.x + acc.y;
+      // P(t) goes over the first 32 columns of its own S buffer
+      tmem_st32_u(tmem + lane_addr + L::colS(m, buf), pk);
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sh.p_full[m]);
+      mbar_arrive(&sh.p_full[m][buf]);
     }
-    if (ok) ok = mbar_wait(&sh.pv_done[m], (n_tiles - 1) & 1, abort);
+    if (ok)
+      ok = mbar_wait(&sh.pv_done[m][(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort);
     if (ok) {
       tc_fence_after();
       const float inv = 1.f / l_run;
-      const int hq = h * G + g;
+      const int hq = head0 + g;
       const int64_t orow = (int64_t(b) * n_q_heads + hq) * s_len + int64_t(j) * kQBlock + r;
       __nv_bfloat16* odst = o + orow * kD;
       for (int c = 0; c < kD; c += 32) {
         float ov[32];
-        tmem_ld32(tmem + lane_addr + L::kColO + m * kD + c, ov);
+        tmem_ld32(tmem + lane_addr + L::colO(m) + c, ov);
         tmem_wait_ld();
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {

@@ -133,20 +133,19 @@ hga_status_t launch_fwd_tc(const hga_config_t* cfg, const void* q, const void* k
                            int64_t ctx_cap, int64_t q_begin, int32_t s_len,
                            const int32_t* sel_grp, void* o, float* lse, cudaStream_t s) {
   using L = fwdtc::Layout<MT>;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq;
   const uint64_t q_rows = uint64_t(cfg->batch) * cfg->n_q_heads * s_len;
-  const uint64_t kv_rows = uint64_t(cfg->batch) * cfg->n_kv_heads * ctx_cap;
-  if (!make_map_bf16_d128(&tq, q, q_rows, 64) || !make_map_bf16_d128(&tk, k, kv_rows, 8) ||
-      !make_map_bf16_d128(&tv, v, kv_rows, 8))
-    return HGA_ERR_CUDA;
-  hga_status_t e = ensure_smem(reinterpret_cast<const void*>(&fwdtc::attn_fwd_tc_kernel<MT>),
-                               L::kDynSmem);
+  if (!make_map_bf16_d128(&tq, q, q_rows, 64)) return HGA_ERR_CUDA;
+  hga_status_t e = ensure_smem(
+      reinterpret_cast<const void*>(&fwdtc::attn_fwd_tc_kernel<MT>), L::kDynSmem);
   if (e != HGA_OK) return e;
-  dim3 grid(s_len / kQBlock, cfg->n_kv_heads, cfg->batch);
+  const int sets = cfg->n_q_heads / cfg->n_kv_heads / (2 * MT);
+  dim3 grid((s_len / kQBlock) * sets, cfg->n_kv_heads, cfg->batch);
   const float scale_log2 = cfg->scale * 1.4426950408889634f;
   return traced_launch(HGA_K_FWD_TC, s, [&] {
     fwdtc::attn_fwd_tc_kernel<MT><<<grid, L::kThreads, L::kDynSmem, s>>>(
-        tq, tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups,
+        tq, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), ctx_cap,
+        q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups,
         sel_grp, scale_log2, static_cast<__nv_bfloat16*>(o), lse, cfg->flags);
   });
 }
@@ -368,7 +367,7 @@ hga_status_t hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k,
   const int n_qb = s_len / kQBlock;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (use_tensor_cores(cfg, ctx_cap, s_len)) {
-    if (cfg->n_q_heads / cfg->n_kv_heads == 4)
+    if ((cfg->n_q_heads / cfg->n_kv_heads) % 4 == 0)
       return launch_fwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, s);
     return launch_fwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, s);
   }
