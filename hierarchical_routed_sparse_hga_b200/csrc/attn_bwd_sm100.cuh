@@ -107,12 +107,14 @@ __device__ __forceinline__ void build_schedule(SH& sh, const int32_t* srow, int 
   }
 }
 
+constexpr int kDqProducers = 96;  // warps 0, 2, 3
+
 template <int MT>
 __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_do,
-                          const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, int64_t ctx_cap,
+                          const __nv_bfloat16* __restrict__ k,
+                          const __nv_bfloat16* __restrict__ v, int64_t ctx_cap,
                           int64_t q_begin, int s_len, int n_q_heads, int n_kv_heads,
                           int topk_groups, const int32_t* __restrict__ sel_grp, float scale,
                           float scale_log2, const __nv_bfloat16* __restrict__ o,
@@ -136,7 +138,7 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
   if (tid == 0) {
     mbar_init(&sh.q_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&sh.kv_full[s], 1);
+      mbar_init(&sh.kv_full[s], kDqProducers);
       mbar_init(&sh.kv_empty[s], 1);
     }
     for (int m = 0; m < 2; ++m) {
@@ -162,12 +164,12 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
   const uint32_t tmem = sh.tmem_base;
   const int n_tiles = sh.n_tiles;
 
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp == 0 || warp == 2 || warp == 3) {
+    // ---------------- producers: Q, dO by TMA; K/V groups by cp.async ----------------
+    const int ptid = warp == 0 ? lane : 32 * (warp - 1) + lane;
+    if (tid == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_do);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
       mbar_arrive_expect_tx(&sh.q_full, MT * 65536);
       for (int g = 0; g < G; ++g) {
         const int32_t row = int32_t((int64_t(b) * n_q_heads + h * G + g) * s_len + j * kQBlock);
@@ -177,73 +179,92 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
           tma_load_2d(smem + L::kDO + off, &tm_do, &sh.q_full, hf * 64, row);
         }
       }
-      const int64_t kv_row0 = (int64_t(b) * n_kv_heads + h) * ctx_cap;
-      int issued = 0;
-      for (int t = 0; t < n_tiles; ++t) {
-        const int st = t & 1;
-        if (t >= 2 && !mbar_wait(&sh.kv_empty[st], ((t >> 1) - 1) & 1, abort)) break;
-        mbar_arrive_expect_tx(&sh.kv_full[st], L::kStageBytes);
-        uint8_t* kdst = smem + L::kKV + st * L::kStageBytes;
-        for (int gi = 0; gi < 8; ++gi) {
-          const int32_t row = int32_t(kv_row0 + int64_t(sh.grp[t * 8 + gi]) * kGroup);
-          for (int hf = 0; hf < 2; ++hf) {
-            tma_load_2d(kdst + hf * 8192 + gi * 1024, &tm_k, &sh.kv_full[st], hf * 64, row);
-            tma_load_2d(kdst + 16384 + hf * 8192 + gi * 1024, &tm_v, &sh.kv_full[st], hf * 64,
-                        row);
-          }
-        }
-        issued = t + 1;
-      }
-      int never = 0;
-      mbar_wait(&sh.q_full, 0, &never);
-      for (int t = issued - 1; t >= 0 && t >= issued - 2; --t)
-        mbar_wait(&sh.kv_full[t & 1], (t >> 1) & 1, &never);
     }
+    const __nv_bfloat16* kh = k + (int64_t(b) * n_kv_heads + h) * ctx_cap * kD;
+    const __nv_bfloat16* vh = v + (int64_t(b) * n_kv_heads + h) * ctx_cap * kD;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int st = t & 1;
+      if (t >= 2 && !mbar_wait(&sh.kv_empty[st], ((t >> 1) - 1) & 1, abort)) break;
+      const uint32_t kdst = sKV + st * L::kStageBytes;
+      for (int c = ptid; c < 2048; c += kDqProducers) {
+        const int tensor = c >> 10, rc = c & 1023, r = rc >> 4, ch = rc & 15;
+        const int64_t row = int64_t(sh.grp[t * 8 + (r >> 3)]) * kGroup + (r & 7);
+        const __nv_bfloat16* src = (tensor ? vh : kh) + row * kD + ch * 8;
+        cp_async16(kdst + tensor * 16384 + (ch >> 3) * 8192 + r * 128 + (((ch & 7) ^ (r & 7)) << 4),
+                   src);
+      }
+      cp_async_arrive(&sh.kv_full[st]);
+    }
+    int never = 0;
+    if (tid == 0) mbar_wait(&sh.q_full, 0, &never);
+    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 1) {
+    // ---------------- MMA issuer (event driven) ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kD, 0, 1);
       bool ok = mbar_wait(&sh.q_full, 0, abort);
       bool issued_any = false;
-      tc_fence_after();
-      for (int t = 0; ok && t <= n_tiles; ++t) {
-        if (t < n_tiles) {
-          const int st = t & 1;
-          if (!(ok = mbar_wait(&sh.kv_full[st], (t >> 1) & 1, abort))) break;
-          for (int m = 0; m < MT && ok; ++m)
-            if (t >= 1) ok = mbar_wait(&sh.sdp_free[m], (t - 1) & 1, abort);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t kb = sKV + st * L::kStageBytes;
-          for (int m = 0; m < MT; ++m) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32;
-              const uint32_t bo = (k >> 2) * 8192 + (k & 3) * 32;
-              mma_bf16(tmem + L::colS(m), smem_desc_sw128(sQ + m * 32768 + ko, 16, 1024),
-                       smem_desc_sw128(kb + bo, 16, 1024), idesc_s, k > 0);
-              mma_bf16(tmem + L::colDP(m), smem_desc_sw128(sDO + m * 32768 + ko, 16, 1024),
-                       smem_desc_sw128(kb + 16384 + bo, 16, 1024), idesc_s, k > 0);
-            }
-            mma_commit(&sh.sdp_full[m]);
-          }
-          issued_any = true;
-        }
-        if (t >= 1) {
-          const int tt = t - 1, st = tt & 1;
-          const uint32_t kb = sKV + st * L::kStageBytes;
-          for (int m = 0; m < MT; ++m) {
-            if (!(ok = mbar_wait(&sh.ds_full[m], tt & 1, abort))) break;
+      int next_sdp = 0, next_dq = 0;
+      long long t0 = clock64();
+      while (ok && next_dq < n_tiles) {
+        bool progressed = false;
+        if (next_dq < next_sdp) {
+          bool ready = true;
+          for (int m = 0; m < MT; ++m) ready = ready && mbar_try_wait(&sh.ds_full[m], next_dq & 1);
+          if (ready) {
+            const int tt = next_dq;
+            const uint32_t kb = sKV + (tt & 1) * L::kStageBytes;
             tc_fence_after();
+            for (int m = 0; m < MT; ++m) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_bf16(tmem + L::colDQ(m), smem_desc_sw128(sDS + m * 16384 + k * 32, 16, 1024),
-                       smem_desc_sw128(kb + k * 2048, 8192, 1024), idesc_dq,
-                       (tt > 0 || k > 0) ? 1u : 0u);
-            mma_commit(&sh.ds_done[m]);
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tmem + L::colDQ(m), smem_desc_sw128(sDS + m * 16384 + kk * 32, 16, 1024),
+                         smem_desc_sw128(kb + kk * 2048, 8192, 1024), idesc_dq,
+                         (tt > 0 || kk > 0) ? 1u : 0u);
+              mma_commit(&sh.ds_done[m]);
+            }
+            mma_commit(&sh.kv_empty[tt & 1]);
+            ++next_dq;
+            progressed = true;
           }
-          if (!ok) break;
-          mma_commit(&sh.kv_empty[st]);
+        }
+        // S/dP(t) may run one tile ahead of dQ: its TMEM columns are free once
+        // the softmax has loaded S/dP(t-1)
+        if (!progressed && next_sdp < n_tiles && next_sdp <= next_dq + 1) {
+          const int t = next_sdp, st = t & 1;
+          bool ready = mbar_try_wait(&sh.kv_full[st], (t >> 1) & 1);
+          for (int m = 0; m < MT && ready && t >= 1; ++m)
+            ready = mbar_try_wait(&sh.sdp_free[m], (t - 1) & 1);
+          if (ready) {
+            fence_proxy_async_smem();  // cp.async data -> tensor-core reads
+            tc_fence_after();
+            const uint32_t kb = sKV + st * L::kStageBytes;
+            for (int m = 0; m < MT; ++m) {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+                const uint32_t bo = (kk >> 2) * 8192 + (kk & 3) * 32;
+                mma_bf16(tmem + L::colS(m), smem_desc_sw128(sQ + m * 32768 + ko, 16, 1024),
+                         smem_desc_sw128(kb + bo, 16, 1024), idesc_s, kk > 0);
+                mma_bf16(tmem + L::colDP(m), smem_desc_sw128(sDO + m * 32768 + ko, 16, 1024),
+                         smem_desc_sw128(kb + 16384 + bo, 16, 1024), idesc_s, kk > 0);
+              }
+              mma_commit(&sh.sdp_full[m]);
+            }
+            ++next_sdp;
+            issued_any = true;
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          t0 = clock64();
+        } else if (*abort) {
+          ok = false;
+        } else if (clock64() - t0 > 2000000000LL) {
+          latch_status(HGA_ERR_TIMEOUT);
+          *abort = 1;
+          ok = false;
         }
       }
       if (issued_any) {
@@ -253,23 +274,40 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
       }
     }
   } else if (warp >= 4) {
-    const int m = (warp - 4) >> 2, wq = (warp - 4) & 3;
+    const int m = (warp - 4) >> 2, wq = warp & 3;
     const int row = wq * 32 + lane;
     const int grow = m * 128 + row, g = grow >> 6, r = grow & 63;
     const uint32_t lane_addr = uint32_t(wq * 32) << 16;
     const int hq = h * G + g;
     const int64_t rix = (int64_t(b) * n_q_heads + hq) * s_len + int64_t(j) * kQBlock + r;
-    // D = rowsum(dO * O), saved for the dK/dV kernel
+    // D = rowsum(dO * O), saved for the dK/dV kernel (all loads issued first)
     float dsum = 0.f;
-    for (int c = 0; c < kD; c += 8) {
-      float a[8], bb[8];
-      load8(d_o + rix * kD + c, a);
-      load8(o + rix * kD + c, bb);
+    {
+      uint4 a[16], bb[16];
+      const uint4* ap = reinterpret_cast<const uint4*>(d_o + rix * kD);
+      const uint4* bp = reinterpret_cast<const uint4*>(o + rix * kD);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) dsum = fmaf(a[i], bb[i], dsum);
+      for (int c = 0; c < 16; ++c) {
+        a[c] = ap[c];
+        bb[c] = bp[c];
+      }
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint32_t wa[4] = {a[c].x, a[c].y, a[c].z, a[c].w};
+        const uint32_t wb[4] = {bb[c].x, bb[c].y, bb[c].z, bb[c].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          dsum = fmaf(__uint_as_float(wa[i] << 16), __uint_as_float(wb[i] << 16), dsum);
+          dsum = fmaf(__uint_as_float(wa[i] & 0xffff0000u), __uint_as_float(wb[i] & 0xffff0000u),
+                      dsum);
+        }
+      }
     }
     dvec[rix] = dsum;
     const float lse2 = lse[rix] * 1.4426950408889634f;
+    const float2 c2 = make_float2(scale_log2, scale_log2);
+    const float2 nl = make_float2(-lse2, -lse2);
+    const float2 nd = make_float2(-dsum, -dsum);
     bool ok = true;
     uint8_t* drow = smem + L::kDS + m * 16384 + row * 128;
     for (int t = 0; t < n_tiles && ok; ++t) {
@@ -277,6 +315,7 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
       tc_fence_after();
       const bool own = t == n_tiles - 1;
       const uint32_t mask = sh.tile_mask[t];
+      const bool full = !own && mask == 0xffu;
       uint32_t packed[32];
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
@@ -284,18 +323,21 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
         tmem_ld32(tmem + lane_addr + L::colS(m) + hb * 32, sv);
         tmem_ld32(tmem + lane_addr + L::colDP(m) + hb * 32, dp);
         tmem_wait_ld();
+        if (!full) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int key = hb * 32 + i;
+            const bool valid = ((mask >> (key >> 3)) & 1u) && (!own || key <= r);
+            if (!valid) sv[i] = -INFINITY;
+          }
+        }
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          float ds2[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int key = hb * 32 + i + u;
-            const bool valid = ((mask >> (key >> 3)) & 1u) && (!own || key <= r);
-            const float p = valid ? exp2f(sv[i + u] * scale_log2 - lse2) : 0.f;
-            ds2[u] = p * (dp[i + u] - dsum);
-          }
-          __nv_bfloat162 pr = __floats2bfloat162_rn(ds2[0], ds2[1]);
-          packed[hb * 16 + i / 2] = *reinterpret_cast<uint32_t*>(&pr);
+          float2 x = __ffma2_rn(make_float2(sv[i], sv[i + 1]), c2, nl);
+          x.x = ex2_approx(x.x);
+          x.y = ex2_approx(x.y);
+          const float2 y = __fmul2_rn(x, __fadd2_rn(make_float2(dp[i], dp[i + 1]), nd));
+          packed[hb * 16 + i / 2] = pack_bf16x2(y.x, y.y);
         }
       }
       tc_fence_before();
@@ -314,14 +356,14 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
       tc_fence_after();
       __nv_bfloat16* dst = dq + rix * kD;
       for (int c = 0; c < kD; c += 32) {
-        float v[32];
-        tmem_ld32(tmem + lane_addr + L::colDQ(m) + c, v);
+        float vv[32];
+        tmem_ld32(tmem + lane_addr + L::colDQ(m) + c, vv);
         tmem_wait_ld();
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
           float f[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) f[i] = v[8 * q8 + i] * scale;
+          for (int i = 0; i < 8; ++i) f[i] = vv[8 * q8 + i] * scale;
           store8(dst + c + 8 * q8, f);
         }
       }
@@ -340,40 +382,44 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
 // ------------------------------------------------------------------------
 // dK / dV kernel
 // ------------------------------------------------------------------------
-template <int MT>
+// Work item = (attending query block jj, M tile m): 128 query rows = two heads
+// x 64 tokens.  Items run through two buffers (u = item & 1): Q_m / dO_m by
+// TMA (64-row boxes), S / dP in TMEM, P / dS in shared memory; warp group u
+// does the softmax of the items of buffer u, so one group's softmax overlaps
+// the other buffer's MMAs and loads.
 struct KvLayout {
-  static constexpr uint32_t kK = 0;                  // [2 halves][64][128 B]
+  static constexpr uint32_t kK = 0;                    // [2 halves][64][128 B]
   static constexpr uint32_t kV = 16384;
-  static constexpr uint32_t kQ = 32768;              // [MT][2][128][128 B]
-  static constexpr uint32_t kDO = kQ + MT * 32768;
-  static constexpr uint32_t kP = kDO + MT * 32768;   // [MT][128][128 B]
-  static constexpr uint32_t kDS = kP + MT * 16384;
-  static constexpr uint32_t kBytes = kDS + MT * 16384;
+  static constexpr uint32_t kQD = 32768;               // [buf][Q_m 32 KB | dO_m 32 KB]
+  static constexpr uint32_t kQDBytes = 65536;
+  static constexpr uint32_t kPD = kQD + 2 * kQDBytes;  // [buf][P 16 KB | dS 16 KB]
+  static constexpr uint32_t kPDBytes = 32768;
+  static constexpr uint32_t kBytes = kPD + 2 * kPDBytes;
   static constexpr uint32_t kDynSmem = kBytes + 1024;
-  static constexpr uint32_t kThreads = 128 + 128 * MT;
+  static constexpr uint32_t kThreads = 384;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t colS(int m) { return m * 64; }
-  static constexpr uint32_t colDP(int m) { return MT * 64 + m * 64; }
-  static constexpr uint32_t kColDV = MT * 128;
-  static constexpr uint32_t kColDK = MT * 128 + 64;
+  static constexpr uint32_t colS(int u) { return u * 128; }
+  static constexpr uint32_t colDP(int u) { return u * 128 + 64; }
+  static constexpr uint32_t kColDV = 256;
+  static constexpr uint32_t kColDK = 320;
 };
 
 struct KvShared {
   uint64_t kv_full;
-  uint64_t qd_full;
-  uint64_t qd_empty;
+  uint64_t qd_full[2];
+  uint64_t qd_empty[2];
   uint64_t sdp_full[2];
-  uint64_t pds_full;
+  uint64_t pds_full[2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
-  int n_iter;
+  int n_items;
   int masks[64];
   int js[64];
 };
 
 template <int MT>
-__global__ void __launch_bounds__(KvLayout<MT>::kThreads, 1)
+__global__ void __launch_bounds__(KvLayout::kThreads, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                             const __grid_constant__ CUtensorMap tm_do,
                             const __grid_constant__ CUtensorMap tm_k,
@@ -383,15 +429,14 @@ __global__ void __launch_bounds__(KvLayout<MT>::kThreads, 1)
                             float scale_log2, const float* __restrict__ lse,
                             const float* __restrict__ dvec, __nv_bfloat16* __restrict__ dk,
                             __nv_bfloat16* __restrict__ dv) {
-  using L = KvLayout<MT>;
+  using L = KvLayout;
   constexpr int G = 2 * MT;
   extern __shared__ uint8_t dsmem_raw[];
   __shared__ KvShared sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
-  const uint32_t sQ = smem_u32(smem + L::kQ), sDO = smem_u32(smem + L::kDO);
-  const uint32_t sP = smem_u32(smem + L::kP), sDS = smem_u32(smem + L::kDS);
+  const uint32_t sQD = smem_u32(smem + L::kQD), sPD = smem_u32(smem + L::kPD);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -402,11 +447,12 @@ __global__ void __launch_bounds__(KvLayout<MT>::kThreads, 1)
   for (int i = tid; i < 64; i += blockDim.x) sh.masks[i] = (i == kb) ? 0xff : 0;
   if (tid == 0) {
     mbar_init(&sh.kv_full, 1);
-    mbar_init(&sh.qd_full, 1);
-    mbar_init(&sh.qd_empty, 1);
-    mbar_init(&sh.sdp_full[0], 1);
-    mbar_init(&sh.sdp_full[1], 1);
-    mbar_init(&sh.pds_full, 128 * MT);
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&sh.qd_full[u], 1);
+      mbar_init(&sh.qd_empty[u], 1);
+      mbar_init(&sh.sdp_full[u], 1);
+      mbar_init(&sh.pds_full[u], 128);
+    }
     mbar_init(&sh.mma_done, 1);
     sh.abort = 0;
     fence_barrier_init();
@@ -436,15 +482,16 @@ __global__ void __launch_bounds__(KvLayout<MT>::kThreads, 1)
       if (on) sh.js[n + __popc(ball & ((1u << lane) - 1u))] = jj;
       n += __popc(ball);
     }
-    if (lane == 0) sh.n_iter = n;
+    if (lane == 0) sh.n_items = n * MT;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
-  const int n_iter = sh.n_iter;
+  const int n_items = sh.n_items;
 
   if (warp == 0) {
+    // ---------------- TMA producer ----------------
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_do);
@@ -460,60 +507,87 @@ __global__ void __launch_bounds__(KvLayout<MT>::kThreads, 1)
                       krow + gi * kGroup);
         }
       int issued = 0;
-      for (int it = 0; it < n_iter; ++it) {
-        if (it > 0 && !mbar_wait(&sh.qd_empty, (it - 1) & 1, abort)) break;
-        const int jj = sh.js[it];
-        mbar_arrive_expect_tx(&sh.qd_full, MT * 65536);
-        for (int g = 0; g < G; ++g) {
+      for (int it = 0; it < n_items; ++it) {
+        const int u = it & 1;
+        if (it >= 2 && !mbar_wait(&sh.qd_empty[u], ((it >> 1) - 1) & 1, abort)) break;
+        const int jj = sh.js[it / MT], m = it % MT;
+        mbar_arrive_expect_tx(&sh.qd_full[u], 65536);
+        uint8_t* dst = smem + L::kQD + u * L::kQDBytes;
+        for (int g = 0; g < 2; ++g) {
           const int32_t row =
-              int32_t((int64_t(b) * n_q_heads + h * G + g) * s_len + jj * kQBlock);
+              int32_t((int64_t(b) * n_q_heads + h * G + 2 * m + g) * s_len + jj * kQBlock);
           for (int hf = 0; hf < 2; ++hf) {
-            const uint32_t off = (g >> 1) * 32768 + hf * 16384 + (g & 1) * 8192;
-            tma_load_2d(smem + L::kQ + off, &tm_q, &sh.qd_full, hf * 64, row);
-            tma_load_2d(smem + L::kDO + off, &tm_do, &sh.qd_full, hf * 64, row);
+            tma_load_2d(dst + hf * 16384 + g * 8192, &tm_q, &sh.qd_full[u], hf * 64, row);
+            tma_load_2d(dst + 32768 + hf * 16384 + g * 8192, &tm_do, &sh.qd_full[u], hf * 64,
+                        row);
           }
         }
         issued = it + 1;
       }
       int never = 0;
       mbar_wait(&sh.kv_full, 0, &never);
-      if (issued > 0) mbar_wait(&sh.qd_full, (issued - 1) & 1, &never);
+      for (int it = issued - 1; it >= 0 && it >= issued - 2; --it)
+        mbar_wait(&sh.qd_full[it & 1], (it >> 1) & 1, &never);
     }
   } else if (warp == 1) {
+    // ---------------- MMA issuer (event driven) ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t idesc_t = idesc_bf16_f32(128, 64, 1, 1);
       bool ok = mbar_wait(&sh.kv_full, 0, abort);
       bool issued_any = false;
-      for (int it = 0; ok && it < n_iter; ++it) {
-        if (!(ok = mbar_wait(&sh.qd_full, it & 1, abort))) break;
-        tc_fence_after();
-        for (int m = 0; m < MT; ++m) {
+      int next_s = 0, next_t = 0;  // items with S/dP issued, with dV/dK issued
+      long long t0 = clock64();
+      while (ok && next_t < n_items) {
+        bool progressed = false;
+        if (next_t < next_s && mbar_try_wait(&sh.pds_full[next_t & 1], (next_t >> 1) & 1)) {
+          // dV^T += dO^T P and dK^T += Q^T dS over this item's 128 query rows
+          const int u = next_t & 1;
+          const uint32_t qd = sQD + u * L::kQDBytes, pd = sPD + u * L::kPDBytes;
+          tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint32_t ao = m * 32768 + (k >> 2) * 16384 + (k & 3) * 32;
-            const uint32_t bo = (k >> 2) * 8192 + (k & 3) * 32;
-            mma_bf16(tmem + L::colS(m), smem_desc_sw128(sQ + ao, 16, 1024),
-                     smem_desc_sw128(sK + bo, 16, 1024), idesc_s, k > 0);
-            mma_bf16(tmem + L::colDP(m), smem_desc_sw128(sDO + ao, 16, 1024),
-                     smem_desc_sw128(sV + bo, 16, 1024), idesc_s, k > 0);
+          for (int s8 = 0; s8 < 8; ++s8) {
+            const uint32_t ro = s8 * 2048;
+            const uint32_t acc = (next_t > 0 || s8 > 0) ? 1u : 0u;
+            mma_bf16(tmem + L::kColDV, smem_desc_sw128(qd + 32768 + ro, 16384, 1024),
+                     smem_desc_sw128(pd + ro, 8192, 1024), idesc_t, acc);
+            mma_bf16(tmem + L::kColDK, smem_desc_sw128(qd + ro, 16384, 1024),
+                     smem_desc_sw128(pd + 16384 + ro, 8192, 1024), idesc_t, acc);
           }
-          mma_commit(&sh.sdp_full[m]);
+          mma_commit(&sh.qd_empty[u]);
+          ++next_t;
+          progressed = true;
         }
-        issued_any = true;
-        if (!(ok = mbar_wait(&sh.pds_full, it & 1, abort))) break;
-        tc_fence_after();
-        // dV^T += dO^T P and dK^T += Q^T dS: K runs over the MT*128 query rows
-        for (int s = 0; s < MT * 8; ++s) {
-          const int m = s >> 3;
-          const uint32_t ro = (s & 7) * 2048;
-          const uint32_t acc = (it > 0 || s > 0) ? 1u : 0u;
-          mma_bf16(tmem + L::kColDV, smem_desc_sw128(sDO + m * 32768 + ro, 16384, 1024),
-                   smem_desc_sw128(sP + m * 16384 + ro, 8192, 1024), idesc_t, acc);
-          mma_bf16(tmem + L::kColDK, smem_desc_sw128(sQ + m * 32768 + ro, 16384, 1024),
-                   smem_desc_sw128(sDS + m * 16384 + ro, 8192, 1024), idesc_t, acc);
+        // S/dP(i) into buffer i & 1, free once dV/dK(i-2) has been issued
+        // (its softmax has then finished with that buffer)
+        if (!progressed && next_s < n_items && next_s < next_t + 2 &&
+            mbar_try_wait(&sh.qd_full[next_s & 1], (next_s >> 1) & 1)) {
+          const int u = next_s & 1;
+          const uint32_t qd = sQD + u * L::kQDBytes;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t ao = (kk >> 2) * 16384 + (kk & 3) * 32;
+            const uint32_t bo = (kk >> 2) * 8192 + (kk & 3) * 32;
+            mma_bf16(tmem + L::colS(u), smem_desc_sw128(qd + ao, 16, 1024),
+                     smem_desc_sw128(sK + bo, 16, 1024), idesc_s, kk > 0);
+            mma_bf16(tmem + L::colDP(u), smem_desc_sw128(qd + 32768 + ao, 16, 1024),
+                     smem_desc_sw128(sV + bo, 16, 1024), idesc_s, kk > 0);
+          }
+          mma_commit(&sh.sdp_full[u]);
+          ++next_s;
+          issued_any = true;
+          progressed = true;
         }
-        mma_commit(&sh.qd_empty);
+        if (progressed) {
+          t0 = clock64();
+        } else if (*abort) {
+          ok = false;
+        } else if (clock64() - t0 > 2000000000LL) {
+          latch_status(HGA_ERR_TIMEOUT);
+          *abort = 1;
+          ok = false;
+        }
       }
       if (issued_any) {
         int never = 0;
@@ -522,48 +596,50 @@ __global__ void __launch_bounds__(KvLayout<MT>::kThreads, 1)
       }
     }
   } else if (warp >= 4) {
-    const int m = (warp - 4) >> 2, wq = (warp - 4) & 3;
+    // ---------------- softmax (two warp groups, one per buffer) ----------------
+    const int u = (warp - 4) >> 2, wq = warp & 3;
     const int row = wq * 32 + lane;
-    const int grow = m * 128 + row, g = grow >> 6, r = grow & 63;
+    const int g = row >> 6, r = row & 63;
     const uint32_t lane_addr = uint32_t(wq * 32) << 16;
-    const int hq = h * G + g;
+    const float2 c2 = make_float2(scale_log2, scale_log2);
     bool ok = true;
-    uint8_t* prow = smem + L::kP + m * 16384 + row * 128;
-    uint8_t* drow = smem + L::kDS + m * 16384 + row * 128;
-    for (int it = 0; it < n_iter && ok; ++it) {
-      const int jj = sh.js[it];
+    uint8_t* prow = smem + L::kPD + u * L::kPDBytes + row * 128;
+    uint8_t* drow = prow + 16384;
+    for (int it = u; it < n_items && ok; it += 2) {
+      const int jj = sh.js[it / MT], m = it % MT;
       const bool own = jj == kb;
       const uint32_t mask = sh.masks[jj];
+      const int hq = h * G + 2 * m + g;
       const int64_t rix = (int64_t(b) * n_q_heads + hq) * s_len + int64_t(jj) * kQBlock + r;
       const float lse2 = lse[rix] * 1.4426950408889634f;
       const float dsum = dvec[rix];
-      if (!(ok = mbar_wait(&sh.sdp_full[m], it & 1, abort))) break;
-      // the previous iteration's dV/dK MMAs must be done reading P and dS (this
-      // phase already completed: the producer waited for it before loading the
-      // Q/dO tiles that this iteration's S and dP were computed from)
-      if (it > 0 && !(ok = mbar_wait(&sh.qd_empty, (it - 1) & 1, abort))) break;
+      const float2 nl = make_float2(-lse2, -lse2), nd = make_float2(-dsum, -dsum);
+      if (!(ok = mbar_wait(&sh.sdp_full[u], (it >> 1) & 1, abort))) break;
       tc_fence_after();
+      const bool full = !own && mask == 0xffu;
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
         float sv[32], dp[32];
-        tmem_ld32(tmem + lane_addr + L::colS(m) + hb * 32, sv);
-        tmem_ld32(tmem + lane_addr + L::colDP(m) + hb * 32, dp);
+        tmem_ld32(tmem + lane_addr + L::colS(u) + hb * 32, sv);
+        tmem_ld32(tmem + lane_addr + L::colDP(u) + hb * 32, dp);
         tmem_wait_ld();
+        if (!full) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int key = hb * 32 + i;
+            const bool valid = ((mask >> (key >> 3)) & 1u) && (!own || key <= r);
+            if (!valid) sv[i] = -INFINITY;
+          }
+        }
         uint32_t pk[16], dk2[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          float p2[2], d2[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int key = hb * 32 + i + u;
-            const bool valid = ((mask >> (key >> 3)) & 1u) && (!own || key <= r);
-            p2[u] = valid ? exp2f(sv[i + u] * scale_log2 - lse2) : 0.f;
-            d2[u] = p2[u] * (dp[i + u] - dsum);
-          }
-          __nv_bfloat162 pp = __floats2bfloat162_rn(p2[0], p2[1]);
-          __nv_bfloat162 dd = __floats2bfloat162_rn(d2[0], d2[1]);
-          pk[i / 2] = *reinterpret_cast<uint32_t*>(&pp);
-          dk2[i / 2] = *reinterpret_cast<uint32_t*>(&dd);
+          float2 p = __ffma2_rn(make_float2(sv[i], sv[i + 1]), c2, nl);
+          p.x = ex2_approx(p.x);
+          p.y = ex2_approx(p.y);
+          const float2 d2 = __fmul2_rn(p, __fadd2_rn(make_float2(dp[i], dp[i + 1]), nd));
+          pk[i / 2] = pack_bf16x2(p.x, p.y);
+          dk2[i / 2] = pack_bf16x2(d2.x, d2.y);
         }
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
@@ -577,11 +653,14 @@ __global__ void __launch_bounds__(KvLayout<MT>::kThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&sh.pds_full);
+      mbar_arrive(&sh.pds_full[u]);
     }
     // epilogue: warp group 0 owns TMEM lanes 0..127 = the 128 head dims
-    if (m == 0) {
-      if (ok && n_iter > 0) ok = mbar_wait(&sh.qd_empty, (n_iter - 1) & 1, abort);
+    if (u == 0) {
+      // mma_done completes exactly once, after the last dV/dK MMA; a parity
+      // wait on a per-buffer barrier here could pass a phase early, because
+      // the earlier phase of that barrier need not have completed yet
+      if (ok) ok = mbar_wait(&sh.mma_done, 0, abort);
       if (ok) {
         tc_fence_after();
         const int dcol = row;
@@ -594,8 +673,8 @@ __global__ void __launch_bounds__(KvLayout<MT>::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int64_t at = base + int64_t(c + i) * kD + dcol;
-            dv[at] = __float2bfloat16_rn(n_iter > 0 ? vv[i] : 0.f);
-            dk[at] = __float2bfloat16_rn(n_iter > 0 ? kk[i] * scale : 0.f);
+            dv[at] = __float2bfloat16_rn(n_items > 0 ? vv[i] : 0.f);
+            dk[at] = __float2bfloat16_rn(n_items > 0 ? kk[i] * scale : 0.f);
           }
         }
       }

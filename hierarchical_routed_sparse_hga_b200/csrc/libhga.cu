@@ -157,7 +157,7 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
                            const void* d_o, void* dq, void* dk, void* dv, float* dvec,
                            cudaStream_t s) {
   using LQ = bwdtc::DqLayout<MT>;
-  using LK = bwdtc::KvLayout<MT>;
+  using LK = bwdtc::KvLayout;
   CUtensorMap tq, tdo, tk, tv;
   const uint64_t q_rows = uint64_t(cfg->batch) * cfg->n_q_heads * s_len;
   const uint64_t kv_rows = uint64_t(cfg->batch) * cfg->n_kv_heads * ctx_cap;
@@ -174,7 +174,8 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
   const float scale_log2 = cfg->scale * 1.4426950408889634f;
   e = traced_launch(HGA_K_BWD_DQ_TC, s, [&] {
     bwdtc::attn_bwd_dq_tc_kernel<MT><<<grid, LQ::kThreads, LQ::kDynSmem, s>>>(
-        tq, tdo, tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads,
+        tq, tdo, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+        ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads,
         cfg->topk_groups, sel_grp, cfg->scale, scale_log2, static_cast<const __nv_bfloat16*>(o),
         static_cast<const __nv_bfloat16*>(d_o), lse, static_cast<__nv_bfloat16*>(dq), dvec);
   });

@@ -23,7 +23,7 @@
 namespace hga {
 
 constexpr int kRouteThreads = 256;
-constexpr int kScoreChunk = 64;  // candidate blocks per block_score CTA
+constexpr int kScoreChunk = 16;  // candidate blocks per block_score CTA
 
 struct RouteWs {
   float* qbar;     // [B, Hkv, n_qb, D]
@@ -45,12 +45,24 @@ __global__ void __launch_bounds__(kRouteThreads)
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  for (int r = rs; r < rows; r += RS) {
-    const int hq = h * G + r / kQBlock, t = j * kQBlock + r % kQBlock;
-    float f[8];
-    load8(q + ((int64_t(b) * n_q_heads + hq) * s_len + t) * D + ch * 8, f);
+  // 8 rows per pass with all loads issued before the adds (8 x 16 B in flight)
+  for (int r0 = rs; r0 < rows; r0 += 8 * RS) {
+    float f[8][8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += f[e];
+    for (int u = 0; u < 8; ++u) {
+      const int r = r0 + u * RS;
+      if (r < rows) {
+        const int hq = h * G + r / kQBlock, t = j * kQBlock + r % kQBlock;
+        load8(q + ((int64_t(b) * n_q_heads + hq) * s_len + t) * D + ch * 8, f[u]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[u][e] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += f[u][e];
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) part[rs][ch * 8 + e] = acc[e];
@@ -63,7 +75,7 @@ __global__ void __launch_bounds__(kRouteThreads)
   }
 }
 
-// grid (ceil(j_max / 64), Hkv, B); dynamic smem: (n_qb*D + D*65) floats
+// grid (ceil(j_max / 16), Hkv, B); dynamic smem: (n_qb*D + D*17) floats
 template <int D>
 __global__ void __launch_bounds__(kRouteThreads)
     block_score_kernel(const float* __restrict__ qbar, const float* __restrict__ bsum,
@@ -71,7 +83,7 @@ __global__ void __launch_bounds__(kRouteThreads)
                        float* __restrict__ scores, int64_t jstride) {
   extern __shared__ float smem[];
   float* qb = smem;                // [n_qb][D]
-  float* bsT = smem + n_qb * D;    // [D][65] transposed chunk (padded: no bank conflicts)
+  float* bsT = smem + n_qb * D;    // [D][17] transposed chunk (padded: no bank conflicts)
   const int h = blockIdx.y, b = blockIdx.z;
   const int64_t head = int64_t(b) * n_kv_heads + h;
   const int64_t c0 = int64_t(blockIdx.x) * kScoreChunk;
@@ -86,7 +98,7 @@ __global__ void __launch_bounds__(kRouteThreads)
   }
   __syncthreads();
   const int cl = threadIdx.x % kScoreChunk;
-  const int jg = threadIdx.x / kScoreChunk;  // 4 query-block lanes
+  const int jg = threadIdx.x / kScoreChunk;  // query-block lane
   constexpr int JG = kRouteThreads / kScoreChunk;
   const int64_t c = c0 + cl;
   for (int j0 = jg; j0 < n_qb; j0 += 4 * JG) {
@@ -177,33 +189,45 @@ __global__ void __launch_bounds__(kRouteThreads)
   constexpr int V4 = D / 4;  // float4 per summary row
   const float4* qb4 = reinterpret_cast<const float4*>(qb);
   const float* gbase = gsum + head * (ctx_cap / kGroup) * D;
-  for (int p0 = warp * 4; p0 < n2; p0 += NW * 4) {
-    float part[4] = {0.f, 0.f, 0.f, 0.f};
+  // 16 candidate rows per warp pass, all loads issued before any use
+  constexpr int kU = 16;
+  constexpr int kE = (V4 + 31) / 32;  // float4 per lane per row
+  for (int p0 = warp * kU; p0 < n2; p0 += NW * kU) {
+    float4 x[kU][kE];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kU; ++u) {
       const int p = p0 + u;
-      if (p < n2) {
-        const int64_t g = int64_t(blocks[p >> 3]) * kGroupsPerBlock + (p & 7);
-        const float4* row = reinterpret_cast<const float4*>(gbase + g * D);
-        for (int e = lane; e < V4; e += 32) {
-          const float4 x = row[e], y = qb4[e];
-          part[u] = fmaf(x.x, y.x, part[u]);
-          part[u] = fmaf(x.y, y.y, part[u]);
-          part[u] = fmaf(x.z, y.z, part[u]);
-          part[u] = fmaf(x.w, y.w, part[u]);
-        }
+      const int64_t g = p < n2 ? int64_t(blocks[p >> 3]) * kGroupsPerBlock + (p & 7) : 0;
+      const float4* row = reinterpret_cast<const float4*>(gbase + g * D);
+#pragma unroll
+      for (int i = 0; i < kE; ++i) {
+        const int e = lane + 32 * i;
+        x[u][i] = (p < n2 && e < V4) ? row[e] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
+    float part[kU];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kU; ++u) {
+      part[u] = 0.f;
+#pragma unroll
+      for (int i = 0; i < kE; ++i) {
+        const int e = lane + 32 * i;
+        if (e < V4) {
+          const float4 y = qb4[e];
+          part[u] = fmaf(x[u][i].x, y.x, part[u]);
+          part[u] = fmaf(x[u][i].y, y.y, part[u]);
+          part[u] = fmaf(x[u][i].z, y.z, part[u]);
+          part[u] = fmaf(x[u][i].w, y.w, part[u]);
+        }
+      }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) part[u] += __shfl_xor_sync(0xffffffffu, part[u], o);
     }
-    if (lane < 4 && p0 + lane < n2) {
+    if (lane < kU && p0 + lane < n2) {
       float v = part[0];
-      if (lane == 1) v = part[1];
-      if (lane == 2) v = part[2];
-      if (lane == 3) v = part[3];
+#pragma unroll
+      for (int u = 1; u < kU; ++u)
+        if (lane == u) v = part[u];
       key2[p0 + lane] = ordered_key(v);
     }
   }
