@@ -121,15 +121,32 @@ __device__ int block_enumerate(int n, Pred pred, Fn f, int* scratch) {
 // ---------------------------------------------------------------------------
 // block-wide top-k of n distinct-or-not uint32 keys held in shared memory:
 // sets sel[i] = 1 for the k largest keys, ties broken toward the lower index.
-// Radix select on 8-bit digits (MSB first) finds the k-th largest key T; keys
-// above T are taken, and among keys equal to T the lowest indices fill the
-// remaining slots.  Needs hist[256] and scratch (see block_enumerate).
+// Up to 512 keys: rank counting (below).  Otherwise a radix select on 8-bit
+// digits (MSB first) finds the k-th largest key T; keys above T are taken,
+// and among keys equal to T the lowest indices fill the remaining slots.
+// Needs hist[256] and scratch (see block_enumerate).
 // ---------------------------------------------------------------------------
 __device__ void block_topk(const uint32_t* key, int n, int k, uint8_t* sel, int* hist,
                            int* scratch) {
   const int nt = blockDim.x, tid = threadIdx.x;
   if (k >= n) {
     for (int i = tid; i < n; i += nt) sel[i] = 1;
+    __syncthreads();
+    return;
+  }
+  if (n <= 512) {
+    // rank by counting: rank(i) = #{keys above key[i]} + #{equal keys before i};
+    // the k smallest ranks are the k largest keys, ties to the lower index.
+    // O(n^2) comparisons with broadcast shared-memory reads, no barrier.
+    for (int i = tid; i < n; i += nt) {
+      const uint32_t ki = key[i];
+      int rank = 0;
+      for (int jdx = 0; jdx < n; ++jdx) {
+        const uint32_t kj = key[jdx];
+        rank += (kj > ki) || (kj == ki && jdx < i);
+      }
+      sel[i] = rank < k ? 1 : 0;
+    }
     __syncthreads();
     return;
   }

@@ -200,7 +200,8 @@ RouteCarve route_carve(const hga_config_t* c, int32_t s_len, int64_t q_begin, vo
   const int64_t heads = int64_t(c->batch) * c->n_kv_heads;
   RouteCarve r;
   r.jstride = ((q_begin / kBlock + n_qb) + 3) & ~int64_t(3);
-  const size_t qbar_bytes = align256(size_t(heads * n_qb * c->head_dim) * 4);
+  const int64_t G = c->n_q_heads / c->n_kv_heads;
+  const size_t qbar_bytes = align256(size_t(heads * n_qb * G * c->head_dim) * 4);
   const size_t score_bytes = align256(size_t(heads * n_qb * r.jstride) * 4);
   r.qbar = static_cast<float*>(base);
   r.scores = base ? reinterpret_cast<float*>(static_cast<char*>(base) + qbar_bytes) : nullptr;
@@ -324,31 +325,32 @@ hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, 
   const int64_t own0 = q_begin / kBlock;
   const int64_t j_max = own0 + n_qb - 1;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int G = cfg->n_q_heads / cfg->n_kv_heads;
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
-    dim3 g1(n_qb, cfg->n_kv_heads, cfg->batch);
+    dim3 g0(n_qb * G, cfg->n_kv_heads, cfg->batch);
     hga_status_t e = traced_launch(HGA_K_QMEAN, s, [&] {
-      qmean_kernel<T, D><<<g1, kRouteThreads, 0, s>>>(static_cast<const T*>(q), cfg->n_q_heads,
+      qmean_kernel<T, D><<<g0, kQmeanThreads, 0, s>>>(static_cast<const T*>(q), cfg->n_q_heads,
                                                       cfg->n_kv_heads, s_len, ws.qbar);
     });
     if (e != HGA_OK) return e;
     if (j_max > 0) {
-      const size_t sm2 = size_t(n_qb * D + D * (kScoreChunk + 1)) * 4;
-      e = ensure_smem(reinterpret_cast<const void*>(&block_score_kernel<D>), sm2);
-      if (e != HGA_OK) return e;
-      dim3 g2(unsigned((j_max + kScoreChunk - 1) / kScoreChunk), cfg->n_kv_heads, cfg->batch);
+      const int n_cc = int((j_max + kScoreCands - 1) / kScoreCands);
+      const int n_jc = (n_qb + kScoreQbs - 1) / kScoreQbs;
+      dim3 g2(unsigned(n_cc * n_jc), cfg->n_kv_heads, cfg->batch);
       e = traced_launch(HGA_K_BLOCK_SCORE, s, [&] {
-        block_score_kernel<D><<<g2, kRouteThreads, sm2, s>>>(ws.qbar, bsum, ctx_cap,
-                                                             cfg->n_kv_heads, n_qb, own0,
-                                                             ws.scores, ws.jstride);
+        block_score_kernel<D><<<g2, kRouteThreads, 0, s>>>(ws.qbar, bsum, ctx_cap,
+                                                           cfg->n_kv_heads, G, n_qb, own0,
+                                                           ws.scores, ws.jstride);
       });
       if (e != HGA_OK) return e;
     }
+    dim3 g1(n_qb, cfg->n_kv_heads, cfg->batch);
     const size_t sm3 = select_layout(own0 + n_qb, cfg->topk_blocks, D).total;
     e = ensure_smem(reinterpret_cast<const void*>(&select_kernel<D>), sm3);
     if (e != HGA_OK) return e;
     return traced_launch(HGA_K_SELECT, s, [&] {
       select_kernel<D><<<g1, kRouteThreads, sm3, s>>>(ws.qbar, ws.scores, gsum, ctx_cap,
-                                                      cfg->n_kv_heads, n_qb, own0, ws.jstride,
+                                                      cfg->n_kv_heads, G, n_qb, own0, ws.jstride,
                                                       cfg->topk_blocks, cfg->topk_groups,
                                                       sel_blk, sel_grp);
     });

@@ -4,12 +4,11 @@
 // scores the existing projected keys).
 //
 // Three launches, all HBM/L2-bound:
-//   qmean_kernel        qbar[b,h,j] = mean of the 64 x G query rows of query
-//                       block j (reads Q once, coalesced 16-byte loads);
-//   block_score_kernel  S[b,h,j,c] = qbar[b,h,j] . bsum[b,h,c] for a 64-block
-//                       chunk of candidates and every query block of the
-//                       segment -- one read of each block summary per KV head
-//                       instead of one per query block;
+//   qmean_kernel        per (query block j, query head): that head's share of
+//                       qbar[b,h,j], the mean of the 64 x G query rows (reads Q
+//                       once, 1024 CTAs for Qwen3 shapes, one load round);
+//   block_score_kernel  S[b,h,j,c] = qbar[b,h,j] . bsum[b,h,c] on tiles of 32
+//                       candidate blocks x 8 query blocks;
 //   select_kernel       per (b,h,j): radix top-k over the J candidate scores,
 //                       gather the selected blocks' 8*kb group summaries,
 //                       score them, radix top-k again, write both selections in
@@ -25,99 +24,114 @@ namespace hga {
 constexpr int kRouteThreads = 256;
 constexpr int kScoreChunk = 16;  // candidate blocks per block_score CTA
 
-struct RouteWs {
-  float* qbar;     // [B, Hkv, n_qb, D]
-  float* scores;   // [B, Hkv, n_qb, jstride]
-  int64_t jstride;
-};
+// grid (n_qb * G, Hkv, B), 128 threads: the 64 rows of one query head of one
+// query block (16 KB), all loads issued in one round; writes that head's
+// share of the mean, qpart[b, h, j, g, :] = sum of its rows / (64 G).  The
+// consumers add the G shares in a fixed order (deterministic).
+constexpr int kQmeanThreads = 128;
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kRouteThreads)
+__global__ void __launch_bounds__(kQmeanThreads)
     qmean_kernel(const T* __restrict__ q, int n_q_heads, int n_kv_heads, int s_len,
-                 float* __restrict__ qbar) {
-  constexpr int CH = D / 8;
-  constexpr int RS = kRouteThreads / CH;  // row slots
+                 float* __restrict__ qpart) {
+  constexpr int CH = D / 8;                    // 16-byte chunks per row
+  constexpr int RS = kQmeanThreads / CH;       // row slots
+  constexpr int PASSES = kQBlock / RS;
   __shared__ float part[RS][D];
-  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int G = n_q_heads / n_kv_heads;
-  const int rows = G * kQBlock;
+  const int j = blockIdx.x / G, g = blockIdx.x % G, h = blockIdx.y, b = blockIdx.z;
+  const int hq = h * G + g;
   const int ch = threadIdx.x % CH, rs = threadIdx.x / CH;
+  const T* src = q + ((int64_t(b) * n_q_heads + hq) * s_len + int64_t(j) * kQBlock) * D + ch * 8;
+  float f[PASSES][8];
+#pragma unroll
+  for (int u = 0; u < PASSES; ++u) load8(src + int64_t(rs + u * RS) * D, f[u]);
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  // 8 rows per pass with all loads issued before the adds (8 x 16 B in flight)
-  for (int r0 = rs; r0 < rows; r0 += 8 * RS) {
-    float f[8][8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int r = r0 + u * RS;
-      if (r < rows) {
-        const int hq = h * G + r / kQBlock, t = j * kQBlock + r % kQBlock;
-        load8(q + ((int64_t(b) * n_q_heads + hq) * s_len + t) * D + ch * 8, f[u]);
-      } else {
+  for (int u = 0; u < PASSES; ++u)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) f[u][e] = 0.f;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += f[u][e];
-  }
+    for (int e = 0; e < 8; ++e) acc[e] += f[u][e];
 #pragma unroll
   for (int e = 0; e < 8; ++e) part[rs][ch * 8 + e] = acc[e];
   __syncthreads();
   const int n_qb = s_len / kQBlock;
-  for (int e = threadIdx.x; e < D; e += kRouteThreads) {
-    float s = 0.f;
-    for (int r = 0; r < RS; ++r) s += part[r][e];
-    qbar[((int64_t(b) * n_kv_heads + h) * n_qb + j) * D + e] = s / float(rows);
+  const float inv = 1.f / float(G * kQBlock);
+  for (int e = threadIdx.x; e < D; e += kQmeanThreads) {
+    float sum = 0.f;
+#pragma unroll
+    for (int r = 0; r < RS; ++r) sum += part[r][e];
+    qpart[(((int64_t(b) * n_kv_heads + h) * n_qb + j) * G + g) * D + e] = sum * inv;
   }
 }
 
-// grid (ceil(j_max / 16), Hkv, B); dynamic smem: (n_qb*D + D*17) floats
+// qbar of (b, h, j) = sum over the G shares (G <= 8), added in order
+// g = 0 .. G-1; all G loads are issued before the adds
+__device__ __forceinline__ float qbar_elem(const float* qpart_bhj, int G, int D, int e) {
+  float x[8];
+#pragma unroll
+  for (int g = 0; g < 8; ++g) x[g] = g < G ? qpart_bhj[g * D + e] : 0.f;
+  float v = x[0];
+#pragma unroll
+  for (int g = 1; g < 8; ++g)
+    if (g < G) v += x[g];
+  return v;
+}
+
+// grid (ceil(j_max / 32) * ceil(n_qb / 8), Hkv, B), 256 threads: a tile of
+// 32 candidate blocks x 8 query blocks, one score per thread, operands
+// staged in shared memory (candidates transposed and padded: conflict-free).
+constexpr int kScoreCands = 32;
+constexpr int kScoreQbs = 8;
+
 template <int D>
 __global__ void __launch_bounds__(kRouteThreads)
-    block_score_kernel(const float* __restrict__ qbar, const float* __restrict__ bsum,
-                       int64_t ctx_cap, int n_kv_heads, int n_qb, int64_t own0,
+    block_score_kernel(const float* __restrict__ qpart, const float* __restrict__ bsum,
+                       int64_t ctx_cap, int n_kv_heads, int G, int n_qb, int64_t own0,
                        float* __restrict__ scores, int64_t jstride) {
-  extern __shared__ float smem[];
-  float* qb = smem;                // [n_qb][D]
-  float* bsT = smem + n_qb * D;    // [D][17] transposed chunk (padded: no bank conflicts)
+  __shared__ float qb[kScoreQbs][D];
+  __shared__ float bsT[D][kScoreCands + 1];
   const int h = blockIdx.y, b = blockIdx.z;
+  const int n_jc = (n_qb + kScoreQbs - 1) / kScoreQbs;
+  const int cc = blockIdx.x / n_jc, jc = blockIdx.x % n_jc;
   const int64_t head = int64_t(b) * n_kv_heads + h;
-  const int64_t c0 = int64_t(blockIdx.x) * kScoreChunk;
-  const int64_t j_max = own0 + n_qb - 1;  // candidates of the last query block
-  const float* qsrc = qbar + head * n_qb * D;
-  for (int i = threadIdx.x; i < n_qb * D; i += kRouteThreads) qb[i] = qsrc[i];
+  const int64_t c0 = int64_t(cc) * kScoreCands;
+  const int j0 = jc * kScoreQbs;
+  const int64_t j_max = own0 + n_qb - 1;
+  constexpr int kQ = kScoreQbs * D / kRouteThreads;     // elements per thread
+  constexpr int kB = kScoreCands * D / kRouteThreads;
   const float* bsrc = bsum + head * (ctx_cap / kBlock) * D;
-  for (int i = threadIdx.x; i < kScoreChunk * D; i += kRouteThreads) {
-    const int cl = i / D, e = i % D;
+  float qv[kQ], bv[kB];
+#pragma unroll
+  for (int u = 0; u < kQ; ++u) {
+    const int i = threadIdx.x + u * kRouteThreads, jl = i / D, e = i % D, j = j0 + jl;
+    qv[u] = j < n_qb ? qbar_elem(qpart + ((head * n_qb + j) * G) * D, G, D, e) : 0.f;
+  }
+#pragma unroll
+  for (int u = 0; u < kB; ++u) {
+    const int i = threadIdx.x + u * kRouteThreads, cl = i / D, e = i % D;
     const int64_t c = c0 + cl;
-    bsT[e * (kScoreChunk + 1) + cl] = c < j_max ? bsrc[c * D + e] : 0.f;
+    bv[u] = c < j_max ? bsrc[c * D + e] : 0.f;
+  }
+#pragma unroll
+  for (int u = 0; u < kQ; ++u) {
+    const int i = threadIdx.x + u * kRouteThreads;
+    qb[i / D][i % D] = qv[u];
+  }
+#pragma unroll
+  for (int u = 0; u < kB; ++u) {
+    const int i = threadIdx.x + u * kRouteThreads;
+    bsT[i % D][i / D] = bv[u];
   }
   __syncthreads();
-  const int cl = threadIdx.x % kScoreChunk;
-  const int jg = threadIdx.x / kScoreChunk;  // query-block lane
-  constexpr int JG = kRouteThreads / kScoreChunk;
+  const int cl = threadIdx.x % kScoreCands, jl = threadIdx.x / kScoreCands;
   const int64_t c = c0 + cl;
-  for (int j0 = jg; j0 < n_qb; j0 += 4 * JG) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-    for (int e = 0; e < D; ++e) {
-      const float bv = bsT[e * (kScoreChunk + 1) + cl];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = j0 + u * JG;
-        if (j < n_qb) acc[u] = fmaf(qb[j * D + e], bv, acc[u]);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int j = j0 + u * JG;
-      if (j < n_qb && c < own0 + j) scores[(head * n_qb + j) * jstride + c] = acc[u];
-    }
-  }
+  const int j = j0 + jl;
+  float acc = 0.f;
+#pragma unroll 16
+  for (int e = 0; e < D; ++e) acc = fmaf(qb[jl][e], bsT[e][cl], acc);
+  if (j < n_qb && c < own0 + j) scores[(head * n_qb + j) * jstride + c] = acc;
 }
 
 // Shared-memory layout of select_kernel (16-byte aligned sections).
@@ -145,8 +159,8 @@ __host__ __device__ inline SelectLayout select_layout(int64_t j_cap, int topk_bl
 // grid (n_qb, Hkv, B); dynamic smem select_layout(...).total
 template <int D>
 __global__ void __launch_bounds__(kRouteThreads)
-    select_kernel(const float* __restrict__ qbar, const float* __restrict__ scores,
-                  const float* __restrict__ gsum, int64_t ctx_cap, int n_kv_heads, int n_qb,
+    select_kernel(const float* __restrict__ qpart, const float* __restrict__ scores,
+                  const float* __restrict__ gsum, int64_t ctx_cap, int n_kv_heads, int G, int n_qb,
                   int64_t own0, int64_t jstride, int topk_blocks, int topk_groups,
                   int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp) {
   extern __shared__ __align__(16) unsigned char sm_raw[];
@@ -169,7 +183,8 @@ __global__ void __launch_bounds__(kRouteThreads)
 
   const float* srow = scores + (head * n_qb + j) * jstride;
   for (int64_t i = threadIdx.x; i < J; i += kRouteThreads) key1[i] = ordered_key(srow[i]);
-  for (int i = threadIdx.x; i < D; i += kRouteThreads) qb[i] = qbar[(head * n_qb + j) * D + i];
+  for (int i = threadIdx.x; i < D; i += kRouteThreads)
+    qb[i] = qbar_elem(qpart + ((head * n_qb + j) * G) * D, G, D, i);
   __syncthreads();
 
   // level 1

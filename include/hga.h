@@ -184,8 +184,8 @@ HGA_API hga_status_t hga_attn_fwd(const hga_config_t* cfg, const void* q, const 
  * The array is HGA_NOALLOC_SCRATCH_BYTES (4 MiB) of device memory that every
  * GPU which loads the library holds until the process exits.  A call whose
  * hga_route_workspace_size() exceeds it returns HGA_ERR_WORKSPACE and
- * launches nothing (for the Qwen3-8B shape -- 8 KV heads, d = 128, 2048-token
- * segments, batch 1 -- contexts up to 253,952 tokens fit).
+ * launches nothing (for the Qwen3-8B shape -- 32 query / 8 KV heads, d = 128,
+ * 2048-token segments, batch 1 -- contexts up to 229,376 tokens fit).
  *
  * The first call on each device looks up the array's device address (with
  * that device current) and caches it; make that first call before any stream

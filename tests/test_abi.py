@@ -84,8 +84,10 @@ def test_host_argument_checks():
 
 def test_workspace_sizes():
     c = cfg()
-    # qbar 8 heads x 32 blocks x 128 floats + scores 8 x 32 x 256 floats (256-B aligned)
-    assert hga.hga_route_workspace_size(c, 2048, 14336) == 8 * 32 * 128 * 4 + 8 * 32 * 256 * 4
+    # per-head shares of qbar: 8 KV heads x 32 blocks x 4 query heads x 128 floats,
+    # + block scores 8 x 32 x 256 floats (each part 256-B aligned)
+    assert hga.hga_route_workspace_size(c, 2048, 14336) == (8 * 32 * 4 * 128 * 4
+                                                           + 8 * 32 * 256 * 4)
     assert hga.hga_attn_bwd_workspace_size(c, 2048) == 32 * 2048 * 4
     assert hga.hga_route_workspace_size(cfg(head_dim=100), 2048, 0) == 0
 

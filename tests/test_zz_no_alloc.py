@@ -65,5 +65,5 @@ def test_route_noalloc_rejects_work_beyond_its_scratch():
     cfg = Config(1, 32, 8, 128, 16, 64)
     fake = 0x10000  # never dereferenced: the size check fails before any launch
     with pytest.raises(HgaError) as e:
-        hga_route_noalloc(cfg, fake, 253952, 2048, 256000, fake, fake, None, fake, 0)
+        hga_route_noalloc(cfg, fake, 227392, 2048, 229440, fake, fake, None, fake, 0)
     assert e.value.status == HGA_ERR_WORKSPACE
