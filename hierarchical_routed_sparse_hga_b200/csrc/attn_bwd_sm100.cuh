@@ -280,29 +280,51 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     const uint32_t lane_addr = uint32_t(wq * 32) << 16;
     const int hq = h * G + g;
     const int64_t rix = (int64_t(b) * n_q_heads + hq) * s_len + int64_t(j) * kQBlock + r;
-    // D = rowsum(dO * O), saved for the dK/dV kernel (all loads issued first)
-    float dsum = 0.f;
+    // D = rowsum(dO * O), saved for the dK/dV kernel.  Computed cooperatively:
+    // a warp takes two rows per step (16 lanes x 16 B each), O read with
+    // coalesced 256-byte row loads, dO from the shared-memory tile.
     {
-      uint4 a[16], bb[16];
-      const uint4* ap = reinterpret_cast<const uint4*>(d_o + rix * kD);
-      const uint4* bp = reinterpret_cast<const uint4*>(o + rix * kD);
+      if (!mbar_wait(&sh.q_full, 0, abort)) {
+      } else {
+        const int half = lane >> 4, c = lane & 15;   // row of the pair, 16-byte chunk
+        const uint8_t* dO_m = smem + L::kDO + m * 32768;
+        // scratch: the first bytes of this warp's own dS rows, which only
+        // this warp writes, and only after it has read its D values
+        float* dsh = reinterpret_cast<float*>(smem + L::kDS + m * 16384 + wq * 32 * 128);
+        // all 16 row-pair loads of O issued before any use
+        uint4 ov[16];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        a[c] = ap[c];
-        bb[c] = bp[c];
-      }
+        for (int p2 = 0; p2 < 16; ++p2) {
+          const int rw = wq * 32 + 2 * p2 + half;    // row in the M tile
+          const int gw = (m * 128 + rw) >> 6, tw = (m * 128 + rw) & 63;
+          const int64_t orow =
+              (int64_t(b) * n_q_heads + h * G + gw) * s_len + int64_t(j) * kQBlock + tw;
+          ov[p2] = *reinterpret_cast<const uint4*>(o + orow * kD + c * 8);
+        }
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const uint32_t wa[4] = {a[c].x, a[c].y, a[c].z, a[c].w};
-        const uint32_t wb[4] = {bb[c].x, bb[c].y, bb[c].z, bb[c].w};
+        for (int p2 = 0; p2 < 16; ++p2) {
+          const int rw = wq * 32 + 2 * p2 + half;
+          float df[8];
+          load8(reinterpret_cast<const __nv_bfloat16*>(
+                    dO_m + (c >> 3) * 16384 + rw * 128 + (((c & 7) ^ (rw & 7)) << 4)),
+                df);
+          const uint32_t w4[4] = {ov[p2].x, ov[p2].y, ov[p2].z, ov[p2].w};
+          float part = 0.f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          dsum = fmaf(__uint_as_float(wa[i] << 16), __uint_as_float(wb[i] << 16), dsum);
-          dsum = fmaf(__uint_as_float(wa[i] & 0xffff0000u), __uint_as_float(wb[i] & 0xffff0000u),
-                      dsum);
+          for (int i = 0; i < 4; ++i) {
+            part = fmaf(__uint_as_float(w4[i] << 16), df[2 * i], part);
+            part = fmaf(__uint_as_float(w4[i] & 0xffff0000u), df[2 * i + 1], part);
+          }
+#pragma unroll
+          for (int off = 8; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+          if (c == 0) dsh[2 * p2 + half] = part;
         }
       }
+      __syncwarp();
     }
+    const float dsum = reinterpret_cast<const float*>(smem + L::kDS + m * 16384 +
+                                                      wq * 32 * 128)[lane];
+    __syncwarp();
     dvec[rix] = dsum;
     const float lse2 = lse[rix] * 1.4426950408889634f;
     const float2 c2 = make_float2(scale_log2, scale_log2);

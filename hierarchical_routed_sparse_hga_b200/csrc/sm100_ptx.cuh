@@ -86,6 +86,12 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Bulk prefetch of [src, src + bytes) into L2 (no destination, no completion
+// to wait for); src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // 16-byte asynchronous global -> shared copy (L2 only), and the arrive on an
 // mbarrier once every copy this thread issued so far has landed (the barrier's
 // expected count must include one arrival per issuing thread).
