@@ -9,14 +9,12 @@
 // all of them.
 //
 // Roles (128 + 128*MT threads, one CTA per SM):
-//   warps 0,2,3 producers: Q once by TMA (64 x 64 boxes); then per key tile
-//               the 8 selected groups of K and V (a group is a contiguous
-//               2 KiB run of [B,Hkv,T,d]) by 16-byte cp.async copies, 96
-//               threads x ~21 copies, written straight into the 128-byte-
-//               swizzled operand layout of a 4-stage ring -- far faster than
-//               8-row TMA boxes, whose per-box cost capped the gather at ~16 B
-//               per cycle per SM; the gather latency of one tile hides behind
-//               three others;
+//   warp 0      TMA producer: Q once (64 x 64 boxes); then per key tile the
+//               8 selected groups of K and V, each group (a contiguous 2 KiB
+//               run of [B,Hkv,T,d]) one 3-D box of 64 columns x 8 rows x 2
+//               column halves, issued from 8 lanes, into a 4-stage ring laid
+//               out [group][d half][8 rows][128 B] (128-byte swizzle; UMMA
+//               stride 2048 B between 8-row groups);
 //   warp 1      TMEM owner and MMA issuer.  It issues, as soon as each one's
 //               inputs are ready, S = Q K^T into double-buffered TMEM and
 //               O += P V with P read straight from TMEM (A operand in tensor
@@ -45,7 +43,6 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kStages = 4;
-constexpr int kProducers = 96;  // warps 0, 2, 3
 constexpr int kMaxTiles = 33;  // 256 groups / 8 + own block
 
 template <int MT>
@@ -84,8 +81,8 @@ constexpr uint32_t kTestDropFirstTile = 0x80000000u;  // test hook, see hga.h
 template <int MT>
 __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
-                       const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
-                       int64_t ctx_cap, int64_t q_begin, int s_len, int n_q_heads, int n_kv_heads,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, int64_t ctx_cap, int64_t q_begin, int s_len, int n_q_heads, int n_kv_heads,
                        int topk_groups, const int32_t* __restrict__ sel_grp, float scale_log2,
                        __nv_bfloat16* __restrict__ o, float* __restrict__ lse, uint32_t flags) {
   using L = Layout<MT>;
@@ -109,7 +106,7 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
   if (tid == 0) {
     mbar_init(&sh.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sh.kv_full[s], kProducers);
+      mbar_init(&sh.kv_full[s], 1);
       mbar_init(&sh.kv_empty[s], 1);
     }
     for (int m = 0; m < 2; ++m)
@@ -162,11 +159,14 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
   const uint32_t tmem = sh.tmem_base;
   const int n_tiles = sh.n_tiles;
 
-  if (warp == 0 || warp == 2 || warp == 3) {
-    // ---------------- producers ----------------
-    const int ptid = warp == 0 ? lane : 32 * (warp - 1) + lane;  // 0..95
-    if (tid == 0) {
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    // K/V tile layout: group gi at gi * 2048: [d half][8 rows][128 B], one
+    // 3-D box (64 columns x 8 rows x 2 halves) per group and tensor
+    if (lane == 0) {
       prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
       mbar_arrive_expect_tx(&sh.q_full, MT * 32768);
       for (int g = 0; g < 2 * MT; ++g) {
         const int32_t row =
@@ -177,32 +177,43 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
         }
       }
     }
-    const __nv_bfloat16* kh = k + (int64_t(b) * n_kv_heads + h) * ctx_cap * kD;
-    const __nv_bfloat16* vh = v + (int64_t(b) * n_kv_heads + h) * ctx_cap * kD;
+    __syncwarp();
+    const int64_t kv_row0 = (int64_t(b) * n_kv_heads + h) * ctx_cap;
     int issued = 0;
     for (int t = 0; t < n_tiles; ++t) {
       const int st = t % kStages;
-      if (t >= kStages && !mbar_wait(&sh.kv_empty[st], ((t / kStages) - 1) & 1, abort)) break;
-      if ((flags & kTestDropFirstTile) && t == 0) continue;  // test hook: never arrives
-      const uint32_t kdst = sKV + st * L::kStageBytes;
-      // 2 tensors x 64 rows x 16 chunks of 16 B; a row's 16 chunks go to 16
-      // consecutive threads (coalesced 256-byte reads)
-      for (int c = ptid; c < 2048; c += kProducers) {
-        const int tensor = c >> 10, rc = c & 1023, r = rc >> 4, ch = rc & 15;
-        const int64_t row = int64_t(sh.grp[t * 8 + (r >> 3)]) * kGroup + (r & 7);
-        const __nv_bfloat16* src = (tensor ? vh : kh) + row * kD + ch * 8;
-        const uint32_t dst = kdst + tensor * 16384 + (ch >> 3) * 8192 + r * 128 +
-                             (((ch & 7) ^ (r & 7)) << 4);
-        cp_async16(dst, src);
+      bool go = true;
+      if (lane == 0) {
+        if (t >= kStages && !mbar_wait(&sh.kv_empty[st], ((t / kStages) - 1) & 1, abort))
+          go = false;
+        else if ((flags & kTestDropFirstTile) && t == 0)
+          go = false;  // test hook: never armed
+        else
+          mbar_arrive_expect_tx(&sh.kv_full[st], L::kStageBytes);
       }
-      cp_async_arrive(&sh.kv_full[st]);
+      go = __shfl_sync(0xffffffffu, go, 0);
+      if (!go) {
+        if ((flags & kTestDropFirstTile) && t == 0 && !*abort) continue;
+        break;
+      }
+      if (lane < 8) {
+        uint8_t* kdst = smem + L::kKV + st * L::kStageBytes + lane * 2048;
+        const int32_t row = int32_t(kv_row0 + int64_t(sh.grp[t * 8 + lane]) * kGroup);
+        tma_load_3d(kdst, &tm_k, &sh.kv_full[st], 0, row, 0);
+        tma_load_3d(kdst + 16384, &tm_v, &sh.kv_full[st], 0, row, 0);
+      }
+      __syncwarp();
       issued = t + 1;
     }
     // drain: wait (bounded, independent of abort) for the copies in flight
-    int never = 0;
-    if (tid == 0) mbar_wait(&sh.q_full, 0, &never);
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    (void)issued;
+    if (lane == 0) {
+      int never = 0;
+      mbar_wait(&sh.q_full, 0, &never);
+      for (int t = issued - 1; t >= 0 && t >= issued - kStages; --t) {
+        if ((flags & kTestDropFirstTile) && t == 0) continue;
+        mbar_wait(&sh.kv_full[t % kStages], (t / kStages) & 1, &never);
+      }
+    }
   } else if (warp == 1) {
     // ---------------- MMA issuer (event driven) ----------------
     if (lane == 0) {
@@ -226,7 +237,7 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
             for (int m = 0; m < MT; ++m) {
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
-                const uint64_t bd = smem_desc_sw128(vbase + k * 2048, 8192, 1024);
+                const uint64_t bd = smem_desc_sw128(vbase + k * 4096, 1024, 2048);
                 mma_bf16_tmem_a(tmem + L::colO(m), tmem + L::colS(m, tt & 1) + k * 8, bd,
                                 idesc_pv, (tt > 0 || k > 0) ? 1u : 0u);
               }
@@ -245,7 +256,6 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
           for (int m = 0; m < MT && ready && t >= 2; ++m)
             ready = mbar_try_wait(&sh.pv_done[m][buf], ((t - 2) >> 1) & 1);
           if (ready) {
-            fence_proxy_async_smem();  // cp.async (generic proxy) data -> tensor-core reads
             tc_fence_after();
             const uint32_t kbase = sKV + st * L::kStageBytes;
             for (int m = 0; m < MT; ++m) {
@@ -254,7 +264,7 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
                 const uint64_t a =
                     smem_desc_sw128(sQ + m * 32768 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
                 const uint64_t bd =
-                    smem_desc_sw128(kbase + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024);
+                    smem_desc_sw128(kbase + (k >> 2) * 1024 + (k & 3) * 32, 16, 2048);
                 mma_bf16(tmem + L::colS(m, buf), a, bd, idesc_qk, k > 0);
               }
               mma_commit(&sh.s_full[m][buf]);

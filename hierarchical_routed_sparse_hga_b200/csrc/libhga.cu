@@ -118,6 +118,22 @@ bool make_map_bf16_d128(CUtensorMap* map, const void* base, uint64_t rows, uint3
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same matrix seen as [halves = 2][rows][64 columns] (global strides
+// 128 B for a half, 256 B for a row), boxes of 64 x box_rows x 2 land in
+// shared memory as [half][row][128 B]: a group of 8 rows in one copy.
+bool make_map_bf16_d128_groups(CUtensorMap* map, const void* base, uint64_t rows,
+                               uint32_t box_rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, rows, 2};
+  cuuint64_t strides[2] = {256, 128};
+  cuuint32_t box[3] = {64, box_rows, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool use_tensor_cores(const hga_config_t* c, int64_t ctx_cap, int32_t s_len) {
   const int G = c->n_q_heads / c->n_kv_heads;
   if (c->flags & HGA_FLAG_SIMT) return false;
@@ -133,9 +149,13 @@ hga_status_t launch_fwd_tc(const hga_config_t* cfg, const void* q, const void* k
                            int64_t ctx_cap, int64_t q_begin, int32_t s_len,
                            const int32_t* sel_grp, void* o, float* lse, cudaStream_t s) {
   using L = fwdtc::Layout<MT>;
-  CUtensorMap tq;
+  CUtensorMap tq, tk, tv;
   const uint64_t q_rows = uint64_t(cfg->batch) * cfg->n_q_heads * s_len;
-  if (!make_map_bf16_d128(&tq, q, q_rows, 64)) return HGA_ERR_CUDA;
+  const uint64_t kv_rows = uint64_t(cfg->batch) * cfg->n_kv_heads * ctx_cap;
+  if (!make_map_bf16_d128(&tq, q, q_rows, 64) ||
+      !make_map_bf16_d128_groups(&tk, k, kv_rows, 8) ||
+      !make_map_bf16_d128_groups(&tv, v, kv_rows, 8))
+    return HGA_ERR_CUDA;
   hga_status_t e = ensure_smem(
       reinterpret_cast<const void*>(&fwdtc::attn_fwd_tc_kernel<MT>), L::kDynSmem);
   if (e != HGA_OK) return e;
@@ -144,8 +164,7 @@ hga_status_t launch_fwd_tc(const hga_config_t* cfg, const void* q, const void* k
   const float scale_log2 = cfg->scale * 1.4426950408889634f;
   return traced_launch(HGA_K_FWD_TC, s, [&] {
     fwdtc::attn_fwd_tc_kernel<MT><<<grid, L::kThreads, L::kDynSmem, s>>>(
-        tq, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), ctx_cap,
-        q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups,
+        tq, tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups,
         sel_grp, scale_log2, static_cast<__nv_bfloat16*>(o), lse, cfg->flags);
   });
 }
