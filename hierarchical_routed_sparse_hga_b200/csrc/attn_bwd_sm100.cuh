@@ -199,23 +199,23 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     if (tid == 0) mbar_wait(&sh.q_full, 0, &never);
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 1) {
-    // ---------------- MMA issuer (event driven) ----------------
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);
-      constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kD, 0, 1);
-      bool ok = mbar_wait(&sh.q_full, 0, abort);
-      bool issued_any = false;
-      int next_sdp = 0, next_dq = 0;
-      long long t0 = clock64();
-      while (ok && next_dq < n_tiles) {
-        bool progressed = false;
-        if (next_dq < next_sdp) {
-          bool ready = true;
-          for (int m = 0; m < MT; ++m) ready = ready && mbar_try_wait(&sh.ds_full[m], next_dq & 1);
-          if (ready) {
-            const int tt = next_dq;
-            const uint32_t kb = sKV + (tt & 1) * L::kStageBytes;
-            tc_fence_after();
+    // ---------------- MMA issuer (event driven; whole warp, one lane issues) --
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);
+    constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kD, 0, 1);
+    bool ok = __all_sync(kFullMask, mbar_wait(&sh.q_full, 0, abort));
+    bool issued_any = false;
+    int next_sdp = 0, next_dq = 0;
+    long long t0 = clock64();
+    while (ok && next_dq < n_tiles) {
+      bool progressed = false;
+      if (next_dq < next_sdp) {
+        bool ready = true;
+        for (int m = 0; m < MT; ++m) ready = ready && mbar_test(&sh.ds_full[m], next_dq & 1);
+        if (__all_sync(kFullMask, ready)) {
+          const int tt = next_dq;
+          const uint32_t kb = sKV + (tt & 1) * L::kStageBytes;
+          tc_fence_after();
+          if (elect_one()) {
             for (int m = 0; m < MT; ++m) {
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
@@ -225,21 +225,24 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
               mma_commit(&sh.ds_done[m]);
             }
             mma_commit(&sh.kv_empty[tt & 1]);
-            ++next_dq;
-            progressed = true;
           }
+          __syncwarp();
+          ++next_dq;
+          progressed = true;
         }
-        // S/dP(t) may run one tile ahead of dQ: its TMEM columns are free once
-        // the softmax has loaded S/dP(t-1)
-        if (!progressed && next_sdp < n_tiles && next_sdp <= next_dq + 1) {
-          const int t = next_sdp, st = t & 1;
-          bool ready = mbar_try_wait(&sh.kv_full[st], (t >> 1) & 1);
-          for (int m = 0; m < MT && ready && t >= 1; ++m)
-            ready = mbar_try_wait(&sh.sdp_free[m], (t - 1) & 1);
-          if (ready) {
-            fence_proxy_async_smem();  // cp.async data -> tensor-core reads
-            tc_fence_after();
-            const uint32_t kb = sKV + st * L::kStageBytes;
+      }
+      // S/dP(t) may run one tile ahead of dQ: its TMEM columns are free once
+      // the softmax has loaded S/dP(t-1)
+      if (!progressed && next_sdp < n_tiles && next_sdp <= next_dq + 1) {
+        const int t = next_sdp, st = t & 1;
+        bool ready = mbar_test(&sh.kv_full[st], (t >> 1) & 1);
+        for (int m = 0; m < MT && t >= 1; ++m)
+          ready = ready && mbar_test(&sh.sdp_free[m], (t - 1) & 1);
+        if (__all_sync(kFullMask, ready)) {
+          fence_proxy_async_smem();  // cp.async data -> tensor-core reads
+          tc_fence_after();
+          const uint32_t kb = sKV + st * L::kStageBytes;
+          if (elect_one()) {
             for (int m = 0; m < MT; ++m) {
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk) {
@@ -252,26 +255,20 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
               }
               mma_commit(&sh.sdp_full[m]);
             }
-            ++next_sdp;
-            issued_any = true;
-            progressed = true;
           }
-        }
-        if (progressed) {
-          t0 = clock64();
-        } else if (*abort) {
-          ok = false;
-        } else if (clock64() - t0 > 2000000000LL) {
-          latch_status(HGA_ERR_TIMEOUT);
-          *abort = 1;
-          ok = false;
+          __syncwarp();
+          ++next_sdp;
+          issued_any = true;
+          progressed = true;
         }
       }
-      if (issued_any) {
-        int never = 0;
-        mma_commit(&sh.mma_done);
-        mbar_wait(&sh.mma_done, 0, &never);
-      }
+      ok = warp_event_continue(progressed, t0, abort);
+    }
+    if (issued_any) {
+      if (elect_one()) mma_commit(&sh.mma_done);
+      __syncwarp();
+      int never = 0;
+      mbar_wait(&sh.mma_done, 0, &never);
     }
   } else if (warp >= 4) {
     const int m = (warp - 4) >> 2, wq = warp & 3;
@@ -513,8 +510,8 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
   const int n_items = sh.n_items;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
+    // ---------------- TMA producer (whole warp; one elected lane issues) ----
+    if (elect_one()) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_do);
       prefetch_tmap(&tm_k);
@@ -528,11 +525,15 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
           tma_load_2d(smem + L::kV + hf * 8192 + gi * 1024, &tm_v, &sh.kv_full, hf * 64,
                       krow + gi * kGroup);
         }
-      int issued = 0;
-      for (int it = 0; it < n_items; ++it) {
-        const int u = it & 1;
-        if (it >= 2 && !mbar_wait(&sh.qd_empty[u], ((it >> 1) - 1) & 1, abort)) break;
-        const int jj = sh.js[it / MT], m = it % MT;
+    }
+    __syncwarp();
+    int issued = 0;
+    for (int it = 0; it < n_items; ++it) {
+      const int u = it & 1;
+      const bool free_ok = it < 2 || mbar_wait(&sh.qd_empty[u], ((it >> 1) - 1) & 1, abort);
+      if (!__all_sync(kFullMask, free_ok)) break;
+      const int jj = sh.js[it / MT], m = it % MT;
+      if (elect_one()) {
         mbar_arrive_expect_tx(&sh.qd_full[u], 65536);
         uint8_t* dst = smem + L::kQD + u * L::kQDBytes;
         for (int g = 0; g < 2; ++g) {
@@ -544,29 +545,33 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
                         row);
           }
         }
-        issued = it + 1;
       }
+      __syncwarp();
+      issued = it + 1;
+    }
+    if (lane == 0) {
       int never = 0;
       mbar_wait(&sh.kv_full, 0, &never);
       for (int it = issued - 1; it >= 0 && it >= issued - 2; --it)
         mbar_wait(&sh.qd_full[it & 1], (it >> 1) & 1, &never);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer (event driven) ----------------
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);
-      constexpr uint32_t idesc_t = idesc_bf16_f32(128, 64, 1, 1);
-      bool ok = mbar_wait(&sh.kv_full, 0, abort);
-      bool issued_any = false;
-      int next_s = 0, next_t = 0;  // items with S/dP issued, with dV/dK issued
-      long long t0 = clock64();
-      while (ok && next_t < n_items) {
-        bool progressed = false;
-        if (next_t < next_s && mbar_try_wait(&sh.pds_full[next_t & 1], (next_t >> 1) & 1)) {
-          // dV^T += dO^T P and dK^T += Q^T dS over this item's 128 query rows
-          const int u = next_t & 1;
-          const uint32_t qd = sQD + u * L::kQDBytes, pd = sPD + u * L::kPDBytes;
-          tc_fence_after();
+    // ---------------- MMA issuer (event driven; whole warp, one lane issues) --
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);
+    constexpr uint32_t idesc_t = idesc_bf16_f32(128, 64, 1, 1);
+    bool ok = __all_sync(kFullMask, mbar_wait(&sh.kv_full, 0, abort));
+    bool issued_any = false;
+    int next_s = 0, next_t = 0;  // items with S/dP issued, with dV/dK issued
+    long long t0 = clock64();
+    while (ok && next_t < n_items) {
+      bool progressed = false;
+      if (next_t < next_s &&
+          __all_sync(kFullMask, mbar_test(&sh.pds_full[next_t & 1], (next_t >> 1) & 1))) {
+        // dV^T += dO^T P and dK^T += Q^T dS over this item's 128 query rows
+        const int u = next_t & 1;
+        const uint32_t qd = sQD + u * L::kQDBytes, pd = sPD + u * L::kPDBytes;
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
           for (int s8 = 0; s8 < 8; ++s8) {
             const uint32_t ro = s8 * 2048;
@@ -577,16 +582,19 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
                      smem_desc_sw128(pd + 16384 + ro, 8192, 1024), idesc_t, acc);
           }
           mma_commit(&sh.qd_empty[u]);
-          ++next_t;
-          progressed = true;
         }
-        // S/dP(i) into buffer i & 1, free once dV/dK(i-2) has been issued
-        // (its softmax has then finished with that buffer)
-        if (!progressed && next_s < n_items && next_s < next_t + 2 &&
-            mbar_try_wait(&sh.qd_full[next_s & 1], (next_s >> 1) & 1)) {
-          const int u = next_s & 1;
-          const uint32_t qd = sQD + u * L::kQDBytes;
-          tc_fence_after();
+        __syncwarp();
+        ++next_t;
+        progressed = true;
+      }
+      // S/dP(i) into buffer i & 1, free once dV/dK(i-2) has been issued
+      // (its softmax has then finished with that buffer)
+      if (!progressed && next_s < n_items && next_s < next_t + 2 &&
+          __all_sync(kFullMask, mbar_test(&sh.qd_full[next_s & 1], (next_s >> 1) & 1))) {
+        const int u = next_s & 1;
+        const uint32_t qd = sQD + u * L::kQDBytes;
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t ao = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -597,25 +605,19 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
                      smem_desc_sw128(sV + bo, 16, 1024), idesc_s, kk > 0);
           }
           mma_commit(&sh.sdp_full[u]);
-          ++next_s;
-          issued_any = true;
-          progressed = true;
         }
-        if (progressed) {
-          t0 = clock64();
-        } else if (*abort) {
-          ok = false;
-        } else if (clock64() - t0 > 2000000000LL) {
-          latch_status(HGA_ERR_TIMEOUT);
-          *abort = 1;
-          ok = false;
-        }
+        __syncwarp();
+        ++next_s;
+        issued_any = true;
+        progressed = true;
       }
-      if (issued_any) {
-        int never = 0;
-        mma_commit(&sh.mma_done);
-        mbar_wait(&sh.mma_done, 0, &never);
-      }
+      ok = warp_event_continue(progressed, t0, abort);
+    }
+    if (issued_any) {
+      if (elect_one()) mma_commit(&sh.mma_done);
+      __syncwarp();
+      int never = 0;
+      mbar_wait(&sh.mma_done, 0, &never);
     }
   } else if (warp >= 4) {
     // ---------------- softmax (two warp groups, one per buffer) ----------------

@@ -12,20 +12,20 @@
 //   warp 0      TMA producer: Q once (64 x 64 boxes); then per key tile the
 //               8 selected groups of K and V, each group (a contiguous 2 KiB
 //               run of [B,Hkv,T,d]) one 3-D box of 64 columns x 8 rows x 2
-//               column halves, issued from 8 lanes, into a 4-stage ring laid
+//               column halves, into a 4-stage ring laid
 //               out [group][d half][8 rows][128 B] (128-byte swizzle; UMMA
 //               stride 2048 B between 8-row groups);
-//   warp 1      TMEM owner and MMA issuer.  It issues, as soon as each one's
-//               inputs are ready, S = Q K^T into double-buffered TMEM and
-//               O += P V with P read straight from TMEM (A operand in tensor
-//               memory) -- whichever is ready first, so a late K/V tile never
-//               holds back the PV of the tile before it;
+//   warp 1      TMEM owner and MMA issuer: S = Q K^T into double-buffered
+//               TMEM and O += P V with P read straight from TMEM (A operand
+//               in tensor memory), in a fixed order with blocking waits;
 //   warps 4..   softmax, one warp group per M tile, one thread per row (TMEM
 //               lane): masks (padding slots, causal own block; skipped for
 //               full routed tiles), online softmax in the log2 domain with
 //               packed f32x2 arithmetic and lazy rescaling (O is rescaled only
 //               when the running max grows by more than 2^8), P written back as
 //               bf16 over its own S columns, epilogue O / l and LSE.
+// The producer and issuer loops run in all 32 lanes of their warp, so loop
+// state and operand descriptors are warp-uniform; one elected lane issues.
 // Every wait is bounded; a timeout latches HGA_ERR_TIMEOUT, raises a shared
 // abort flag, drains the copies and MMAs in flight and frees TMEM.
 #pragma once
@@ -160,10 +160,10 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
   const int n_tiles = sh.n_tiles;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (whole warp; one elected lane issues) ----
     // K/V tile layout: group gi at gi * 2048: [d half][8 rows][128 B], one
     // 3-D box (64 columns x 8 rows x 2 halves) per group and tensor
-    if (lane == 0) {
+    if (elect_one()) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
@@ -182,25 +182,23 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
     int issued = 0;
     for (int t = 0; t < n_tiles; ++t) {
       const int st = t % kStages;
-      bool go = true;
-      if (lane == 0) {
-        if (t >= kStages && !mbar_wait(&sh.kv_empty[st], ((t / kStages) - 1) & 1, abort))
-          go = false;
-        else if ((flags & kTestDropFirstTile) && t == 0)
-          go = false;  // test hook: never armed
-        else
-          mbar_arrive_expect_tx(&sh.kv_full[st], L::kStageBytes);
+      const bool free_ok =
+          t < kStages || mbar_wait(&sh.kv_empty[st], ((t / kStages) - 1) & 1, abort);
+      if (!__all_sync(kFullMask, free_ok)) break;
+      if ((flags & kTestDropFirstTile) && t == 0) {
+        // test hook: tile 0 is never armed, so its consumers must time out
+        if (__any_sync(kFullMask, *abort != 0)) break;
+        continue;
       }
-      go = __shfl_sync(0xffffffffu, go, 0);
-      if (!go) {
-        if ((flags & kTestDropFirstTile) && t == 0 && !*abort) continue;
-        break;
-      }
-      if (lane < 8) {
-        uint8_t* kdst = smem + L::kKV + st * L::kStageBytes + lane * 2048;
-        const int32_t row = int32_t(kv_row0 + int64_t(sh.grp[t * 8 + lane]) * kGroup);
-        tma_load_3d(kdst, &tm_k, &sh.kv_full[st], 0, row, 0);
-        tma_load_3d(kdst + 16384, &tm_v, &sh.kv_full[st], 0, row, 0);
+      if (elect_one()) {
+        mbar_arrive_expect_tx(&sh.kv_full[st], L::kStageBytes);
+        uint8_t* kdst = smem + L::kKV + st * L::kStageBytes;
+#pragma unroll
+        for (int gi = 0; gi < 8; ++gi) {
+          const int32_t row = int32_t(kv_row0 + int64_t(sh.grp[t * 8 + gi]) * kGroup);
+          tma_load_3d(kdst + gi * 2048, &tm_k, &sh.kv_full[st], 0, row, 0);
+          tma_load_3d(kdst + gi * 2048 + 16384, &tm_v, &sh.kv_full[st], 0, row, 0);
+        }
       }
       __syncwarp();
       issued = t + 1;
@@ -215,81 +213,74 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer (event driven) ----------------
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kD, 0, 1);
-      bool ok = mbar_wait(&sh.q_full, 0, abort);
-      bool issued_any = false;
-      int next_qk = 0, next_pv = 0;  // next tile to issue S = QK^T for / O += PV for
-      long long t0 = clock64();
-      while (ok && next_pv < n_tiles) {
-        bool progressed = false;
-        // PV(next_pv) once every M tile's P is in TMEM
-        if (next_pv < next_qk) {
-          bool ready = true;
-          for (int m = 0; m < MT; ++m)
-            ready = ready && mbar_try_wait(&sh.p_full[m][next_pv & 1], (next_pv >> 1) & 1);
-          if (ready) {
-            const int tt = next_pv, st = tt % kStages;
-            const uint32_t vbase = sKV + st * L::kStageBytes + 16384;
-            tc_fence_after();
-            for (int m = 0; m < MT; ++m) {
+    // ---------------- MMA issuer (whole warp, one lane issues) --------------
+    // Fixed order S(0), S(1), then PV(t), S(t+2) for t = 0, 1, ...: S(t+2)
+    // reuses the TMEM columns that hold P(t) until PV(t) has read them.  The
+    // waits block (the warp is parked until the phase completes), which
+    // leaves the issue slots of its sub-partition to the softmax warps.
+    constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, 0, 0);
+    constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kD, 0, 1);
+    bool issued_any = false;
+    auto issue_qk = [&](int t) -> bool {
+      const int st = t % kStages, buf = t & 1;
+      bool ready = mbar_wait(&sh.kv_full[st], (t / kStages) & 1, abort);
+      for (int m = 0; m < MT && t >= 2; ++m)
+        ready = ready && mbar_wait(&sh.pv_done[m][buf], ((t - 2) >> 1) & 1, abort);
+      if (!__all_sync(kFullMask, ready)) return false;
+      tc_fence_after();
+      const uint32_t kbase = sKV + st * L::kStageBytes;
+      if (elect_one()) {
+        for (int m = 0; m < MT; ++m) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const uint64_t bd = smem_desc_sw128(vbase + k * 4096, 1024, 2048);
-                mma_bf16_tmem_a(tmem + L::colO(m), tmem + L::colS(m, tt & 1) + k * 8, bd,
-                                idesc_pv, (tt > 0 || k > 0) ? 1u : 0u);
-              }
-              mma_commit(&sh.pv_done[m][tt & 1]);
-            }
-            mma_commit(&sh.kv_empty[st]);
-            ++next_pv;
-            progressed = true;
+          for (int k = 0; k < 8; ++k) {
+            const uint64_t a =
+                smem_desc_sw128(sQ + m * 32768 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(kbase + (k >> 2) * 1024 + (k & 3) * 32, 16, 2048);
+            mma_bf16(tmem + L::colS(m, buf), a, bd, idesc_qk, k > 0);
           }
-        }
-        // S(next_qk) once its K/V tile is in and its S buffer is free again:
-        // P(next_qk - 2) lives there until PV(next_qk - 2) has read it
-        if (!progressed && next_qk < n_tiles && next_qk < next_pv + 2) {
-          const int t = next_qk, st = t % kStages, buf = t & 1;
-          bool ready = mbar_try_wait(&sh.kv_full[st], (t / kStages) & 1);
-          for (int m = 0; m < MT && ready && t >= 2; ++m)
-            ready = mbar_try_wait(&sh.pv_done[m][buf], ((t - 2) >> 1) & 1);
-          if (ready) {
-            tc_fence_after();
-            const uint32_t kbase = sKV + st * L::kStageBytes;
-            for (int m = 0; m < MT; ++m) {
-#pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const uint64_t a =
-                    smem_desc_sw128(sQ + m * 32768 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-                const uint64_t bd =
-                    smem_desc_sw128(kbase + (k >> 2) * 1024 + (k & 3) * 32, 16, 2048);
-                mma_bf16(tmem + L::colS(m, buf), a, bd, idesc_qk, k > 0);
-              }
-              mma_commit(&sh.s_full[m][buf]);
-            }
-            ++next_qk;
-            issued_any = true;
-            progressed = true;
-          }
-        }
-        if (progressed) {
-          t0 = clock64();
-        } else if (*abort) {
-          ok = false;
-        } else if (clock64() - t0 > 2000000000LL) {
-          latch_status(HGA_ERR_TIMEOUT);
-          *abort = 1;
-          ok = false;
+          mma_commit(&sh.s_full[m][buf]);
         }
       }
-      if (issued_any) {
-        // every MMA this thread issued must finish before TMEM is freed
-        int never = 0;
-        mma_commit(&sh.mma_done);
-        mbar_wait(&sh.mma_done, 0, &never);
+      __syncwarp();
+      issued_any = true;
+      return true;
+    };
+    auto issue_pv = [&](int t) -> bool {
+      bool ready = true;
+      for (int m = 0; m < MT; ++m)
+        ready = ready && mbar_wait(&sh.p_full[m][t & 1], (t >> 1) & 1, abort);
+      if (!__all_sync(kFullMask, ready)) return false;
+      const int st = t % kStages;
+      const uint32_t vbase = sKV + st * L::kStageBytes + 16384;
+      tc_fence_after();
+      if (elect_one()) {
+        for (int m = 0; m < MT; ++m) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t bd = smem_desc_sw128(vbase + k * 4096, 1024, 2048);
+            mma_bf16_tmem_a(tmem + L::colO(m), tmem + L::colS(m, t & 1) + k * 8, bd, idesc_pv,
+                            (t > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(&sh.pv_done[m][t & 1]);
+        }
+        mma_commit(&sh.kv_empty[st]);
       }
+      __syncwarp();
+      return true;
+    };
+    bool ok = __all_sync(kFullMask, mbar_wait(&sh.q_full, 0, abort));
+    if (ok) ok = issue_qk(0);
+    if (ok && n_tiles > 1) ok = issue_qk(1);
+    for (int t = 0; ok && t < n_tiles; ++t) {
+      ok = issue_pv(t);
+      if (ok && t + 2 < n_tiles) ok = issue_qk(t + 2);
+    }
+    if (issued_any) {
+      // every MMA this warp issued must finish before TMEM is freed
+      if (elect_one()) mma_commit(&sh.mma_done);
+      __syncwarp();
+      int never = 0;
+      mbar_wait(&sh.mma_done, 0, &never);
     }
   } else if (warp >= 4) {
     // ---------------- softmax / epilogue ----------------

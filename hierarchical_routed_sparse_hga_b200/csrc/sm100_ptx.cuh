@@ -55,6 +55,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of a phase (never suspends the thread, unlike try_wait,
+// which may park it for a while): for issuers that poll several barriers and
+// must act on whichever completes first.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr unsigned kFullMask = 0xffffffffu;
+
+// True in exactly one lane of a converged warp: elect.sync picks the leader
+// among the active lanes of the mask, the same lane each time the whole warp
+// runs it.  Issue loops run in all 32 lanes (so every operand and loop
+// variable is warp-uniform) and only the issuing instruction sits under this.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // Bounded wait: spins until the phase with `parity` completes, another role
 // has raised *abort, or about `limit_cycles` SM cycles pass.  On timeout it
 // latches HGA_ERR_TIMEOUT and raises *abort.  Returns true iff the phase
@@ -72,6 +103,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       return false;
     }
   }
+}
+
+// One step of the idle bookkeeping of an event loop run by a whole warp:
+// after progress the idle clock restarts; otherwise the loop ends (false) if
+// another role raised *abort, or -- latching HGA_ERR_TIMEOUT and raising
+// *abort -- once nothing has progressed for about 2e9 cycles.  The result is
+// the same in every lane.
+__device__ __forceinline__ bool warp_event_continue(bool progressed, long long& t0,
+                                                    volatile int* abort) {
+  if (progressed) {
+    t0 = clock64();
+    return true;
+  }
+  if (__any_sync(kFullMask, *abort != 0)) return false;
+  if (__any_sync(kFullMask, clock64() - t0 > 2000000000LL)) {
+    if ((threadIdx.x & 31) == 0) {
+      latch_status(HGA_ERR_TIMEOUT);
+      *abort = 1;
+    }
+    __syncwarp();
+    return false;
+  }
+  return true;
 }
 
 // ---------------------------------------------------------------------------
