@@ -96,6 +96,11 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def job_throughput(units_per_rank_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job rate: the units all ranks processed over the slowest rank's time."""
+    return world * units_per_rank_step * steps / (max_ms / 1e3)
+
+
 def barrier(world: int, device=None):
     if world > 1:
         import torch.distributed as dist
@@ -505,7 +510,7 @@ def run_gpu(args, rank, world, local):
 
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(step_ms), world, device)
-    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+    value = job_throughput(tokens_per_step, args.steps, world, total_ms)
 
     # per-kernel table and the dominant kernel's roofline
     table = timing_table()
@@ -560,7 +565,7 @@ def run_gpu(args, rank, world, local):
         barrier(world, device)
         e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
         h2d, d2h = run.io_bytes()
-        e2e = {"value": round(world * tokens_per_step * args.steps / (e_ms / 1e3), 1),
+        e2e = {"value": round(job_throughput(tokens_per_step, args.steps, world, e_ms), 1),
                "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = None
