@@ -8,13 +8,16 @@ The shared library is loaded on first use; build it with
 """
 from ._lib import (EXPORTS, HGA_BF16, HGA_ERR_CUDA, HGA_ERR_DEVICE_CHECK,  # noqa: F401
                    HGA_ERR_INVALID_ARG, HGA_ERR_TIMEOUT, HGA_ERR_UNSUPPORTED,
-                   HGA_ERR_WORKSPACE, HGA_F32, HGA_FLAG_SIMT, HGA_OK, Config, HgaError,
+                   HGA_ERR_WORKSPACE, HGA_F32, HGA_FLAG_SIMT, HGA_K_COUNT, HGA_OK, Config,
+                   HgaError,
                    hga_attn_bwd, hga_attn_bwd_workspace_size, hga_attn_fwd,
                    hga_build_summaries, hga_build_summaries_seg, hga_tier_append, hga_tier_gather,
-                   hga_tier_stage_rows, hga_tier_workspace_size, hga_get_device_status, hga_kernel_name,
+                   hga_tier_stage_rows, hga_tier_workspace_size, hga_get_device_status,
+                   hga_kernel_name,
                    hga_launch_count, hga_route, hga_route_noalloc,
                    hga_route_workspace_size, hga_status_string,
-                   hga_timing_collect, hga_timing_enable, hga_timing_get, hga_timing_reset,
+                   hga_timing_collect, hga_timing_enable, hga_timing_get, hga_timing_kinds,
+                   hga_timing_reset,
                    hga_version, load, timing_table)
 
 

@@ -26,7 +26,8 @@ EXPORTS = ("hga_version", "hga_status_string", "hga_build_summaries",
            "hga_route_workspace_size", "hga_route", "hga_attn_fwd",
            "hga_attn_bwd_workspace_size", "hga_attn_bwd", "hga_get_device_status",
            "hga_kernel_name", "hga_launch_count", "hga_timing_enable", "hga_timing_collect",
-           "hga_timing_get", "hga_timing_reset", "hga_route_noalloc", "hga_build_summaries_seg",
+           "hga_timing_get", "hga_timing_reset", "hga_timing_kinds", "hga_route_noalloc",
+           "hga_build_summaries_seg",
            "hga_tier_stage_rows", "hga_tier_workspace_size", "hga_tier_gather",
            "hga_tier_append")
 HGA_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -98,6 +99,7 @@ def load() -> ctypes.CDLL:
         "hga_timing_get": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_double),
                                           ctypes.POINTER(ctypes.c_uint64)]),
         "hga_timing_reset": (None, []),
+        "hga_timing_kinds": (None, [ctypes.c_uint32]),
         "hga_route_noalloc": (ctypes.c_int, [CFG, P, I64, I32, I64, P, P, P, P, P]),
         "hga_build_summaries_seg": (ctypes.c_int, [CFG, P, I64, I64, I64, I64, P, P, P]),
         "hga_tier_stage_rows": (I64, [CFG, I64, I32]),
@@ -286,6 +288,10 @@ def hga_timing_get(kind: int):
 
 def hga_timing_reset():
     load().hga_timing_reset()
+
+
+def hga_timing_kinds(mask: int):
+    load().hga_timing_kinds(mask & 0xFFFFFFFF)
 
 
 def timing_table() -> dict:

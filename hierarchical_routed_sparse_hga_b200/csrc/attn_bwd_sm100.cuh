@@ -134,6 +134,7 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
   const int n_qb = s_len / kQBlock;
   const int64_t own_blk = (q_begin + int64_t(j) * kQBlock) / kBlock;
   volatile int* abort = &sh.abort;
+  pdl_launch_dependents();
 
   if (tid == 0) {
     mbar_init(&sh.q_full, 1);
@@ -151,6 +152,9 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     sh.abort = 0;
     fence_barrier_init();
   }
+  // the previous kernel may still hold this SM's tensor memory or write
+  // this kernel's inputs: wait for it before allocating or reading
+  pdl_wait();
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, L::kTmemCols);
     tmem_relinquish();
@@ -462,6 +466,7 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
   const int n_qb = s_len / kQBlock;
   const int64_t gblk = q_begin / kBlock + kb;  // global index of this key block
   volatile int* abort = &sh.abort;
+  pdl_launch_dependents();
 
   for (int i = tid; i < 64; i += blockDim.x) sh.masks[i] = (i == kb) ? 0xff : 0;
   if (tid == 0) {
@@ -476,6 +481,9 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
     sh.abort = 0;
     fence_barrier_init();
   }
+  // the previous kernel may still hold this SM's tensor memory or write
+  // this kernel's inputs: wait for it before allocating or reading
+  pdl_wait();
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, L::kTmemCols);
     tmem_relinquish();

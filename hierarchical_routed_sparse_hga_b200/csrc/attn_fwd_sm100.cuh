@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
   const int n_qb = s_len / kQBlock;
   const int64_t own_blk = (q_begin + int64_t(j) * kQBlock) / kBlock;
   volatile int* abort = &sh.abort;
+  pdl_launch_dependents();
 
   // ---- set-up: barriers, TMEM, the tile schedule -------------------------
   if (tid == 0) {
@@ -119,6 +120,9 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
     sh.abort = 0;
     fence_barrier_init();
   }
+  // the previous kernel may still hold this SM's tensor memory or write
+  // this kernel's inputs: wait for it before allocating or reading
+  pdl_wait();
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, L::kTmemCols);
     tmem_relinquish();

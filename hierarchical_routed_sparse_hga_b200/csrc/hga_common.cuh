@@ -23,6 +23,19 @@ __device__ __forceinline__ void latch_status(int code) {
   atomicCAS(&g_device_status, 0, code);
 }
 
+// Programmatic dependent launch.  The hot-path kernels are launched with
+// programmatic stream serialization: pdl_launch_dependents() lets the next
+// kernel on the stream be scheduled once every CTA of this grid has run it
+// (so no CTA of this grid can be kept off an SM by its dependents), and
+// pdl_wait() blocks until the previous kernel has completed and its writes
+// are visible.  Every thread calls pdl_wait() before its first access to
+// global memory that a previous kernel may write or read.  Both are no-ops
+// in a launch without the attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------
 // element loads: 8 consecutive elements -> 8 floats (16 B for bf16, 32 B for f32)
 // ---------------------------------------------------------------------------

@@ -163,9 +163,9 @@ hga_status_t launch_fwd_tc(const hga_config_t* cfg, const void* q, const void* k
   dim3 grid((s_len / kQBlock) * sets, cfg->n_kv_heads, cfg->batch);
   const float scale_log2 = cfg->scale * 1.4426950408889634f;
   return traced_launch(HGA_K_FWD_TC, s, [&] {
-    fwdtc::attn_fwd_tc_kernel<MT><<<grid, L::kThreads, L::kDynSmem, s>>>(
-        tq, tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups,
-        sel_grp, scale_log2, static_cast<__nv_bfloat16*>(o), lse, cfg->flags);
+    return launch_pdl(fwdtc::attn_fwd_tc_kernel<MT>, grid, dim3(L::kThreads), L::kDynSmem, s, tq,
+        tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups, sel_grp,
+        scale_log2, static_cast<__nv_bfloat16*>(o), lse, cfg->flags);
   });
 }
 
@@ -192,18 +192,18 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
   dim3 grid(s_len / kQBlock, cfg->n_kv_heads, cfg->batch);
   const float scale_log2 = cfg->scale * 1.4426950408889634f;
   e = traced_launch(HGA_K_BWD_DQ_TC, s, [&] {
-    bwdtc::attn_bwd_dq_tc_kernel<MT><<<grid, LQ::kThreads, LQ::kDynSmem, s>>>(
+    return launch_pdl(bwdtc::attn_bwd_dq_tc_kernel<MT>, grid, dim3(LQ::kThreads), LQ::kDynSmem, s,
         tq, tdo, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-        ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads,
-        cfg->topk_groups, sel_grp, cfg->scale, scale_log2, static_cast<const __nv_bfloat16*>(o),
+        ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups, sel_grp,
+        cfg->scale, scale_log2, static_cast<const __nv_bfloat16*>(o),
         static_cast<const __nv_bfloat16*>(d_o), lse, static_cast<__nv_bfloat16*>(dq), dvec);
   });
   if (e != HGA_OK) return e;
   return traced_launch(HGA_K_BWD_DKDV_TC, s, [&] {
-    bwdtc::attn_bwd_dkdv_tc_kernel<MT><<<grid, LK::kThreads, LK::kDynSmem, s>>>(
-        tq, tdo, tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads,
-        cfg->topk_groups, sel_grp, cfg->scale, scale_log2, lse, dvec,
-        static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
+    return launch_pdl(bwdtc::attn_bwd_dkdv_tc_kernel<MT>, grid, dim3(LK::kThreads), LK::kDynSmem, s,
+        tq, tdo, tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups,
+        sel_grp, cfg->scale, scale_log2, lse, dvec, static_cast<__nv_bfloat16*>(dk),
+        static_cast<__nv_bfloat16*>(dv));
   });
 }
 
@@ -292,9 +292,8 @@ hga_status_t hga_build_summaries(const hga_config_t* cfg, const void* k, int64_t
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
     dim3 grid(unsigned(n_blk), cfg->n_kv_heads, cfg->batch);
     return traced_launch(HGA_K_SUMMARIES, s, [&] {
-      summaries_kernel<T, D><<<grid, D, 0, s>>>(static_cast<const T*>(k), ctx_cap, t_begin,
-                                                ctx_cap, t_begin / kBlock, cfg->n_kv_heads,
-                                                gsum, bsum);
+      return launch_pdl(summaries_kernel<T, D>, grid, dim3(D), 0, s, static_cast<const T*>(k),
+          ctx_cap, t_begin, ctx_cap, t_begin / kBlock, cfg->n_kv_heads, gsum, bsum);
     });
   });
 }
@@ -316,9 +315,8 @@ hga_status_t hga_build_summaries_seg(const hga_config_t* cfg, const void* k_seg,
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
     dim3 grid(unsigned(n_blk), cfg->n_kv_heads, cfg->batch);
     return traced_launch(HGA_K_SUMMARIES, s, [&] {
-      summaries_kernel<T, D><<<grid, D, 0, s>>>(static_cast<const T*>(k_seg), seg_cap, 0,
-                                                ctx_cap, t_begin / kBlock, cfg->n_kv_heads,
-                                                gsum, bsum);
+      return launch_pdl(summaries_kernel<T, D>, grid, dim3(D), 0, s, static_cast<const T*>(k_seg),
+          seg_cap, 0, ctx_cap, t_begin / kBlock, cfg->n_kv_heads, gsum, bsum);
     });
   });
 }
@@ -348,8 +346,8 @@ hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, 
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
     dim3 g0(n_qb * G, cfg->n_kv_heads, cfg->batch);
     hga_status_t e = traced_launch(HGA_K_QMEAN, s, [&] {
-      qmean_kernel<T, D><<<g0, kQmeanThreads, 0, s>>>(static_cast<const T*>(q), cfg->n_q_heads,
-                                                      cfg->n_kv_heads, s_len, ws.qbar);
+      return launch_pdl(qmean_kernel<T, D>, g0, dim3(kQmeanThreads), 0, s, static_cast<const T*>(q),
+          cfg->n_q_heads, cfg->n_kv_heads, s_len, ws.qbar);
     });
     if (e != HGA_OK) return e;
     if (j_max > 0) {
@@ -357,9 +355,8 @@ hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, 
       const int n_jc = (n_qb + kScoreQbs - 1) / kScoreQbs;
       dim3 g2(unsigned(n_cc * n_jc), cfg->n_kv_heads, cfg->batch);
       e = traced_launch(HGA_K_BLOCK_SCORE, s, [&] {
-        block_score_kernel<D><<<g2, kRouteThreads, 0, s>>>(ws.qbar, bsum, ctx_cap,
-                                                           cfg->n_kv_heads, G, n_qb, own0,
-                                                           ws.scores, ws.jstride);
+        return launch_pdl(block_score_kernel<D>, g2, dim3(kRouteThreads), 0, s, ws.qbar, bsum,
+            ctx_cap, cfg->n_kv_heads, G, n_qb, own0, ws.scores, ws.jstride);
       });
       if (e != HGA_OK) return e;
     }
@@ -368,10 +365,9 @@ hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, 
     e = ensure_smem(reinterpret_cast<const void*>(&select_kernel<D>), sm3);
     if (e != HGA_OK) return e;
     return traced_launch(HGA_K_SELECT, s, [&] {
-      select_kernel<D><<<g1, kRouteThreads, sm3, s>>>(ws.qbar, ws.scores, gsum, ctx_cap,
-                                                      cfg->n_kv_heads, G, n_qb, own0, ws.jstride,
-                                                      cfg->topk_blocks, cfg->topk_groups,
-                                                      sel_blk, sel_grp);
+      return launch_pdl(select_kernel<D>, g1, dim3(kRouteThreads), sm3, s, ws.qbar, ws.scores, gsum,
+          ctx_cap, cfg->n_kv_heads, G, n_qb, own0, ws.jstride, cfg->topk_blocks, cfg->topk_groups,
+          sel_blk, sel_grp);
     });
   });
 }
@@ -619,6 +615,12 @@ hga_status_t hga_timing_enable(int32_t slots) {
   t.on = slots > 0;
   t.next = 0;
   return HGA_OK;
+}
+
+void hga_timing_kinds(uint32_t mask) {
+  Tracer& t = tracer();
+  std::lock_guard<std::mutex> lock(t.mu);
+  t.kinds = mask;
 }
 
 hga_status_t hga_timing_collect(void) {

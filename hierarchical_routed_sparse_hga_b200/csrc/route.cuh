@@ -34,6 +34,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kQmeanThreads)
     qmean_kernel(const T* __restrict__ q, int n_q_heads, int n_kv_heads, int s_len,
                  float* __restrict__ qpart) {
+  pdl_launch_dependents();
+  pdl_wait();
   constexpr int CH = D / 8;                    // 16-byte chunks per row
   constexpr int RS = kQmeanThreads / CH;       // row slots
   constexpr int PASSES = kQBlock / RS;
@@ -90,6 +92,8 @@ __global__ void __launch_bounds__(kRouteThreads)
     block_score_kernel(const float* __restrict__ qpart, const float* __restrict__ bsum,
                        int64_t ctx_cap, int n_kv_heads, int G, int n_qb, int64_t own0,
                        float* __restrict__ scores, int64_t jstride) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ float qb[kScoreQbs][D];
   __shared__ float bsT[D][kScoreCands + 1];
   const int h = blockIdx.y, b = blockIdx.z;
@@ -163,6 +167,8 @@ __global__ void __launch_bounds__(kRouteThreads)
                   const float* __restrict__ gsum, int64_t ctx_cap, int n_kv_heads, int G, int n_qb,
                   int64_t own0, int64_t jstride, int topk_blocks, int topk_groups,
                   int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ __align__(16) unsigned char sm_raw[];
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int64_t head = int64_t(b) * n_kv_heads + h;

@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(D) summaries_kernel(const T* __restrict__ k, i
                                                       int64_t blk0, int n_kv_heads,
                                                       float* __restrict__ gsum,
                                                       float* __restrict__ bsum) {
+  pdl_launch_dependents();
+  pdl_wait();
   constexpr int CH = D / 8;  // column chunks per row
   __shared__ float part[kGroupsPerBlock][D];
   const int64_t c = blk0 + blockIdx.x;  // global block index

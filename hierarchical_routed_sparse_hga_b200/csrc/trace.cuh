@@ -6,6 +6,8 @@
 
 #include <atomic>
 #include <mutex>
+#include <type_traits>
+#include <utility>
 #include <vector>
 
 #include "hga.h"
@@ -21,6 +23,7 @@ struct Tracer {
   std::mutex mu;
   std::atomic<uint64_t> launches{0};
   bool on = false;
+  uint32_t kinds = ~0u;  // kinds whose launches are bracketed (bit per kind)
   std::vector<TimingSlot> slots;
   size_t next = 0;
   double ms[HGA_K_COUNT] = {};
@@ -47,7 +50,7 @@ hga_status_t traced_launch(int kind, cudaStream_t s, F&& launch) {
   Tracer& t = tracer();
   t.launches.fetch_add(1, std::memory_order_relaxed);
   TimingSlot* slot = nullptr;
-  if (t.on) {
+  if (t.on && ((t.kinds >> kind) & 1u)) {
     std::lock_guard<std::mutex> lock(t.mu);
     if (t.next < t.slots.size()) {
       slot = &t.slots[t.next++];
@@ -55,10 +58,36 @@ hga_status_t traced_launch(int kind, cudaStream_t s, F&& launch) {
     }
   }
   if (slot && record(slot->begin, s) != cudaSuccess) return HGA_ERR_CUDA;
-  launch();
+  if constexpr (std::is_same_v<decltype(launch()), cudaError_t>) {
+    if (launch() != cudaSuccess) {
+      cudaGetLastError();
+      return HGA_ERR_CUDA;
+    }
+  } else {
+    launch();
+  }
   if (cudaGetLastError() != cudaSuccess) return HGA_ERR_CUDA;
   if (slot && record(slot->end, s) != cudaSuccess) return HGA_ERR_CUDA;
   return HGA_OK;
+}
+
+// Launches `kernel` on stream s with programmatic stream serialization, so
+// that it may be scheduled while the kernel before it drains (the kernel
+// itself orders its reads with pdl_wait()).  Returns the launch status.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace hga

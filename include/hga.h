@@ -273,6 +273,10 @@ HGA_API hga_status_t hga_get_device_status(void* stream);
  * Diagnostics: launch counting and per-kernel timing.
  *
  * Every kernel launch of the library increments a process-wide counter.
+ * The hot-path kernels (summaries, routing, tensor-core attention) are
+ * launched with programmatic stream serialization: each may be scheduled
+ * while the kernel before it on the stream drains, and waits for that
+ * kernel's completion on the device before touching memory.
  * When timing is enabled, each launch is bracketed by two CUDA events
  * recorded on its stream (as external event nodes while the stream is being
  * captured into a CUDA graph, so graph replays are timed too).  Events come
@@ -319,6 +323,12 @@ HGA_API hga_status_t hga_timing_get(int kind, double* ms, uint64_t* launches);
 
 /* Zeroes the per-kind totals. */
 HGA_API void hga_timing_reset(void);
+
+/* Restricts timing to the kinds whose bit (1u << kind) is set in `mask`
+ * (initially all).  Launches of other kinds are counted but not bracketed,
+ * so they keep their programmatic dependency on the kernel before them
+ * (an event between two kernels orders them fully). */
+HGA_API void hga_timing_kinds(uint32_t mask);
 
 #ifdef __cplusplus
 }
