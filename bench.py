@@ -116,11 +116,36 @@ def barrier(world: int, device=None):
 # ----------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clock and clock-event reasons sampled during the timed region (read
+    only).  NVML polled every 5 ms from a thread; nvidia-smi at 100 ms if the
+    NVML binding is missing."""
+
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = (("sw_power_cap", 0x4), ("hw_slowdown", 0x8),
+                   ("sw_thermal_slowdown", 0x20), ("hw_thermal_slowdown", 0x40))
 
     def __init__(self, gpu_id=None):
+        self.proc = self.thread = None
+        self.samples = []
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = (pynvml.nvmlDeviceGetHandleByUUID(gpu_id) if gpu_id
+                 else pynvml.nvmlDeviceGetHandleByIndex(0))
+            self.nvml, self.handle = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nvml = None
+        if self.nvml is not None:
+            import threading
+            self.stop_evt = threading.Event()
+            self.sample()
+            self.thread = threading.Thread(target=self.poll, daemon=True)
+            self.thread.start()
+            return
         self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                "-lms", "100"]
@@ -131,7 +156,32 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def sample(self):
+        nv, h = self.nvml, self.handle
+        try:
+            mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.samples.append((float(mhz), int(get(h))))
+        except Exception:
+            pass
+
+    def poll(self):
+        while not self.stop_evt.wait(0.005):
+            self.sample()
+
     def stop(self):
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
+            self.sample()
+            if not self.samples:
+                return None
+            reasons = {name for _, bits in self.samples for name, bit in self.REASON_BITS
+                       if bits & bit}
+            return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                    "sm_max_mhz": float(self.max_mhz), "samples": len(self.samples),
+                    "reasons": sorted(reasons), "source": "nvml, 5 ms"}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -157,7 +207,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
-                "reasons": sorted(reasons)}
+                "reasons": sorted(reasons), "source": "nvidia-smi, 100 ms"}
 
 
 # ----------------------------------------------------------------------------
@@ -543,36 +593,45 @@ def run_gpu(args, rank, world, local):
     value = job_throughput(tokens_per_step, args.steps, world, total_ms)
 
     # per-kernel table and the dominant kernel's roofline: in graph mode the
-    # table comes from the fully bracketed graph, the dominant kernel's
-    # launch time from the timed replays
+    # table comes from the fully bracketed graph (3 untimed replays), the
+    # dominant kernel's launch time from the timed replays
+    pk = peaks()
+    pcie_peak = []
+
+    def roof(bound):
+        """(peak, unit, scale to that unit, note) for a bound."""
+        if bound == "tensor":
+            return pk["tc_sustained"], "TFLOP/s", 1e12, f"bf16 dense, sustained ({pk['source']})"
+        if bound == "alu":
+            return (FP32_ALU_TFLOPS, "TFLOP/s", 1e12,
+                    "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz")
+        if bound == "pcie":
+            if not pcie_peak:
+                pcie_peak.append(round(pcie_probe(device), 2))
+            return (pcie_peak[0], "GB/s", 1e9,
+                    "pinned host-to-device cudaMemcpyAsync probe, 256 MiB, best of 5")
+        return pk["hbm"], "GB/s", 1e9, f"HBM copy ({pk['source']})"
+
     table = timing_table()
-    shown = table_all if table_all is not None else table
+    shown, reps = (table_all, 3) if table_all is not None else (table, args.steps)
     kernels = {}
+    tot_ms = max(sum(v[0] for v in shown.values()), 1e-12)
     for name, (ms, n) in shown.items():
-        kernels[name] = {"launches": n, "ms_total": round(ms, 4),
-                         "share": round(ms / max(sum(v[0] for v in shown.values()), 1e-12), 4)}
+        work, unit, bound = kernel_work(name, w, sels, unique_groups)
+        per_launch = work / (n / reps)
+        peak, punit, scale, _ = roof(bound)
+        achieved = per_launch / (ms / n / 1e3) / scale
+        kernels[name] = {"launches": n, "ms_total": round(ms, 4), "share": round(ms / tot_ms, 4),
+                         "avg_us": round(ms / n * 1e3, 3), "bound": bound,
+                         "achieved": round(achieved, 3), "unit": punit,
+                         "frac": round(achieved / peak, 4)}
     dom = max(table, key=lambda k: table[k][0])
     dom_ms, dom_n = table[dom]
     work, unit, bound = kernel_work(dom, w, sels, unique_groups)
     work_per_launch = work / (dom_n / args.steps)
-    pk = peaks()
     avg_s = dom_ms / dom_n / 1e3
-    if bound == "tensor":
-        achieved = work_per_launch / avg_s / 1e12
-        peak, punit = pk["tc_sustained"], "TFLOP/s"
-        peak_note = f"bf16 dense, sustained ({pk['source']})"
-    elif bound == "alu":
-        achieved = work_per_launch / avg_s / 1e12
-        peak, punit = FP32_ALU_TFLOPS, "TFLOP/s"
-        peak_note = "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz"
-    elif bound == "pcie":
-        achieved = work_per_launch / avg_s / 1e9
-        peak, punit = round(pcie_probe(device), 2), "GB/s"
-        peak_note = "pinned host-to-device cudaMemcpyAsync probe, 256 MiB, best of 5"
-    else:
-        achieved = work_per_launch / avg_s / 1e9
-        peak, punit = pk["hbm"], "GB/s"
-        peak_note = f"HBM copy ({pk['source']})"
+    peak, punit, scale, peak_note = roof(bound)
+    achieved = work_per_launch / avg_s / scale
     roofline = {"kernel": dom, "bound": bound, "achieved": round(achieved, 3),
                 "peak": peak, "unit": punit, "frac": round(achieved / peak, 4),
                 "traffic": measured_traffic(dom, args.workload),
