@@ -74,39 +74,6 @@ struct DqShared {
   uint8_t tile_mask[kMaxTiles];
 };
 
-// Builds the key-tile schedule of query block j exactly as the forward does:
-// valid selected groups in order, last routed tile padded with the first
-// valid group (masked), then the own block.  Executed by one full warp.
-template <typename SH>
-__device__ __forceinline__ void build_schedule(SH& sh, const int32_t* srow, int topk_groups,
-                                               int64_t own_blk, int lane) {
-  int n_valid = 0;
-  for (int c0 = 0; c0 < topk_groups; c0 += 32) {
-    const int idx = c0 + lane;
-    const int g = idx < topk_groups ? srow[idx] : -1;
-    bool ok = false;
-    if (idx < topk_groups && g != -1) {
-      ok = g >= 0 && int64_t(g) < own_blk * kGroupsPerBlock;
-      if (!ok) latch_status(HGA_ERR_DEVICE_CHECK);
-    }
-    const unsigned ball = __ballot_sync(0xffffffffu, ok);
-    if (ok) sh.grp[n_valid + __popc(ball & ((1u << lane) - 1u))] = g;
-    n_valid += __popc(ball);
-  }
-  __syncwarp();
-  const int n_rt = (n_valid + 7) / 8;
-  for (int i = n_valid + lane; i < n_rt * 8; i += 32) sh.grp[i] = sh.grp[0];
-  for (int t = lane; t < n_rt; t += 32) {
-    const int left = n_valid - 8 * t;
-    sh.tile_mask[t] = left >= 8 ? 0xffu : uint8_t((1u << left) - 1u);
-  }
-  for (int i = lane; i < 8; i += 32) sh.grp[n_rt * 8 + i] = int(own_blk * kGroupsPerBlock + i);
-  if (lane == 0) {
-    sh.tile_mask[n_rt] = 0xffu;
-    sh.n_tiles = n_rt + 1;
-  }
-}
-
 constexpr int kDqProducers = 96;  // warps 0, 2, 3
 
 template <int MT>
@@ -155,13 +122,27 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
   // the previous kernel may still hold this SM's tensor memory or write
   // this kernel's inputs: wait for it before allocating or reading
   pdl_wait();
+  if (tid == 0) {
+    // Q and dO first: they do not depend on the selection
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_do);
+    mbar_arrive_expect_tx(&sh.q_full, MT * 65536);
+    for (int g = 0; g < G; ++g) {
+      const int32_t row = int32_t((int64_t(b) * n_q_heads + h * G + g) * s_len + j * kQBlock);
+      for (int hf = 0; hf < 2; ++hf) {
+        const uint32_t off = (g >> 1) * 32768 + hf * 16384 + (g & 1) * 8192;
+        tma_load_2d(smem + L::kQ + off, &tm_q, &sh.q_full, hf * 64, row);
+        tma_load_2d(smem + L::kDO + off, &tm_do, &sh.q_full, hf * 64, row);
+      }
+    }
+  }
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, L::kTmemCols);
     tmem_relinquish();
   }
   if (warp == 0)
-    build_schedule(sh, sel_grp + ((int64_t(b) * n_kv_heads + h) * n_qb + j) * topk_groups,
-                   topk_groups, own_blk, lane);
+    build_tile_schedule(sh, sel_grp + ((int64_t(b) * n_kv_heads + h) * n_qb + j) * topk_groups,
+                        topk_groups, own_blk, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -171,19 +152,6 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
   if (warp == 0 || warp == 2 || warp == 3) {
     // ---------------- producers: Q, dO by TMA; K/V groups by cp.async ----------------
     const int ptid = warp == 0 ? lane : 32 * (warp - 1) + lane;
-    if (tid == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_do);
-      mbar_arrive_expect_tx(&sh.q_full, MT * 65536);
-      for (int g = 0; g < G; ++g) {
-        const int32_t row = int32_t((int64_t(b) * n_q_heads + h * G + g) * s_len + j * kQBlock);
-        for (int hf = 0; hf < 2; ++hf) {
-          const uint32_t off = (g >> 1) * 32768 + hf * 16384 + (g & 1) * 8192;
-          tma_load_2d(smem + L::kQ + off, &tm_q, &sh.q_full, hf * 64, row);
-          tma_load_2d(smem + L::kDO + off, &tm_do, &sh.q_full, hf * 64, row);
-        }
-      }
-    }
     const __nv_bfloat16* kh = k + (int64_t(b) * n_kv_heads + h) * ctx_cap * kD;
     const __nv_bfloat16* vh = v + (int64_t(b) * n_kv_heads + h) * ctx_cap * kD;
     for (int t = 0; t < n_tiles; ++t) {
@@ -484,6 +452,22 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
   // the previous kernel may still hold this SM's tensor memory or write
   // this kernel's inputs: wait for it before allocating or reading
   pdl_wait();
+  if (tid == 0) {
+    // this block's keys and values first: they do not depend on the selection
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_do);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    const int32_t krow = int32_t((int64_t(b) * n_kv_heads + h) * ctx_cap + gblk * kBlock);
+    mbar_arrive_expect_tx(&sh.kv_full, 32768);
+    for (int gi = 0; gi < 8; ++gi)
+      for (int hf = 0; hf < 2; ++hf) {
+        tma_load_2d(smem + L::kK + hf * 8192 + gi * 1024, &tm_k, &sh.kv_full, hf * 64,
+                    krow + gi * kGroup);
+        tma_load_2d(smem + L::kV + hf * 8192 + gi * 1024, &tm_v, &sh.kv_full, hf * 64,
+                    krow + gi * kGroup);
+      }
+  }
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, L::kTmemCols);
     tmem_relinquish();
@@ -491,13 +475,27 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
   __syncthreads();
   // which later query blocks of the segment selected groups of this block
   const int32_t* sel_bh = sel_grp + (int64_t(b) * n_kv_heads + h) * n_qb * topk_groups;
-  for (int idx = tid; idx < n_qb * topk_groups; idx += blockDim.x) {
-    const int jj = idx / topk_groups;
-    if (jj <= kb) continue;
-    const int g = sel_bh[idx];
-    const int64_t own_jj = q_begin / kBlock + jj;
-    if (g >= 0 && int64_t(g) < own_jj * kGroupsPerBlock && int64_t(g) / kGroupsPerBlock == gblk)
-      atomicOr(&sh.masks[jj], 1 << (g % kGroupsPerBlock));
+  // (only query blocks after kb can select it; 4 loads per thread in flight)
+  {
+    const int first = (kb + 1) * topk_groups, total = n_qb * topk_groups;
+    const int nt = blockDim.x;
+    for (int base = first + tid; base < total; base += 4 * nt) {
+      int gv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int idx = base + u * nt;
+        gv[u] = idx < total ? sel_bh[idx] : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int idx = base + u * nt, g = gv[u];
+        if (idx >= total || g < 0) continue;
+        const int jj = idx / topk_groups;
+        const int64_t own_jj = q_begin / kBlock + jj;
+        if (int64_t(g) < own_jj * kGroupsPerBlock && int64_t(g) / kGroupsPerBlock == gblk)
+          atomicOr(&sh.masks[jj], 1 << (g % kGroupsPerBlock));
+      }
+    }
   }
   __syncthreads();
   if (warp == 0) {
@@ -519,22 +517,6 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
 
   if (warp == 0) {
     // ---------------- TMA producer (whole warp; one elected lane issues) ----
-    if (elect_one()) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_do);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      const int32_t krow = int32_t((int64_t(b) * n_kv_heads + h) * ctx_cap + gblk * kBlock);
-      mbar_arrive_expect_tx(&sh.kv_full, 32768);
-      for (int gi = 0; gi < 8; ++gi)
-        for (int hf = 0; hf < 2; ++hf) {
-          tma_load_2d(smem + L::kK + hf * 8192 + gi * 1024, &tm_k, &sh.kv_full, hf * 64,
-                      krow + gi * kGroup);
-          tma_load_2d(smem + L::kV + hf * 8192 + gi * 1024, &tm_v, &sh.kv_full, hf * 64,
-                      krow + gi * kGroup);
-        }
-    }
-    __syncwarp();
     int issued = 0;
     for (int it = 0; it < n_items; ++it) {
       const int u = it & 1;

@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
   volatile int* abort = &sh.abort;
   pdl_launch_dependents();
 
-  // ---- set-up: barriers, TMEM, the tile schedule -------------------------
+  // ---- set-up: barriers, the Q load, TMEM, the tile schedule -------------
   if (tid == 0) {
     mbar_init(&sh.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
@@ -123,40 +123,27 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
   // the previous kernel may still hold this SM's tensor memory or write
   // this kernel's inputs: wait for it before allocating or reading
   pdl_wait();
+  if (tid == 0) {
+    // Q first: it does not depend on the selection
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    mbar_arrive_expect_tx(&sh.q_full, MT * 32768);
+    for (int g = 0; g < 2 * MT; ++g) {
+      const int32_t row = int32_t((int64_t(b) * n_q_heads + head0 + g) * s_len + j * kQBlock);
+      for (int hf = 0; hf < 2; ++hf) {
+        uint8_t* dst = smem + L::kQ + (g >> 1) * 32768 + hf * 16384 + (g & 1) * 8192;
+        tma_load_2d(dst, &tm_q, &sh.q_full, hf * 64, row);
+      }
+    }
+  }
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, L::kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 0) {
-    // compact the valid selected groups (ascending order kept), pad the last
-    // routed tile with copies of the first valid group (masked out later)
-    const int32_t* srow = sel_grp + ((int64_t(b) * n_kv_heads + h) * n_qb + j) * topk_groups;
-    int n_valid = 0;
-    for (int c0 = 0; c0 < topk_groups; c0 += 32) {
-      const int idx = c0 + lane;
-      const int g = idx < topk_groups ? srow[idx] : -1;
-      bool ok = false;
-      if (idx < topk_groups && g != -1) {
-        ok = g >= 0 && int64_t(g) < own_blk * kGroupsPerBlock;
-        if (!ok) latch_status(HGA_ERR_DEVICE_CHECK);
-      }
-      const unsigned ball = __ballot_sync(0xffffffffu, ok);
-      if (ok) sh.grp[n_valid + __popc(ball & ((1u << lane) - 1u))] = g;
-      n_valid += __popc(ball);
-    }
-    __syncwarp();
-    const int n_rt = (n_valid + 7) / 8;
-    for (int i = n_valid + lane; i < n_rt * 8; i += 32) sh.grp[i] = sh.grp[0];
-    for (int t = lane; t < n_rt; t += 32) {
-      const int left = n_valid - 8 * t;
-      sh.tile_mask[t] = left >= 8 ? 0xffu : uint8_t((1u << left) - 1u);
-    }
-    for (int i = lane; i < 8; i += 32) sh.grp[n_rt * 8 + i] = int(own_blk * kGroupsPerBlock + i);
-    if (lane == 0) {
-      sh.tile_mask[n_rt] = 0xffu;
-      sh.n_tiles = n_rt + 1;
-    }
-  }
+  if (warp == 0)
+    build_tile_schedule(sh, sel_grp + ((int64_t(b) * n_kv_heads + h) * n_qb + j) * topk_groups,
+                        topk_groups, own_blk, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -166,22 +153,8 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
   if (warp == 0) {
     // ---------------- TMA producer (whole warp; one elected lane issues) ----
     // K/V tile layout: group gi at gi * 2048: [d half][8 rows][128 B], one
-    // 3-D box (64 columns x 8 rows x 2 halves) per group and tensor
-    if (elect_one()) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(&sh.q_full, MT * 32768);
-      for (int g = 0; g < 2 * MT; ++g) {
-        const int32_t row =
-            int32_t((int64_t(b) * n_q_heads + head0 + g) * s_len + j * kQBlock);
-        for (int hf = 0; hf < 2; ++hf) {
-          uint8_t* dst = smem + L::kQ + (g >> 1) * 32768 + hf * 16384 + (g & 1) * 8192;
-          tma_load_2d(dst, &tm_q, &sh.q_full, hf * 64, row);
-        }
-      }
-    }
-    __syncwarp();
+    // 3-D box (64 columns x 8 rows x 2 halves) per group and tensor (Q was
+    // issued during set-up)
     const int64_t kv_row0 = (int64_t(b) * n_kv_heads + h) * ctx_cap;
     int issued = 0;
     for (int t = 0; t < n_tiles; ++t) {
