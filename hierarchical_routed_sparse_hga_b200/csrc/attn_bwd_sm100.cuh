@@ -14,8 +14,12 @@
 //   shared memory), and dQ += dS K accumulates in TMEM; dQ = scale * dQ at the
 //   end.  D = rowsum(dO * O) is computed here and saved for the next kernel.
 //
-// attn_bwd_dkdv_tc_kernel -- one CTA per (batch, KV head, 64-key block of the
-//   active segment).  It visits, in increasing order, every query block of the
+// attn_bwd_dkdv_tc_kernel -- persistent: at most one CTA per SM, each taking
+//   work units (batch, KV head, 64-key block of the active segment) from a
+//   counter in the workspace (zeroed by the dQ kernel) until none is left,
+//   the key blocks that the most query blocks can select first, so the
+//   uneven units balance out over the SMs.  Per unit it visits, in
+//   increasing order, every query block of the
 //   segment that attends to the block (its own block causally, later blocks
 //   through the groups of it they selected) and accumulates the transposed
 //   gradients dV^T += dO^T P and dK^T += Q^T dS in TMEM (M = head_dim = 128,
@@ -86,7 +90,8 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
                           int topk_groups, const int32_t* __restrict__ sel_grp, float scale,
                           float scale_log2, const __nv_bfloat16* __restrict__ o,
                           const __nv_bfloat16* __restrict__ d_o, const float* __restrict__ lse,
-                          __nv_bfloat16* __restrict__ dq, float* __restrict__ dvec) {
+                          __nv_bfloat16* __restrict__ dq, float* __restrict__ dvec,
+                          int* __restrict__ unit_counter) {
   using L = DqLayout<MT>;
   constexpr int G = 2 * MT;
   extern __shared__ uint8_t dsmem_raw[];
@@ -122,6 +127,8 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
   // the previous kernel may still hold this SM's tensor memory or write
   // this kernel's inputs: wait for it before allocating or reading
   pdl_wait();
+  // the dK/dV kernel that follows takes its work units from this counter
+  if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) *unit_counter = 0;
   if (tid == 0) {
     // Q and dO first: they do not depend on the selection
     prefetch_tmap(&tm_q);
@@ -405,6 +412,7 @@ struct KvShared {
   uint32_t tmem_base;
   int abort;
   int n_items;
+  int unit;
   int masks[64];
   int js[64];
 };
@@ -415,11 +423,11 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
                             const __grid_constant__ CUtensorMap tm_do,
                             const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, int64_t ctx_cap,
-                            int64_t q_begin, int s_len, int n_q_heads, int n_kv_heads,
+                            int64_t q_begin, int s_len, int batch, int n_q_heads, int n_kv_heads,
                             int topk_groups, const int32_t* __restrict__ sel_grp, float scale,
                             float scale_log2, const float* __restrict__ lse,
                             const float* __restrict__ dvec, __nv_bfloat16* __restrict__ dk,
-                            __nv_bfloat16* __restrict__ dv) {
+                            __nv_bfloat16* __restrict__ dv, int* __restrict__ unit_counter) {
   using L = KvLayout;
   constexpr int G = 2 * MT;
   extern __shared__ uint8_t dsmem_raw[];
@@ -430,13 +438,11 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
   const uint32_t sQD = smem_u32(smem + L::kQD), sPD = smem_u32(smem + L::kPD);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int n_qb = s_len / kQBlock;
-  const int64_t gblk = q_begin / kBlock + kb;  // global index of this key block
+  const int n_bh = batch * n_kv_heads, n_units = n_qb * n_bh;
   volatile int* abort = &sh.abort;
   pdl_launch_dependents();
 
-  for (int i = tid; i < 64; i += blockDim.x) sh.masks[i] = (i == kb) ? 0xff : 0;
   if (tid == 0) {
     mbar_init(&sh.kv_full, 1);
     for (int u = 0; u < 2; ++u) {
@@ -450,249 +456,280 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
     fence_barrier_init();
   }
   // the previous kernel may still hold this SM's tensor memory or write
-  // this kernel's inputs: wait for it before allocating or reading
+  // this kernel's inputs (the dQ kernel zeroes the unit counter): wait for it
   pdl_wait();
   if (tid == 0) {
-    // this block's keys and values first: they do not depend on the selection
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_do);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
-    const int32_t krow = int32_t((int64_t(b) * n_kv_heads + h) * ctx_cap + gblk * kBlock);
-    mbar_arrive_expect_tx(&sh.kv_full, 32768);
-    for (int gi = 0; gi < 8; ++gi)
-      for (int hf = 0; hf < 2; ++hf) {
-        tma_load_2d(smem + L::kK + hf * 8192 + gi * 1024, &tm_k, &sh.kv_full, hf * 64,
-                    krow + gi * kGroup);
-        tma_load_2d(smem + L::kV + hf * 8192 + gi * 1024, &tm_v, &sh.kv_full, hf * 64,
-                    krow + gi * kGroup);
-      }
   }
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, L::kTmemCols);
     tmem_relinquish();
   }
-  __syncthreads();
-  // which later query blocks of the segment selected groups of this block
-  const int32_t* sel_bh = sel_grp + (int64_t(b) * n_kv_heads + h) * n_qb * topk_groups;
-  // (only query blocks after kb can select it; 4 loads per thread in flight)
-  {
-    const int first = (kb + 1) * topk_groups, total = n_qb * topk_groups;
-    const int nt = blockDim.x;
-    for (int base = first + tid; base < total; base += 4 * nt) {
-      int gv[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int idx = base + u * nt;
-        gv[u] = idx < total ? sel_bh[idx] : -1;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int idx = base + u * nt, g = gv[u];
-        if (idx >= total || g < 0) continue;
-        const int jj = idx / topk_groups;
-        const int64_t own_jj = q_begin / kBlock + jj;
-        if (int64_t(g) < own_jj * kGroupsPerBlock && int64_t(g) / kGroupsPerBlock == gblk)
-          atomicOr(&sh.masks[jj], 1 << (g % kGroupsPerBlock));
-      }
-    }
-  }
-  __syncthreads();
-  if (warp == 0) {
-    int n = 0;
-    for (int c0 = 0; c0 < n_qb; c0 += 32) {
-      const int jj = c0 + lane;
-      const bool on = jj < n_qb && jj >= kb && sh.masks[jj] != 0;
-      const unsigned ball = __ballot_sync(0xffffffffu, on);
-      if (on) sh.js[n + __popc(ball & ((1u << lane) - 1u))] = jj;
-      n += __popc(ball);
-    }
-    if (lane == 0) sh.n_items = n * MT;
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
-  const int n_items = sh.n_items;
 
-  if (warp == 0) {
-    // ---------------- TMA producer (whole warp; one elected lane issues) ----
-    int issued = 0;
-    for (int it = 0; it < n_items; ++it) {
-      const int u = it & 1;
-      const bool free_ok = it < 2 || mbar_wait(&sh.qd_empty[u], ((it >> 1) - 1) & 1, abort);
-      if (!__all_sync(kFullMask, free_ok)) break;
-      const int jj = sh.js[it / MT], m = it % MT;
-      if (elect_one()) {
-        mbar_arrive_expect_tx(&sh.qd_full[u], 65536);
-        uint8_t* dst = smem + L::kQD + u * L::kQDBytes;
-        for (int g = 0; g < 2; ++g) {
-          const int32_t row =
-              int32_t((int64_t(b) * n_q_heads + h * G + 2 * m + g) * s_len + jj * kQBlock);
-          for (int hf = 0; hf < 2; ++hf) {
-            tma_load_2d(dst + hf * 16384 + g * 8192, &tm_q, &sh.qd_full[u], hf * 64, row);
-            tma_load_2d(dst + 32768 + hf * 16384 + g * 8192, &tm_do, &sh.qd_full[u], hf * 64,
-                        row);
-          }
+  // Work units (key block kb, batch x KV head) in order of kb, so the blocks
+  // that the most query blocks can select come first; each CTA takes the
+  // next unit from the counter until none is left.  Item indices run on
+  // across units (it_base), so every barrier's phase sequence continues.
+  int it_base = 0;
+  for (int un = 0;; ++un) {
+    if (tid == 0) sh.unit = *abort ? n_units : atomicAdd(unit_counter, 1);
+    for (int i = tid; i < 64; i += blockDim.x) sh.masks[i] = 0;
+    __syncthreads();
+    const int w = sh.unit;
+    if (w >= n_units) break;
+    const int kb = w / n_bh, bh = w % n_bh, b = bh / n_kv_heads, h = bh % n_kv_heads;
+    const int64_t gblk = q_begin / kBlock + kb;  // global index of this key block
+    if (tid == 0) {
+      // this block's keys and values first: they do not depend on the selection
+      // (the previous unit's MMAs have all completed: see the end of the loop)
+      sh.masks[kb] = 0xff;
+      const int32_t krow = int32_t((int64_t(b) * n_kv_heads + h) * ctx_cap + gblk * kBlock);
+      mbar_arrive_expect_tx(&sh.kv_full, 32768);
+      for (int gi = 0; gi < 8; ++gi)
+        for (int hf = 0; hf < 2; ++hf) {
+          tma_load_2d(smem + L::kK + hf * 8192 + gi * 1024, &tm_k, &sh.kv_full, hf * 64,
+                      krow + gi * kGroup);
+          tma_load_2d(smem + L::kV + hf * 8192 + gi * 1024, &tm_v, &sh.kv_full, hf * 64,
+                      krow + gi * kGroup);
+        }
+    }
+    // which later query blocks of the segment selected groups of this block
+    // (only query blocks after kb can; 4 loads per thread in flight)
+    const int32_t* sel_bh = sel_grp + (int64_t(b) * n_kv_heads + h) * n_qb * topk_groups;
+    {
+      const int first = (kb + 1) * topk_groups, total = n_qb * topk_groups;
+      const int nt = blockDim.x;
+      for (int base = first + tid; base < total; base += 4 * nt) {
+        int gv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int idx = base + u * nt;
+          gv[u] = idx < total ? sel_bh[idx] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int idx = base + u * nt, g = gv[u];
+          if (idx >= total || g < 0) continue;
+          const int jj = idx / topk_groups;
+          const int64_t own_jj = q_begin / kBlock + jj;
+          if (int64_t(g) < own_jj * kGroupsPerBlock && int64_t(g) / kGroupsPerBlock == gblk)
+            atomicOr(&sh.masks[jj], 1 << (g % kGroupsPerBlock));
         }
       }
-      __syncwarp();
-      issued = it + 1;
     }
-    if (lane == 0) {
-      int never = 0;
-      mbar_wait(&sh.kv_full, 0, &never);
-      for (int it = issued - 1; it >= 0 && it >= issued - 2; --it)
-        mbar_wait(&sh.qd_full[it & 1], (it >> 1) & 1, &never);
+    __syncthreads();
+    if (warp == 0) {
+      int n = 0;
+      for (int c0 = 0; c0 < n_qb; c0 += 32) {
+        const int jj = c0 + lane;
+        const bool on = jj < n_qb && jj >= kb && sh.masks[jj] != 0;
+        const unsigned ball = __ballot_sync(0xffffffffu, on);
+        if (on) sh.js[n + __popc(ball & ((1u << lane) - 1u))] = jj;
+        n += __popc(ball);
+      }
+      if (lane == 0) sh.n_items = n * MT;  // >= MT: the own block is always in
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer (event driven; whole warp, one lane issues) --
-    constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);
-    constexpr uint32_t idesc_t = idesc_bf16_f32(128, 64, 1, 1);
-    bool ok = __all_sync(kFullMask, mbar_wait(&sh.kv_full, 0, abort));
-    bool issued_any = false;
-    int next_s = 0, next_t = 0;  // items with S/dP issued, with dV/dK issued
-    long long t0 = clock64();
-    while (ok && next_t < n_items) {
-      bool progressed = false;
-      if (next_t < next_s &&
-          __all_sync(kFullMask, mbar_test(&sh.pds_full[next_t & 1], (next_t >> 1) & 1))) {
-        // dV^T += dO^T P and dK^T += Q^T dS over this item's 128 query rows
-        const int u = next_t & 1;
-        const uint32_t qd = sQD + u * L::kQDBytes, pd = sPD + u * L::kPDBytes;
-        tc_fence_after();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const int n_items = sh.n_items;
+
+    if (warp == 0) {
+      // ---------------- TMA producer (whole warp; one elected lane issues) --
+      int issued = 0;
+      for (int it = 0; it < n_items; ++it) {
+        const int gi = it_base + it, u = gi & 1;
+        const bool free_ok =
+            gi < 2 || mbar_wait(&sh.qd_empty[u], ((gi >> 1) - 1) & 1, abort);
+        if (!__all_sync(kFullMask, free_ok)) break;
+        const int jj = sh.js[it / MT], m = it % MT;
         if (elect_one()) {
-#pragma unroll
-          for (int s8 = 0; s8 < 8; ++s8) {
-            const uint32_t ro = s8 * 2048;
-            const uint32_t acc = (next_t > 0 || s8 > 0) ? 1u : 0u;
-            mma_bf16(tmem + L::kColDV, smem_desc_sw128(qd + 32768 + ro, 16384, 1024),
-                     smem_desc_sw128(pd + ro, 8192, 1024), idesc_t, acc);
-            mma_bf16(tmem + L::kColDK, smem_desc_sw128(qd + ro, 16384, 1024),
-                     smem_desc_sw128(pd + 16384 + ro, 8192, 1024), idesc_t, acc);
+          mbar_arrive_expect_tx(&sh.qd_full[u], 65536);
+          uint8_t* dst = smem + L::kQD + u * L::kQDBytes;
+          for (int g = 0; g < 2; ++g) {
+            const int32_t row =
+                int32_t((int64_t(b) * n_q_heads + h * G + 2 * m + g) * s_len + jj * kQBlock);
+            for (int hf = 0; hf < 2; ++hf) {
+              tma_load_2d(dst + hf * 16384 + g * 8192, &tm_q, &sh.qd_full[u], hf * 64, row);
+              tma_load_2d(dst + 32768 + hf * 16384 + g * 8192, &tm_do, &sh.qd_full[u],
+                          hf * 64, row);
+            }
           }
-          mma_commit(&sh.qd_empty[u]);
         }
         __syncwarp();
-        ++next_t;
-        progressed = true;
+        issued = it + 1;
       }
-      // S/dP(i) into buffer i & 1, free once dV/dK(i-2) has been issued
-      // (its softmax has then finished with that buffer)
-      if (!progressed && next_s < n_items && next_s < next_t + 2 &&
-          __all_sync(kFullMask, mbar_test(&sh.qd_full[next_s & 1], (next_s >> 1) & 1))) {
-        const int u = next_s & 1;
-        const uint32_t qd = sQD + u * L::kQDBytes;
-        tc_fence_after();
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t ao = (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint32_t bo = (kk >> 2) * 8192 + (kk & 3) * 32;
-            mma_bf16(tmem + L::colS(u), smem_desc_sw128(qd + ao, 16, 1024),
-                     smem_desc_sw128(sK + bo, 16, 1024), idesc_s, kk > 0);
-            mma_bf16(tmem + L::colDP(u), smem_desc_sw128(qd + 32768 + ao, 16, 1024),
-                     smem_desc_sw128(sV + bo, 16, 1024), idesc_s, kk > 0);
-          }
-          mma_commit(&sh.sdp_full[u]);
+      // drain: wait (bounded, independent of abort) for the copies in flight
+      if (lane == 0) {
+        int never = 0;
+        mbar_wait(&sh.kv_full, un & 1, &never);
+        for (int it = issued - 1; it >= 0 && it >= issued - 2; --it) {
+          const int gi = it_base + it;
+          mbar_wait(&sh.qd_full[gi & 1], (gi >> 1) & 1, &never);
         }
-        __syncwarp();
-        ++next_s;
-        issued_any = true;
-        progressed = true;
       }
-      ok = warp_event_continue(progressed, t0, abort);
-    }
-    if (issued_any) {
+    } else if (warp == 1) {
+      // ---------------- MMA issuer (event driven; whole warp, one lane issues)
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);
+      constexpr uint32_t idesc_t = idesc_bf16_f32(128, 64, 1, 1);
+      bool ok = __all_sync(kFullMask, mbar_wait(&sh.kv_full, un & 1, abort));
+      int next_s = 0, next_t = 0;  // items with S/dP issued, with dV/dK issued
+      long long t0 = clock64();
+      while (ok && next_t < n_items) {
+        bool progressed = false;
+        const int gt = it_base + next_t, gs = it_base + next_s;
+        if (next_t < next_s &&
+            __all_sync(kFullMask, mbar_test(&sh.pds_full[gt & 1], (gt >> 1) & 1))) {
+          // dV^T += dO^T P and dK^T += Q^T dS over this item's 128 query rows
+          const int u = gt & 1;
+          const uint32_t qd = sQD + u * L::kQDBytes, pd = sPD + u * L::kPDBytes;
+          tc_fence_after();
+          if (elect_one()) {
+#pragma unroll
+            for (int s8 = 0; s8 < 8; ++s8) {
+              const uint32_t ro = s8 * 2048;
+              const uint32_t acc = (next_t > 0 || s8 > 0) ? 1u : 0u;
+              mma_bf16(tmem + L::kColDV, smem_desc_sw128(qd + 32768 + ro, 16384, 1024),
+                       smem_desc_sw128(pd + ro, 8192, 1024), idesc_t, acc);
+              mma_bf16(tmem + L::kColDK, smem_desc_sw128(qd + ro, 16384, 1024),
+                       smem_desc_sw128(pd + 16384 + ro, 8192, 1024), idesc_t, acc);
+            }
+            mma_commit(&sh.qd_empty[u]);
+          }
+          __syncwarp();
+          ++next_t;
+          progressed = true;
+        }
+        // S/dP(i) into buffer i & 1, free once dV/dK(i-2) has been issued
+        // (its softmax has then finished with that buffer)
+        if (!progressed && next_s < n_items && next_s < next_t + 2 &&
+            __all_sync(kFullMask, mbar_test(&sh.qd_full[gs & 1], (gs >> 1) & 1))) {
+          const int u = gs & 1;
+          const uint32_t qd = sQD + u * L::kQDBytes;
+          tc_fence_after();
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t ao = (kk >> 2) * 16384 + (kk & 3) * 32;
+              const uint32_t bo = (kk >> 2) * 8192 + (kk & 3) * 32;
+              mma_bf16(tmem + L::colS(u), smem_desc_sw128(qd + ao, 16, 1024),
+                       smem_desc_sw128(sK + bo, 16, 1024), idesc_s, kk > 0);
+              mma_bf16(tmem + L::colDP(u), smem_desc_sw128(qd + 32768 + ao, 16, 1024),
+                       smem_desc_sw128(sV + bo, 16, 1024), idesc_s, kk > 0);
+            }
+            mma_commit(&sh.sdp_full[u]);
+          }
+          __syncwarp();
+          ++next_s;
+          progressed = true;
+        }
+        ok = warp_event_continue(progressed, t0, abort);
+      }
+      // one mma_done phase per unit: every MMA of this unit has finished
+      // before its epilogue reads TMEM and before the next unit overwrites
+      // the tiles in shared memory (a commit with none pending arrives at once)
       if (elect_one()) mma_commit(&sh.mma_done);
       __syncwarp();
       int never = 0;
-      mbar_wait(&sh.mma_done, 0, &never);
-    }
-  } else if (warp >= 4) {
-    // ---------------- softmax (two warp groups, one per buffer) ----------------
-    const int u = (warp - 4) >> 2, wq = warp & 3;
-    const int row = wq * 32 + lane;
-    const int g = row >> 6, r = row & 63;
-    const uint32_t lane_addr = uint32_t(wq * 32) << 16;
-    const float2 c2 = make_float2(scale_log2, scale_log2);
-    bool ok = true;
-    uint8_t* prow = smem + L::kPD + u * L::kPDBytes + row * 128;
-    uint8_t* drow = prow + 16384;
-    for (int it = u; it < n_items && ok; it += 2) {
-      const int jj = sh.js[it / MT], m = it % MT;
-      const bool own = jj == kb;
-      const uint32_t mask = sh.masks[jj];
-      const int hq = h * G + 2 * m + g;
-      const int64_t rix = (int64_t(b) * n_q_heads + hq) * s_len + int64_t(jj) * kQBlock + r;
-      const float lse2 = lse[rix] * 1.4426950408889634f;
-      const float dsum = dvec[rix];
-      const float2 nl = make_float2(-lse2, -lse2), nd = make_float2(-dsum, -dsum);
-      if (!(ok = mbar_wait(&sh.sdp_full[u], (it >> 1) & 1, abort))) break;
-      tc_fence_after();
-      const bool full = !own && mask == 0xffu;
-#pragma unroll
-      for (int hb = 0; hb < 2; ++hb) {
-        float sv[32], dp[32];
-        tmem_ld32(tmem + lane_addr + L::colS(u) + hb * 32, sv);
-        tmem_ld32(tmem + lane_addr + L::colDP(u) + hb * 32, dp);
-        tmem_wait_ld();
-        if (!full) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int key = hb * 32 + i;
-            const bool valid = ((mask >> (key >> 3)) & 1u) && (!own || key <= r);
-            if (!valid) sv[i] = -INFINITY;
-          }
-        }
-        uint32_t pk[16], dk2[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float2 p = __ffma2_rn(make_float2(sv[i], sv[i + 1]), c2, nl);
-          p.x = ex2_approx(p.x);
-          p.y = ex2_approx(p.y);
-          const float2 d2 = __fmul2_rn(p, __fadd2_rn(make_float2(dp[i], dp[i + 1]), nd));
-          pk[i / 2] = pack_bf16x2(p.x, p.y);
-          dk2[i / 2] = pack_bf16x2(d2.x, d2.y);
-        }
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int c = hb * 4 + cc;
-          const int off = (c ^ (row & 7)) << 4;
-          *reinterpret_cast<uint4*>(prow + off) =
-              make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-          *reinterpret_cast<uint4*>(drow + off) =
-              make_uint4(dk2[4 * cc], dk2[4 * cc + 1], dk2[4 * cc + 2], dk2[4 * cc + 3]);
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&sh.pds_full[u]);
-    }
-    // epilogue: warp group 0 owns TMEM lanes 0..127 = the 128 head dims
-    if (u == 0) {
-      // mma_done completes exactly once, after the last dV/dK MMA; a parity
-      // wait on a per-buffer barrier here could pass a phase early, because
-      // the earlier phase of that barrier need not have completed yet
-      if (ok) ok = mbar_wait(&sh.mma_done, 0, abort);
-      if (ok) {
+      mbar_wait(&sh.mma_done, un & 1, &never);
+    } else if (warp >= 4) {
+      // ---------------- softmax (two warp groups, one per buffer) --------------
+      const int u = (warp - 4) >> 2, wq = warp & 3;
+      const int row = wq * 32 + lane;
+      const int g = row >> 6, r = row & 63;
+      const uint32_t lane_addr = uint32_t(wq * 32) << 16;
+      const float2 c2 = make_float2(scale_log2, scale_log2);
+      bool ok = true;
+      uint8_t* prow = smem + L::kPD + u * L::kPDBytes + row * 128;
+      uint8_t* drow = prow + 16384;
+      // this group's items: those whose running index has parity u
+      for (int it = (u - it_base) & 1; it < n_items && ok; it += 2) {
+        const int gi = it_base + it;
+        const int jj = sh.js[it / MT], m = it % MT;
+        const bool own = jj == kb;
+        const uint32_t mask = sh.masks[jj];
+        const int hq = h * G + 2 * m + g;
+        const int64_t rix = (int64_t(b) * n_q_heads + hq) * s_len + int64_t(jj) * kQBlock + r;
+        const float lse2 = lse[rix] * 1.4426950408889634f;
+        const float dsum = dvec[rix];
+        const float2 nl = make_float2(-lse2, -lse2), nd = make_float2(-dsum, -dsum);
+        if (!(ok = mbar_wait(&sh.sdp_full[u], (gi >> 1) & 1, abort))) break;
         tc_fence_after();
-        const int dcol = row;
-        const int64_t base = ((int64_t(b) * n_kv_heads + h) * s_len + int64_t(kb) * kBlock) * kD;
-        for (int c = 0; c < 64; c += 32) {
-          float vv[32], kk[32];
-          tmem_ld32(tmem + lane_addr + L::kColDV + c, vv);
-          tmem_ld32(tmem + lane_addr + L::kColDK + c, kk);
-          tmem_wait_ld();
+        const bool full = !own && mask == 0xffu;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int64_t at = base + int64_t(c + i) * kD + dcol;
-            dv[at] = __float2bfloat16_rn(n_items > 0 ? vv[i] : 0.f);
-            dk[at] = __float2bfloat16_rn(n_items > 0 ? kk[i] * scale : 0.f);
+        for (int hb = 0; hb < 2; ++hb) {
+          float sv[32], dp[32];
+          tmem_ld32(tmem + lane_addr + L::colS(u) + hb * 32, sv);
+          tmem_ld32(tmem + lane_addr + L::colDP(u) + hb * 32, dp);
+          tmem_wait_ld();
+          if (!full) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int key = hb * 32 + i;
+              const bool valid = ((mask >> (key >> 3)) & 1u) && (!own || key <= r);
+              if (!valid) sv[i] = -INFINITY;
+            }
+          }
+          uint32_t pk[16], dk2[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float2 p = __ffma2_rn(make_float2(sv[i], sv[i + 1]), c2, nl);
+            p.x = ex2_approx(p.x);
+            p.y = ex2_approx(p.y);
+            const float2 d2 = __fmul2_rn(p, __fadd2_rn(make_float2(dp[i], dp[i + 1]), nd));
+            pk[i / 2] = pack_bf16x2(p.x, p.y);
+            dk2[i / 2] = pack_bf16x2(d2.x, d2.y);
+          }
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            const int c = hb * 4 + cc;
+            const int off = (c ^ (row & 7)) << 4;
+            *reinterpret_cast<uint4*>(prow + off) =
+                make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+            *reinterpret_cast<uint4*>(drow + off) =
+                make_uint4(dk2[4 * cc], dk2[4 * cc + 1], dk2[4 * cc + 2], dk2[4 * cc + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sh.pds_full[u]);
+      }
+      // epilogue: warp group 0 owns TMEM lanes 0..127 = the 128 head dims
+      if (u == 0) {
+        if (ok) ok = mbar_wait(&sh.mma_done, un & 1, abort);
+        if (ok) {
+          tc_fence_after();
+          const int dcol = row;
+          const int64_t base =
+              ((int64_t(b) * n_kv_heads + h) * s_len + int64_t(kb) * kBlock) * kD;
+          for (int c = 0; c < 64; c += 32) {
+            float vv[32], kk[32];
+            tmem_ld32(tmem + lane_addr + L::kColDV + c, vv);
+            tmem_ld32(tmem + lane_addr + L::kColDK + c, kk);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int64_t at = base + int64_t(c + i) * kD + dcol;
+              dv[at] = __float2bfloat16_rn(vv[i]);
+              dk[at] = __float2bfloat16_rn(kk[i] * scale);
+            }
           }
         }
       }
     }
+    it_base += n_items;
+    // end of the unit: every role is done with its barriers, tiles and TMEM
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (*abort) break;
   }
 
   tc_fence_before();

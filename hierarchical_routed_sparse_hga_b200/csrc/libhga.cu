@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -134,6 +135,20 @@ bool make_map_bf16_d128_groups(CUtensorMap* map, const void* base, uint64_t rows
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// SM count of the current device (cached per device)
+int sm_count() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 bool use_tensor_cores(const hga_config_t* c, int64_t ctx_cap, int32_t s_len) {
   const int G = c->n_q_heads / c->n_kv_heads;
   if (c->flags & HGA_FLAG_SIMT) return false;
@@ -174,7 +189,7 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
                            int64_t ctx_cap, int64_t q_begin, int32_t s_len,
                            const int32_t* sel_grp, const void* o, const float* lse,
                            const void* d_o, void* dq, void* dk, void* dv, float* dvec,
-                           cudaStream_t s) {
+                           int* unit_counter, cudaStream_t s) {
   using LQ = bwdtc::DqLayout<MT>;
   using LK = bwdtc::KvLayout;
   CUtensorMap tq, tdo, tk, tv;
@@ -196,14 +211,18 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
         tq, tdo, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
         ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups, sel_grp,
         cfg->scale, scale_log2, static_cast<const __nv_bfloat16*>(o),
-        static_cast<const __nv_bfloat16*>(d_o), lse, static_cast<__nv_bfloat16*>(dq), dvec);
+        static_cast<const __nv_bfloat16*>(d_o), lse, static_cast<__nv_bfloat16*>(dq), dvec,
+        unit_counter);
   });
   if (e != HGA_OK) return e;
+  // persistent: at most one CTA per SM over the (key block, head) units
+  const int n_units = (s_len / kBlock) * cfg->batch * cfg->n_kv_heads;
+  dim3 grid_kv(unsigned(std::min(n_units, sm_count())));
   return traced_launch(HGA_K_BWD_DKDV_TC, s, [&] {
-    return launch_pdl(bwdtc::attn_bwd_dkdv_tc_kernel<MT>, grid, dim3(LK::kThreads), LK::kDynSmem, s,
-        tq, tdo, tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups,
-        sel_grp, cfg->scale, scale_log2, lse, dvec, static_cast<__nv_bfloat16*>(dk),
-        static_cast<__nv_bfloat16*>(dv));
+    return launch_pdl(bwdtc::attn_bwd_dkdv_tc_kernel<MT>, grid_kv, dim3(LK::kThreads),
+        LK::kDynSmem, s, tq, tdo, tk, tv, ctx_cap, q_begin, s_len, cfg->batch, cfg->n_q_heads,
+        cfg->n_kv_heads, cfg->topk_groups, sel_grp, cfg->scale, scale_log2, lse, dvec,
+        static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), unit_counter);
   });
 }
 
@@ -419,9 +438,15 @@ hga_status_t hga_route_noalloc(const hga_config_t* cfg, const void* q, int64_t q
                    HGA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+// backward workspace: D = rowsum(dO * O) [B, Hq, S] fp32, then (256-B aligned)
+// the work-unit counter of the persistent dK/dV kernel
+static size_t bwd_dvec_bytes(const hga_config_t* cfg, int32_t s_len) {
+  return align256(size_t(cfg->batch) * cfg->n_q_heads * size_t(s_len) * 4);
+}
+
 size_t hga_attn_bwd_workspace_size(const hga_config_t* cfg, int32_t s_len) {
   if (check_cfg(cfg) != HGA_OK || s_len <= 0) return 0;
-  return align256(size_t(cfg->batch) * cfg->n_q_heads * size_t(s_len) * 4);
+  return bwd_dvec_bytes(cfg, s_len) + 256;
 }
 
 hga_status_t hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k, const void* v,
@@ -438,13 +463,15 @@ hga_status_t hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k,
   if (ws_bytes < hga_attn_bwd_workspace_size(cfg, s_len)) return HGA_ERR_WORKSPACE;
   const int n_qb = s_len / kQBlock;
   float* dvec = static_cast<float*>(workspace);
+  int* unit_counter =
+      reinterpret_cast<int*>(static_cast<char*>(workspace) + bwd_dvec_bytes(cfg, s_len));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (use_tensor_cores(cfg, ctx_cap, s_len)) {
     if (cfg->n_q_heads / cfg->n_kv_heads == 4)
       return launch_bwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq,
-                              dk, dv, dvec, s);
+                              dk, dv, dvec, unit_counter, s);
     return launch_bwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk,
-                            dv, dvec, s);
+                            dv, dvec, unit_counter, s);
   }
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
     const size_t sm1 = size_t(simt_fwd_smem_floats<D>()) * 4;

@@ -201,7 +201,9 @@ HGA_API hga_status_t hga_route_noalloc(const hga_config_t* cfg, const void* q, i
                                        const float* gsum, int32_t* sel_blk, int32_t* sel_grp,
                                        void* stream);
 
-/* Bytes of device workspace hga_attn_bwd needs for this segment. */
+/* Bytes of device workspace hga_attn_bwd needs for this segment: D =
+ * rowsum(dO * O) as [B, Hq, S] fp32 (256-byte aligned), then 256 bytes for
+ * the work counter of the tensor-core dK/dV kernel. */
 HGA_API size_t hga_attn_bwd_workspace_size(const hga_config_t* cfg, int32_t s_len);
 
 /*
