@@ -257,6 +257,12 @@ def kernel_work(name, w, sels, unique_groups=None):
         elif name == "route_select":
             tot += B * Hkv * sum(J * 4 + 8 * k * d * 4 + d * 4 + 4 * (w.topk_blocks + w.topk_groups)
                                  for J, k in zip(Js, kb))
+        elif name == "route_fused":
+            # Q once, each block summary of the head once, the kept blocks'
+            # group summaries, the two selections written
+            tot += B * Hq * S * d * el + B * Hkv * (
+                (own0 + n_qb - 1) * d * 4
+                + sum(8 * k * d * 4 + 4 * (w.topk_blocks + w.topk_groups) for k in kb))
         elif name == "tier_copy":
             tot += 2 * 2 * unique_groups.get(q_begin, 0) * 8 * d * el   # read host + write HBM
         elif name == "tier_dedup":

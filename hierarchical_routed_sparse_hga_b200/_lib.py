@@ -31,7 +31,7 @@ EXPORTS = ("hga_version", "hga_status_string", "hga_build_summaries",
            "hga_tier_stage_rows", "hga_tier_workspace_size", "hga_tier_gather",
            "hga_tier_append")
 HGA_NOALLOC_SCRATCH_BYTES = 4 << 20
-HGA_K_COUNT = 12
+HGA_K_COUNT = 13
 
 
 class HgaError(RuntimeError):

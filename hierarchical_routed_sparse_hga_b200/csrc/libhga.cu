@@ -363,6 +363,19 @@ hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int G = cfg->n_q_heads / cfg->n_kv_heads;
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
+    if (j_max <= kFusedRouteMaxBlocks) {
+      // the whole routing in one launch (every CTA reads all J block summaries)
+      dim3 g1(n_qb, cfg->n_kv_heads, cfg->batch);
+      const size_t smf = fused_route_smem<D>(own0 + n_qb, cfg->topk_blocks);
+      hga_status_t e = ensure_smem(reinterpret_cast<const void*>(&route_fused_kernel<T, D>), smf);
+      if (e != HGA_OK) return e;
+      return traced_launch(HGA_K_ROUTE_FUSED, s, [&] {
+        return launch_pdl(route_fused_kernel<T, D>, g1, dim3(kRouteThreads), smf, s,
+                          static_cast<const T*>(q), bsum, gsum, ctx_cap, cfg->n_q_heads,
+                          cfg->n_kv_heads, s_len, own0, cfg->topk_blocks, cfg->topk_groups,
+                          sel_blk, sel_grp);
+      });
+    }
     dim3 g0(n_qb * G, cfg->n_kv_heads, cfg->batch);
     hga_status_t e = traced_launch(HGA_K_QMEAN, s, [&] {
       return launch_pdl(qmean_kernel<T, D>, g0, dim3(kQmeanThreads), 0, s, static_cast<const T*>(q),
@@ -623,7 +636,8 @@ const char* hga_kernel_name(int kind) {
   static const char* names[HGA_K_COUNT] = {
       "summaries",      "route_qmean",       "route_block_score",   "route_select",
       "attn_fwd_simt",  "attn_bwd_dq_simt",  "attn_bwd_dkdv_simt",  "attn_fwd_tc",
-      "attn_bwd_dq_tc", "attn_bwd_dkdv_tc",  "tier_dedup",          "tier_copy"};
+      "attn_bwd_dq_tc", "attn_bwd_dkdv_tc",  "tier_dedup",          "tier_copy",
+      "route_fused"};
   return (kind >= 0 && kind < HGA_K_COUNT) ? names[kind] : "unknown";
 }
 

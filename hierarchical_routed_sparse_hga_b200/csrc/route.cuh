@@ -3,7 +3,8 @@
 // are opened at 8-token-group level, the router uses no learned weights and
 // scores the existing projected keys).
 //
-// Three launches, all HBM/L2-bound:
+// One launch (route_fused_kernel) while the candidate blocks number at most
+// kFusedRouteMaxBlocks; beyond that three launches, all HBM/L2-bound:
 //   qmean_kernel        per (query block j, query head): that head's share of
 //                       qbar[b,h,j], the mean of the 64 x G query rows (reads Q
 //                       once, 1024 CTAs for Qwen3 shapes, one load round);
@@ -160,70 +161,29 @@ __host__ __device__ inline SelectLayout select_layout(int64_t j_cap, int topk_bl
   return L;
 }
 
-// grid (n_qb, Hkv, B); dynamic smem select_layout(...).total
-template <int D>
-__global__ void __launch_bounds__(kRouteThreads)
-    select_kernel(const float* __restrict__ qpart, const float* __restrict__ scores,
-                  const float* __restrict__ gsum, int64_t ctx_cap, int n_kv_heads, int G, int n_qb,
-                  int64_t own0, int64_t jstride, int topk_blocks, int topk_groups,
-                  int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp) {
-  pdl_launch_dependents();
-  pdl_wait();
-  extern __shared__ __align__(16) unsigned char sm_raw[];
-  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int64_t head = int64_t(b) * n_kv_heads + h;
-  const int64_t J = own0 + j;                 // candidate blocks [0, J)
-  const int kb = int(J < topk_blocks ? J : topk_blocks);
-  const int64_t j_cap = own0 + n_qb;
-  const int n2 = 8 * kb;
-
-  const SelectLayout L = select_layout(j_cap, topk_blocks, D);
-  float* qb = reinterpret_cast<float*>(sm_raw + L.qb);
-  uint32_t* key1 = reinterpret_cast<uint32_t*>(sm_raw + L.key1);
-  uint32_t* key2 = reinterpret_cast<uint32_t*>(sm_raw + L.key2);
-  int* blocks = reinterpret_cast<int*>(sm_raw + L.blocks);
-  int* hist = reinterpret_cast<int*>(sm_raw + L.hist);
-  int* scratch = reinterpret_cast<int*>(sm_raw + L.scratch);
-  uint8_t* sel1 = sm_raw + L.sel1;
-  uint8_t* sel2 = sm_raw + L.sel2;
-
-  const float* srow = scores + (head * n_qb + j) * jstride;
-  for (int64_t i = threadIdx.x; i < J; i += kRouteThreads) key1[i] = ordered_key(srow[i]);
-  for (int i = threadIdx.x; i < D; i += kRouteThreads)
-    qb[i] = qbar_elem(qpart + ((head * n_qb + j) * G) * D, G, D, i);
-  __syncthreads();
-
-  // level 1
-  block_topk(key1, int(J), kb, sel1, hist, scratch);
-  block_enumerate(
-      int(J), [&](int i) { return sel1[i] != 0; }, [&](int i, int r) { blocks[r] = i; },
-      scratch);
-  int32_t* out_blk = sel_blk ? sel_blk + (head * n_qb + j) * topk_blocks : nullptr;
-  if (out_blk)
-    for (int i = threadIdx.x; i < topk_blocks; i += kRouteThreads)
-      out_blk[i] = i < kb ? blocks[i] : -1;
-
-  // level 2: score the 8 groups of every kept block (candidate p -> group
-  // blocks[p/8]*8 + p%8, which is ascending in p)
+// Scores n rows of a summary table against q-bar (in shared memory): key[p]
+// = ordered_key(qb . rows[row_of(p)]).  A warp takes 16 rows per pass, lanes
+// across the d dimension, all 16 row loads issued before any use.
+template <int D, typename RowOf>
+__device__ __forceinline__ void score_rows(const float* __restrict__ table, const float* qb,
+                                           int n, RowOf row_of, uint32_t* key) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NW = kRouteThreads / 32;
   constexpr int V4 = D / 4;  // float4 per summary row
   const float4* qb4 = reinterpret_cast<const float4*>(qb);
-  const float* gbase = gsum + head * (ctx_cap / kGroup) * D;
-  // 16 candidate rows per warp pass, all loads issued before any use
   constexpr int kU = 16;
   constexpr int kE = (V4 + 31) / 32;  // float4 per lane per row
-  for (int p0 = warp * kU; p0 < n2; p0 += NW * kU) {
+  for (int p0 = warp * kU; p0 < n; p0 += NW * kU) {
     float4 x[kU][kE];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int p = p0 + u;
-      const int64_t g = p < n2 ? int64_t(blocks[p >> 3]) * kGroupsPerBlock + (p & 7) : 0;
-      const float4* row = reinterpret_cast<const float4*>(gbase + g * D);
+      const int64_t r = p < n ? row_of(p) : 0;
+      const float4* row = reinterpret_cast<const float4*>(table + r * D);
 #pragma unroll
       for (int i = 0; i < kE; ++i) {
         const int e = lane + 32 * i;
-        x[u][i] = (p < n2 && e < V4) ? row[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[u][i] = (p < n && e < V4) ? row[e] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
     float part[kU];
@@ -244,14 +204,53 @@ __global__ void __launch_bounds__(kRouteThreads)
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) part[u] += __shfl_xor_sync(0xffffffffu, part[u], o);
     }
-    if (lane < kU && p0 + lane < n2) {
+    if (lane < kU && p0 + lane < n) {
       float v = part[0];
 #pragma unroll
       for (int u = 1; u < kU; ++u)
         if (lane == u) v = part[u];
-      key2[p0 + lane] = ordered_key(v);
+      key[p0 + lane] = ordered_key(v);
     }
   }
+}
+
+// The two selections of one (b, h, j) once q-bar is in qb and the J block
+// scores are in key1: top-k_b blocks, their 8 groups scored, top-k_g groups,
+// both written in ascending index order (-1 padded).
+template <int D>
+__device__ __forceinline__ void select_levels(const SelectLayout& L, unsigned char* sm_raw,
+                                              const float* __restrict__ gsum, int64_t head,
+                                              int64_t ctx_cap, int n_qb, int j, int64_t J,
+                                              int topk_blocks, int topk_groups,
+                                              int32_t* __restrict__ sel_blk,
+                                              int32_t* __restrict__ sel_grp) {
+  const float* qb = reinterpret_cast<const float*>(sm_raw + L.qb);
+  uint32_t* key1 = reinterpret_cast<uint32_t*>(sm_raw + L.key1);
+  uint32_t* key2 = reinterpret_cast<uint32_t*>(sm_raw + L.key2);
+  int* blocks = reinterpret_cast<int*>(sm_raw + L.blocks);
+  int* hist = reinterpret_cast<int*>(sm_raw + L.hist);
+  int* scratch = reinterpret_cast<int*>(sm_raw + L.scratch);
+  uint8_t* sel1 = sm_raw + L.sel1;
+  uint8_t* sel2 = sm_raw + L.sel2;
+  const int kb = int(J < topk_blocks ? J : topk_blocks);
+  const int n2 = 8 * kb;
+
+  // level 1
+  block_topk(key1, int(J), kb, sel1, hist, scratch);
+  block_enumerate(
+      int(J), [&](int i) { return sel1[i] != 0; }, [&](int i, int r) { blocks[r] = i; },
+      scratch);
+  int32_t* out_blk = sel_blk ? sel_blk + (head * n_qb + j) * topk_blocks : nullptr;
+  if (out_blk)
+    for (int i = threadIdx.x; i < topk_blocks; i += kRouteThreads)
+      out_blk[i] = i < kb ? blocks[i] : -1;
+
+  // level 2: score the 8 groups of every kept block (candidate p -> group
+  // blocks[p/8]*8 + p%8, which is ascending in p)
+  const float* gbase = gsum + head * (ctx_cap / kGroup) * D;
+  score_rows<D>(gbase, qb, n2,
+                [&](int p) { return int64_t(blocks[p >> 3]) * kGroupsPerBlock + (p & 7); },
+                key2);
   __syncthreads();
   const int kg = n2 < topk_groups ? n2 : topk_groups;
   block_topk(key2, n2, kg, sel2, hist, scratch);
@@ -260,6 +259,102 @@ __global__ void __launch_bounds__(kRouteThreads)
       n2, [&](int p) { return sel2[p] != 0; },
       [&](int p, int r) { out_grp[r] = blocks[p >> 3] * kGroupsPerBlock + (p & 7); }, scratch);
   for (int i = kg + threadIdx.x; i < topk_groups; i += kRouteThreads) out_grp[i] = -1;
+}
+
+// grid (n_qb, Hkv, B); dynamic smem select_layout(...).total
+template <int D>
+__global__ void __launch_bounds__(kRouteThreads)
+    select_kernel(const float* __restrict__ qpart, const float* __restrict__ scores,
+                  const float* __restrict__ gsum, int64_t ctx_cap, int n_kv_heads, int G, int n_qb,
+                  int64_t own0, int64_t jstride, int topk_blocks, int topk_groups,
+                  int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp) {
+  pdl_launch_dependents();
+  pdl_wait();
+  extern __shared__ __align__(16) unsigned char sm_raw[];
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int64_t head = int64_t(b) * n_kv_heads + h;
+  const int64_t J = own0 + j;                 // candidate blocks [0, J)
+  const int64_t j_cap = own0 + n_qb;
+  const SelectLayout L = select_layout(j_cap, topk_blocks, D);
+  float* qb = reinterpret_cast<float*>(sm_raw + L.qb);
+  uint32_t* key1 = reinterpret_cast<uint32_t*>(sm_raw + L.key1);
+  const float* srow = scores + (head * n_qb + j) * jstride;
+  for (int64_t i = threadIdx.x; i < J; i += kRouteThreads) key1[i] = ordered_key(srow[i]);
+  for (int i = threadIdx.x; i < D; i += kRouteThreads)
+    qb[i] = qbar_elem(qpart + ((head * n_qb + j) * G) * D, G, D, i);
+  __syncthreads();
+  select_levels<D>(L, sm_raw, gsum, head, ctx_cap, n_qb, j, J, topk_blocks, topk_groups, sel_blk,
+                   sel_grp);
+}
+
+// The whole routing of one (b, h, j) in one CTA, used while every CTA can
+// afford to read all J block summaries (J <= kFusedRouteMaxBlocks; they stay
+// in L2): q-bar from the G heads' 64 query rows (the loads of several rows in
+// flight per thread), the J block scores, then select_levels.  One launch
+// instead of qmean + block_score + select.  Dynamic shared memory:
+// fused_route_smem(), the select layout followed by the q-bar partial sums.
+constexpr int kFusedRouteMaxBlocks = 512;
+
+template <int D>
+__host__ __device__ constexpr int fused_route_rows() { return kRouteThreads / (D / 8); }
+
+template <int D>
+__host__ __device__ inline size_t fused_route_smem(int64_t j_cap, int topk_blocks) {
+  return select_layout(j_cap, topk_blocks, D).total + size_t(fused_route_rows<D>()) * D * 4;
+}
+
+// grid (n_qb, Hkv, B)
+template <typename T, int D>
+__global__ void __launch_bounds__(kRouteThreads)
+    route_fused_kernel(const T* __restrict__ q, const float* __restrict__ bsum,
+                       const float* __restrict__ gsum, int64_t ctx_cap, int n_q_heads,
+                       int n_kv_heads, int s_len, int64_t own0, int topk_blocks, int topk_groups,
+                       int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp) {
+  pdl_launch_dependents();
+  pdl_wait();
+  extern __shared__ __align__(16) unsigned char sm_raw[];
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int G = n_q_heads / n_kv_heads, n_qb = s_len / kQBlock;
+  const int64_t head = int64_t(b) * n_kv_heads + h;
+  const int64_t J = own0 + j;                 // candidate blocks [0, J)
+  const SelectLayout L = select_layout(own0 + n_qb, topk_blocks, D);
+  float* qb = reinterpret_cast<float*>(sm_raw + L.qb);
+  uint32_t* key1 = reinterpret_cast<uint32_t*>(sm_raw + L.key1);
+  float* part = reinterpret_cast<float*>(sm_raw + L.total);
+
+  // q-bar: thread (row slot rs, 8-column chunk ch) sums rows rs, rs + RS, ...
+  // of the G x 64 query rows; the RS partial rows are then added in order
+  constexpr int CH = D / 8, RS = fused_route_rows<D>();
+  const int ch = threadIdx.x % CH, rs = threadIdx.x / CH;
+  const int rows = G * kQBlock;
+  const T* qh =
+      q + ((int64_t(b) * n_q_heads + int64_t(h) * G) * s_len + int64_t(j) * kQBlock) * D + ch * 8;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 8
+  for (int rr = rs; rr < rows; rr += RS) {
+    float f[8];
+    load8(qh + (int64_t(rr >> 6) * s_len + (rr & 63)) * D, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += f[e];
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[rs * D + ch * 8 + e] = acc[e];
+  __syncthreads();
+  const float inv = 1.f / float(rows);
+  for (int e = threadIdx.x; e < D; e += kRouteThreads) {
+    float sum = 0.f;
+    for (int r = 0; r < RS; ++r) sum += part[r * D + e];
+    qb[e] = sum * inv;
+  }
+  __syncthreads();
+  // level-1 scores of the J candidate blocks
+  score_rows<D>(bsum + head * (ctx_cap / kBlock) * D, qb, int(J),
+                [](int p) { return int64_t(p); }, key1);
+  __syncthreads();
+  select_levels<D>(L, sm_raw, gsum, head, ctx_cap, n_qb, j, J, topk_blocks, topk_groups, sel_blk,
+                   sel_grp);
 }
 
 }  // namespace hga

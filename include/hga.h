@@ -300,7 +300,8 @@ typedef enum {
   HGA_K_BWD_DKDV_TC = 9,
   HGA_K_TIER_DEDUP = 10,
   HGA_K_TIER_COPY = 11,
-  HGA_K_COUNT = 12
+  HGA_K_ROUTE_FUSED = 12,
+  HGA_K_COUNT = 13
 } hga_kernel_kind_t;
 
 /* Name of a kernel kind ("attn_fwd_simt", ...). */
