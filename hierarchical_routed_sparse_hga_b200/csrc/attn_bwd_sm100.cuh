@@ -9,10 +9,12 @@
 //
 // attn_bwd_dq_tc_kernel -- one CTA per (batch, KV head, query block), the G
 //   heads stacked into M = 64 G rows as in the forward.  Per key tile (the
-//   same tiles as the forward): S = Q K^T and dP = dO V^T into TMEM, then one
-//   thread per row forms P = exp2(S c - LSE2), dS = P (dP - D) (bf16 into
-//   shared memory), and dQ += dS K accumulates in TMEM; dQ = scale * dQ at the
-//   end.  D = rowsum(dO * O) is computed here and saved for the next kernel.
+//   same tiles as the forward, gathered by cp.async into a 3-stage ring) and
+//   M tile: S = Q K^T and dP = dO V^T into one of two TMEM regions, then one
+//   thread per row forms P = exp2(S c - LSE2), dS = P (dP - D) and stores it
+//   as bf16 over the region's S columns, and dQ += dS K (A operand in tensor
+//   memory) accumulates in TMEM; dQ = scale * dQ at the end.  D = rowsum(dO * O)
+//   is computed here (warp shuffles) and saved for the next kernel.
 //
 // attn_bwd_dkdv_tc_kernel -- persistent: at most one CTA per SM, each taking
 //   work units (batch, KV head, 64-key block of the active segment) from a
@@ -48,28 +50,29 @@ template <int MT>
 struct DqLayout {
   static constexpr uint32_t kQ = 0;                              // [MT][2][128][128 B]
   static constexpr uint32_t kDO = MT * 32768;                    // same layout
-  static constexpr uint32_t kKV = 2 * MT * 32768;                // [2 stages][K | V]
-  static constexpr uint32_t kStages = 2;
+  static constexpr uint32_t kKV = 2 * MT * 32768;                // [3 stages][K | V]
+  static constexpr uint32_t kStages = 3;
   static constexpr uint32_t kStageBytes = 32768;
-  static constexpr uint32_t kDS = kKV + kStages * kStageBytes;   // [MT][128][128 B]
-  static constexpr uint32_t kBytes = kDS + MT * 16384;
+  static constexpr uint32_t kBytes = kKV + kStages * kStageBytes;
   static constexpr uint32_t kDynSmem = kBytes + 1024;
   static constexpr uint32_t kThreads = 128 + 128 * MT;
-  static constexpr uint32_t kTmemCols = MT == 2 ? 512 : 256;
-  // TMEM columns: S_m, dP_m (64 each), dQ_m (128)
-  static constexpr uint32_t colS(int m) { return m * 64; }
-  static constexpr uint32_t colDP(int m) { return MT * 64 + m * 64; }
-  static constexpr uint32_t colDQ(int m) { return MT * 128 + m * 128; }
+  static constexpr uint32_t kTmemCols = 512;
+  // TMEM columns: two S | dP regions (64 + 64 each); dS of an op, as bf16
+  // pairs, goes over the first 32 columns of its own region once S and dP
+  // are in registers; dQ of each M tile (128)
+  static constexpr uint32_t colS(int r) { return r * 128; }
+  static constexpr uint32_t colDP(int r) { return r * 128 + 64; }
+  static constexpr uint32_t colDQ(int m) { return 256 + m * 128; }
 };
 
 struct DqShared {
   uint64_t q_full;
-  uint64_t kv_full[2];
-  uint64_t kv_empty[2];
-  uint64_t sdp_full[2];
-  uint64_t sdp_free[2];
-  uint64_t ds_full[2];
-  uint64_t ds_done[2];
+  uint64_t kv_full[3];
+  uint64_t kv_empty[3];
+  // [region]: op s = t * MT + m (tile t, M tile m) runs in region s & 1
+  uint64_t sdp_full[2];   // S, dP of the op are in the region
+  uint64_t ds_full[2];    // its dS is in the region
+  uint64_t ds_done[2];    // dQ += dS K has completed: the region is free
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
@@ -94,12 +97,13 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
                           int* __restrict__ unit_counter) {
   using L = DqLayout<MT>;
   constexpr int G = 2 * MT;
+  constexpr int kSt = L::kStages;
   extern __shared__ uint8_t dsmem_raw[];
   __shared__ DqShared sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sQ = smem_u32(smem + L::kQ), sDO = smem_u32(smem + L::kDO);
-  const uint32_t sKV = smem_u32(smem + L::kKV), sDS = smem_u32(smem + L::kDS);
+  const uint32_t sKV = smem_u32(smem + L::kKV);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -110,15 +114,14 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
 
   if (tid == 0) {
     mbar_init(&sh.q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kSt; ++s) {
       mbar_init(&sh.kv_full[s], kDqProducers);
       mbar_init(&sh.kv_empty[s], 1);
     }
-    for (int m = 0; m < 2; ++m) {
-      mbar_init(&sh.sdp_full[m], 1);
-      mbar_init(&sh.sdp_free[m], 128);
-      mbar_init(&sh.ds_full[m], 128);
-      mbar_init(&sh.ds_done[m], 1);
+    for (int r = 0; r < 2; ++r) {
+      mbar_init(&sh.sdp_full[r], 1);
+      mbar_init(&sh.ds_full[r], 128);
+      mbar_init(&sh.ds_done[r], 1);
     }
     mbar_init(&sh.mma_done, 1);
     sh.abort = 0;
@@ -157,13 +160,14 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
   const int n_tiles = sh.n_tiles;
 
   if (warp == 0 || warp == 2 || warp == 3) {
-    // ---------------- producers: Q, dO by TMA; K/V groups by cp.async ----------------
+    // ---------------- producers: K/V groups by cp.async into a 3-stage ring ------
+    // stage layout [K | V][d half][64 rows][128 B], 128-byte swizzle
     const int ptid = warp == 0 ? lane : 32 * (warp - 1) + lane;
     const __nv_bfloat16* kh = k + (int64_t(b) * n_kv_heads + h) * ctx_cap * kD;
     const __nv_bfloat16* vh = v + (int64_t(b) * n_kv_heads + h) * ctx_cap * kD;
     for (int t = 0; t < n_tiles; ++t) {
-      const int st = t & 1;
-      if (t >= 2 && !mbar_wait(&sh.kv_empty[st], ((t >> 1) - 1) & 1, abort)) break;
+      const int st = t % kSt;
+      if (t >= kSt && !mbar_wait(&sh.kv_empty[st], ((t / kSt) - 1) & 1, abort)) break;
       const uint32_t kdst = sKV + st * L::kStageBytes;
       for (int c = ptid; c < 2048; c += kDqProducers) {
         const int tensor = c >> 10, rc = c & 1023, r = rc >> 4, ch = rc & 15;
@@ -179,64 +183,60 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 1) {
     // ---------------- MMA issuer (event driven; whole warp, one lane issues) --
+    // Ops s = t * MT + m (tile t, M tile m) alternate between the two TMEM
+    // regions (region s & 1).  S/dP of op s needs the K/V of tile t and its
+    // region back from op s - 2 (whose dQ has read its dS); dQ of op s needs
+    // its dS, and the last dQ of a tile frees the tile's K/V stage.
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);
     constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kD, 0, 1);
     bool ok = __all_sync(kFullMask, mbar_wait(&sh.q_full, 0, abort));
     bool issued_any = false;
-    int next_sdp = 0, next_dq = 0;
+    const int n_ops = n_tiles * MT;
+    int next_s = 0, next_q = 0;  // next S/dP op, next dQ op
     long long t0 = clock64();
-    while (ok && next_dq < n_tiles) {
+    while (ok && next_q < n_ops) {
       bool progressed = false;
-      if (next_dq < next_sdp) {
-        bool ready = true;
-        for (int m = 0; m < MT; ++m) ready = ready && mbar_test(&sh.ds_full[m], next_dq & 1);
-        if (__all_sync(kFullMask, ready)) {
-          const int tt = next_dq;
-          const uint32_t kb = sKV + (tt & 1) * L::kStageBytes;
+      if (next_q < next_s) {
+        const int t = next_q / MT, m = next_q % MT, rg = next_q & 1;
+        if (__all_sync(kFullMask, mbar_test(&sh.ds_full[rg], (next_q >> 1) & 1))) {
+          const uint32_t kb = sKV + (t % kSt) * L::kStageBytes;
           tc_fence_after();
           if (elect_one()) {
-            for (int m = 0; m < MT; ++m) {
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + L::colDQ(m), smem_desc_sw128(sDS + m * 16384 + kk * 32, 16, 1024),
-                         smem_desc_sw128(kb + kk * 2048, 8192, 1024), idesc_dq,
-                         (tt > 0 || kk > 0) ? 1u : 0u);
-              mma_commit(&sh.ds_done[m]);
-            }
-            mma_commit(&sh.kv_empty[tt & 1]);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_tmem_a(tmem + L::colDQ(m), tmem + L::colS(rg) + kk * 8,
+                              smem_desc_sw128(kb + kk * 2048, 8192, 1024), idesc_dq,
+                              (t > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&sh.ds_done[rg]);
+            if (m == MT - 1) mma_commit(&sh.kv_empty[t % kSt]);
           }
           __syncwarp();
-          ++next_dq;
+          ++next_q;
           progressed = true;
         }
       }
-      // S/dP(t) may run one tile ahead of dQ: its TMEM columns are free once
-      // the softmax has loaded S/dP(t-1)
-      if (!progressed && next_sdp < n_tiles && next_sdp <= next_dq + 1) {
-        const int t = next_sdp, st = t & 1;
-        bool ready = mbar_test(&sh.kv_full[st], (t >> 1) & 1);
-        for (int m = 0; m < MT && t >= 1; ++m)
-          ready = ready && mbar_test(&sh.sdp_free[m], (t - 1) & 1);
+      if (!progressed && next_s < n_ops && next_s < next_q + 2) {
+        const int t = next_s / MT, m = next_s % MT, rg = next_s & 1;
+        bool ready = m != 0 || mbar_test(&sh.kv_full[t % kSt], (t / kSt) & 1);
+        if (next_s >= 2) ready = ready && mbar_test(&sh.ds_done[rg], ((next_s - 2) >> 1) & 1);
         if (__all_sync(kFullMask, ready)) {
           fence_proxy_async_smem();  // cp.async data -> tensor-core reads
           tc_fence_after();
-          const uint32_t kb = sKV + st * L::kStageBytes;
+          const uint32_t kb = sKV + (t % kSt) * L::kStageBytes;
           if (elect_one()) {
-            for (int m = 0; m < MT; ++m) {
 #pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-                const uint32_t bo = (kk >> 2) * 8192 + (kk & 3) * 32;
-                mma_bf16(tmem + L::colS(m), smem_desc_sw128(sQ + m * 32768 + ko, 16, 1024),
-                         smem_desc_sw128(kb + bo, 16, 1024), idesc_s, kk > 0);
-                mma_bf16(tmem + L::colDP(m), smem_desc_sw128(sDO + m * 32768 + ko, 16, 1024),
-                         smem_desc_sw128(kb + 16384 + bo, 16, 1024), idesc_s, kk > 0);
-              }
-              mma_commit(&sh.sdp_full[m]);
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+              const uint32_t bo = (kk >> 2) * 8192 + (kk & 3) * 32;
+              mma_bf16(tmem + L::colS(rg), smem_desc_sw128(sQ + m * 32768 + ko, 16, 1024),
+                       smem_desc_sw128(kb + bo, 16, 1024), idesc_s, kk > 0);
+              mma_bf16(tmem + L::colDP(rg), smem_desc_sw128(sDO + m * 32768 + ko, 16, 1024),
+                       smem_desc_sw128(kb + 16384 + bo, 16, 1024), idesc_s, kk > 0);
             }
+            mma_commit(&sh.sdp_full[rg]);
           }
           __syncwarp();
-          ++next_sdp;
+          ++next_s;
           issued_any = true;
           progressed = true;
         }
@@ -256,100 +256,87 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     const uint32_t lane_addr = uint32_t(wq * 32) << 16;
     const int hq = h * G + g;
     const int64_t rix = (int64_t(b) * n_q_heads + hq) * s_len + int64_t(j) * kQBlock + r;
-    // D = rowsum(dO * O), saved for the dK/dV kernel.  Computed cooperatively:
-    // a warp takes two rows per step (16 lanes x 16 B each), O read with
-    // coalesced 256-byte row loads, dO from the shared-memory tile.
-    {
-      if (!mbar_wait(&sh.q_full, 0, abort)) {
-      } else {
-        const int half = lane >> 4, c = lane & 15;   // row of the pair, 16-byte chunk
-        const uint8_t* dO_m = smem + L::kDO + m * 32768;
-        // scratch: the first bytes of this warp's own dS rows, which only
-        // this warp writes, and only after it has read its D values
-        float* dsh = reinterpret_cast<float*>(smem + L::kDS + m * 16384 + wq * 32 * 128);
-        // all 16 row-pair loads of O issued before any use
-        uint4 ov[16];
+    // D = rowsum(dO * O), saved for the dK/dV kernel.  A warp takes two rows
+    // per step (16 lanes x 16 B each): O by coalesced 256-byte row loads, all
+    // issued first, dO from shared memory; lane i keeps the sum of row i.
+    float dsum = 0.f;
+    if (mbar_wait(&sh.q_full, 0, abort)) {
+      const int half = lane >> 4, c = lane & 15;   // row of the pair, 16-byte chunk
+      const uint8_t* dO_m = smem + L::kDO + m * 32768;
+      uint4 ov[16];
 #pragma unroll
-        for (int p2 = 0; p2 < 16; ++p2) {
-          const int rw = wq * 32 + 2 * p2 + half;    // row in the M tile
-          const int gw = (m * 128 + rw) >> 6, tw = (m * 128 + rw) & 63;
-          const int64_t orow =
-              (int64_t(b) * n_q_heads + h * G + gw) * s_len + int64_t(j) * kQBlock + tw;
-          ov[p2] = *reinterpret_cast<const uint4*>(o + orow * kD + c * 8);
-        }
-#pragma unroll
-        for (int p2 = 0; p2 < 16; ++p2) {
-          const int rw = wq * 32 + 2 * p2 + half;
-          float df[8];
-          load8(reinterpret_cast<const __nv_bfloat16*>(
-                    dO_m + (c >> 3) * 16384 + rw * 128 + (((c & 7) ^ (rw & 7)) << 4)),
-                df);
-          const uint32_t w4[4] = {ov[p2].x, ov[p2].y, ov[p2].z, ov[p2].w};
-          float part = 0.f;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            part = fmaf(__uint_as_float(w4[i] << 16), df[2 * i], part);
-            part = fmaf(__uint_as_float(w4[i] & 0xffff0000u), df[2 * i + 1], part);
-          }
-#pragma unroll
-          for (int off = 8; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-          if (c == 0) dsh[2 * p2 + half] = part;
-        }
+      for (int p2 = 0; p2 < 16; ++p2) {
+        const int rw = wq * 32 + 2 * p2 + half;    // row in the M tile
+        const int gw = (m * 128 + rw) >> 6, tw = (m * 128 + rw) & 63;
+        const int64_t orow =
+            (int64_t(b) * n_q_heads + h * G + gw) * s_len + int64_t(j) * kQBlock + tw;
+        ov[p2] = *reinterpret_cast<const uint4*>(o + orow * kD + c * 8);
       }
-      __syncwarp();
+#pragma unroll
+      for (int p2 = 0; p2 < 16; ++p2) {
+        const int rw = wq * 32 + 2 * p2 + half;
+        float df[8];
+        load8(reinterpret_cast<const __nv_bfloat16*>(
+                  dO_m + (c >> 3) * 16384 + rw * 128 + (((c & 7) ^ (rw & 7)) << 4)),
+              df);
+        const uint32_t w4[4] = {ov[p2].x, ov[p2].y, ov[p2].z, ov[p2].w};
+        float part = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          part = fmaf(__uint_as_float(w4[i] << 16), df[2 * i], part);
+          part = fmaf(__uint_as_float(w4[i] & 0xffff0000u), df[2 * i + 1], part);
+        }
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+        // row 2 p2 + h' is now in every lane of half h': lane 2 p2 + h' takes it
+        const float mine = __shfl_sync(0xffffffffu, part, 16 * (lane & 1));
+        if ((lane >> 1) == p2) dsum = mine;
+      }
     }
-    const float dsum = reinterpret_cast<const float*>(smem + L::kDS + m * 16384 +
-                                                      wq * 32 * 128)[lane];
-    __syncwarp();
     dvec[rix] = dsum;
     const float lse2 = lse[rix] * 1.4426950408889634f;
     const float2 c2 = make_float2(scale_log2, scale_log2);
     const float2 nl = make_float2(-lse2, -lse2);
     const float2 nd = make_float2(-dsum, -dsum);
     bool ok = true;
-    uint8_t* drow = smem + L::kDS + m * 16384 + row * 128;
     for (int t = 0; t < n_tiles && ok; ++t) {
-      if (!(ok = mbar_wait(&sh.sdp_full[m], t & 1, abort))) break;
+      const int op = t * MT + m, rg = op & 1;
+      if (!(ok = mbar_wait(&sh.sdp_full[rg], (op >> 1) & 1, abort))) break;
       tc_fence_after();
+      float sv[64], dp[64];
+      tmem_ld32(tmem + lane_addr + L::colS(rg), sv);
+      tmem_ld32(tmem + lane_addr + L::colS(rg) + 32, sv + 32);
+      tmem_ld32(tmem + lane_addr + L::colDP(rg), dp);
+      tmem_ld32(tmem + lane_addr + L::colDP(rg) + 32, dp + 32);
+      tmem_wait_ld();
       const bool own = t == n_tiles - 1;
       const uint32_t mask = sh.tile_mask[t];
-      const bool full = !own && mask == 0xffu;
-      uint32_t packed[32];
+      if (own || mask != 0xffu) {
 #pragma unroll
-      for (int hb = 0; hb < 2; ++hb) {
-        float sv[32], dp[32];
-        tmem_ld32(tmem + lane_addr + L::colS(m) + hb * 32, sv);
-        tmem_ld32(tmem + lane_addr + L::colDP(m) + hb * 32, dp);
-        tmem_wait_ld();
-        if (!full) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int key = hb * 32 + i;
-            const bool valid = ((mask >> (key >> 3)) & 1u) && (!own || key <= r);
-            if (!valid) sv[i] = -INFINITY;
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float2 x = __ffma2_rn(make_float2(sv[i], sv[i + 1]), c2, nl);
-          x.x = ex2_approx(x.x);
-          x.y = ex2_approx(x.y);
-          const float2 y = __fmul2_rn(x, __fadd2_rn(make_float2(dp[i], dp[i + 1]), nd));
-          packed[hb * 16 + i / 2] = pack_bf16x2(y.x, y.y);
+        for (int i = 0; i < 64; ++i) {
+          const bool valid = ((mask >> (i >> 3)) & 1u) && (!own || i <= r);
+          if (!valid) sv[i] = -INFINITY;
         }
       }
-      tc_fence_before();
-      mbar_arrive(&sh.sdp_free[m]);
-      if (t > 0 && !(ok = mbar_wait(&sh.ds_done[m], (t - 1) & 1, abort))) break;
+      uint32_t packed[32];
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(drow + ((c ^ (row & 7)) << 4)) =
-            make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-      fence_proxy_async_smem();
+      for (int i = 0; i < 64; i += 2) {
+        float2 x = __ffma2_rn(make_float2(sv[i], sv[i + 1]), c2, nl);
+        x.x = ex2_approx(x.x);
+        x.y = ex2_approx(x.y);
+        const float2 y = __fmul2_rn(x, __fadd2_rn(make_float2(dp[i], dp[i + 1]), nd));
+        packed[i / 2] = pack_bf16x2(y.x, y.y);
+      }
+      // dS over the S columns of this op's region (A operand of dQ += dS K)
+      tmem_st32_u(tmem + lane_addr + L::colS(rg), packed);
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sh.ds_full[m]);
+      mbar_arrive(&sh.ds_full[rg]);
     }
-    if (ok) ok = mbar_wait(&sh.ds_done[m], (n_tiles - 1) & 1, abort);
+    if (ok) {
+      const int op = (n_tiles - 1) * MT + m;
+      ok = mbar_wait(&sh.ds_done[op & 1], (op >> 1) & 1, abort);
+    }
     if (ok) {
       tc_fence_after();
       __nv_bfloat16* dst = dq + rix * kD;
