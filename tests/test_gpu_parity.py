@@ -50,6 +50,18 @@ def test_qwen3_fwd_128k_sampled():
     run_and_compare(w, segments=[0, 31 * 2048, 63 * 2048], kv_heads=[0, 5])
 
 
+def test_largest_segment_and_topk():
+    # the largest segment (4096 tokens: 64 query blocks, which fills the dK/dV
+    # kernel's per-unit query-block lists) with the largest k_g (256 groups:
+    # 32 routed 8-group tiles plus the own block in the forward and dQ
+    # schedules) and k_b = 32 blocks opened, at the Qwen3 head layout; the
+    # second segment is checked on one KV head
+    w = synth.custom(n_q_heads=32, n_kv_heads=8, head_dim=128, ctx_len=12288, seg_len=4096,
+                     topk_blocks=32, topk_groups=256, dtype="bf16", scaled=True, rope_base=1e6,
+                     seed=5, first_seg=1)
+    run_and_compare(w, segments=[8192], kv_heads=[3])
+
+
 @pytest.mark.parametrize("kw", [
     # ragged: k_g not a multiple of 8, more k_b than candidates early on
     dict(n_q_heads=4, n_kv_heads=1, head_dim=64, ctx_len=576, seg_len=192, topk_blocks=5,
