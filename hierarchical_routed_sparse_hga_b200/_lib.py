@@ -24,7 +24,8 @@ HGA_FLAG_SIMT = 1
 
 EXPORTS = ("hga_version", "hga_status_string", "hga_build_summaries",
            "hga_route_workspace_size", "hga_route", "hga_attn_fwd",
-           "hga_attn_bwd_workspace_size", "hga_attn_bwd", "hga_get_device_status",
+           "hga_attn_bwd_workspace_size", "hga_attn_bwd", "hga_attn_fwd_bwd",
+           "hga_get_device_status",
            "hga_kernel_name", "hga_launch_count", "hga_timing_enable", "hga_timing_collect",
            "hga_timing_get", "hga_timing_reset", "hga_timing_kinds", "hga_route_noalloc",
            "hga_build_summaries_seg",
@@ -91,6 +92,8 @@ def load() -> ctypes.CDLL:
         "hga_attn_bwd_workspace_size": (SZ, [CFG, I32]),
         "hga_attn_bwd": (ctypes.c_int, [CFG, P, P, P, I64, I64, I32, P, P, P, P, P, P, P,
                                         P, SZ, P]),
+        "hga_attn_fwd_bwd": (ctypes.c_int, [CFG, P, P, P, I64, I64, I32, P, P, P, P, P, P, P,
+                                            P, SZ, P]),
         "hga_get_device_status": (ctypes.c_int, [P]),
         "hga_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
         "hga_launch_count": (ctypes.c_uint64, []),
@@ -251,6 +254,18 @@ def hga_attn_bwd(cfg: Config, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse,
     c = cfg.c()
     ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
     _check("hga_attn_bwd", load().hga_attn_bwd(
+        ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), ctx_cap, q_begin, s_len, _ptr(sel_grp),
+        _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes,
+        _stream(stream)))
+
+
+def hga_attn_fwd_bwd(cfg: Config, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq,
+                     dk, dv, workspace, ws_bytes=None, stream=None):
+    """hga_attn_fwd then hga_attn_bwd in one call (the kernels overlap);
+    the workspace's flag sections must be zero before its first use."""
+    c = cfg.c()
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check("hga_attn_fwd_bwd", load().hga_attn_fwd_bwd(
         ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), ctx_cap, q_begin, s_len, _ptr(sel_grp),
         _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes,
         _stream(stream)))

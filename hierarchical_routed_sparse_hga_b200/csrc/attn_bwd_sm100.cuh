@@ -77,6 +77,7 @@ struct DqShared {
   uint32_t tmem_base;
   int abort;
   int n_tiles;
+  int d_arrived;          // rows whose D is written (fused forward + backward)
   int grp[kMaxTiles * 8];
   uint8_t tile_mask[kMaxTiles];
 };
@@ -94,7 +95,8 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
                           float scale_log2, const __nv_bfloat16* __restrict__ o,
                           const __nv_bfloat16* __restrict__ d_o, const float* __restrict__ lse,
                           __nv_bfloat16* __restrict__ dq, float* __restrict__ dvec,
-                          int* __restrict__ unit_counter) {
+                          int* __restrict__ unit_counter, const int* __restrict__ fwd_done,
+                          int* __restrict__ d_done, uint32_t token) {
   using L = DqLayout<MT>;
   constexpr int G = 2 * MT;
   constexpr int kSt = L::kStages;
@@ -109,10 +111,11 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int n_qb = s_len / kQBlock;
   const int64_t own_blk = (q_begin + int64_t(j) * kQBlock) / kBlock;
+  const int item = j + n_qb * (h + gridDim.y * b);
   volatile int* abort = &sh.abort;
-  pdl_launch_dependents();
 
   if (tid == 0) {
+    sh.d_arrived = 0;
     mbar_init(&sh.q_full, 1);
     for (int s = 0; s < kSt; ++s) {
       mbar_init(&sh.kv_full[s], kDqProducers);
@@ -128,10 +131,18 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     fence_barrier_init();
   }
   // the previous kernel may still hold this SM's tensor memory or write
-  // this kernel's inputs: wait for it before allocating or reading
-  pdl_wait();
+  // this kernel's inputs: wait for it before allocating or reading.  In a
+  // fused forward + backward the previous kernel is that forward: this CTA
+  // waits only for its own item's O and LSE (fwd_done), and everything the
+  // forward waited for has completed (it let this grid start only then);
+  // the two kernels' CTAs cannot share an SM (shared memory), so no forward
+  // CTA holds this SM's tensor memory.
+  if (!fwd_done) pdl_wait();
   // the dK/dV kernel that follows takes its work units from this counter
-  if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) *unit_counter = 0;
+  if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) {
+    *unit_counter = 0;
+    __threadfence();
+  }
   if (tid == 0) {
     // Q and dO first: they do not depend on the selection
     prefetch_tmap(&tm_q);
@@ -156,6 +167,7 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_launch_dependents();  // after CTA 0 has zeroed the unit counter
   const uint32_t tmem = sh.tmem_base;
   const int n_tiles = sh.n_tiles;
 
@@ -260,7 +272,8 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     // per step (16 lanes x 16 B each): O by coalesced 256-byte row loads, all
     // issued first, dO from shared memory; lane i keeps the sum of row i.
     float dsum = 0.f;
-    if (mbar_wait(&sh.q_full, 0, abort)) {
+    if ((!fwd_done || flag_wait(fwd_done + item, token, abort)) &&
+        mbar_wait(&sh.q_full, 0, abort)) {
       const int half = lane >> 4, c = lane & 15;   // row of the pair, 16-byte chunk
       const uint8_t* dO_m = smem + L::kDO + m * 32768;
       uint4 ov[16];
@@ -294,6 +307,12 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
       }
     }
     dvec[rix] = dsum;
+    if (d_done) {
+      // fused: the last of this CTA's rows to write D publishes the item
+      __threadfence();
+      if (atomicAdd(&sh.d_arrived, 1) == 128 * MT - 1 && !*abort)
+        flag_release(d_done + item, token);
+    }
     const float lse2 = lse[rix] * 1.4426950408889634f;
     const float2 c2 = make_float2(scale_log2, scale_log2);
     const float2 nl = make_float2(-lse2, -lse2);
@@ -362,6 +381,9 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }
+  // fused: this grid completes only after the forward grid has, so that the
+  // kernels after it on the stream see both complete
+  if (fwd_done) pdl_wait();
 }
 
 // ------------------------------------------------------------------------
@@ -414,7 +436,8 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
                             int topk_groups, const int32_t* __restrict__ sel_grp, float scale,
                             float scale_log2, const float* __restrict__ lse,
                             const float* __restrict__ dvec, __nv_bfloat16* __restrict__ dk,
-                            __nv_bfloat16* __restrict__ dv, int* __restrict__ unit_counter) {
+                            __nv_bfloat16* __restrict__ dv, int* __restrict__ unit_counter,
+                            const int* __restrict__ d_done, uint32_t token) {
   using L = KvLayout;
   constexpr int G = 2 * MT;
   extern __shared__ uint8_t dsmem_raw[];
@@ -443,8 +466,11 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
     fence_barrier_init();
   }
   // the previous kernel may still hold this SM's tensor memory or write
-  // this kernel's inputs (the dQ kernel zeroes the unit counter): wait for it
-  pdl_wait();
+  // this kernel's inputs (the dQ kernel zeroes the unit counter): wait for
+  // it.  In a fused forward + backward each unit instead waits for the D of
+  // the query blocks it visits (d_done); the counter was zeroed before the
+  // dQ grid let this one start, and the two kernels' CTAs cannot share an SM.
+  if (!d_done) pdl_wait();
   if (tid == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_do);
@@ -527,6 +553,12 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const int n_items = sh.n_items;
+    if (d_done) {
+      // fused: D (and, through the dQ kernel, LSE) of every visited query block
+      for (int q = tid; q < n_items / MT; q += blockDim.x)
+        flag_wait(d_done + bh * n_qb + sh.js[q], token, abort);
+      __syncthreads();
+    }
 
     if (warp == 0) {
       // ---------------- TMA producer (whole warp; one elected lane issues) --
@@ -726,6 +758,8 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }
+  // fused: this grid completes only after the dQ grid has
+  if (d_done) pdl_wait();
 }
 
 }  // namespace bwdtc

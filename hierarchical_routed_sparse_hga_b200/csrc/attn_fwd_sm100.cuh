@@ -84,7 +84,8 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, int64_t ctx_cap, int64_t q_begin, int s_len, int n_q_heads, int n_kv_heads,
                        int topk_groups, const int32_t* __restrict__ sel_grp, float scale_log2,
-                       __nv_bfloat16* __restrict__ o, float* __restrict__ lse, uint32_t flags) {
+                       __nv_bfloat16* __restrict__ o, float* __restrict__ lse, uint32_t flags,
+                       int* __restrict__ done, uint32_t token) {
   using L = Layout<MT>;
   extern __shared__ uint8_t dsmem_raw[];
   __shared__ Shared sh;
@@ -101,7 +102,6 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
   const int n_qb = s_len / kQBlock;
   const int64_t own_blk = (q_begin + int64_t(j) * kQBlock) / kBlock;
   volatile int* abort = &sh.abort;
-  pdl_launch_dependents();
 
   // ---- set-up: barriers, the Q load, TMEM, the tile schedule -------------
   if (tid == 0) {
@@ -121,8 +121,11 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
     fence_barrier_init();
   }
   // the previous kernel may still hold this SM's tensor memory or write
-  // this kernel's inputs: wait for it before allocating or reading
+  // this kernel's inputs: wait for it before allocating or reading.  The
+  // next kernel may be scheduled from here on: everything before this
+  // kernel on the stream has completed.
   pdl_wait();
+  pdl_launch_dependents();
   if (tid == 0) {
     // Q first: it does not depend on the selection
     prefetch_tmap(&tm_q);
@@ -353,6 +356,7 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
       }
       lse[orow] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
     }
+    if (done) __threadfence();  // O and LSE before this item's completion flag
   }
 
   tc_fence_before();
@@ -362,6 +366,9 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }
+  // fused forward + backward: this item's O and LSE are written
+  if (done && tid == 0 && !*abort)
+    flag_release(done + blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z), token);
 }
 
 }  // namespace fwdtc

@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -162,7 +163,8 @@ bool use_tensor_cores(const hga_config_t* c, int64_t ctx_cap, int32_t s_len) {
 template <int MT>
 hga_status_t launch_fwd_tc(const hga_config_t* cfg, const void* q, const void* k, const void* v,
                            int64_t ctx_cap, int64_t q_begin, int32_t s_len,
-                           const int32_t* sel_grp, void* o, float* lse, cudaStream_t s) {
+                           const int32_t* sel_grp, void* o, float* lse, int* done,
+                           uint32_t token, cudaStream_t s) {
   using L = fwdtc::Layout<MT>;
   CUtensorMap tq, tk, tv;
   const uint64_t q_rows = uint64_t(cfg->batch) * cfg->n_q_heads * s_len;
@@ -180,7 +182,7 @@ hga_status_t launch_fwd_tc(const hga_config_t* cfg, const void* q, const void* k
   return traced_launch(HGA_K_FWD_TC, s, [&] {
     return launch_pdl(fwdtc::attn_fwd_tc_kernel<MT>, grid, dim3(L::kThreads), L::kDynSmem, s, tq,
         tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups, sel_grp,
-        scale_log2, static_cast<__nv_bfloat16*>(o), lse, cfg->flags);
+        scale_log2, static_cast<__nv_bfloat16*>(o), lse, cfg->flags, done, token);
   });
 }
 
@@ -189,7 +191,8 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
                            int64_t ctx_cap, int64_t q_begin, int32_t s_len,
                            const int32_t* sel_grp, const void* o, const float* lse,
                            const void* d_o, void* dq, void* dk, void* dv, float* dvec,
-                           int* unit_counter, cudaStream_t s) {
+                           int* unit_counter, const int* fwd_done, int* d_done, uint32_t token,
+                           cudaStream_t s) {
   using LQ = bwdtc::DqLayout<MT>;
   using LK = bwdtc::KvLayout;
   CUtensorMap tq, tdo, tk, tv;
@@ -212,7 +215,7 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
         ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups, sel_grp,
         cfg->scale, scale_log2, static_cast<const __nv_bfloat16*>(o),
         static_cast<const __nv_bfloat16*>(d_o), lse, static_cast<__nv_bfloat16*>(dq), dvec,
-        unit_counter);
+        unit_counter, fwd_done, d_done, token);
   });
   if (e != HGA_OK) return e;
   // persistent: at most one CTA per SM over the (key block, head) units
@@ -222,7 +225,8 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
     return launch_pdl(bwdtc::attn_bwd_dkdv_tc_kernel<MT>, grid_kv, dim3(LK::kThreads),
         LK::kDynSmem, s, tq, tdo, tk, tv, ctx_cap, q_begin, s_len, cfg->batch, cfg->n_q_heads,
         cfg->n_kv_heads, cfg->topk_groups, sel_grp, cfg->scale, scale_log2, lse, dvec,
-        static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), unit_counter);
+        static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), unit_counter,
+        fwd_done ? d_done : nullptr, token);
   });
 }
 
@@ -418,8 +422,9 @@ hga_status_t hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (use_tensor_cores(cfg, ctx_cap, s_len)) {
     if ((cfg->n_q_heads / cfg->n_kv_heads) % 4 == 0)
-      return launch_fwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, s);
-    return launch_fwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, s);
+      return launch_fwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, nullptr, 0,
+                              s);
+    return launch_fwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, nullptr, 0, s);
   }
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
     const size_t sm = size_t(simt_fwd_smem_floats<D>()) * 4;
@@ -451,15 +456,20 @@ hga_status_t hga_route_noalloc(const hga_config_t* cfg, const void* q, int64_t q
                    HGA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
-// backward workspace: D = rowsum(dO * O) [B, Hq, S] fp32, then (256-B aligned)
-// the work-unit counter of the persistent dK/dV kernel
+// backward workspace, 256-byte aligned sections: D = rowsum(dO * O)
+// [B, Hq, S] fp32; the work-unit counter of the persistent dK/dV kernel;
+// the per-item completion flags of a fused forward + backward, forward
+// items then dQ items, [B, Hkv, S/64] int32 each
 static size_t bwd_dvec_bytes(const hga_config_t* cfg, int32_t s_len) {
   return align256(size_t(cfg->batch) * cfg->n_q_heads * size_t(s_len) * 4);
+}
+static size_t bwd_flag_bytes(const hga_config_t* cfg, int32_t s_len) {
+  return align256(size_t(cfg->batch) * cfg->n_kv_heads * size_t(s_len / kQBlock) * 4);
 }
 
 size_t hga_attn_bwd_workspace_size(const hga_config_t* cfg, int32_t s_len) {
   if (check_cfg(cfg) != HGA_OK || s_len <= 0) return 0;
-  return bwd_dvec_bytes(cfg, s_len) + 256;
+  return bwd_dvec_bytes(cfg, s_len) + 256 + 2 * bwd_flag_bytes(cfg, s_len);
 }
 
 hga_status_t hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k, const void* v,
@@ -482,9 +492,9 @@ hga_status_t hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k,
   if (use_tensor_cores(cfg, ctx_cap, s_len)) {
     if (cfg->n_q_heads / cfg->n_kv_heads == 4)
       return launch_bwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq,
-                              dk, dv, dvec, unit_counter, s);
+                              dk, dv, dvec, unit_counter, nullptr, nullptr, 0, s);
     return launch_bwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk,
-                            dv, dvec, unit_counter, s);
+                            dv, dvec, unit_counter, nullptr, nullptr, 0, s);
   }
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
     const size_t sm1 = size_t(simt_fwd_smem_floats<D>()) * 4;
@@ -512,6 +522,49 @@ hga_status_t hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k,
           static_cast<T*>(dv));
     });
   });
+}
+
+hga_status_t hga_attn_fwd_bwd(const hga_config_t* cfg, const void* q, const void* k,
+                              const void* v, int64_t ctx_cap, int64_t q_begin, int32_t s_len,
+                              const int32_t* sel_grp, void* o, float* lse, const void* d_o,
+                              void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                              void* stream) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
+  const void* ptrs[] = {q, k, v, sel_grp, o, lse, d_o, dq, dk, dv, workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return HGA_ERR_INVALID_ARG;
+  if (ws_bytes < hga_attn_bwd_workspace_size(cfg, s_len)) return HGA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!use_tensor_cores(cfg, ctx_cap, s_len)) {
+    st = hga_attn_fwd(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, stream);
+    if (st != HGA_OK) return st;
+    return hga_attn_bwd(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk, dv,
+                        workspace, ws_bytes, stream);
+  }
+  char* ws = static_cast<char*>(workspace);
+  float* dvec = reinterpret_cast<float*>(ws);
+  int* unit_counter = reinterpret_cast<int*>(ws + bwd_dvec_bytes(cfg, s_len));
+  int* fwd_done = reinterpret_cast<int*>(ws + bwd_dvec_bytes(cfg, s_len) + 256);
+  int* d_done = reinterpret_cast<int*>(reinterpret_cast<char*>(fwd_done) +
+                                       bwd_flag_bytes(cfg, s_len));
+  // a fresh token per call: flags left by earlier calls never match it
+  static std::atomic<uint32_t> next_token{0};
+  uint32_t token = ++next_token;
+  if (token == 0) token = ++next_token;
+  if (cfg->n_q_heads / cfg->n_kv_heads == 4) {
+    st = launch_fwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, fwd_done,
+                          token, s);
+    if (st != HGA_OK) return st;
+    return launch_bwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk,
+                            dv, dvec, unit_counter, fwd_done, d_done, token, s);
+  }
+  st = launch_fwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, fwd_done, token,
+                        s);
+  if (st != HGA_OK) return st;
+  return launch_bwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk,
+                          dv, dvec, unit_counter, fwd_done, d_done, token, s);
 }
 
 namespace {

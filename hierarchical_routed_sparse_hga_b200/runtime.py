@@ -41,7 +41,8 @@ class HgaLayer:
                                 device=self.device)
         ws = max(_lib.hga_route_workspace_size(cfg, seg_len, ctx_cap - seg_len), 256)
         self.route_ws = torch.empty(ws, dtype=torch.uint8, device=self.device)
-        self.bwd_ws = torch.empty(max(_lib.hga_attn_bwd_workspace_size(cfg, seg_len), 256),
+        # zeroed once: hga_attn_fwd_bwd's completion flags live in it
+        self.bwd_ws = torch.zeros(max(_lib.hga_attn_bwd_workspace_size(cfg, seg_len), 256),
                                   dtype=torch.uint8, device=self.device)
         self.sel_blk = torch.empty((B, Hkv, n_qb, cfg.topk_blocks), dtype=torch.int32,
                                    device=self.device)
@@ -71,13 +72,21 @@ class HgaLayer:
                           self.sel_grp, self.o, self.lse, d_o, self.dq, self.dk, self.dv,
                           self.bwd_ws, stream=stream)
 
+    def forward_backward(self, q, d_o, q_begin: int, stream=None):
+        _lib.hga_attn_fwd_bwd(self.cfg, q, self.k, self.v, self.ctx_cap, q_begin, self.seg_len,
+                              self.sel_grp, self.o, self.lse, d_o, self.dq, self.dk, self.dv,
+                              self.bwd_ws, stream=stream)
+
     def segment(self, q, q_begin: int, d_o=None, stream=None):
-        """One segment: summaries, routing, forward and (if d_o) backward."""
+        """One segment: summaries, routing, forward and (if d_o) backward
+        (fused, so that the backward of each query block starts as soon as
+        its forward is done)."""
         self.summarize(q_begin, stream)
         self.route(q, q_begin, stream)
-        self.forward(q, q_begin, stream)
-        if d_o is not None:
-            self.backward(q, d_o, q_begin, stream)
+        if d_o is None:
+            self.forward(q, q_begin, stream)
+        else:
+            self.forward_backward(q, d_o, q_begin, stream)
 
 
 class HgaTieredLayer:

@@ -201,9 +201,11 @@ HGA_API hga_status_t hga_route_noalloc(const hga_config_t* cfg, const void* q, i
                                        const float* gsum, int32_t* sel_blk, int32_t* sel_grp,
                                        void* stream);
 
-/* Bytes of device workspace hga_attn_bwd needs for this segment: D =
- * rowsum(dO * O) as [B, Hq, S] fp32 (256-byte aligned), then 256 bytes for
- * the work counter of the tensor-core dK/dV kernel. */
+/* Bytes of device workspace hga_attn_bwd and hga_attn_fwd_bwd need for this
+ * segment: D = rowsum(dO * O) as [B, Hq, S] fp32, 256 bytes for the work
+ * counter of the tensor-core dK/dV kernel, and two arrays of per-item
+ * completion flags ([B, Hkv, S/64] int32 each) used by hga_attn_fwd_bwd;
+ * every section starts on a 256-byte boundary. */
 HGA_API size_t hga_attn_bwd_workspace_size(const hga_config_t* cfg, int32_t s_len);
 
 /*
@@ -222,6 +224,25 @@ HGA_API hga_status_t hga_attn_bwd(const hga_config_t* cfg, const void* q, const 
                           const int32_t* sel_grp, const void* o, const float* lse,
                           const void* d_o, void* dq, void* dk, void* dv, void* workspace,
                           size_t ws_bytes, void* stream);
+
+/*
+ * Steps a4 + a5 in one call: hga_attn_fwd then hga_attn_bwd for the same
+ * segment, with the same arguments and results (o, lse, dq, dk, dv).  On the
+ * tensor-core path the three kernels overlap: the dQ work of a query block
+ * starts as soon as that block's forward is done, and the dK/dV work of a
+ * key block as soon as D of the query blocks that attend to it is, through
+ * per-item completion flags in the workspace instead of whole-grid waits.
+ * The flag sections of the workspace must be zero before its first use in
+ * this call (e.g. one cudaMemset of the whole workspace after allocating
+ * it); each call leaves them holding its own token, which later calls never
+ * reuse.  Not to be called concurrently with another call on the same
+ * workspace.
+ */
+HGA_API hga_status_t hga_attn_fwd_bwd(const hga_config_t* cfg, const void* q, const void* k,
+                              const void* v, int64_t ctx_cap, int64_t q_begin, int32_t s_len,
+                              const int32_t* sel_grp, void* o, float* lse, const void* d_o,
+                              void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                              void* stream);
 
 /*
  * Step a7 -- the host tier [A] ("older KV is detached into RAM or NVMe, and

@@ -11,7 +11,7 @@ import pytest
 
 from hierarchical_routed_sparse_hga_b200 import synth
 
-from hga_testlib import Segmenter, compare_segment
+from hga_testlib import Segmenter, compare_segment, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -48,6 +48,30 @@ def test_qwen3_fwd_128k_sampled():
     # 64 segments on the GPU; segments 0, 31 and 63 checked on two KV heads
     w = WL["qwen3_fwd_128k"]
     run_and_compare(w, segments=[0, 31 * 2048, 63 * 2048], kv_heads=[0, 5])
+
+
+def test_fused_call_equals_separate_calls():
+    # hga_attn_fwd_bwd (kernels chained by per-item flags) against
+    # hga_attn_fwd + hga_attn_bwd (whole-grid waits) on the same inputs: the
+    # same kernels and arithmetic, so every output is bit-identical; two
+    # segments in a row exercise the flags' per-call tokens
+    import torch
+    w = WL["qwen3_fwdbwd_16k"]
+    seg = Segmenter(w)
+    L = seg.layer
+    for q_begin in (12288, 14336):
+        q = to_device(synth.queries(w, q_begin), w)
+        d_o = to_device(synth.douts(w, q_begin), w)
+        L.summarize(q_begin)
+        L.route(q, q_begin)
+        L.forward_backward(q, d_o, q_begin)
+        torch.cuda.synchronize()
+        fused = [t.clone() for t in (L.o, L.lse, L.dq, L.dk, L.dv)]
+        L.forward(q, q_begin)
+        L.backward(q, d_o, q_begin)
+        torch.cuda.synchronize()
+        for a, b in zip(fused, (L.o, L.lse, L.dq, L.dk, L.dv)):
+            assert torch.equal(a, b), q_begin
 
 
 def test_largest_segment_and_topk():
