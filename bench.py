@@ -345,19 +345,56 @@ class Runner:
                 record_sel.append((q_begin, L.sel_grp.cpu().numpy()))
 
     def e2e_step(self, out_host):
-        """Host buffers in, host buffers out: H2D of the step's inputs, the step,
-        D2H of every segment's outputs (all on the current stream)."""
-        L = self.layer
-        L.k.copy_(self.k_host, non_blocking=True)
-        L.v.copy_(self.v_host, non_blocking=True)
+        """Host buffers in, host buffers out, through the runtime: every
+        segment's K/V rows, Q and dO go up on an upload stream (segment i's
+        while segment i-1 computes), the segment runs on the current stream,
+        and its outputs come down on a download stream while the next segment
+        computes (two output sets alternate).  The step ends when the last
+        outputs are on the host."""
+        import torch
+        L, w = self.layer, self.w
+        if not hasattr(self, "s_up"):
+            self.s_up = torch.cuda.Stream(self.device)
+            self.s_down = torch.cuda.Stream(self.device)
+            self.out_sets = [L.make_outputs() for _ in range(2)]
+        comp = torch.cuda.current_stream(self.device)
+        # this step's uploads overwrite what the previous step computed from
+        self.s_up.wait_stream(comp)
+        up_done = []
+        with torch.cuda.stream(self.s_up):
+            for i, q_begin in enumerate(self.segs):
+                lo = 0 if i == 0 else q_begin          # history rows go with the first
+                hi = q_begin + w.seg_len
+                # one contiguous block per (batch, KV head): a strided slice
+                # copy from pinned memory is staged through the host
+                for bb in range(w.batch):
+                    for hh in range(w.n_kv_heads):
+                        L.k[bb, hh, lo:hi].copy_(self.k_host[bb, hh, lo:hi], non_blocking=True)
+                        L.v[bb, hh, lo:hi].copy_(self.v_host[bb, hh, lo:hi], non_blocking=True)
+                self.q[i].copy_(self.q_host[i], non_blocking=True)
+                if w.backward:
+                    self.do[i].copy_(self.do_host[i], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(self.s_up)
+                up_done.append(ev)
+        down_done = []
         for i, q_begin in enumerate(self.segs):
-            self.q[i].copy_(self.q_host[i], non_blocking=True)
-            if self.w.backward:
-                self.do[i].copy_(self.do_host[i], non_blocking=True)
-            L.segment(self.q[i], q_begin, self.do[i] if self.w.backward else None)
-            outs = (L.o, L.dq, L.dk, L.dv) if self.w.backward else (L.o,)
-            for dst, src in zip(out_host[i], outs):
-                dst.copy_(src, non_blocking=True)
+            comp.wait_event(up_done[i])
+            if i >= 2:
+                comp.wait_event(down_done[i - 2])       # its output set is free again
+            out = self.out_sets[i & 1]
+            L.segment(self.q[i], q_begin, self.do[i] if w.backward else None, out=out)
+            ev = torch.cuda.Event()
+            ev.record(comp)
+            self.s_down.wait_event(ev)
+            srcs = (out[0], out[2], out[3], out[4]) if w.backward else (out[0],)
+            with torch.cuda.stream(self.s_down):
+                for dst, src in zip(out_host[i], srcs):
+                    dst.copy_(src, non_blocking=True)
+                ev2 = torch.cuda.Event()
+                ev2.record(self.s_down)
+                down_done.append(ev2)
+        comp.wait_stream(self.s_down)
 
     def io_bytes(self):
         nb = lambda t: t.numel() * t.element_size()  # noqa: E731

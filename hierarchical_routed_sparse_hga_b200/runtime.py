@@ -63,30 +63,41 @@ class HgaLayer:
         _lib.hga_route(self.cfg, q, q_begin, self.seg_len, self.ctx_cap, self.bsum,
                        self.gsum, self.sel_blk, self.sel_grp, self.route_ws, stream=stream)
 
-    def forward(self, q, q_begin: int, stream=None):
+    def make_outputs(self):
+        """A fresh set of per-segment outputs (o, lse, dq, dk, dv), for callers
+        that keep one segment's results while the next one is computed."""
+        return (torch.empty_like(self.o), torch.empty_like(self.lse), torch.empty_like(self.dq),
+                torch.empty_like(self.dk), torch.empty_like(self.dv))
+
+    def _out(self, out):
+        return (self.o, self.lse, self.dq, self.dk, self.dv) if out is None else out
+
+    def forward(self, q, q_begin: int, stream=None, out=None):
+        o, lse = self._out(out)[:2]
         _lib.hga_attn_fwd(self.cfg, q, self.k, self.v, self.ctx_cap, q_begin, self.seg_len,
-                          self.sel_grp, self.o, self.lse, stream)
+                          self.sel_grp, o, lse, stream)
 
-    def backward(self, q, d_o, q_begin: int, stream=None):
+    def backward(self, q, d_o, q_begin: int, stream=None, out=None):
+        o, lse, dq, dk, dv = self._out(out)
         _lib.hga_attn_bwd(self.cfg, q, self.k, self.v, self.ctx_cap, q_begin, self.seg_len,
-                          self.sel_grp, self.o, self.lse, d_o, self.dq, self.dk, self.dv,
-                          self.bwd_ws, stream=stream)
+                          self.sel_grp, o, lse, d_o, dq, dk, dv, self.bwd_ws, stream=stream)
 
-    def forward_backward(self, q, d_o, q_begin: int, stream=None):
+    def forward_backward(self, q, d_o, q_begin: int, stream=None, out=None):
+        o, lse, dq, dk, dv = self._out(out)
         _lib.hga_attn_fwd_bwd(self.cfg, q, self.k, self.v, self.ctx_cap, q_begin, self.seg_len,
-                              self.sel_grp, self.o, self.lse, d_o, self.dq, self.dk, self.dv,
-                              self.bwd_ws, stream=stream)
+                              self.sel_grp, o, lse, d_o, dq, dk, dv, self.bwd_ws, stream=stream)
 
-    def segment(self, q, q_begin: int, d_o=None, stream=None):
+    def segment(self, q, q_begin: int, d_o=None, stream=None, out=None):
         """One segment: summaries, routing, forward and (if d_o) backward
         (fused, so that the backward of each query block starts as soon as
-        its forward is done)."""
+        its forward is done).  Results go to `out` (from make_outputs) if
+        given, else to the layer's own o, lse, dq, dk, dv."""
         self.summarize(q_begin, stream)
         self.route(q, q_begin, stream)
         if d_o is None:
-            self.forward(q, q_begin, stream)
+            self.forward(q, q_begin, stream, out)
         else:
-            self.forward_backward(q, d_o, q_begin, stream)
+            self.forward_backward(q, d_o, q_begin, stream, out)
 
 
 class HgaTieredLayer:
