@@ -74,6 +74,26 @@ def test_fused_call_equals_separate_calls():
             assert torch.equal(a, b), q_begin
 
 
+def test_segment_into_caller_output_set():
+    # HgaLayer.segment(..., out=make_outputs()): the same results, written to
+    # the caller's tensors (used to download one segment while the next runs)
+    import torch
+    w = WL["qwen3_fwdbwd_16k"]
+    seg = Segmenter(w)
+    L = seg.layer
+    q_begin = 14336
+    q = to_device(synth.queries(w, q_begin), w)
+    d_o = to_device(synth.douts(w, q_begin), w)
+    L.segment(q, q_begin, d_o)
+    torch.cuda.synchronize()
+    own = [t.clone() for t in (L.o, L.lse, L.dq, L.dk, L.dv)]
+    out = L.make_outputs()
+    L.segment(q, q_begin, d_o, out=out)
+    torch.cuda.synchronize()
+    for a, b in zip(own, out):
+        assert torch.equal(a, b)
+
+
 def test_largest_segment_and_topk():
     # the largest segment (4096 tokens: 64 query blocks, which fills the dK/dV
     # kernel's per-unit query-block lists) with the largest k_g (256 groups:
