@@ -180,7 +180,7 @@ __device__ int block_enumerate(int n, Pred pred, Fn f, int* scratch) {
 // ---------------------------------------------------------------------------
 // block-wide top-k of n distinct-or-not uint32 keys held in shared memory:
 // sets sel[i] = 1 for the k largest keys, ties broken toward the lower index.
-// Up to 512 keys: rank counting (below).  Otherwise a radix select on 8-bit
+// Up to 128 keys: rank counting (below).  Otherwise a radix select on 8-bit
 // digits (MSB first) finds the k-th largest key T; keys above T are taken,
 // and among keys equal to T the lowest indices fill the remaining slots.
 // Needs hist[256] and scratch (see block_enumerate).
@@ -193,7 +193,7 @@ __device__ void block_topk(const uint32_t* key, int n, int k, uint8_t* sel, int*
     __syncthreads();
     return;
   }
-  if (n <= 512) {
+  if (n <= 128) {
     // rank by counting: rank(i) = #{keys above key[i]} + #{equal keys before i};
     // the k smallest ranks are the k largest keys, ties to the lower index.
     // O(n^2) comparisons with broadcast shared-memory reads, no barrier.
