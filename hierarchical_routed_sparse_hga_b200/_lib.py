@@ -25,6 +25,7 @@ HGA_FLAG_SIMT = 1
 EXPORTS = ("hga_version", "hga_status_string", "hga_build_summaries",
            "hga_route_workspace_size", "hga_route", "hga_attn_fwd",
            "hga_attn_bwd_workspace_size", "hga_attn_bwd", "hga_attn_fwd_bwd",
+           "hga_segment_workspace_size", "hga_segment_fwd_bwd",
            "hga_get_device_status",
            "hga_kernel_name", "hga_launch_count", "hga_timing_enable", "hga_timing_collect",
            "hga_timing_get", "hga_timing_reset", "hga_timing_kinds", "hga_route_noalloc",
@@ -94,6 +95,9 @@ def load() -> ctypes.CDLL:
                                         P, SZ, P]),
         "hga_attn_fwd_bwd": (ctypes.c_int, [CFG, P, P, P, I64, I64, I32, P, P, P, P, P, P, P,
                                             P, SZ, P]),
+        "hga_segment_workspace_size": (SZ, [CFG, I32, I64]),
+        "hga_segment_fwd_bwd": (ctypes.c_int, [CFG, P, P, P, I64, I64, I32, P, P, P, P, P, P,
+                                               P, P, P, P, P, SZ, P]),
         "hga_get_device_status": (ctypes.c_int, [P]),
         "hga_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
         "hga_launch_count": (ctypes.c_uint64, []),
@@ -270,6 +274,24 @@ def hga_attn_fwd_bwd(cfg: Config, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, 
         _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes,
         _stream(stream)))
 
+
+def hga_segment_workspace_size(cfg: Config, s_len, q_begin) -> int:
+    c = cfg.c()
+    return int(load().hga_segment_workspace_size(ctypes.byref(c), s_len, q_begin))
+
+
+def hga_segment_fwd_bwd(cfg: Config, q, k, v, ctx_cap, q_begin, s_len, bsum, gsum, sel_blk,
+                        sel_grp, o, lse, d_o, dq, dk, dv, workspace, ws_bytes=None,
+                        stream=None):
+    """hga_route then hga_attn_fwd_bwd in one call (the forward of a query
+    block waits only for its own selection); sel_blk may be None; the
+    workspace's flag sections must be zero before its first use."""
+    c = cfg.c()
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check("hga_segment_fwd_bwd", load().hga_segment_fwd_bwd(
+        ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), ctx_cap, q_begin, s_len, _ptr(bsum),
+        _ptr(gsum), _ptr(sel_blk), _ptr(sel_grp), _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq),
+        _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, _stream(stream)))
 
 def hga_get_device_status(stream=None) -> int:
     return int(load().hga_get_device_status(_stream(stream)))

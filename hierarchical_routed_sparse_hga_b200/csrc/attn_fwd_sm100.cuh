@@ -85,7 +85,8 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
                        const __grid_constant__ CUtensorMap tm_v, int64_t ctx_cap, int64_t q_begin, int s_len, int n_q_heads, int n_kv_heads,
                        int topk_groups, const int32_t* __restrict__ sel_grp, float scale_log2,
                        __nv_bfloat16* __restrict__ o, float* __restrict__ lse, uint32_t flags,
-                       int* __restrict__ done, uint32_t token) {
+                       const int* __restrict__ route_done, int* __restrict__ done,
+                       uint32_t token) {
   using L = Layout<MT>;
   extern __shared__ uint8_t dsmem_raw[];
   __shared__ Shared sh;
@@ -121,11 +122,11 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
     fence_barrier_init();
   }
   // the previous kernel may still hold this SM's tensor memory or write
-  // this kernel's inputs: wait for it before allocating or reading.  The
-  // next kernel may be scheduled from here on: everything before this
-  // kernel on the stream has completed.
-  pdl_wait();
-  pdl_launch_dependents();
+  // this kernel's inputs: wait for it before allocating or reading.  In a
+  // chained segment call the previous kernel is the routing, which has no
+  // tensor memory and let this grid start only once everything before it
+  // had completed: only this item's selection is waited for (route_done).
+  if (!route_done) pdl_wait();
   if (tid == 0) {
     // Q first: it does not depend on the selection
     prefetch_tmap(&tm_q);
@@ -144,12 +145,19 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
     tmem_alloc(&sh.tmem_base, L::kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 0)
+  if (warp == 0) {
+    if (route_done)
+      flag_wait(route_done + blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z),
+                token, abort);
     build_tile_schedule(sh, sel_grp + ((int64_t(b) * n_kv_heads + h) * n_qb + j) * topk_groups,
                         topk_groups, own_blk, lane);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the next kernel may be scheduled from here on (this item's selection,
+  // and everything the routing waited for, are complete)
+  pdl_launch_dependents();
   const uint32_t tmem = sh.tmem_base;
   const int n_tiles = sh.n_tiles;
 
@@ -369,6 +377,8 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
   // fused forward + backward: this item's O and LSE are written
   if (done && tid == 0 && !*abort)
     flag_release(done + blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z), token);
+  // chained: this grid completes only after the routing grid has
+  if (route_done) pdl_wait();
 }
 
 }  // namespace fwdtc

@@ -36,6 +36,32 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Per-item completion flags between the kernels of one fused call: the
+// producing CTA stores the call's token with release semantics after its
+// writes (every writing thread fenced first); the consuming thread waits,
+// bounded, until it reads the token with acquire semantics.  On timeout it
+// latches HGA_ERR_TIMEOUT, raises *abort and returns false.
+__device__ __forceinline__ void flag_release(int* flag, uint32_t token) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(token) : "memory");
+}
+
+__device__ __forceinline__ bool flag_wait(const int* flag, uint32_t token, volatile int* abort,
+                                          long long limit_cycles = 2000000000LL) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v == token) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > limit_cycles) {
+      latch_status(HGA_ERR_TIMEOUT);
+      *abort = 1;
+      return false;
+    }
+    __nanosleep(100);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // element loads: 8 consecutive elements -> 8 floats (16 B for bf16, 32 B for f32)
 // ---------------------------------------------------------------------------

@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <initializer_list>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -163,8 +164,8 @@ bool use_tensor_cores(const hga_config_t* c, int64_t ctx_cap, int32_t s_len) {
 template <int MT>
 hga_status_t launch_fwd_tc(const hga_config_t* cfg, const void* q, const void* k, const void* v,
                            int64_t ctx_cap, int64_t q_begin, int32_t s_len,
-                           const int32_t* sel_grp, void* o, float* lse, int* done,
-                           uint32_t token, cudaStream_t s) {
+                           const int32_t* sel_grp, void* o, float* lse, const int* route_done,
+                           int* done, uint32_t token, cudaStream_t s) {
   using L = fwdtc::Layout<MT>;
   CUtensorMap tq, tk, tv;
   const uint64_t q_rows = uint64_t(cfg->batch) * cfg->n_q_heads * s_len;
@@ -182,7 +183,7 @@ hga_status_t launch_fwd_tc(const hga_config_t* cfg, const void* q, const void* k
   return traced_launch(HGA_K_FWD_TC, s, [&] {
     return launch_pdl(fwdtc::attn_fwd_tc_kernel<MT>, grid, dim3(L::kThreads), L::kDynSmem, s, tq,
         tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups, sel_grp,
-        scale_log2, static_cast<__nv_bfloat16*>(o), lse, cfg->flags, done, token);
+        scale_log2, static_cast<__nv_bfloat16*>(o), lse, cfg->flags, route_done, done, token);
   });
 }
 
@@ -349,9 +350,14 @@ size_t hga_route_workspace_size(const hga_config_t* cfg, int32_t s_len, int64_t 
   return route_carve(cfg, s_len, q_begin, nullptr).bytes;
 }
 
-hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, int32_t s_len,
-                       int64_t ctx_cap, const float* bsum, const float* gsum, int32_t* sel_blk,
-                       int32_t* sel_grp, void* workspace, size_t ws_bytes, void* stream) {
+// The routing of hga_route.  With `done`, a fused routing launch also stores
+// `token` into done[item] once item's selections are written (chained
+// segment call); the three-launch path ignores it.
+static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q_begin,
+                               int32_t s_len, int64_t ctx_cap, const float* bsum,
+                               const float* gsum, int32_t* sel_blk, int32_t* sel_grp,
+                               void* workspace, size_t ws_bytes, int* done, uint32_t token,
+                               cudaStream_t s) {
   hga_status_t st = check_cfg(cfg);
   if (st != HGA_OK) return st;
   if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
@@ -364,7 +370,6 @@ hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, 
   const int n_qb = s_len / kQBlock;
   const int64_t own0 = q_begin / kBlock;
   const int64_t j_max = own0 + n_qb - 1;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int G = cfg->n_q_heads / cfg->n_kv_heads;
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
     if (j_max <= kFusedRouteMaxBlocks) {
@@ -377,7 +382,7 @@ hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, 
         return launch_pdl(route_fused_kernel<T, D>, g1, dim3(kRouteThreads), smf, s,
                           static_cast<const T*>(q), bsum, gsum, ctx_cap, cfg->n_q_heads,
                           cfg->n_kv_heads, s_len, own0, cfg->topk_blocks, cfg->topk_groups,
-                          sel_blk, sel_grp);
+                          sel_blk, sel_grp, done, token);
       });
     }
     dim3 g0(n_qb * G, cfg->n_kv_heads, cfg->batch);
@@ -408,6 +413,18 @@ hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, 
   });
 }
 
+// whether route_impl takes the one-launch path
+static bool route_fused(int64_t q_begin, int32_t s_len) {
+  return q_begin / kBlock + s_len / kQBlock - 1 <= kFusedRouteMaxBlocks;
+}
+
+hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, int32_t s_len,
+                       int64_t ctx_cap, const float* bsum, const float* gsum, int32_t* sel_blk,
+                       int32_t* sel_grp, void* workspace, size_t ws_bytes, void* stream) {
+  return route_impl(cfg, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp, workspace,
+                    ws_bytes, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
+
 hga_status_t hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k, const void* v,
                           int64_t ctx_cap, int64_t q_begin, int32_t s_len,
                           const int32_t* sel_grp, void* o, float* lse, void* stream) {
@@ -422,9 +439,10 @@ hga_status_t hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (use_tensor_cores(cfg, ctx_cap, s_len)) {
     if ((cfg->n_q_heads / cfg->n_kv_heads) % 4 == 0)
-      return launch_fwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, nullptr, 0,
-                              s);
-    return launch_fwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, nullptr, 0, s);
+      return launch_fwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, nullptr,
+                              nullptr, 0, s);
+    return launch_fwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, nullptr,
+                            nullptr, 0, s);
   }
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
     const size_t sm = size_t(simt_fwd_smem_floats<D>()) * 4;
@@ -524,24 +542,26 @@ hga_status_t hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k,
   });
 }
 
-hga_status_t hga_attn_fwd_bwd(const hga_config_t* cfg, const void* q, const void* k,
-                              const void* v, int64_t ctx_cap, int64_t q_begin, int32_t s_len,
-                              const int32_t* sel_grp, void* o, float* lse, const void* d_o,
-                              void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
-                              void* stream) {
-  hga_status_t st = check_cfg(cfg);
-  if (st != HGA_OK) return st;
-  if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
-  const void* ptrs[] = {q, k, v, sel_grp, o, lse, d_o, dq, dk, dv, workspace};
-  for (const void* p : ptrs)
-    if (!p || !aligned16(p)) return HGA_ERR_INVALID_ARG;
-  if (ws_bytes < hga_attn_bwd_workspace_size(cfg, s_len)) return HGA_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+static uint32_t next_call_token() {
+  // a fresh token per chained call: flags left by earlier calls never match
+  static std::atomic<uint32_t> next{0};
+  uint32_t token = ++next;
+  if (token == 0) token = ++next;
+  return token;
+}
+
+// hga_attn_fwd_bwd on a checked configuration; with route_done, the forward
+// waits for each item's routing flag instead of the whole routing grid
+static hga_status_t fwd_bwd_impl(const hga_config_t* cfg, const void* q, const void* k,
+                                 const void* v, int64_t ctx_cap, int64_t q_begin, int32_t s_len,
+                                 const int32_t* sel_grp, void* o, float* lse, const void* d_o,
+                                 void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                                 const int* route_done, uint32_t token, cudaStream_t s) {
   if (!use_tensor_cores(cfg, ctx_cap, s_len)) {
-    st = hga_attn_fwd(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, stream);
+    hga_status_t st = hga_attn_fwd(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, s);
     if (st != HGA_OK) return st;
     return hga_attn_bwd(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk, dv,
-                        workspace, ws_bytes, stream);
+                        workspace, ws_bytes, s);
   }
   char* ws = static_cast<char*>(workspace);
   float* dvec = reinterpret_cast<float*>(ws);
@@ -549,22 +569,77 @@ hga_status_t hga_attn_fwd_bwd(const hga_config_t* cfg, const void* q, const void
   int* fwd_done = reinterpret_cast<int*>(ws + bwd_dvec_bytes(cfg, s_len) + 256);
   int* d_done = reinterpret_cast<int*>(reinterpret_cast<char*>(fwd_done) +
                                        bwd_flag_bytes(cfg, s_len));
-  // a fresh token per call: flags left by earlier calls never match it
-  static std::atomic<uint32_t> next_token{0};
-  uint32_t token = ++next_token;
-  if (token == 0) token = ++next_token;
+  hga_status_t st;
   if (cfg->n_q_heads / cfg->n_kv_heads == 4) {
-    st = launch_fwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, fwd_done,
-                          token, s);
+    st = launch_fwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, route_done,
+                          fwd_done, token, s);
     if (st != HGA_OK) return st;
     return launch_bwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk,
                             dv, dvec, unit_counter, fwd_done, d_done, token, s);
   }
-  st = launch_fwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, fwd_done, token,
-                        s);
+  st = launch_fwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, route_done,
+                        fwd_done, token, s);
   if (st != HGA_OK) return st;
   return launch_bwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk,
                           dv, dvec, unit_counter, fwd_done, d_done, token, s);
+}
+
+static hga_status_t check_fwd_bwd_args(const hga_config_t* cfg, int64_t ctx_cap, int64_t q_begin,
+                                       int32_t s_len, std::initializer_list<const void*> ptrs) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return HGA_ERR_INVALID_ARG;
+  return HGA_OK;
+}
+
+hga_status_t hga_attn_fwd_bwd(const hga_config_t* cfg, const void* q, const void* k,
+                              const void* v, int64_t ctx_cap, int64_t q_begin, int32_t s_len,
+                              const int32_t* sel_grp, void* o, float* lse, const void* d_o,
+                              void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                              void* stream) {
+  hga_status_t st = check_fwd_bwd_args(cfg, ctx_cap, q_begin, s_len,
+                                       {q, k, v, sel_grp, o, lse, d_o, dq, dk, dv, workspace});
+  if (st != HGA_OK) return st;
+  if (ws_bytes < hga_attn_bwd_workspace_size(cfg, s_len)) return HGA_ERR_WORKSPACE;
+  return fwd_bwd_impl(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk, dv,
+                      workspace, ws_bytes, nullptr, next_call_token(),
+                      static_cast<cudaStream_t>(stream));
+}
+
+size_t hga_segment_workspace_size(const hga_config_t* cfg, int32_t s_len, int64_t q_begin) {
+  if (check_cfg(cfg) != HGA_OK || s_len <= 0 || q_begin < 0) return 0;
+  return hga_attn_bwd_workspace_size(cfg, s_len) + bwd_flag_bytes(cfg, s_len) +
+         align256(hga_route_workspace_size(cfg, s_len, q_begin));
+}
+
+hga_status_t hga_segment_fwd_bwd(const hga_config_t* cfg, const void* q, const void* k,
+                                 const void* v, int64_t ctx_cap, int64_t q_begin, int32_t s_len,
+                                 const float* bsum, const float* gsum, int32_t* sel_blk,
+                                 int32_t* sel_grp, void* o, float* lse, const void* d_o, void* dq,
+                                 void* dk, void* dv, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  hga_status_t st = check_fwd_bwd_args(
+      cfg, ctx_cap, q_begin, s_len,
+      {q, k, v, bsum, gsum, sel_grp, o, lse, d_o, dq, dk, dv, workspace});
+  if (st != HGA_OK) return st;
+  if (sel_blk && !aligned16(sel_blk)) return HGA_ERR_INVALID_ARG;
+  if (ws_bytes < hga_segment_workspace_size(cfg, s_len, q_begin)) return HGA_ERR_WORKSPACE;
+  // workspace: [backward workspace][routing flags][routing workspace]
+  const size_t bwd_bytes = hga_attn_bwd_workspace_size(cfg, s_len);
+  char* ws = static_cast<char*>(workspace);
+  int* route_done = reinterpret_cast<int*>(ws + bwd_bytes);
+  char* route_ws = ws + bwd_bytes + bwd_flag_bytes(cfg, s_len);
+  const size_t route_bytes = ws_bytes - bwd_bytes - bwd_flag_bytes(cfg, s_len);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint32_t token = next_call_token();
+  const bool chain = use_tensor_cores(cfg, ctx_cap, s_len) && route_fused(q_begin, s_len);
+  st = route_impl(cfg, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp, route_ws,
+                  route_bytes, chain ? route_done : nullptr, token, s);
+  if (st != HGA_OK) return st;
+  return fwd_bwd_impl(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk, dv,
+                      workspace, bwd_bytes, chain ? route_done : nullptr, token, s);
 }
 
 namespace {

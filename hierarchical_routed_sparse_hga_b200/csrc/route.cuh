@@ -309,9 +309,12 @@ __global__ void __launch_bounds__(kRouteThreads)
     route_fused_kernel(const T* __restrict__ q, const float* __restrict__ bsum,
                        const float* __restrict__ gsum, int64_t ctx_cap, int n_q_heads,
                        int n_kv_heads, int s_len, int64_t own0, int topk_blocks, int topk_groups,
-                       int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp) {
-  pdl_launch_dependents();
+                       int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp,
+                       int* __restrict__ done, uint32_t token) {
+  // the next kernel may be scheduled once everything before this one has
+  // completed (a chained forward reads only its own item's selection)
   pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(16) unsigned char sm_raw[];
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int G = n_q_heads / n_kv_heads, n_qb = s_len / kQBlock;
@@ -355,6 +358,13 @@ __global__ void __launch_bounds__(kRouteThreads)
   __syncthreads();
   select_levels<D>(L, sm_raw, gsum, head, ctx_cap, n_qb, j, J, topk_blocks, topk_groups, sel_blk,
                    sel_grp);
+  if (done) {
+    // chained segment call: this item's selections are written
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0)
+      flag_release(done + blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z), token);
+  }
 }
 
 }  // namespace hga

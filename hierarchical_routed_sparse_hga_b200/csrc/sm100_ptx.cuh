@@ -105,32 +105,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// Per-item completion flags between the kernels of one fused call: the
-// producing CTA stores the call's token with release semantics after its
-// writes (every writing thread fenced first); the consuming thread waits,
-// bounded, until it reads the token with acquire semantics.  On timeout it
-// latches HGA_ERR_TIMEOUT, raises *abort and returns false.
-__device__ __forceinline__ void flag_release(int* flag, uint32_t token) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(token) : "memory");
-}
-
-__device__ __forceinline__ bool flag_wait(const int* flag, uint32_t token, volatile int* abort,
-                                          long long limit_cycles = 2000000000LL) {
-  const long long t0 = clock64();
-  while (true) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
-    if (v == token) return true;
-    if (*abort) return false;
-    if (clock64() - t0 > limit_cycles) {
-      latch_status(HGA_ERR_TIMEOUT);
-      *abort = 1;
-      return false;
-    }
-    __nanosleep(100);
-  }
-}
-
 // One step of the idle bookkeeping of an event loop run by a whole warp:
 // after progress the idle clock restarts; otherwise the loop ends (false) if
 // another role raised *abort, or -- latching HGA_ERR_TIMEOUT and raising

@@ -44,6 +44,10 @@ class HgaLayer:
         # zeroed once: hga_attn_fwd_bwd's completion flags live in it
         self.bwd_ws = torch.zeros(max(_lib.hga_attn_bwd_workspace_size(cfg, seg_len), 256),
                                   dtype=torch.uint8, device=self.device)
+        # zeroed once: hga_segment_fwd_bwd's completion flags live in it
+        self.seg_ws = torch.zeros(
+            max(_lib.hga_segment_workspace_size(cfg, seg_len, ctx_cap - seg_len), 256),
+            dtype=torch.uint8, device=self.device)
         self.sel_blk = torch.empty((B, Hkv, n_qb, cfg.topk_blocks), dtype=torch.int32,
                                    device=self.device)
         self.sel_grp = torch.empty((B, Hkv, n_qb, cfg.topk_groups), dtype=torch.int32,
@@ -87,17 +91,24 @@ class HgaLayer:
         _lib.hga_attn_fwd_bwd(self.cfg, q, self.k, self.v, self.ctx_cap, q_begin, self.seg_len,
                               self.sel_grp, o, lse, d_o, dq, dk, dv, self.bwd_ws, stream=stream)
 
+    def route_forward_backward(self, q, d_o, q_begin: int, stream=None, out=None):
+        o, lse, dq, dk, dv = self._out(out)
+        _lib.hga_segment_fwd_bwd(self.cfg, q, self.k, self.v, self.ctx_cap, q_begin,
+                                 self.seg_len, self.bsum, self.gsum, self.sel_blk, self.sel_grp,
+                                 o, lse, d_o, dq, dk, dv, self.seg_ws, stream=stream)
+
     def segment(self, q, q_begin: int, d_o=None, stream=None, out=None):
         """One segment: summaries, routing, forward and (if d_o) backward
-        (fused, so that the backward of each query block starts as soon as
-        its forward is done).  Results go to `out` (from make_outputs) if
-        given, else to the layer's own o, lse, dq, dk, dv."""
+        (chained, so that the forward of each query block starts as soon as
+        its selection is written and its backward as soon as its forward is
+        done).  Results go to `out` (from make_outputs) if given, else to the
+        layer's own o, lse, dq, dk, dv."""
         self.summarize(q_begin, stream)
-        self.route(q, q_begin, stream)
         if d_o is None:
+            self.route(q, q_begin, stream)
             self.forward(q, q_begin, stream, out)
         else:
-            self.forward_backward(q, d_o, q_begin, stream, out)
+            self.route_forward_backward(q, d_o, q_begin, stream, out)
 
 
 class HgaTieredLayer:

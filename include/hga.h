@@ -244,6 +244,32 @@ HGA_API hga_status_t hga_attn_fwd_bwd(const hga_config_t* cfg, const void* q, co
                               void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
                               void* stream);
 
+/* Bytes of device workspace hga_segment_fwd_bwd needs: the backward
+ * workspace (hga_attn_bwd_workspace_size), one more array of per-item flags
+ * ([B, Hkv, S/64] int32, 256-byte aligned) and the routing workspace
+ * (hga_route_workspace_size, rounded up to 256 bytes), in that order. */
+HGA_API size_t hga_segment_workspace_size(const hga_config_t* cfg, int32_t s_len, int64_t q_begin);
+
+/*
+ * Steps a3 + a4 + a5 in one call: hga_route, then hga_attn_fwd_bwd, for one
+ * segment, with the same arguments and results (sel_blk, sel_grp, o, lse, dq,
+ * dk, dv; sel_blk may be NULL).  Where the routing runs as one kernel (up to
+ * 512 key blocks of context) and the attention on the tensor-core path, the
+ * forward of a query block starts as soon as that block's selection is
+ * written, through a third array of per-item flags; otherwise the steps run
+ * one after another.  bsum and gsum are the summaries of the context
+ * (hga_summaries), as for hga_route.  The flag sections follow the rule of
+ * hga_attn_fwd_bwd: zero before the workspace's first use, never used by two
+ * calls at once.  workspace: at least hga_segment_workspace_size() bytes of
+ * device memory, 16-byte aligned.
+ */
+HGA_API hga_status_t hga_segment_fwd_bwd(const hga_config_t* cfg, const void* q, const void* k,
+                                         const void* v, int64_t ctx_cap, int64_t q_begin,
+                                         int32_t s_len, const float* bsum, const float* gsum,
+                                         int32_t* sel_blk, int32_t* sel_grp, void* o, float* lse,
+                                         const void* d_o, void* dq, void* dk, void* dv,
+                                         void* workspace, size_t ws_bytes, void* stream);
+
 /*
  * Step a7 -- the host tier [A] ("older KV is detached into RAM or NVMe, and
  * HGA loads a bounded set of exact historical tokens for each query block").

@@ -80,6 +80,13 @@ def test_host_argument_checks():
     need = hga.hga_attn_bwd_workspace_size(c, 2048)
     assert status_of(hga.hga_attn_bwd, c, FAKE, FAKE, FAKE, 16384, 14336, 2048, FAKE, FAKE,
                      FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 4, 0) == 6
+    need = hga.hga_segment_workspace_size(c, 2048, 14336)
+    assert status_of(hga.hga_segment_fwd_bwd, c, FAKE, FAKE, FAKE, 16384, 14336, 2048, FAKE,
+                     FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 16,
+                     0) == 6
+    # sel_grp is required
+    assert status_of(hga.hga_segment_fwd_bwd, c, FAKE, FAKE, FAKE, 16384, 14336, 2048, FAKE,
+                     FAKE, None, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, 0) == 1
 
 
 def test_workspace_sizes():
@@ -92,6 +99,12 @@ def test_workspace_sizes():
     # two arrays of per-item flags (8 KV heads x 32 query blocks) for the fused call
     assert hga.hga_attn_bwd_workspace_size(c, 2048) == 32 * 2048 * 4 + 256 + 2 * 8 * 32 * 4
     assert hga.hga_route_workspace_size(cfg(head_dim=100), 2048, 0) == 0
+    # the chained segment call: the backward workspace, a third flag array,
+    # then the routing workspace
+    assert hga.hga_segment_workspace_size(c, 2048, 14336) == (
+        hga.hga_attn_bwd_workspace_size(c, 2048) + 8 * 32 * 4
+        + hga.hga_route_workspace_size(c, 2048, 14336))
+    assert hga.hga_segment_workspace_size(cfg(head_dim=100), 2048, 0) == 0
 
 
 def test_diagnostics_without_gpu():

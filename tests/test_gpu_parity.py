@@ -74,6 +74,32 @@ def test_fused_call_equals_separate_calls():
             assert torch.equal(a, b), q_begin
 
 
+def test_chained_segment_call_equals_separate_calls():
+    # hga_segment_fwd_bwd (routing chained into the forward by per-item
+    # flags) against hga_route + hga_attn_fwd + hga_attn_bwd: the same kernels
+    # and arithmetic, so the selections and every output are bit-identical;
+    # the first segment (no history) and two later ones in a row
+    import torch
+    w = WL["qwen3_fwdbwd_16k"]
+    seg = Segmenter(w)
+    L = seg.layer
+    for q_begin in (0, 12288, 14336):
+        q = to_device(synth.queries(w, q_begin), w)
+        d_o = to_device(synth.douts(w, q_begin), w)
+        L.summarize(q_begin)
+        L.sel_blk.fill_(-7)
+        L.sel_grp.fill_(-7)
+        L.route_forward_backward(q, d_o, q_begin)
+        torch.cuda.synchronize()
+        chained = [t.clone() for t in (L.sel_blk, L.sel_grp, L.o, L.lse, L.dq, L.dk, L.dv)]
+        L.route(q, q_begin)
+        L.forward(q, q_begin)
+        L.backward(q, d_o, q_begin)
+        torch.cuda.synchronize()
+        for a, b in zip(chained, (L.sel_blk, L.sel_grp, L.o, L.lse, L.dq, L.dk, L.dv)):
+            assert torch.equal(a, b), q_begin
+
+
 def test_segment_into_caller_output_set():
     # HgaLayer.segment(..., out=make_outputs()): the same results, written to
     # the caller's tensors (used to download one segment while the next runs)
