@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
                           int topk_groups, const int32_t* __restrict__ sel_grp, float scale,
                           float scale_log2, const __nv_bfloat16* __restrict__ o,
                           const __nv_bfloat16* __restrict__ d_o, const float* __restrict__ lse,
-                          __nv_bfloat16* __restrict__ dq, float* __restrict__ dvec,
+                          const __grid_constant__ CUtensorMap tm_dq, float* __restrict__ dvec,
                           int* __restrict__ unit_counter, const int* __restrict__ fwd_done,
                           int* __restrict__ d_done, uint32_t token) {
   using L = DqLayout<MT>;
@@ -356,21 +356,42 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
       const int op = (n_tiles - 1) * MT + m;
       ok = mbar_wait(&sh.ds_done[op & 1], (op >> 1) & 1, abort);
     }
+    // dQ of this M tile goes out through shared memory, over its own Q tile
+    // (every MMA that reads it has completed), in the layout Q came in; one
+    // TMA store per head and column half
+    uint8_t* stage = smem + L::kQ + m * 32768 + (row >> 6) * 8192 + r * 128;
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16* dst = dq + rix * kD;
       for (int c = 0; c < kD; c += 32) {
         float vv[32];
         tmem_ld32(tmem + lane_addr + L::colDQ(m) + c, vv);
         tmem_wait_ld();
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
-          float f[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) f[i] = vv[8 * q8 + i] * scale;
-          store8(dst + c + 8 * q8, f);
+          const int ch = c / 8 + q8;
+          const float* f = vv + 8 * q8;
+          *reinterpret_cast<uint4*>(stage + (ch >> 3) * 16384 + (((ch & 7) ^ (r & 7)) << 4)) =
+              make_uint4(pack_bf16x2(f[0] * scale, f[1] * scale),
+                         pack_bf16x2(f[2] * scale, f[3] * scale),
+                         pack_bf16x2(f[4] * scale, f[5] * scale),
+                         pack_bf16x2(f[6] * scale, f[7] * scale));
         }
       }
+      fence_proxy_async_smem();
+    }
+    if (m == 0)
+      named_barrier<1, 128>();
+    else
+      named_barrier<2, 128>();
+    if (ok && row == 0) {
+      for (int gg = 0; gg < 2; ++gg) {
+        const int32_t row0 =
+            int32_t((int64_t(b) * n_q_heads + h * G + 2 * m + gg) * s_len + j * kQBlock);
+        for (int hf = 0; hf < 2; ++hf)
+          tma_store_2d(&tm_dq, smem + L::kQ + m * 32768 + hf * 16384 + gg * 8192, hf * 64, row0);
+      }
+      bulk_commit_group();
+      bulk_wait_read_all();
     }
   }
 

@@ -82,9 +82,11 @@ template <int MT>
 __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, int64_t ctx_cap, int64_t q_begin, int s_len, int n_q_heads, int n_kv_heads,
-                       int topk_groups, const int32_t* __restrict__ sel_grp, float scale_log2,
-                       __nv_bfloat16* __restrict__ o, float* __restrict__ lse, uint32_t flags,
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_o, int64_t ctx_cap, int64_t q_begin,
+                       int s_len, int n_q_heads, int n_kv_heads, int topk_groups,
+                       const int32_t* __restrict__ sel_grp, float scale_log2,
+                       float* __restrict__ lse, uint32_t flags,
                        const int* __restrict__ route_done, int* __restrict__ done,
                        uint32_t token) {
   using L = Layout<MT>;
@@ -344,25 +346,52 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
     }
     if (ok)
       ok = mbar_wait(&sh.pv_done[m][(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort);
+    // O of this M tile goes out through shared memory, over its own Q tile
+    // (every MMA that reads it has completed), in the layout Q came in:
+    // [head][column half][64 rows][128 B], 128-byte swizzle; one TMA store
+    // per head and column half
+    uint8_t* stage = smem + L::kQ + m * 32768 + (row >> 6) * 8192 + r * 128;
     if (ok) {
       tc_fence_after();
       const float inv = 1.f / l_run;
-      const int hq = head0 + g;
-      const int64_t orow = (int64_t(b) * n_q_heads + hq) * s_len + int64_t(j) * kQBlock + r;
-      __nv_bfloat16* odst = o + orow * kD;
       for (int c = 0; c < kD; c += 32) {
         float ov[32];
         tmem_ld32(tmem + lane_addr + L::colO(m) + c, ov);
         tmem_wait_ld();
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
-          float f[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) f[i] = ov[8 * q8 + i] * inv;
-          store8(odst + c + 8 * q8, f);
+          const int ch = c / 8 + q8;
+          const float* f = ov + 8 * q8;
+          *reinterpret_cast<uint4*>(stage + (ch >> 3) * 16384 + (((ch & 7) ^ (r & 7)) << 4)) =
+              make_uint4(pack_bf16x2(f[0] * inv, f[1] * inv), pack_bf16x2(f[2] * inv, f[3] * inv),
+                         pack_bf16x2(f[4] * inv, f[5] * inv), pack_bf16x2(f[6] * inv, f[7] * inv));
         }
       }
+      const int64_t orow =
+          (int64_t(b) * n_q_heads + head0 + g) * s_len + int64_t(j) * kQBlock + r;
       lse[orow] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+      fence_proxy_async_smem();
+    }
+    if (m == 0)
+      named_barrier<1, 128>();
+    else
+      named_barrier<2, 128>();
+    if (ok && row == 0) {
+      for (int gg = 0; gg < 2; ++gg) {
+        const int32_t orow0 =
+            int32_t((int64_t(b) * n_q_heads + head0 + 2 * m + gg) * s_len + j * kQBlock);
+        for (int hf = 0; hf < 2; ++hf)
+          tma_store_2d(&tm_o, smem + L::kQ + m * 32768 + hf * 16384 + gg * 8192, hf * 64, orow0);
+      }
+      bulk_commit_group();
+      // a chained dQ kernel reads O once this item's flag is set: the stores
+      // must have completed, not only read shared memory
+      if (done) {
+        bulk_wait_all();
+        fence_proxy_async_global();
+      } else {
+        bulk_wait_read_all();
+      }
     }
     if (done) __threadfence();  // O and LSE before this item's completion flag
   }

@@ -203,6 +203,42 @@ __device__ int block_enumerate(int n, Pred pred, Fn f, int* scratch) {
   return total;
 }
 
+// The same contract for short ranges (a few times the block size): element
+// i goes to thread i % blockDim.x in round i / blockDim.x, and its rank is
+// the count of earlier predicates in that round (warp ballots, one table of
+// per-warp counts) plus the counts of the earlier rounds.  Needs `scratch` of
+// blockDim.x/32 ints.
+template <typename Pred, typename Fn>
+__device__ int block_enumerate_rounds(int n, Pred pred, Fn f, int* scratch) {
+  const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = nt >> 5;
+  int done = 0;
+  for (int base = 0; base < n; base += nt) {
+    const int i = base + tid;
+    const bool p = i < n && pred(i);
+    const unsigned ball = __ballot_sync(0xffffffffu, p);
+    if (lane == 0) scratch[warp] = __popc(ball);
+    __syncthreads();
+    int before = done, total = done;
+    for (int w = 0; w < nwarps; ++w) {
+      const int c = scratch[w];
+      before += w < warp ? c : 0;
+      total += c;
+    }
+    if (p) f(i, before + __popc(ball & ((1u << lane) - 1u)));
+    done = total;
+    __syncthreads();
+  }
+  return done;
+}
+
+// block_enumerate or block_enumerate_rounds, whichever takes fewer barriers
+template <typename Pred, typename Fn>
+__device__ int block_enumerate_any(int n, Pred pred, Fn f, int* scratch) {
+  if (n <= 2 * int(blockDim.x)) return block_enumerate_rounds(n, pred, f, scratch);
+  return block_enumerate(n, pred, f, scratch);
+}
+
 // ---------------------------------------------------------------------------
 // block-wide top-k of n distinct-or-not uint32 keys held in shared memory:
 // sets sel[i] = 1 for the k largest keys, ties broken toward the lower index.
@@ -222,11 +258,23 @@ __device__ void block_topk(const uint32_t* key, int n, int k, uint8_t* sel, int*
   if (n <= 128) {
     // rank by counting: rank(i) = #{keys above key[i]} + #{equal keys before i};
     // the k smallest ranks are the k largest keys, ties to the lower index.
-    // O(n^2) comparisons with broadcast shared-memory reads, no barrier.
+    // O(n^2) comparisons with broadcast shared-memory reads (four keys per
+    // 16-byte load; `key` is 16-byte aligned), no barrier.
+    const uint4* key4 = reinterpret_cast<const uint4*>(key);
+    const int n4 = n >> 2;
     for (int i = tid; i < n; i += nt) {
       const uint32_t ki = key[i];
       int rank = 0;
-      for (int jdx = 0; jdx < n; ++jdx) {
+#pragma unroll 4
+      for (int q = 0; q < n4; ++q) {
+        const uint4 v = key4[q];
+        const int j0 = 4 * q;
+        rank += (v.x > ki) || (v.x == ki && j0 < i);
+        rank += (v.y > ki) || (v.y == ki && j0 + 1 < i);
+        rank += (v.z > ki) || (v.z == ki && j0 + 2 < i);
+        rank += (v.w > ki) || (v.w == ki && j0 + 3 < i);
+      }
+      for (int jdx = 4 * n4; jdx < n; ++jdx) {
         const uint32_t kj = key[jdx];
         rank += (kj > ki) || (kj == ki && jdx < i);
       }
@@ -244,9 +292,18 @@ __device__ void block_topk(const uint32_t* key, int n, int k, uint8_t* sel, int*
     for (int i = tid; i < 256; i += nt) hist[i] = 0;
     __syncthreads();
     const uint32_t prefix = s_prefix, mask = s_mask;
-    for (int i = tid; i < n; i += nt) {
-      uint32_t kk = key[i];
-      if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255u], 1);
+    // warp-aggregated: the lanes holding the same digit add their count once
+    // (the top digits of nearby scores are mostly equal)
+    for (int base = 0; base < n; base += nt) {
+      const int i = base + tid;
+      const uint32_t kk = i < n ? key[i] : 0u;
+      const bool act = i < n && (kk & mask) == prefix;
+      const unsigned am = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const uint32_t dg = (kk >> shift) & 255u;
+        const unsigned peers = __match_any_sync(am, dg);
+        if ((tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[dg], __popc(peers));
+      }
     }
     __syncthreads();
     if (tid < 32) {
@@ -288,7 +345,7 @@ __device__ void block_topk(const uint32_t* key, int n, int k, uint8_t* sel, int*
   const int need_equal = s_remaining;  // how many keys equal to thr are taken
   for (int i = tid; i < n; i += nt) sel[i] = key[i] > thr ? 1 : 0;
   __syncthreads();
-  block_enumerate(
+  block_enumerate_any(
       n, [&](int i) { return key[i] == thr; },
       [&](int i, int rank) {
         if (rank < need_equal) sel[i] = 1;

@@ -167,10 +167,10 @@ hga_status_t launch_fwd_tc(const hga_config_t* cfg, const void* q, const void* k
                            const int32_t* sel_grp, void* o, float* lse, const int* route_done,
                            int* done, uint32_t token, cudaStream_t s) {
   using L = fwdtc::Layout<MT>;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   const uint64_t q_rows = uint64_t(cfg->batch) * cfg->n_q_heads * s_len;
   const uint64_t kv_rows = uint64_t(cfg->batch) * cfg->n_kv_heads * ctx_cap;
-  if (!make_map_bf16_d128(&tq, q, q_rows, 64) ||
+  if (!make_map_bf16_d128(&tq, q, q_rows, 64) || !make_map_bf16_d128(&to, o, q_rows, 64) ||
       !make_map_bf16_d128_groups(&tk, k, kv_rows, 8) ||
       !make_map_bf16_d128_groups(&tv, v, kv_rows, 8))
     return HGA_ERR_CUDA;
@@ -182,8 +182,8 @@ hga_status_t launch_fwd_tc(const hga_config_t* cfg, const void* q, const void* k
   const float scale_log2 = cfg->scale * 1.4426950408889634f;
   return traced_launch(HGA_K_FWD_TC, s, [&] {
     return launch_pdl(fwdtc::attn_fwd_tc_kernel<MT>, grid, dim3(L::kThreads), L::kDynSmem, s, tq,
-        tk, tv, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups, sel_grp,
-        scale_log2, static_cast<__nv_bfloat16*>(o), lse, cfg->flags, route_done, done, token);
+        tk, tv, to, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups,
+        sel_grp, scale_log2, lse, cfg->flags, route_done, done, token);
   });
 }
 
@@ -196,10 +196,11 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
                            cudaStream_t s) {
   using LQ = bwdtc::DqLayout<MT>;
   using LK = bwdtc::KvLayout;
-  CUtensorMap tq, tdo, tk, tv;
+  CUtensorMap tq, tdo, tk, tv, tdq;
   const uint64_t q_rows = uint64_t(cfg->batch) * cfg->n_q_heads * s_len;
   const uint64_t kv_rows = uint64_t(cfg->batch) * cfg->n_kv_heads * ctx_cap;
   if (!make_map_bf16_d128(&tq, q, q_rows, 64) || !make_map_bf16_d128(&tdo, d_o, q_rows, 64) ||
+      !make_map_bf16_d128(&tdq, dq, q_rows, 64) ||
       !make_map_bf16_d128(&tk, k, kv_rows, 8) || !make_map_bf16_d128(&tv, v, kv_rows, 8))
     return HGA_ERR_CUDA;
   hga_status_t e = ensure_smem(
@@ -215,7 +216,7 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
         tq, tdo, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
         ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups, sel_grp,
         cfg->scale, scale_log2, static_cast<const __nv_bfloat16*>(o),
-        static_cast<const __nv_bfloat16*>(d_o), lse, static_cast<__nv_bfloat16*>(dq), dvec,
+        static_cast<const __nv_bfloat16*>(d_o), lse, tdq, dvec,
         unit_counter, fwd_done, d_done, token);
   });
   if (e != HGA_OK) return e;

@@ -237,7 +237,7 @@ __device__ __forceinline__ void select_levels(const SelectLayout& L, unsigned ch
 
   // level 1
   block_topk(key1, int(J), kb, sel1, hist, scratch);
-  block_enumerate(
+  block_enumerate_any(
       int(J), [&](int i) { return sel1[i] != 0; }, [&](int i, int r) { blocks[r] = i; },
       scratch);
   int32_t* out_blk = sel_blk ? sel_blk + (head * n_qb + j) * topk_blocks : nullptr;
@@ -255,7 +255,7 @@ __device__ __forceinline__ void select_levels(const SelectLayout& L, unsigned ch
   const int kg = n2 < topk_groups ? n2 : topk_groups;
   block_topk(key2, n2, kg, sel2, hist, scratch);
   int32_t* out_grp = sel_grp + (head * n_qb + j) * topk_groups;
-  block_enumerate(
+  block_enumerate_any(
       n2, [&](int p) { return sel2[p] != 0; },
       [&](int p, int r) { out_grp[r] = blocks[p >> 3] * kGroupsPerBlock + (p & 7); }, scratch);
   for (int i = kg + threadIdx.x; i < topk_groups; i += kRouteThreads) out_grp[i] = -1;
