@@ -73,7 +73,7 @@ struct DqShared {
   uint64_t sdp_full[2];   // S, dP of the op are in the region
   uint64_t ds_full[2];    // its dS is in the region
   uint64_t ds_done[2];    // dQ += dS K has completed: the region is free
-  uint64_t mma_done;
+  uint64_t mma_done[2];   // every MMA of issuer 0 (S, dP) / issuer 1 (dQ) has completed
   uint32_t tmem_base;
   int abort;
   int n_tiles;
@@ -82,7 +82,7 @@ struct DqShared {
   uint8_t tile_mask[kMaxTiles];
 };
 
-constexpr int kDqProducers = 96;  // warps 0, 2, 3
+constexpr int kDqProducers = 64;  // warps 0, 2
 
 template <int MT>
 __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
@@ -119,14 +119,15 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     mbar_init(&sh.q_full, 1);
     for (int s = 0; s < kSt; ++s) {
       mbar_init(&sh.kv_full[s], kDqProducers);
-      mbar_init(&sh.kv_empty[s], 1);
+      mbar_init(&sh.kv_empty[s], 2);  // the last S/dP and the last dQ of the tile
     }
     for (int r = 0; r < 2; ++r) {
       mbar_init(&sh.sdp_full[r], 1);
       mbar_init(&sh.ds_full[r], 128);
       mbar_init(&sh.ds_done[r], 1);
     }
-    mbar_init(&sh.mma_done, 1);
+    mbar_init(&sh.mma_done[0], 1);
+    mbar_init(&sh.mma_done[1], 1);
     sh.abort = 0;
     fence_barrier_init();
   }
@@ -171,10 +172,10 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
   const uint32_t tmem = sh.tmem_base;
   const int n_tiles = sh.n_tiles;
 
-  if (warp == 0 || warp == 2 || warp == 3) {
+  if (warp == 0 || warp == 2) {
     // ---------------- producers: K/V groups by cp.async into a 3-stage ring ------
     // stage layout [K | V][d half][64 rows][128 B], 128-byte swizzle
-    const int ptid = warp == 0 ? lane : 32 * (warp - 1) + lane;
+    const int ptid = warp == 0 ? lane : 32 + lane;
     const __nv_bfloat16* kh = k + (int64_t(b) * n_kv_heads + h) * ctx_cap * kD;
     const __nv_bfloat16* vh = v + (int64_t(b) * n_kv_heads + h) * ctx_cap * kD;
     for (int t = 0; t < n_tiles; ++t) {
@@ -193,73 +194,67 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     int never = 0;
     if (tid == 0) mbar_wait(&sh.q_full, 0, &never);
     asm volatile("cp.async.wait_all;" ::: "memory");
-  } else if (warp == 1) {
-    // ---------------- MMA issuer (event driven; whole warp, one lane issues) --
+  } else if (warp == 1 || warp == 3) {
+    // ---------------- MMA issuers (whole warp each, one lane issues) ----------
     // Ops s = t * MT + m (tile t, M tile m) alternate between the two TMEM
-    // regions (region s & 1).  S/dP of op s needs the K/V of tile t and its
-    // region back from op s - 2 (whose dQ has read its dS); dQ of op s needs
-    // its dS, and the last dQ of a tile frees the tile's K/V stage.
+    // regions (region s & 1).  Warp 1 issues S = Q K^T and dP = dO V^T of op
+    // s once the K/V of tile t are in and the region is back from op s - 2
+    // (whose dQ has read its dS); warp 3 issues dQ += dS K of op s once its
+    // dS is in.  Two issuers, so that a dQ never queues behind the sixteen
+    // S/dP MMAs of the other M tile: the tensor core takes both streams.  The
+    // stage of tile t is free once the last S/dP and the last dQ of the tile
+    // have completed (two commits on kv_empty).
+    const int iss = warp == 1 ? 0 : 1;
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);
     constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kD, 0, 1);
     bool ok = __all_sync(kFullMask, mbar_wait(&sh.q_full, 0, abort));
     bool issued_any = false;
     const int n_ops = n_tiles * MT;
-    int next_s = 0, next_q = 0;  // next S/dP op, next dQ op
-    long long t0 = clock64();
-    while (ok && next_q < n_ops) {
-      bool progressed = false;
-      if (next_q < next_s) {
-        const int t = next_q / MT, m = next_q % MT, rg = next_q & 1;
-        if (__all_sync(kFullMask, mbar_test(&sh.ds_full[rg], (next_q >> 1) & 1))) {
-          const uint32_t kb = sKV + (t % kSt) * L::kStageBytes;
-          tc_fence_after();
-          if (elect_one()) {
+    for (int op = 0; ok && op < n_ops; ++op) {
+      const int t = op / MT, m = op % MT, rg = op & 1;
+      const uint32_t kb = sKV + (t % kSt) * L::kStageBytes;
+      if (iss == 0) {
+        bool ready = m != 0 || mbar_wait(&sh.kv_full[t % kSt], (t / kSt) & 1, abort);
+        if (op >= 2) ready = ready && mbar_wait(&sh.ds_done[rg], ((op - 2) >> 1) & 1, abort);
+        if (!(ok = __all_sync(kFullMask, ready))) break;
+        fence_proxy_async_smem();  // cp.async data -> tensor-core reads
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_tmem_a(tmem + L::colDQ(m), tmem + L::colS(rg) + kk * 8,
-                              smem_desc_sw128(kb + kk * 2048, 8192, 1024), idesc_dq,
-                              (t > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&sh.ds_done[rg]);
-            if (m == MT - 1) mma_commit(&sh.kv_empty[t % kSt]);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+            const uint32_t bo = (kk >> 2) * 8192 + (kk & 3) * 32;
+            mma_bf16(tmem + L::colS(rg), smem_desc_sw128(sQ + m * 32768 + ko, 16, 1024),
+                     smem_desc_sw128(kb + bo, 16, 1024), idesc_s, kk > 0);
+            mma_bf16(tmem + L::colDP(rg), smem_desc_sw128(sDO + m * 32768 + ko, 16, 1024),
+                     smem_desc_sw128(kb + 16384 + bo, 16, 1024), idesc_s, kk > 0);
           }
-          __syncwarp();
-          ++next_q;
-          progressed = true;
+          mma_commit(&sh.sdp_full[rg]);
+          if (m == MT - 1) mma_commit(&sh.kv_empty[t % kSt]);
+        }
+      } else {
+        if (!(ok = __all_sync(kFullMask, mbar_wait(&sh.ds_full[rg], (op >> 1) & 1, abort))))
+          break;
+        tc_fence_after();
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_tmem_a(tmem + L::colDQ(m), tmem + L::colS(rg) + kk * 8,
+                            smem_desc_sw128(kb + kk * 2048, 8192, 1024), idesc_dq,
+                            (t > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&sh.ds_done[rg]);
+          if (m == MT - 1) mma_commit(&sh.kv_empty[t % kSt]);
         }
       }
-      if (!progressed && next_s < n_ops && next_s < next_q + 2) {
-        const int t = next_s / MT, m = next_s % MT, rg = next_s & 1;
-        bool ready = m != 0 || mbar_test(&sh.kv_full[t % kSt], (t / kSt) & 1);
-        if (next_s >= 2) ready = ready && mbar_test(&sh.ds_done[rg], ((next_s - 2) >> 1) & 1);
-        if (__all_sync(kFullMask, ready)) {
-          fence_proxy_async_smem();  // cp.async data -> tensor-core reads
-          tc_fence_after();
-          const uint32_t kb = sKV + (t % kSt) * L::kStageBytes;
-          if (elect_one()) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-              const uint32_t bo = (kk >> 2) * 8192 + (kk & 3) * 32;
-              mma_bf16(tmem + L::colS(rg), smem_desc_sw128(sQ + m * 32768 + ko, 16, 1024),
-                       smem_desc_sw128(kb + bo, 16, 1024), idesc_s, kk > 0);
-              mma_bf16(tmem + L::colDP(rg), smem_desc_sw128(sDO + m * 32768 + ko, 16, 1024),
-                       smem_desc_sw128(kb + 16384 + bo, 16, 1024), idesc_s, kk > 0);
-            }
-            mma_commit(&sh.sdp_full[rg]);
-          }
-          __syncwarp();
-          ++next_s;
-          issued_any = true;
-          progressed = true;
-        }
-      }
-      ok = warp_event_continue(progressed, t0, abort);
+      __syncwarp();
+      issued_any = true;
     }
     if (issued_any) {
-      if (elect_one()) mma_commit(&sh.mma_done);
+      // every MMA this warp issued must finish before TMEM is freed
+      if (elect_one()) mma_commit(&sh.mma_done[iss]);
       __syncwarp();
       int never = 0;
-      mbar_wait(&sh.mma_done, 0, &never);
+      mbar_wait(&sh.mma_done[iss], 0, &never);
     }
   } else if (warp >= 4) {
     const int m = (warp - 4) >> 2, wq = warp & 3;
