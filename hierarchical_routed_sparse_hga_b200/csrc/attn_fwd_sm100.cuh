@@ -67,7 +67,7 @@ struct Shared {
   uint64_t s_full[2][2];
   uint64_t p_full[2][2];
   uint64_t pv_done[2][2];
-  uint64_t mma_done;
+  uint64_t mma_done[2];  // every MMA of issuer 0 (S) / issuer 1 (PV) has completed
   uint32_t tmem_base;
   int abort;
   int n_tiles;
@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
     mbar_init(&sh.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sh.kv_full[s], 1);
-      mbar_init(&sh.kv_empty[s], 1);
+      mbar_init(&sh.kv_empty[s], 2);  // the last S and the last PV of the tile
     }
     for (int m = 0; m < 2; ++m)
       for (int u = 0; u < 2; ++u) {
@@ -119,7 +119,8 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
         mbar_init(&sh.p_full[m][u], 128);
         mbar_init(&sh.pv_done[m][u], 1);
       }
-    mbar_init(&sh.mma_done, 1);
+    mbar_init(&sh.mma_done[0], 1);
+    mbar_init(&sh.mma_done[1], 1);
     sh.abort = 0;
     fence_barrier_init();
   }
@@ -202,75 +203,69 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
         mbar_wait(&sh.kv_full[t % kStages], (t / kStages) & 1, &never);
       }
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer (whole warp, one lane issues) --------------
-    // Fixed order S(0), S(1), then PV(t), S(t+2) for t = 0, 1, ...: S(t+2)
-    // reuses the TMEM columns that hold P(t) until PV(t) has read them.  The
-    // waits block (the warp is parked until the phase completes), which
-    // leaves the issue slots of its sub-partition to the softmax warps.
+  } else if (warp == 1 || warp == 3) {
+    // ---------------- MMA issuers (whole warp each, one lane issues) --------
+    // Warp 1 issues S(t, m) = Q_m K_t^T once K/V of tile t are in and, for
+    // t >= 2, PV(t-2, m) has completed (S(t, m) reuses the TMEM columns that
+    // hold P(t-2, m) until PV(t-2, m) has read them); warp 3 issues
+    // PV(t, m): O_m += P(t, m) V_t once the softmax has written P(t, m).  Two
+    // issuers, so that a ready PV never queues behind the sixteen S MMAs of
+    // the next tile.  The stage of tile t is free once its last S and its
+    // last PV have completed (two commits on kv_empty).  The waits block
+    // (the warp is parked until the phase completes), which leaves the issue
+    // slots of its sub-partition to the softmax warps.
+    const int iss = warp == 1 ? 0 : 1;
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, 0, 0);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kD, 0, 1);
     bool issued_any = false;
-    auto issue_qk = [&](int t) -> bool {
-      const int st = t % kStages, buf = t & 1;
-      bool ready = mbar_wait(&sh.kv_full[st], (t / kStages) & 1, abort);
-      for (int m = 0; m < MT && t >= 2; ++m)
-        ready = ready && mbar_wait(&sh.pv_done[m][buf], ((t - 2) >> 1) & 1, abort);
-      if (!__all_sync(kFullMask, ready)) return false;
-      tc_fence_after();
-      const uint32_t kbase = sKV + st * L::kStageBytes;
-      if (elect_one()) {
-        for (int m = 0; m < MT; ++m) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint64_t a =
-                smem_desc_sw128(sQ + m * 32768 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(kbase + (k >> 2) * 1024 + (k & 3) * 32, 16, 2048);
-            mma_bf16(tmem + L::colS(m, buf), a, bd, idesc_qk, k > 0);
-          }
-          mma_commit(&sh.s_full[m][buf]);
-        }
-      }
-      __syncwarp();
-      issued_any = true;
-      return true;
-    };
-    auto issue_pv = [&](int t) -> bool {
-      bool ready = true;
-      for (int m = 0; m < MT; ++m)
-        ready = ready && mbar_wait(&sh.p_full[m][t & 1], (t >> 1) & 1, abort);
-      if (!__all_sync(kFullMask, ready)) return false;
-      const int st = t % kStages;
-      const uint32_t vbase = sKV + st * L::kStageBytes + 16384;
-      tc_fence_after();
-      if (elect_one()) {
-        for (int m = 0; m < MT; ++m) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t bd = smem_desc_sw128(vbase + k * 4096, 1024, 2048);
-            mma_bf16_tmem_a(tmem + L::colO(m), tmem + L::colS(m, t & 1) + k * 8, bd, idesc_pv,
-                            (t > 0 || k > 0) ? 1u : 0u);
-          }
-          mma_commit(&sh.pv_done[m][t & 1]);
-        }
-        mma_commit(&sh.kv_empty[st]);
-      }
-      __syncwarp();
-      return true;
-    };
     bool ok = __all_sync(kFullMask, mbar_wait(&sh.q_full, 0, abort));
-    if (ok) ok = issue_qk(0);
-    if (ok && n_tiles > 1) ok = issue_qk(1);
     for (int t = 0; ok && t < n_tiles; ++t) {
-      ok = issue_pv(t);
-      if (ok && t + 2 < n_tiles) ok = issue_qk(t + 2);
+      const int st = t % kStages, buf = t & 1;
+      for (int m = 0; ok && m < MT; ++m) {
+        if (iss == 0) {
+          bool ready = m > 0 || mbar_wait(&sh.kv_full[st], (t / kStages) & 1, abort);
+          if (t >= 2) ready = ready && mbar_wait(&sh.pv_done[m][buf], ((t - 2) >> 1) & 1, abort);
+          if (!(ok = __all_sync(kFullMask, ready))) break;
+          tc_fence_after();
+          const uint32_t kbase = sKV + st * L::kStageBytes;
+          if (elect_one()) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const uint64_t a =
+                  smem_desc_sw128(sQ + m * 32768 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+              const uint64_t bd =
+                  smem_desc_sw128(kbase + (k >> 2) * 1024 + (k & 3) * 32, 16, 2048);
+              mma_bf16(tmem + L::colS(m, buf), a, bd, idesc_qk, k > 0);
+            }
+            mma_commit(&sh.s_full[m][buf]);
+            if (m == MT - 1) mma_commit(&sh.kv_empty[st]);
+          }
+        } else {
+          if (!(ok = __all_sync(kFullMask, mbar_wait(&sh.p_full[m][buf], (t >> 1) & 1, abort))))
+            break;
+          const uint32_t vbase = sKV + st * L::kStageBytes + 16384;
+          tc_fence_after();
+          if (elect_one()) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t bd = smem_desc_sw128(vbase + k * 4096, 1024, 2048);
+              mma_bf16_tmem_a(tmem + L::colO(m), tmem + L::colS(m, buf) + k * 8, bd, idesc_pv,
+                              (t > 0 || k > 0) ? 1u : 0u);
+            }
+            mma_commit(&sh.pv_done[m][buf]);
+            if (m == MT - 1) mma_commit(&sh.kv_empty[st]);
+          }
+        }
+        __syncwarp();
+        issued_any = true;
+      }
     }
     if (issued_any) {
       // every MMA this warp issued must finish before TMEM is freed
-      if (elect_one()) mma_commit(&sh.mma_done);
+      if (elect_one()) mma_commit(&sh.mma_done[iss]);
       __syncwarp();
       int never = 0;
-      mbar_wait(&sh.mma_done, 0, &never);
+      mbar_wait(&sh.mma_done[iss], 0, &never);
     }
   } else if (warp >= 4) {
     // ---------------- softmax / epilogue ----------------
