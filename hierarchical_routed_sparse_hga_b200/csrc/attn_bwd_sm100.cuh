@@ -477,7 +477,7 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
       mbar_init(&sh.sdp_full[u], 1);
       mbar_init(&sh.pds_full[u], 128);
     }
-    mbar_init(&sh.mma_done, 1);
+    mbar_init(&sh.mma_done, 2);  // one commit from each issuer per unit
     sh.abort = 0;
     fence_barrier_init();
   }
@@ -610,44 +610,24 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
           mbar_wait(&sh.qd_full[gi & 1], (gi >> 1) & 1, &never);
         }
       }
-    } else if (warp == 1) {
-      // ---------------- MMA issuer (event driven; whole warp, one lane issues)
+    } else if (warp == 1 || warp == 3) {
+      // ---------------- MMA issuers (whole warp each, one lane issues) ------
+      // Warp 1 issues S/dP(i) into TMEM buffer i & 1 once Q/dO of item i
+      // are in and the softmax of item i - 2 has taken that buffer's S and
+      // dP (its P/dS are then in shared memory); warp 3 issues dV/dK(i) once
+      // P/dS(i) are in.  Two issuers, so that a ready dV/dK never queues
+      // behind the sixteen S/dP MMAs of the next item.
+      const int iss = warp == 1 ? 0 : 1;
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t idesc_t = idesc_bf16_f32(128, 64, 1, 1);
       bool ok = __all_sync(kFullMask, mbar_wait(&sh.kv_full, un & 1, abort));
-      int next_s = 0, next_t = 0;  // items with S/dP issued, with dV/dK issued
-      long long t0 = clock64();
-      while (ok && next_t < n_items) {
-        bool progressed = false;
-        const int gt = it_base + next_t, gs = it_base + next_s;
-        if (next_t < next_s &&
-            __all_sync(kFullMask, mbar_test(&sh.pds_full[gt & 1], (gt >> 1) & 1))) {
-          // dV^T += dO^T P and dK^T += Q^T dS over this item's 128 query rows
-          const int u = gt & 1;
-          const uint32_t qd = sQD + u * L::kQDBytes, pd = sPD + u * L::kPDBytes;
-          tc_fence_after();
-          if (elect_one()) {
-#pragma unroll
-            for (int s8 = 0; s8 < 8; ++s8) {
-              const uint32_t ro = s8 * 2048;
-              const uint32_t acc = (next_t > 0 || s8 > 0) ? 1u : 0u;
-              mma_bf16(tmem + L::kColDV, smem_desc_sw128(qd + 32768 + ro, 16384, 1024),
-                       smem_desc_sw128(pd + ro, 8192, 1024), idesc_t, acc);
-              mma_bf16(tmem + L::kColDK, smem_desc_sw128(qd + ro, 16384, 1024),
-                       smem_desc_sw128(pd + 16384 + ro, 8192, 1024), idesc_t, acc);
-            }
-            mma_commit(&sh.qd_empty[u]);
-          }
-          __syncwarp();
-          ++next_t;
-          progressed = true;
-        }
-        // S/dP(i) into buffer i & 1, free once dV/dK(i-2) has been issued
-        // (its softmax has then finished with that buffer)
-        if (!progressed && next_s < n_items && next_s < next_t + 2 &&
-            __all_sync(kFullMask, mbar_test(&sh.qd_full[gs & 1], (gs >> 1) & 1))) {
-          const int u = gs & 1;
-          const uint32_t qd = sQD + u * L::kQDBytes;
+      for (int it = 0; ok && it < n_items; ++it) {
+        const int gi = it_base + it, u = gi & 1;
+        const uint32_t qd = sQD + u * L::kQDBytes;
+        if (iss == 0) {
+          bool ready = mbar_wait(&sh.qd_full[u], (gi >> 1) & 1, abort);
+          if (it >= 2) ready = ready && mbar_wait(&sh.pds_full[u], ((gi - 2) >> 1) & 1, abort);
+          if (!(ok = __all_sync(kFullMask, ready))) break;
           tc_fence_after();
           if (elect_one()) {
 #pragma unroll
@@ -661,15 +641,31 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
             }
             mma_commit(&sh.sdp_full[u]);
           }
-          __syncwarp();
-          ++next_s;
-          progressed = true;
+        } else {
+          // dV^T += dO^T P and dK^T += Q^T dS over this item's 128 query rows
+          if (!(ok = __all_sync(kFullMask, mbar_wait(&sh.pds_full[u], (gi >> 1) & 1, abort))))
+            break;
+          const uint32_t pd = sPD + u * L::kPDBytes;
+          tc_fence_after();
+          if (elect_one()) {
+#pragma unroll
+            for (int s8 = 0; s8 < 8; ++s8) {
+              const uint32_t ro = s8 * 2048;
+              const uint32_t acc = (it > 0 || s8 > 0) ? 1u : 0u;
+              mma_bf16(tmem + L::kColDV, smem_desc_sw128(qd + 32768 + ro, 16384, 1024),
+                       smem_desc_sw128(pd + ro, 8192, 1024), idesc_t, acc);
+              mma_bf16(tmem + L::kColDK, smem_desc_sw128(qd + ro, 16384, 1024),
+                       smem_desc_sw128(pd + 16384 + ro, 8192, 1024), idesc_t, acc);
+            }
+            mma_commit(&sh.qd_empty[u]);
+          }
         }
-        ok = warp_event_continue(progressed, t0, abort);
+        __syncwarp();
       }
-      // one mma_done phase per unit: every MMA of this unit has finished
-      // before its epilogue reads TMEM and before the next unit overwrites
-      // the tiles in shared memory (a commit with none pending arrives at once)
+      // one mma_done phase per unit (a commit from each issuer): every MMA of
+      // this unit has finished before its epilogue reads TMEM and before the
+      // next unit overwrites the tiles in shared memory (a commit with none
+      // pending arrives at once)
       if (elect_one()) mma_commit(&sh.mma_done);
       __syncwarp();
       int never = 0;
