@@ -96,8 +96,10 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
                           const __nv_bfloat16* __restrict__ d_o, const float* __restrict__ lse,
                           const __grid_constant__ CUtensorMap tm_dq, float* __restrict__ dvec,
                           int* __restrict__ unit_counter, const int* __restrict__ fwd_done,
-                          int* __restrict__ d_done, uint32_t token) {
+                          int* __restrict__ d_done, uint32_t token, int* __restrict__ inv) {
   using L = DqLayout<MT>;
+  // arrivals before this item's D flag: the softmax rows and warp 3's lanes
+  constexpr int kArrive = 128 * MT + 32;
   constexpr int G = 2 * MT;
   constexpr int kSt = L::kStages;
   extern __shared__ uint8_t dsmem_raw[];
@@ -205,6 +207,32 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     // stage of tile t is free once the last S/dP and the last dQ of the tile
     // have completed (two commits on kv_empty).
     const int iss = warp == 1 ? 0 : 1;
+    if (iss == 1) {
+      // the inverted selection for the dK/dV kernel: which groups of each
+      // earlier block kb of the active segment this query block attends,
+      // inv[b, h][kb][j] = token << 8 | mask (every entry of column j is
+      // written, 0 for blocks it does not attend); one lane per block
+      uint32_t mk0 = 0u, mk1 = 0u;
+      const int64_t act0 = q_begin / kGroup;
+      for (int i = 0; i < n_tiles * 8; ++i) {
+        const int64_t ga = int64_t(sh.grp[i]) - act0;
+        if (ga >= 0 && ga < int64_t(j) * kGroupsPerBlock) {
+          const int kb = int(ga / kGroupsPerBlock);
+          const uint32_t bit = 1u << int(ga % kGroupsPerBlock);
+          if (kb == lane) mk0 |= bit;
+          if (kb == lane + 32) mk1 |= bit;
+        }
+      }
+      const uint32_t tk = (token & 0xffffffu) << 8;
+      int* inv_bh = inv + (int64_t(b) * n_kv_heads + h) * n_qb * n_qb;
+      if (lane < n_qb) inv_bh[lane * n_qb + j] = int(tk | mk0);
+      if (lane + 32 < n_qb) inv_bh[(lane + 32) * n_qb + j] = int(tk | mk1);
+      if (d_done) {
+        __threadfence();
+        if (atomicAdd(&sh.d_arrived, 1) == kArrive - 1 && !*abort)
+          flag_release(d_done + item, token);
+      }
+    }
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);
     constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kD, 0, 1);
     bool ok = __all_sync(kFullMask, mbar_wait(&sh.q_full, 0, abort));
@@ -305,7 +333,7 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     if (d_done) {
       // fused: the last of this CTA's rows to write D publishes the item
       __threadfence();
-      if (atomicAdd(&sh.d_arrived, 1) == 128 * MT - 1 && !*abort)
+      if (atomicAdd(&sh.d_arrived, 1) == kArrive - 1 && !*abort)
         flag_release(d_done + item, token);
     }
     const float lse2 = lse[rix] * 1.4426950408889634f;
@@ -453,7 +481,8 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
                             float scale_log2, const float* __restrict__ lse,
                             const float* __restrict__ dvec, __nv_bfloat16* __restrict__ dk,
                             __nv_bfloat16* __restrict__ dv, int* __restrict__ unit_counter,
-                            const int* __restrict__ d_done, uint32_t token) {
+                            const int* __restrict__ d_done, uint32_t token,
+                            const int* __restrict__ inv) {
   using L = KvLayout;
   constexpr int G = 2 * MT;
   extern __shared__ uint8_t dsmem_raw[];
@@ -530,28 +559,22 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
         }
     }
     // which later query blocks of the segment selected groups of this block
-    // (only query blocks after kb can; 4 loads per thread in flight)
-    const int32_t* sel_bh = sel_grp + (int64_t(b) * n_kv_heads + h) * n_qb * topk_groups;
+    // (only query blocks after kb can): their dQ CTAs wrote it, tagged with
+    // the call's token, before releasing their D flags.  Fused: wait for
+    // those flags (and the own block's) first.
     {
-      const int first = (kb + 1) * topk_groups, total = n_qb * topk_groups;
-      const int nt = blockDim.x;
-      for (int base = first + tid; base < total; base += 4 * nt) {
-        int gv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int idx = base + u * nt;
-          gv[u] = idx < total ? sel_bh[idx] : -1;
+      const int* inv_row = inv + (int64_t(bh) * n_qb + kb) * n_qb;
+      const uint32_t tk = token & 0xffffffu;
+      for (int jj = kb + 1 + tid; jj < n_qb; jj += blockDim.x) {
+        if (d_done && !flag_wait(d_done + bh * n_qb + jj, token, abort)) continue;
+        const uint32_t v = uint32_t(inv_row[jj]);
+        if ((v >> 8) != tk) {
+          latch_status(HGA_ERR_DEVICE_CHECK);
+          continue;
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int idx = base + u * nt, g = gv[u];
-          if (idx >= total || g < 0) continue;
-          const int jj = idx / topk_groups;
-          const int64_t own_jj = q_begin / kBlock + jj;
-          if (int64_t(g) < own_jj * kGroupsPerBlock && int64_t(g) / kGroupsPerBlock == gblk)
-            atomicOr(&sh.masks[jj], 1 << (g % kGroupsPerBlock));
-        }
+        if (v & 0xffu) sh.masks[jj] = int(v & 0xffu);
       }
+      if (d_done && tid == blockDim.x - 1) flag_wait(d_done + bh * n_qb + kb, token, abort);
     }
     __syncthreads();
     if (warp == 0) {
@@ -569,12 +592,6 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const int n_items = sh.n_items;
-    if (d_done) {
-      // fused: D (and, through the dQ kernel, LSE) of every visited query block
-      for (int q = tid; q < n_items / MT; q += blockDim.x)
-        flag_wait(d_done + bh * n_qb + sh.js[q], token, abort);
-      __syncthreads();
-    }
 
     if (warp == 0) {
       // ---------------- TMA producer (whole warp; one elected lane issues) --

@@ -193,7 +193,7 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
                            const int32_t* sel_grp, const void* o, const float* lse,
                            const void* d_o, void* dq, void* dk, void* dv, float* dvec,
                            int* unit_counter, const int* fwd_done, int* d_done, uint32_t token,
-                           cudaStream_t s) {
+                           int* inv, cudaStream_t s) {
   using LQ = bwdtc::DqLayout<MT>;
   using LK = bwdtc::KvLayout;
   CUtensorMap tq, tdo, tk, tv, tdq;
@@ -217,7 +217,7 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
         ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups, sel_grp,
         cfg->scale, scale_log2, static_cast<const __nv_bfloat16*>(o),
         static_cast<const __nv_bfloat16*>(d_o), lse, tdq, dvec,
-        unit_counter, fwd_done, d_done, token);
+        unit_counter, fwd_done, d_done, token, inv);
   });
   if (e != HGA_OK) return e;
   // persistent: at most one CTA per SM over the (key block, head) units
@@ -228,7 +228,7 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
         LK::kDynSmem, s, tq, tdo, tk, tv, ctx_cap, q_begin, s_len, cfg->batch, cfg->n_q_heads,
         cfg->n_kv_heads, cfg->topk_groups, sel_grp, cfg->scale, scale_log2, lse, dvec,
         static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), unit_counter,
-        fwd_done ? d_done : nullptr, token);
+        fwd_done ? d_done : nullptr, token, inv);
   });
 }
 
@@ -485,10 +485,41 @@ static size_t bwd_dvec_bytes(const hga_config_t* cfg, int32_t s_len) {
 static size_t bwd_flag_bytes(const hga_config_t* cfg, int32_t s_len) {
   return align256(size_t(cfg->batch) * cfg->n_kv_heads * size_t(s_len / kQBlock) * 4);
 }
+// the inverted selection the dQ kernel writes for the dK/dV kernel,
+// [B, Hkv, S/64 key blocks, S/64 query blocks] int32
+static size_t bwd_inv_bytes(const hga_config_t* cfg, int32_t s_len) {
+  const size_t n = size_t(s_len / kQBlock);
+  return align256(size_t(cfg->batch) * cfg->n_kv_heads * n * n * 4);
+}
+
+// [D][work counter (256 B)][forward flags][dQ flags][inverted selection]
+struct BwdCarve {
+  float* dvec;
+  int* unit_counter;
+  int* fwd_done;
+  int* d_done;
+  int* inv;
+};
+
+static BwdCarve bwd_carve(const hga_config_t* cfg, int32_t s_len, void* workspace) {
+  char* ws = static_cast<char*>(workspace);
+  BwdCarve c;
+  c.dvec = reinterpret_cast<float*>(ws);
+  ws += bwd_dvec_bytes(cfg, s_len);
+  c.unit_counter = reinterpret_cast<int*>(ws);
+  ws += 256;
+  c.fwd_done = reinterpret_cast<int*>(ws);
+  ws += bwd_flag_bytes(cfg, s_len);
+  c.d_done = reinterpret_cast<int*>(ws);
+  ws += bwd_flag_bytes(cfg, s_len);
+  c.inv = reinterpret_cast<int*>(ws);
+  return c;
+}
 
 size_t hga_attn_bwd_workspace_size(const hga_config_t* cfg, int32_t s_len) {
   if (check_cfg(cfg) != HGA_OK || s_len <= 0) return 0;
-  return bwd_dvec_bytes(cfg, s_len) + 256 + 2 * bwd_flag_bytes(cfg, s_len);
+  return bwd_dvec_bytes(cfg, s_len) + 256 + 2 * bwd_flag_bytes(cfg, s_len) +
+         bwd_inv_bytes(cfg, s_len);
 }
 
 hga_status_t hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k, const void* v,
@@ -504,16 +535,15 @@ hga_status_t hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k,
     if (!p || !aligned16(p)) return HGA_ERR_INVALID_ARG;
   if (ws_bytes < hga_attn_bwd_workspace_size(cfg, s_len)) return HGA_ERR_WORKSPACE;
   const int n_qb = s_len / kQBlock;
-  float* dvec = static_cast<float*>(workspace);
-  int* unit_counter =
-      reinterpret_cast<int*>(static_cast<char*>(workspace) + bwd_dvec_bytes(cfg, s_len));
+  const BwdCarve wc = bwd_carve(cfg, s_len, workspace);
+  float* dvec = wc.dvec;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (use_tensor_cores(cfg, ctx_cap, s_len)) {
     if (cfg->n_q_heads / cfg->n_kv_heads == 4)
       return launch_bwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq,
-                              dk, dv, dvec, unit_counter, nullptr, nullptr, 0, s);
+                              dk, dv, dvec, wc.unit_counter, nullptr, nullptr, 0, wc.inv, s);
     return launch_bwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk,
-                            dv, dvec, unit_counter, nullptr, nullptr, 0, s);
+                            dv, dvec, wc.unit_counter, nullptr, nullptr, 0, wc.inv, s);
   }
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
     const size_t sm1 = size_t(simt_fwd_smem_floats<D>()) * 4;
@@ -564,25 +594,24 @@ static hga_status_t fwd_bwd_impl(const hga_config_t* cfg, const void* q, const v
     return hga_attn_bwd(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk, dv,
                         workspace, ws_bytes, s);
   }
-  char* ws = static_cast<char*>(workspace);
-  float* dvec = reinterpret_cast<float*>(ws);
-  int* unit_counter = reinterpret_cast<int*>(ws + bwd_dvec_bytes(cfg, s_len));
-  int* fwd_done = reinterpret_cast<int*>(ws + bwd_dvec_bytes(cfg, s_len) + 256);
-  int* d_done = reinterpret_cast<int*>(reinterpret_cast<char*>(fwd_done) +
-                                       bwd_flag_bytes(cfg, s_len));
+  const BwdCarve wc = bwd_carve(cfg, s_len, workspace);
+  float* dvec = wc.dvec;
+  int* unit_counter = wc.unit_counter;
+  int* fwd_done = wc.fwd_done;
+  int* d_done = wc.d_done;
   hga_status_t st;
   if (cfg->n_q_heads / cfg->n_kv_heads == 4) {
     st = launch_fwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, route_done,
                           fwd_done, token, s);
     if (st != HGA_OK) return st;
     return launch_bwd_tc<2>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk,
-                            dv, dvec, unit_counter, fwd_done, d_done, token, s);
+                            dv, dvec, unit_counter, fwd_done, d_done, token, wc.inv, s);
   }
   st = launch_fwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, route_done,
                         fwd_done, token, s);
   if (st != HGA_OK) return st;
   return launch_bwd_tc<1>(cfg, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, d_o, dq, dk,
-                          dv, dvec, unit_counter, fwd_done, d_done, token, s);
+                          dv, dvec, unit_counter, fwd_done, d_done, token, wc.inv, s);
 }
 
 static hga_status_t check_fwd_bwd_args(const hga_config_t* cfg, int64_t ctx_cap, int64_t q_begin,

@@ -203,9 +203,12 @@ HGA_API hga_status_t hga_route_noalloc(const hga_config_t* cfg, const void* q, i
 
 /* Bytes of device workspace hga_attn_bwd and hga_attn_fwd_bwd need for this
  * segment: D = rowsum(dO * O) as [B, Hq, S] fp32, 256 bytes for the work
- * counter of the tensor-core dK/dV kernel, and two arrays of per-item
- * completion flags ([B, Hkv, S/64] int32 each) used by hga_attn_fwd_bwd;
- * every section starts on a 256-byte boundary. */
+ * counter of the tensor-core dK/dV kernel, two arrays of per-item
+ * completion flags ([B, Hkv, S/64] int32 each) used by hga_attn_fwd_bwd, and
+ * the inverted selection the dQ kernel writes for the dK/dV kernel ([B, Hkv,
+ * S/64 key blocks, S/64 query blocks] int32: which groups of each block of
+ * the segment each query block attends); every section starts on a 256-byte
+ * boundary. */
 HGA_API size_t hga_attn_bwd_workspace_size(const hga_config_t* cfg, int32_t s_len);
 
 /*

@@ -95,9 +95,11 @@ def test_workspace_sizes():
     # + block scores 8 x 32 x 256 floats (each part 256-B aligned)
     assert hga.hga_route_workspace_size(c, 2048, 14336) == (8 * 32 * 4 * 128 * 4
                                                            + 8 * 32 * 256 * 4)
-    # D = rowsum(dO * O) per query row, the dK/dV kernel's work counter, and
-    # two arrays of per-item flags (8 KV heads x 32 query blocks) for the fused call
-    assert hga.hga_attn_bwd_workspace_size(c, 2048) == 32 * 2048 * 4 + 256 + 2 * 8 * 32 * 4
+    # D = rowsum(dO * O) per query row, the dK/dV kernel's work counter, two
+    # arrays of per-item flags (8 KV heads x 32 query blocks) for the fused
+    # call, and the inverted selection (8 KV heads x 32 key blocks x 32 query blocks)
+    assert hga.hga_attn_bwd_workspace_size(c, 2048) == (32 * 2048 * 4 + 256 + 2 * 8 * 32 * 4
+                                                        + 8 * 32 * 32 * 4)
     assert hga.hga_route_workspace_size(cfg(head_dim=100), 2048, 0) == 0
     # the chained segment call: the backward workspace, a third flag array,
     # then the routing workspace
