@@ -466,6 +466,7 @@ struct KvShared {
   int abort;
   int n_items;
   int unit;
+  int pre_issued;  // items whose Q/dO the unit's set-up already requested
   int masks[64];
   int js[64];
 };
@@ -495,6 +496,20 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_qb = s_len / kQBlock;
   const int n_bh = batch * n_kv_heads, n_units = n_qb * n_bh;
+  // Q_m and dO_m of query block jj (two heads x 64 rows) into Q/dO buffer u
+  auto load_qd = [&](int u, int b, int h, int jj, int m) {
+    mbar_arrive_expect_tx(&sh.qd_full[u], 65536);
+    uint8_t* dst = smem + L::kQD + u * L::kQDBytes;
+    for (int g = 0; g < 2; ++g) {
+      const int32_t row =
+          int32_t((int64_t(b) * n_q_heads + h * G + 2 * m + g) * s_len + jj * kQBlock);
+      for (int hf = 0; hf < 2; ++hf) {
+        tma_load_2d(dst + hf * 16384 + g * 8192, &tm_q, &sh.qd_full[u], hf * 64, row);
+        tma_load_2d(dst + 32768 + hf * 16384 + g * 8192, &tm_do, &sh.qd_full[u], hf * 64,
+                    row);
+      }
+    }
+  };
   volatile int* abort = &sh.abort;
   pdl_launch_dependents();
 
@@ -557,6 +572,16 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
           tma_load_2d(smem + L::kV + hf * 8192 + gi * 1024, &tm_v, &sh.kv_full, hf * 64,
                       krow + gi * kGroup);
         }
+      // and the first items, the own block's M tiles (always the first in
+      // the visiting order), before the selection is read
+      int pre = 0;
+      for (int it = 0; it < MT; ++it) {
+        const int gi = it_base + it, u = gi & 1;
+        if (gi >= 2 && !mbar_wait(&sh.qd_empty[u], ((gi >> 1) - 1) & 1, abort)) break;
+        load_qd(u, b, h, kb, it);
+        ++pre;
+      }
+      sh.pre_issued = pre;
     }
     // which later query blocks of the segment selected groups of this block
     // (only query blocks after kb can): their dQ CTAs wrote it, tagged with
@@ -595,26 +620,15 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
 
     if (warp == 0) {
       // ---------------- TMA producer (whole warp; one elected lane issues) --
-      int issued = 0;
-      for (int it = 0; it < n_items; ++it) {
+      int issued = sh.pre_issued;
+      const bool pre_ok = issued == MT;  // else the set-up was aborted
+      for (int it = issued; pre_ok && it < n_items; ++it) {
         const int gi = it_base + it, u = gi & 1;
         const bool free_ok =
             gi < 2 || mbar_wait(&sh.qd_empty[u], ((gi >> 1) - 1) & 1, abort);
         if (!__all_sync(kFullMask, free_ok)) break;
         const int jj = sh.js[it / MT], m = it % MT;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(&sh.qd_full[u], 65536);
-          uint8_t* dst = smem + L::kQD + u * L::kQDBytes;
-          for (int g = 0; g < 2; ++g) {
-            const int32_t row =
-                int32_t((int64_t(b) * n_q_heads + h * G + 2 * m + g) * s_len + jj * kQBlock);
-            for (int hf = 0; hf < 2; ++hf) {
-              tma_load_2d(dst + hf * 16384 + g * 8192, &tm_q, &sh.qd_full[u], hf * 64, row);
-              tma_load_2d(dst + 32768 + hf * 16384 + g * 8192, &tm_do, &sh.qd_full[u],
-                          hf * 64, row);
-            }
-          }
-        }
+        if (elect_one()) load_qd(u, b, h, jj, m);
         __syncwarp();
         issued = it + 1;
       }
