@@ -9,7 +9,7 @@
 //
 // attn_bwd_dq_tc_kernel -- one CTA per (batch, KV head, query block), the G
 //   heads stacked into M = 64 G rows as in the forward.  Per key tile (the
-//   same tiles as the forward, gathered by cp.async into a 3-stage ring) and
+//   same tiles as the forward, gathered by 3-D TMA boxes into a 3-stage ring) and
 //   M tile: S = Q K^T and dP = dO V^T into one of two TMEM regions, then one
 //   thread per row forms P = exp2(S c - LSE2), dS = P (dP - D) and stores it
 //   as bf16 over the region's S columns, and dQ += dS K (A operand in tensor
@@ -50,7 +50,7 @@ template <int MT>
 struct DqLayout {
   static constexpr uint32_t kQ = 0;                              // [MT][2][128][128 B]
   static constexpr uint32_t kDO = MT * 32768;                    // same layout
-  static constexpr uint32_t kKV = 2 * MT * 32768;                // [3 stages][K | V]
+  static constexpr uint32_t kKV = 2 * MT * 32768;                // [3 stages][K | V], group-major
   static constexpr uint32_t kStages = 3;
   static constexpr uint32_t kStageBytes = 32768;
   static constexpr uint32_t kBytes = kKV + kStages * kStageBytes;
@@ -82,14 +82,14 @@ struct DqShared {
   uint8_t tile_mask[kMaxTiles];
 };
 
-constexpr int kDqProducers = 64;  // warps 0, 2
+
 
 template <int MT>
 __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_do,
-                          const __nv_bfloat16* __restrict__ k,
-                          const __nv_bfloat16* __restrict__ v, int64_t ctx_cap,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, int64_t ctx_cap,
                           int64_t q_begin, int s_len, int n_q_heads, int n_kv_heads,
                           int topk_groups, const int32_t* __restrict__ sel_grp, float scale,
                           float scale_log2, const __nv_bfloat16* __restrict__ o,
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     sh.d_arrived = 0;
     mbar_init(&sh.q_full, 1);
     for (int s = 0; s < kSt; ++s) {
-      mbar_init(&sh.kv_full[s], kDqProducers);
+      mbar_init(&sh.kv_full[s], 1);
       mbar_init(&sh.kv_empty[s], 2);  // the last S/dP and the last dQ of the tile
     }
     for (int r = 0; r < 2; ++r) {
@@ -150,6 +150,8 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
     // Q and dO first: they do not depend on the selection
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_do);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
     mbar_arrive_expect_tx(&sh.q_full, MT * 65536);
     for (int g = 0; g < G; ++g) {
       const int32_t row = int32_t((int64_t(b) * n_q_heads + h * G + g) * s_len + j * kQBlock);
@@ -174,28 +176,37 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
   const uint32_t tmem = sh.tmem_base;
   const int n_tiles = sh.n_tiles;
 
-  if (warp == 0 || warp == 2) {
-    // ---------------- producers: K/V groups by cp.async into a 3-stage ring ------
-    // stage layout [K | V][d half][64 rows][128 B], 128-byte swizzle
-    const int ptid = warp == 0 ? lane : 32 + lane;
-    const __nv_bfloat16* kh = k + (int64_t(b) * n_kv_heads + h) * ctx_cap * kD;
-    const __nv_bfloat16* vh = v + (int64_t(b) * n_kv_heads + h) * ctx_cap * kD;
+  if (warp == 0) {
+    // ---------------- TMA producer (whole warp; one elected lane issues) ----
+    // 3-stage ring; stage layout [K | V], each [group][d half][8 rows][128 B]
+    // (128-byte swizzle): one 3-D box (64 columns x 8 rows x 2 halves) per
+    // group and tensor
+    const int64_t kv_row0 = (int64_t(b) * n_kv_heads + h) * ctx_cap;
+    int issued = 0;
     for (int t = 0; t < n_tiles; ++t) {
       const int st = t % kSt;
-      if (t >= kSt && !mbar_wait(&sh.kv_empty[st], ((t / kSt) - 1) & 1, abort)) break;
-      const uint32_t kdst = sKV + st * L::kStageBytes;
-      for (int c = ptid; c < 2048; c += kDqProducers) {
-        const int tensor = c >> 10, rc = c & 1023, r = rc >> 4, ch = rc & 15;
-        const int64_t row = int64_t(sh.grp[t * 8 + (r >> 3)]) * kGroup + (r & 7);
-        const __nv_bfloat16* src = (tensor ? vh : kh) + row * kD + ch * 8;
-        cp_async16(kdst + tensor * 16384 + (ch >> 3) * 8192 + r * 128 + (((ch & 7) ^ (r & 7)) << 4),
-                   src);
+      const bool free_ok = t < kSt || mbar_wait(&sh.kv_empty[st], ((t / kSt) - 1) & 1, abort);
+      if (!__all_sync(kFullMask, free_ok)) break;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(&sh.kv_full[st], L::kStageBytes);
+        uint8_t* kdst = smem + L::kKV + st * L::kStageBytes;
+#pragma unroll
+        for (int gi = 0; gi < 8; ++gi) {
+          const int32_t row = int32_t(kv_row0 + int64_t(sh.grp[t * 8 + gi]) * kGroup);
+          tma_load_3d(kdst + gi * 2048, &tm_k, &sh.kv_full[st], 0, row, 0);
+          tma_load_3d(kdst + 16384 + gi * 2048, &tm_v, &sh.kv_full[st], 0, row, 0);
+        }
       }
-      cp_async_arrive(&sh.kv_full[st]);
+      __syncwarp();
+      issued = t + 1;
     }
-    int never = 0;
-    if (tid == 0) mbar_wait(&sh.q_full, 0, &never);
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    // drain: wait (bounded, independent of abort) for the copies in flight
+    if (lane == 0) {
+      int never = 0;
+      mbar_wait(&sh.q_full, 0, &never);
+      for (int t = issued - 1; t >= 0 && t >= issued - kSt; --t)
+        mbar_wait(&sh.kv_full[t % kSt], (t / kSt) & 1, &never);
+    }
   } else if (warp == 1 || warp == 3) {
     // ---------------- MMA issuers (whole warp each, one lane issues) ----------
     // Ops s = t * MT + m (tile t, M tile m) alternate between the two TMEM
@@ -245,17 +256,16 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
         bool ready = m != 0 || mbar_wait(&sh.kv_full[t % kSt], (t / kSt) & 1, abort);
         if (op >= 2) ready = ready && mbar_wait(&sh.ds_done[rg], ((op - 2) >> 1) & 1, abort);
         if (!(ok = __all_sync(kFullMask, ready))) break;
-        fence_proxy_async_smem();  // cp.async data -> tensor-core reads
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint32_t bo = (kk >> 2) * 8192 + (kk & 3) * 32;
+            const uint32_t bo = (kk >> 2) * 1024 + (kk & 3) * 32;
             mma_bf16(tmem + L::colS(rg), smem_desc_sw128(sQ + m * 32768 + ko, 16, 1024),
-                     smem_desc_sw128(kb + bo, 16, 1024), idesc_s, kk > 0);
+                     smem_desc_sw128(kb + bo, 16, 2048), idesc_s, kk > 0);
             mma_bf16(tmem + L::colDP(rg), smem_desc_sw128(sDO + m * 32768 + ko, 16, 1024),
-                     smem_desc_sw128(kb + 16384 + bo, 16, 1024), idesc_s, kk > 0);
+                     smem_desc_sw128(kb + 16384 + bo, 16, 2048), idesc_s, kk > 0);
           }
           mma_commit(&sh.sdp_full[rg]);
           if (m == MT - 1) mma_commit(&sh.kv_empty[t % kSt]);
@@ -268,7 +278,7 @@ __global__ void __launch_bounds__(DqLayout<MT>::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_bf16_tmem_a(tmem + L::colDQ(m), tmem + L::colS(rg) + kk * 8,
-                            smem_desc_sw128(kb + kk * 2048, 8192, 1024), idesc_dq,
+                            smem_desc_sw128(kb + kk * 4096, 1024, 2048), idesc_dq,
                             (t > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&sh.ds_done[rg]);
           if (m == MT - 1) mma_commit(&sh.kv_empty[t % kSt]);

@@ -196,11 +196,13 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
                            int* inv, cudaStream_t s) {
   using LQ = bwdtc::DqLayout<MT>;
   using LK = bwdtc::KvLayout;
-  CUtensorMap tq, tdo, tk, tv, tdq;
+  CUtensorMap tq, tdo, tk, tv, tdq, tkg, tvg;
   const uint64_t q_rows = uint64_t(cfg->batch) * cfg->n_q_heads * s_len;
   const uint64_t kv_rows = uint64_t(cfg->batch) * cfg->n_kv_heads * ctx_cap;
   if (!make_map_bf16_d128(&tq, q, q_rows, 64) || !make_map_bf16_d128(&tdo, d_o, q_rows, 64) ||
       !make_map_bf16_d128(&tdq, dq, q_rows, 64) ||
+      !make_map_bf16_d128_groups(&tkg, k, kv_rows, 8) ||
+      !make_map_bf16_d128_groups(&tvg, v, kv_rows, 8) ||
       !make_map_bf16_d128(&tk, k, kv_rows, 8) || !make_map_bf16_d128(&tv, v, kv_rows, 8))
     return HGA_ERR_CUDA;
   hga_status_t e = ensure_smem(
@@ -213,8 +215,7 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
   const float scale_log2 = cfg->scale * 1.4426950408889634f;
   e = traced_launch(HGA_K_BWD_DQ_TC, s, [&] {
     return launch_pdl(bwdtc::attn_bwd_dq_tc_kernel<MT>, grid, dim3(LQ::kThreads), LQ::kDynSmem, s,
-        tq, tdo, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-        ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups, sel_grp,
+        tq, tdo, tkg, tvg, ctx_cap, q_begin, s_len, cfg->n_q_heads, cfg->n_kv_heads, cfg->topk_groups, sel_grp,
         cfg->scale, scale_log2, static_cast<const __nv_bfloat16*>(o),
         static_cast<const __nv_bfloat16*>(d_o), lse, tdq, dvec,
         unit_counter, fwd_done, d_done, token, inv);
