@@ -26,8 +26,11 @@ __global__ void __launch_bounds__(D) summaries_kernel(const T* __restrict__ k, i
                                                       int64_t blk0, int n_kv_heads,
                                                       float* __restrict__ gsum,
                                                       float* __restrict__ bsum) {
+  // nothing this kernel reads is written by the kernel before it on the
+  // stream (only the keys of the new blocks, written before that kernel
+  // started): run alongside its tail, but complete only after it, so the
+  // kernels after this one see both complete
   pdl_launch_dependents();
-  pdl_wait();
   constexpr int CH = D / 8;  // column chunks per row
   __shared__ float part[kGroupsPerBlock][D];
   const int64_t c = blk0 + blockIdx.x;  // global block index
@@ -62,6 +65,7 @@ __global__ void __launch_bounds__(D) summaries_kernel(const T* __restrict__ k, i
     for (int g = 0; g < kGroupsPerBlock; ++g) s += part[g][e];
     bsum[(head * (ctx_cap / kBlock) + c) * D + e] = s * (1.0f / kBlock);
   }
+  pdl_wait();
 }
 
 }  // namespace hga
