@@ -311,9 +311,10 @@ __global__ void __launch_bounds__(kRouteThreads)
                        int n_kv_heads, int s_len, int64_t own0, int topk_blocks, int topk_groups,
                        int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp,
                        int* __restrict__ done, uint32_t token) {
-  // the next kernel may be scheduled once everything before this one has
-  // completed (a chained forward reads only its own item's selection)
-  pdl_wait();
+  // q-bar needs only the queries, which the kernels before this one do not
+  // write: it is formed while the kernel before still runs; the summaries
+  // are read only after it has completed (the wait below).  A chained
+  // forward waits for each item's flag, so it may be scheduled at once.
   pdl_launch_dependents();
   extern __shared__ __align__(16) unsigned char sm_raw[];
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -351,6 +352,8 @@ __global__ void __launch_bounds__(kRouteThreads)
     for (int r = 0; r < RS; ++r) sum += part[r * D + e];
     qb[e] = sum * inv;
   }
+  // from here on everything before this kernel has completed
+  pdl_wait();
   __syncthreads();
   // level-1 scores of the J candidate blocks
   score_rows<D>(bsum + head * (ctx_cap / kBlock) * D, qb, int(J),
