@@ -317,6 +317,14 @@ class Runner:
         self.layer = HgaLayer(cfg, w.ctx_len, w.seg_len, device=device,
                               k=self.k_host.to(device), v=self.v_host.to(device))
         self.segs = w.segments()
+        # each segment's K/V rows as one contiguous pinned block [B, Hkv, rows,
+        # d] (the first segment's also holds the history before it), so that
+        # each goes up in one copy per tensor
+        self.kv_host_seg = []
+        for i, q_begin in enumerate(self.segs):
+            lo, hi = (0 if i == 0 else q_begin), q_begin + w.seg_len
+            self.kv_host_seg.append((lo, hi, self.k_host[:, :, lo:hi].contiguous().pin_memory(),
+                                     self.v_host[:, :, lo:hi].contiguous().pin_memory()))
         self.q_host = [self.to_torch(synth.queries(w, s)).pin_memory() for s in self.segs]
         self.q = [t.to(device) for t in self.q_host]
         if w.backward:
@@ -363,14 +371,13 @@ class Runner:
         up_done = []
         with torch.cuda.stream(self.s_up):
             for i, q_begin in enumerate(self.segs):
-                lo = 0 if i == 0 else q_begin          # history rows go with the first
-                hi = q_begin + w.seg_len
-                # one contiguous block per (batch, KV head): a strided slice
-                # copy from pinned memory is staged through the host
-                for bb in range(w.batch):
-                    for hh in range(w.n_kv_heads):
-                        L.k[bb, hh, lo:hi].copy_(self.k_host[bb, hh, lo:hi], non_blocking=True)
-                        L.v[bb, hh, lo:hi].copy_(self.v_host[bb, hh, lo:hi], non_blocking=True)
+                # the segment's K/V block in one copy per tensor (a contiguous
+                # source; the rows land in the whole-context buffers through a
+                # device-side copy, while a strided source would be staged
+                # through the host)
+                lo, hi, kh, vh = self.kv_host_seg[i]
+                L.k[:, :, lo:hi].copy_(kh, non_blocking=True)
+                L.v[:, :, lo:hi].copy_(vh, non_blocking=True)
                 self.q[i].copy_(self.q_host[i], non_blocking=True)
                 if w.backward:
                     self.do[i].copy_(self.do_host[i], non_blocking=True)
@@ -398,7 +405,8 @@ class Runner:
 
     def io_bytes(self):
         nb = lambda t: t.numel() * t.element_size()  # noqa: E731
-        h2d = nb(self.k_host) + nb(self.v_host) + sum(nb(t) for t in self.q_host)
+        h2d = sum(nb(kh) + nb(vh) for _, _, kh, vh in self.kv_host_seg)
+        h2d += sum(nb(t) for t in self.q_host)
         L = self.layer
         outs = (L.o, L.dq, L.dk, L.dv) if self.w.backward else (L.o,)
         if self.w.backward:
