@@ -55,21 +55,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test of a phase (never suspends the thread, unlike try_wait,
-// which may park it for a while): for issuers that poll several barriers and
-// must act on whichever completes first.
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 constexpr unsigned kFullMask = 0xffffffffu;
 
 // True in exactly one lane of a converged warp: elect.sync picks the leader
@@ -105,29 +90,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// One step of the idle bookkeeping of an event loop run by a whole warp:
-// after progress the idle clock restarts; otherwise the loop ends (false) if
-// another role raised *abort, or -- latching HGA_ERR_TIMEOUT and raising
-// *abort -- once nothing has progressed for about 2e9 cycles.  The result is
-// the same in every lane.
-__device__ __forceinline__ bool warp_event_continue(bool progressed, long long& t0,
-                                                    volatile int* abort) {
-  if (progressed) {
-    t0 = clock64();
-    return true;
-  }
-  if (__any_sync(kFullMask, *abort != 0)) return false;
-  if (__any_sync(kFullMask, clock64() - t0 > 2000000000LL)) {
-    if ((threadIdx.x & 31) == 0) {
-      latch_status(HGA_ERR_TIMEOUT);
-      *abort = 1;
-    }
-    __syncwarp();
-    return false;
-  }
-  return true;
-}
-
 // ---------------------------------------------------------------------------
 // TMA (tiled, 2-D, no multicast)
 // ---------------------------------------------------------------------------
@@ -138,25 +100,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
-}
-
-// Bulk prefetch of [src, src + bytes) into L2 (no destination, no completion
-// to wait for); src 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
-// 16-byte asynchronous global -> shared copy (L2 only), and the arrive on an
-// mbarrier once every copy this thread issued so far has landed (the barrier's
-// expected count must include one arrival per issuing thread).
-__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src)
-               : "memory");
-}
-
-__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
 }
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
