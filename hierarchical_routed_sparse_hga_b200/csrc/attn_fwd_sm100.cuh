@@ -15,15 +15,17 @@
 //               column halves, into a 4-stage ring laid
 //               out [group][d half][8 rows][128 B] (128-byte swizzle; UMMA
 //               stride 2048 B between 8-row groups);
-//   warp 1      TMEM owner and MMA issuer: S = Q K^T into double-buffered
-//               TMEM and O += P V with P read straight from TMEM (A operand
-//               in tensor memory), in a fixed order with blocking waits;
+//   warp 1      TMEM owner and S issuer: S = Q K^T into double-buffered
+//               TMEM, in a fixed order with blocking waits;
+//   warp 3      PV issuer: O += P V with P read straight from TMEM (A
+//               operand in tensor memory), as soon as the softmax wrote it;
 //   warps 4..   softmax, one warp group per M tile, one thread per row (TMEM
 //               lane): masks (padding slots, causal own block; skipped for
 //               full routed tiles), online softmax in the log2 domain with
 //               packed f32x2 arithmetic and lazy rescaling (O is rescaled only
 //               when the running max grows by more than 2^8), P written back as
-//               bf16 over its own S columns, epilogue O / l and LSE.
+//               bf16 over its own S columns; epilogue O / l (through shared
+//               memory, TMA stores) and LSE.
 // The producer and issuer loops run in all 32 lanes of their warp, so loop
 // state and operand descriptors are warp-uniform; one elected lane issues.
 // Every wait is bounded; a timeout latches HGA_ERR_TIMEOUT, raises a shared
