@@ -100,6 +100,33 @@ def test_chained_segment_call_equals_separate_calls():
             assert torch.equal(a, b), q_begin
 
 
+def test_chained_segment_call_long_context_routing():
+    # past 512 candidate blocks the routing runs as three kernels and the
+    # chained call waits for the whole routing grid instead of per-item
+    # flags; the selections and outputs still equal the separate calls'
+    import dataclasses
+
+    import torch
+    w = dataclasses.replace(WL["qwen3_fwdbwd_16k"], name="qwen3_fwdbwd_36k_last",
+                            ctx_len=36864, first_seg=17)
+    seg = Segmenter(w)
+    L = seg.layer
+    q_begin = w.ctx_len - w.seg_len
+    assert q_begin // 64 > 512
+    q = to_device(synth.queries(w, q_begin), w)
+    d_o = to_device(synth.douts(w, q_begin), w)
+    L.summarize(q_begin)
+    L.route_forward_backward(q, d_o, q_begin)
+    torch.cuda.synchronize()
+    chained = [t.clone() for t in (L.sel_blk, L.sel_grp, L.o, L.lse, L.dq, L.dk, L.dv)]
+    L.route(q, q_begin)
+    L.forward(q, q_begin)
+    L.backward(q, d_o, q_begin)
+    torch.cuda.synchronize()
+    for a, b in zip(chained, (L.sel_blk, L.sel_grp, L.o, L.lse, L.dq, L.dk, L.dv)):
+        assert torch.equal(a, b)
+
+
 def test_segment_into_caller_output_set():
     # HgaLayer.segment(..., out=make_outputs()): the same results, written to
     # the caller's tensors (used to download one segment while the next runs)
