@@ -742,13 +742,9 @@ def run_gpu(args, rank, world, local):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": args.workload, "batch_per_gpu": w.batch,
-                       "seq_len": w.ctx_len, "seg_len": w.seg_len, "n_q_heads": w.n_q_heads,
-                       "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
-                       "topk_blocks": w.topk_blocks, "topk_groups": w.topk_groups,
-                       "backward": w.backward, "parallelism": f"replicas{world}",
-                       "l2": "flushed between timed steps (512 MiB write, untimed)",
-                       "graph": bool(args.graph), "attention": "simt" if args.simt else "auto"},
+            "config": dict(workload_config(args.workload, w, world),
+                           l2="flushed between timed steps (512 MiB write, untimed)",
+                           graph=bool(args.graph), attention="simt" if args.simt else "auto"),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(launches), "clocks": clocks, "kernels": kernels,
         }
@@ -824,6 +820,15 @@ def args_workload_name(w):
     return w.name
 
 
+def workload_config(name, w, world):
+    """The workload part of the JSON line's config, the same in both arms."""
+    return {"workload": name, "batch_per_gpu": w.batch, "seq_len": w.ctx_len,
+            "seg_len": w.seg_len, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+            "head_dim": w.head_dim, "topk_blocks": w.topk_blocks,
+            "topk_groups": w.topk_groups, "backward": w.backward,
+            "parallelism": f"replicas{world}"}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -844,7 +849,8 @@ def run_reference(args, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "seq_len": w.ctx_len, "seg_len": w.seg_len},
+            "config": dict(workload_config(w.name, w, world),
+                           attention="oracle (float64 NumPy on the host cores)"),
             "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s",
                              "cores": blas_threads(), "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
