@@ -1,0 +1,90 @@
+"""Host-side pieces of bench.py that the reported numbers rest on, on CPU.
+
+* The roofline's algorithmic work counts attended (query row, key) pairs
+  from a realised selection (`segment_pairs`).  Here it is checked against
+  the oracle's own definition of each query's key set (routed groups plus
+  the causal own block), counted one query at a time, and against the
+  active-segment restriction that the dK/dV work uses.
+* The DRAM traffic it reports comes from a committed ncu summary only while
+  that summary was taken on the current kernel sources.
+* Both arms describe the same workload in their JSON line.
+"""
+import importlib.util
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import hga_oracle as orc
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+
+
+def load_bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test",
+                                                  os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+class W:
+    """The fields segment_pairs reads."""
+    group_heads = 4
+    head_dim = 128
+
+
+def random_selection(rng, n_kv, n_qb, k_g, q_begin):
+    sel = np.full((1, n_kv, n_qb, k_g), -1, np.int32)
+    for h in range(n_kv):
+        for j in range(n_qb):
+            own_blk = (q_begin + 64 * j) // 64
+            cands = np.arange(own_blk * 8)          # every group before the own block
+            n = min(int(rng.integers(0, k_g + 1)), len(cands))
+            sel[0, h, j, :n] = np.sort(rng.choice(cands, n, replace=False))
+    return sel
+
+
+@pytest.mark.parametrize("q_begin", [0, 1024, 4096])
+def test_segment_pairs_counts_the_oracle_key_sets(q_begin):
+    bench = load_bench()
+    rng = np.random.default_rng(q_begin + 7)
+    n_kv, n_qb, k_g = 2, 4, 12
+    sel = random_selection(rng, n_kv, n_qb, k_g, q_begin)
+    all_pairs, act_pairs = bench.segment_pairs(W, sel, q_begin)
+    want_all = want_act = 0
+    for h in range(n_kv):
+        for j in range(n_qb):
+            for r in range(64):
+                keys = orc.keyset(q_begin, j, r, sel[0, h, j])
+                want_all += len(keys) * W.group_heads
+                want_act += int((keys >= q_begin).sum()) * W.group_heads
+    assert all_pairs == want_all
+    assert act_pairs == want_act
+
+
+def test_measured_traffic_only_for_the_current_sources(tmp_path, monkeypatch):
+    bench = load_bench()
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    entry = {"bytes_per_launch": 1234, "source_hash": bench.source_hash()}
+    (prof / "dram_traffic.json").write_text(json.dumps({"wl": {"k": entry}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "source_hash", lambda: entry["source_hash"])
+    assert bench.measured_traffic("k", "wl") == 1234
+    assert bench.measured_traffic("other", "wl") is None
+    monkeypatch.setattr(bench, "source_hash", lambda: "changed")
+    assert bench.measured_traffic("k", "wl") is None
+
+
+def test_both_arms_describe_the_same_workload():
+    bench = load_bench()
+    from hierarchical_routed_sparse_hga_b200 import synth
+    w = synth.workloads()["qwen3_fwdbwd_16k"]
+    cfg = bench.workload_config("qwen3_fwdbwd_16k", w, 1)
+    assert cfg["workload"] == "qwen3_fwdbwd_16k"
+    assert (cfg["seq_len"], cfg["seg_len"], cfg["n_q_heads"], cfg["n_kv_heads"],
+            cfg["head_dim"]) == (16384, 2048, 32, 8, 128)
+    assert cfg["backward"] is True and cfg["parallelism"] == "replicas1"
