@@ -114,3 +114,51 @@ def test_diagnostics_without_gpu():
     assert hga.hga_kernel_name(99) == "unknown"
     assert hga.hga_launch_count() >= 0
     assert hga.timing_table() == {}
+
+
+def prototypes():
+    """name -> (return type, [parameter types]) from the header's HGA_API lines."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"HGA_API\s+([\w\s\*]+?)\b(hga_\w+)\s*\(([^)]*)\)\s*;", text):
+        ret, name, params = m.group(1).strip(), m.group(2), m.group(3).strip()
+        types = []
+        if params and params != "void":
+            for p in params.split(","):
+                p = " ".join(p.split())
+                pname = re.search(r"(\w+)\s*$", p).group(1)
+                types.append(p[: len(p) - len(pname)].strip())
+        out[name] = (ret, types)
+    return out
+
+
+def ctype_of(c_type):
+    """The ctypes class the binding must use for a C type of the header."""
+    t = c_type.replace("const ", "").replace(" ", "")
+    if t == "hga_config_t*":
+        return ctypes.POINTER(_lib._Config)
+    if t == "double*":
+        return ctypes.POINTER(ctypes.c_double)
+    if t == "uint64_t*":
+        return ctypes.POINTER(ctypes.c_uint64)
+    if t.endswith("*"):
+        return ctypes.c_char_p if t == "char*" else ctypes.c_void_p
+    return {"int64_t": ctypes.c_int64, "int32_t": ctypes.c_int32, "size_t": ctypes.c_size_t,
+            "int": ctypes.c_int, "uint32_t": ctypes.c_uint32, "uint64_t": ctypes.c_uint64,
+            "hga_status_t": ctypes.c_int, "void": None}[t]
+
+
+def test_binding_signatures_match_the_header():
+    # every argument's width and kind as the header declares it, in order:
+    # a parameter added, dropped or reordered on one side fails here
+    lib = _lib.load()
+    protos = prototypes()
+    assert set(protos) == declared()
+    for name, (ret, params) in protos.items():
+        fn = getattr(lib, name)
+        want = [ctype_of(p) for p in params]
+        got = list(fn.argtypes or [])
+        assert len(got) == len(want), (name, len(got), len(want))
+        for i, (g, w_) in enumerate(zip(got, want)):
+            assert g == w_ or (w_ is ctypes.c_int and g is ctypes.c_int32), (name, i, g, w_)
+        assert fn.restype == ctype_of(ret), (name, fn.restype, ret)
