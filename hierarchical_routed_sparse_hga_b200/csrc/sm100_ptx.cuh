@@ -1,6 +1,6 @@
 // Thin inline-PTX wrappers for the sm_100a building blocks used by the
 // tensor-core attention kernels: mbarriers (with bounded waits), TMA tiled
-// loads (no cluster multicast anywhere), tcgen05 TMEM allocation, MMA,
+// loads (single-CTA tiled copies only), tcgen05 TMEM allocation, MMA,
 // commit, and TMEM loads/stores, plus the UMMA shared-memory and instruction
 // descriptors.
 #pragma once
@@ -91,7 +91,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------
-// TMA (tiled, 2-D, no multicast)
+// TMA (tiled, 2-D, each CTA loads its own tiles)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t x, int32_t y) {

@@ -19,15 +19,26 @@ WL = synth.workloads()
 
 
 def run_and_compare(w, segments=None, kv_heads=None, flags=0):
+    """Every asked-for segment against the oracle.  Prints, per workload, how
+    many (batch, KV head, query block) rows the oracle flags as near ties and
+    on how many of those the GPU picked another valid selection."""
     seg = Segmenter(w, kv_heads=kv_heads, flags=flags)
     n_kv = len(seg.heads)
     want = set(w.segments() if segments is None else segments)
-    flagged = 0
+    flagged = differ = rows = 0
     for q_begin in w.segments():
         out = seg.run_segment(q_begin)
         if q_begin in want:
-            flagged += compare_segment(w, out, q_begin, n_kv, seg.k64, seg.v64, w.backward)
-    return flagged
+            f, dif = compare_segment(w, out, q_begin, n_kv, seg.k64, seg.v64, w.backward)
+            flagged += f
+            differ += dif
+            rows += w.batch * n_kv * (w.seg_len // 64)
+    print(f"[{w.name}] near-tie rows: {flagged} of {rows} flagged, "
+          f"{differ} with another valid selection on the GPU")
+    # the GPU ranks in float32 what the oracle ranks in float64: on a flagged
+    # row it may take the other side of the tie, but it must stay rare
+    assert differ <= max(2, rows // 20), (differ, rows)
+    return flagged, differ
 
 
 def test_tiny_f32_fwd_bwd():

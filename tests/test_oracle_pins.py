@@ -221,6 +221,54 @@ def test_route_first_block_has_no_candidates():
     assert (sb[:, :, 1, 0] == 0).all() and (sb[:, :, 1, 1] == -1).all()
 
 
+def _tie_case(block_x, group_x=None, topk_blocks=2, topk_groups=5):
+    """route() on hand-built summaries (d = 2, one head, one query block whose
+    queries are all (1, 0)), so every score is block_x[c]/sqrt(2) at level 1
+    and group_x[g]/sqrt(2) at level 2.  Returns (sel_blk, sel_grp, flag)."""
+    nb = len(block_x)
+    if group_x is None:                  # well separated: no level-2 tie
+        group_x = [100.0 - 1.7 * g for g in range(8 * nb)]
+    bsum = np.zeros((1, 1, nb + 1, 2))
+    bsum[0, 0, :nb, 0] = block_x
+    gsum = np.zeros((1, 1, 8 * (nb + 1), 2))
+    gsum[0, 0, :8 * nb, 0] = group_x
+    q = np.zeros((1, 1, 64, 2))
+    q[..., 0] = 1.0
+    sb, sg, tie = oracle.route(q, bsum, gsum, 64 * nb, topk_blocks, topk_groups, 1)
+    return list(sb[0, 0, 0]), list(sg[0, 0, 0]), bool(tie[0, 0, 0])
+
+
+def check_near_tie_flags():
+    """The near-tie flag, by hand: set iff the k-th and (k+1)-th sorted scores
+    of a level differ by at most 1e-3 of the larger magnitude."""
+    rel_in, rel_out = 2.0 * (1 - 0.9e-3), 2.0 * (1 - 1.1e-3)
+    # level 1, the gap at the k boundary just inside / just outside the window
+    sb, _, f = _tie_case([3.0, 2.0, rel_in, 0.5])
+    assert f and sb == [0, 1]
+    assert not _tie_case([3.0, 2.0, rel_out, 0.5])[2]
+    # a close pair next to (not at) the boundary does not flag: (k+1, k+2), (k-1, k)
+    assert not _tie_case([3.0, 2.0, 1.0, 0.9995])[2]
+    assert not _tie_case([3.0, 2.9995, 1.0, 0.5])[2]
+    # the window is relative: large scores 0.5 apart flag, tiny ones 5e-4 apart do not
+    assert _tie_case([1000.0, 999.5, 10.0], topk_blocks=1)[2]
+    assert not _tie_case([1e-3, 5e-4, 1e-4], topk_blocks=1)[2]
+    # no (k+1)-th score when k covers every candidate: exact ties do not flag
+    sb, sg, f = _tie_case([1.0, 1.0], group_x=[1.0] * 16, topk_blocks=4, topk_groups=16)
+    assert not f and sb == [0, 1, -1, -1] and sg == list(range(16))
+    # the first query block has no candidates at all
+    assert not _tie_case([], topk_blocks=2)[2]
+    # level 2 alone: blocks 0, 1 clear of block 2; groups' 5th/6th scores in or out
+    gx = [50.0, 40.0, 30.0, 20.0, 10.0, 10.0 * (1 - 0.9e-3), 1.0, 0.5] + [0.1 * i for i in range(8)]
+    _, sg, f = _tie_case([3.0, 2.0, 0.5], group_x=gx + [0.0] * 8)
+    assert f and sg == [0, 1, 2, 3, 4]
+    gx[5] = 10.0 * (1 - 1.1e-3)
+    assert not _tie_case([3.0, 2.0, 0.5], group_x=gx + [0.0] * 8)[2]
+
+
+def test_near_tie_flags():
+    check_near_tie_flags()
+
+
 def test_planted_target_ranks_first():
     # statistical sanity check on the tiny fp32 workload (not an exactness test)
     w = synth.workloads()["tiny_f32"]
@@ -406,12 +454,44 @@ def _mut_summaries_sum(k, t_begin, t_end):
     return g * 8, b                                               # group sum, not mean
 
 
+def _mut_near_tie_next_pair(sorted_scores, k):
+    # compares the (k+1)-th and (k+2)-th scores instead of the k-th and (k+1)-th
+    if k + 1 >= len(sorted_scores) or k == 0:
+        return False
+    a, b = sorted_scores[k], sorted_scores[k + 1]
+    return abs(a - b) <= ho.TIE_REL * max(abs(a), abs(b))
+
+
+def _mut_near_tie_absolute(sorted_scores, k):
+    # an absolute window instead of a relative one
+    if k >= len(sorted_scores) or k == 0:
+        return False
+    return abs(sorted_scores[k - 1] - sorted_scores[k]) <= ho.TIE_REL
+
+
+class _MutNearTieLevel1Only:
+    """route() asks level 1 first and level 2 only when level 1 did not flag;
+    this mutant answers level 2 with False (the level-2 flag dropped)."""
+
+    def __init__(self):
+        self.level2_next = False
+
+    def __call__(self, sorted_scores, k):
+        if self.level2_next:
+            self.level2_next = False
+            return False
+        flag = ORIG["_near_tie"](sorted_scores, k)
+        self.level2_next = not flag
+        return flag
+
+
 ORIG = {"route": ho.route, "_topk_lower_index": ho._topk_lower_index,
-        "_block_keys": ho._block_keys, "build_summaries": ho.build_summaries}
+        "_block_keys": ho._block_keys, "build_summaries": ho.build_summaries,
+        "_near_tie": ho._near_tie}
 
 ALL_PINS = [check_summaries_closed_form, check_route_golden, check_route_bruteforce,
             check_attention_golden, check_dense_equivalence, check_masked_sdpa,
-            check_finite_differences]
+            check_finite_differences, check_near_tie_flags]
 
 
 @pytest.mark.parametrize("target,mutant", [
@@ -419,6 +499,9 @@ ALL_PINS = [check_summaries_closed_form, check_route_golden, check_route_brutefo
     ("_topk_lower_index", _mut_topk_higher_index),
     ("_block_keys", _mut_block_keys_strict),
     ("build_summaries", _mut_summaries_sum),
+    ("_near_tie", _mut_near_tie_next_pair),
+    ("_near_tie", _mut_near_tie_absolute),
+    ("_near_tie", _MutNearTieLevel1Only()),
 ])
 def test_pins_catch_planted_mistakes(monkeypatch, target, mutant):
     monkeypatch.setattr(ho, target, mutant)
@@ -428,7 +511,7 @@ def test_pins_catch_planted_mistakes(monkeypatch, target, mutant):
     for pin in ALL_PINS:
         try:
             pin()
-        except AssertionError:
+        except (AssertionError, IndexError):
             failed += 1
     assert failed >= 1, f"no pin caught the planted mistake in {target}"
 

@@ -3,12 +3,18 @@
 Some callers have no way to call cudaMalloc -- a plugin inside a host runtime
 that owns all device memory and gives its extensions no allocator, or code
 that must not allocate once running because cudaMalloc can synchronise the
-device.  hga_route_noalloc serves them by taking the router's scratch from an
-array built into the library instead of a caller-provided workspace.  This
-test calls it through the C ABI twice in a row, on two different segments (so
-the second call starts from the first call's leftover scratch contents), and
-checks that each result equals the workspace-taking hga_route's.  Selections
-are integer indices, so they must match exactly.
+device.  hga_route_noalloc serves them by taking the router's scratch (the
+mean queries and the block scores) from an array built into the library
+instead of a caller-provided workspace.
+
+The context here is long enough (more than 512 candidate blocks) that the
+routing runs as its three-kernel form, which is the form that writes and
+reads that scratch.  The test calls the entry point through the C ABI twice
+in a row: first at the end of a 40960-token context, then on an earlier
+segment with fewer candidates, so the second call's score rows are shorter
+than the first call's and sit over its leftover contents.  Each result must
+equal the workspace-taking hga_route's exactly (selections are integer
+indices).
 
 The file name sorts last so that a run which stops at the first failure has
 already run every other test.
@@ -28,7 +34,7 @@ def test_route_noalloc_matches_route_on_two_calls_in_a_row():
                                                      hga_build_summaries, hga_route,
                                                      hga_route_noalloc)
 
-    w = synth.custom(n_q_heads=32, n_kv_heads=8, head_dim=128, ctx_len=8192, seg_len=2048,
+    w = synth.custom(n_q_heads=32, n_kv_heads=8, head_dim=128, ctx_len=40960, seg_len=2048,
                      topk_blocks=16, topk_groups=64, dtype="bf16", scaled=True,
                      rope_base=1e6, seed=21)
     dev = torch.device("cuda", 0)
@@ -43,7 +49,8 @@ def test_route_noalloc_matches_route_on_two_calls_in_a_row():
     hga_build_summaries(cfg, layer.k, w.ctx_len, 0, w.ctx_len, layer.gsum, layer.bsum)
 
     n_qb = w.seg_len // 64
-    for q_begin in (6144, 2048):          # two calls in a row, different shapes of work
+    for q_begin in (38912, 34816):        # two calls in a row, the second with shorter rows
+        assert q_begin // 64 > 512        # past the single-kernel routing's limit
         q = bf16(synth.queries(w, q_begin))
         ref_blk = torch.full((1, 8, n_qb, 16), -9, dtype=torch.int32, device=dev)
         ref_grp = torch.full((1, 8, n_qb, 64), -9, dtype=torch.int32, device=dev)
@@ -57,6 +64,9 @@ def test_route_noalloc_matches_route_on_two_calls_in_a_row():
         assert torch.equal(blk, ref_blk), q_begin
         assert torch.equal(grp, ref_grp), q_begin
         assert (grp >= 0).all()           # every slot filled: 16 blocks x 8 groups >= 64
+    # and no device-side check latched an error on the way
+    from hierarchical_routed_sparse_hga_b200 import hga_get_device_status
+    assert hga_get_device_status() == 0
 
 
 def test_route_noalloc_rejects_work_beyond_its_scratch():
