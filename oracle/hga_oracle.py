@@ -302,3 +302,71 @@ def segment_step(q, k, v, do, q_begin: int, gsum, bsum, topk_blocks: int,
         dq, dk, dv = attn_bwd(q, k, v, do, q_begin, sel_grp, n_kv_heads)
         out.update(dq=dq, dk=dk, dv=dv)
     return out
+
+
+# ----------------------------------------------------------------------------
+# decode: one new token per sequence routed against the resident summaries
+# (the adnankhan.ai notes, "Raw Abstract / Excerpt": HGA can also be used for
+# generation).  Readings:
+#   D1  the "query block" of a decode step is the one new token: qbar is the
+#       mean of its query over the G heads of the KV head (R2 with 1 row);
+#   D2  candidates are the complete blocks before the token's own block
+#       (R3): [0, pos // 64); the own block is not complete, so its summary
+#       is never scored;
+#   D3  the token attends to the selected groups' tokens and to its own
+#       block's tokens at positions <= pos (R6), its own K/V included (the
+#       caller writes them into the context before the step).
+# ----------------------------------------------------------------------------
+
+def decode_route(q_tok: np.ndarray, bsum: np.ndarray, gsum: np.ndarray, pos,
+                 topk_blocks: int, topk_groups: int, n_kv_heads: int):
+    """Routing of one token per sequence.  q_tok: [B, Hq, d] float64; pos:
+    global position of each sequence's token.  Returns sel_blk [B,Hkv,k_b],
+    sel_grp [B,Hkv,k_g] (ascending, -1 padded) and near_tie [B,Hkv]."""
+    B, Hq, d = q_tok.shape
+    G = Hq // n_kv_heads
+    sel_blk = np.full((B, n_kv_heads, topk_blocks), -1, np.int32)
+    sel_grp = np.full((B, n_kv_heads, topk_groups), -1, np.int32)
+    near_tie = np.zeros((B, n_kv_heads), bool)
+    inv_sqrt_d = 1.0 / math.sqrt(d)
+    for b in range(B):
+        own = int(pos[b]) // BLOCK                         # D2
+        for h in range(n_kv_heads):
+            qbar = q_tok[b, h * G:(h + 1) * G, :].mean(axis=0)      # D1
+            s1 = (bsum[b, h, :own, :] @ qbar) * inv_sqrt_d
+            kb = min(topk_blocks, own)
+            blocks, s1_sorted = _topk_lower_index(s1, np.arange(own), kb)
+            blocks = np.sort(blocks)
+            groups = (blocks[:, None] * GROUPS_PER_BLOCK
+                      + np.arange(GROUPS_PER_BLOCK)[None, :]).reshape(-1)
+            s2 = (gsum[b, h, groups, :] @ qbar) * inv_sqrt_d
+            kg = min(topk_groups, len(groups))
+            chosen, s2_sorted = _topk_lower_index(s2, groups, kg)
+            sel_blk[b, h, :kb] = blocks
+            sel_grp[b, h, :kg] = np.sort(chosen)
+            near_tie[b, h] = _near_tie(s1_sorted, kb) or _near_tie(s2_sorted, kg)
+    return sel_blk, sel_grp, near_tie
+
+
+def decode_attn(q_tok: np.ndarray, k: np.ndarray, v: np.ndarray, pos, sel_grp: np.ndarray,
+                n_kv_heads: int):
+    """Attention of one token per sequence over its selection (D3).
+    Returns o [B, Hq, d] and lse [B, Hq] (natural log)."""
+    B, Hq, d = q_tok.shape
+    G = Hq // n_kv_heads
+    scale = 1.0 / math.sqrt(d)
+    o = np.zeros_like(q_tok)
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        p = int(pos[b])
+        own0 = (p // BLOCK) * BLOCK
+        for h in range(n_kv_heads):
+            keys = np.concatenate([routed_keys(sel_grp[b, h]), np.arange(own0, p + 1)])
+            kk, vv = k[b, h, keys, :], v[b, h, keys, :]
+            for hq in range(h * G, (h + 1) * G):
+                s = (kk @ q_tok[b, hq]) * scale
+                m = s.max()
+                w = np.exp(s - m)
+                o[b, hq] = (w @ vv) / w.sum()
+                lse[b, hq] = m + math.log(w.sum())
+    return o, lse

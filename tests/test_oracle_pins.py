@@ -554,3 +554,140 @@ def test_tier_stage_preserves_attention():
             sel = sg[b, h]
             want = sorted(set(int(x) for x in sel.ravel() if 0 <= x < q_begin // 8))
             assert list(uniq[b][h]) == want
+
+
+# ----------------------------------------------------------------------------
+# pins: decode (one token per sequence)
+# ----------------------------------------------------------------------------
+
+def decode_case(seed=4, ctx=640, hq=4, hkv=2, d=16, batch=3, topk_blocks=3, topk_groups=7):
+    w = synth.custom(batch=batch, n_q_heads=hq, n_kv_heads=hkv, head_dim=d, ctx_len=ctx,
+                     seg_len=64, topk_blocks=topk_blocks, topk_groups=topk_groups,
+                     seed=seed, first_seg=0)
+    k = synth.widen(synth.keys(w), "f32")
+    v = synth.widen(synth.values(w), "f32")
+    rng = np.random.default_rng(seed)
+    q_tok = rng.standard_normal((batch, hq, d))
+    return w, q_tok, k, v
+
+
+def check_decode_against_prefill():
+    """A query block whose 64 rows all carry the same query routes exactly as
+    a decode step of that query at any position of the block, and row r of
+    its attention is the decode step at position 64J + r."""
+    w, q_tok, k, v = decode_case()
+    B, Hq, d = q_tok.shape
+    g, bl = summaries_upto(k, w.ctx_len)
+    for J in (0, 1, 4, 9):
+        q_blk = np.repeat(q_tok[:, :, None, :], 64, axis=2)
+        sb, sg, tie = oracle.route(q_blk, bl, g, 64 * J, w.topk_blocks, w.topk_groups, 2)
+        o_blk, lse_blk = oracle.attn_fwd(q_blk, k, v, 64 * J, sg, 2)
+        for r in (0, 17, 63):
+            pos = [64 * J + r] * B
+            db, dg, dtie = oracle.decode_route(q_tok, bl, g, pos, w.topk_blocks,
+                                               w.topk_groups, 2)
+            assert np.array_equal(db, sb[:, :, 0]) and np.array_equal(dg, sg[:, :, 0])
+            assert np.array_equal(dtie, tie[:, :, 0])
+            o, lse = oracle.decode_attn(q_tok, k, v, pos, dg, 2)
+            assert close(o, o_blk[:, :, r]) and close(lse, lse_blk[:, :, r])
+
+
+def test_decode_against_prefill():
+    check_decode_against_prefill()
+
+
+def check_decode_dense_equivalence():
+    """top-k covering every candidate: a decode step is dense causal attention
+    of that one query over every earlier token and itself (torch SDPA, f64)."""
+    w, q_tok, k, v = decode_case(topk_blocks=64, topk_groups=256)
+    g, bl = summaries_upto(k, w.ctx_len)
+    pos = [5, 200, 639]
+    _, sg, _ = oracle.decode_route(q_tok, bl, g, pos, 64, 256, 2)
+    o, lse = oracle.decode_attn(q_tok, k, v, pos, sg, 2)
+    G = 2
+    for b, p in enumerate(pos):
+        for hq in range(4):
+            kk = torch.from_numpy(k[b, hq // G, :p + 1])
+            vv = torch.from_numpy(v[b, hq // G, :p + 1])
+            qq = torch.from_numpy(q_tok[b, hq])[None]
+            ref = F.scaled_dot_product_attention(qq[None], kk[None], vv[None])[0, 0].numpy()
+            assert close(o[b, hq], ref)
+            s = (kk.numpy() @ q_tok[b, hq]) / math.sqrt(q_tok.shape[-1])
+            assert abs(lse[b, hq] - (s.max() + math.log(np.exp(s - s.max()).sum()))) < 1e-12
+
+
+def test_decode_dense_equivalence():
+    check_decode_dense_equivalence()
+
+
+def check_decode_route_bruteforce():
+    """Literal definition: block score = mean over the G heads and the
+    block's 64 keys of q.k/sqrt(d); exhaustive sort by (-score, index)."""
+    w, q_tok, k, v = decode_case(seed=8)
+    B, Hq, d = q_tok.shape
+    G = Hq // 2
+    g, bl = summaries_upto(k, w.ctx_len)
+    pos = [64 * 7 + 3, 64 * 9 + 63, 64 * 2]
+    sb, sg, tie = oracle.decode_route(q_tok, bl, g, pos, w.topk_blocks, w.topk_groups, 2)
+    for b in range(B):
+        for h in range(2):
+            if tie[b, h]:
+                continue
+            qs = [q_tok[b, hh] for hh in range(h * G, (h + 1) * G)]
+
+            def score(keys):
+                return sum(float(qq @ k[b, h, t]) for qq in qs for t in keys) / (
+                    len(qs) * len(keys) * math.sqrt(d))
+            J = pos[b] // 64
+            blocks = sorted(range(J), key=lambda c: (-score(range(64 * c, 64 * c + 64)), c))
+            blocks = sorted(blocks[:w.topk_blocks])
+            groups = [8 * c + i for c in blocks for i in range(8)]
+            groups = sorted(groups, key=lambda gg: (-score(range(8 * gg, 8 * gg + 8)), gg))
+            groups = sorted(groups[:w.topk_groups])
+            assert [x for x in sb[b, h] if x >= 0] == blocks
+            assert [x for x in sg[b, h] if x >= 0] == groups
+
+
+def test_decode_route_bruteforce():
+    check_decode_route_bruteforce()
+
+
+def test_decode_first_block_attends_only_itself():
+    w, q_tok, k, v = decode_case()
+    g, bl = summaries_upto(k, w.ctx_len)
+    sb, sg, tie = oracle.decode_route(q_tok, bl, g, [0, 1, 63], 3, 7, 2)
+    assert (sb == -1).all() and (sg == -1).all() and not tie.any()
+    o, lse = oracle.decode_attn(q_tok, k, v, [0, 1, 63], sg, 2)
+    assert close(o[0], np.repeat(v[0, :, 0], 2, axis=0))      # one key: O = its value
+    assert close(lse[0], (q_tok[0] * np.repeat(k[0, :, 0], 2, axis=0)).sum(-1) / 4.0)
+
+
+def _mut_decode_own_block_candidate(q_tok, bsum, gsum, pos, kb, kg, hkv):
+    # the incomplete own block scored as a candidate too
+    return ORIG_DECODE["decode_route"](q_tok, bsum, gsum, [p + 64 for p in pos], kb, kg, hkv)
+
+
+def _mut_decode_attn_without_itself(q_tok, k, v, pos, sel_grp, hkv):
+    # the token does not attend to its own key
+    return ORIG_DECODE["decode_attn"](q_tok, k, v, [p - 1 for p in pos], sel_grp, hkv)
+
+
+ORIG_DECODE = {"decode_route": ho.decode_route, "decode_attn": ho.decode_attn}
+DECODE_PINS = [check_decode_against_prefill, check_decode_dense_equivalence,
+               check_decode_route_bruteforce]
+
+
+@pytest.mark.parametrize("target,mutant", [
+    ("decode_route", _mut_decode_own_block_candidate),
+    ("decode_attn", _mut_decode_attn_without_itself),
+])
+def test_decode_pins_catch_planted_mistakes(monkeypatch, target, mutant):
+    monkeypatch.setattr(ho, target, mutant)
+    monkeypatch.setattr(oracle, target, mutant)
+    failed = 0
+    for pin in DECODE_PINS:
+        try:
+            pin()
+        except (AssertionError, IndexError, ValueError):
+            failed += 1
+    assert failed >= 1, f"no pin caught the planted mistake in {target}"
