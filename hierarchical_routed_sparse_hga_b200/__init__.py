@@ -11,7 +11,7 @@ from ._lib import (EXPORTS, HGA_BF16, HGA_ERR_CUDA, HGA_ERR_DEVICE_CHECK,  # noq
                    HGA_ERR_WORKSPACE, HGA_F32, HGA_FLAG_SIMT, HGA_K_COUNT, HGA_OK, Config,
                    HgaError,
                    hga_attn_bwd, hga_attn_bwd_workspace_size, hga_attn_fwd,
-                   hga_attn_fwd_bwd, hga_segment_fwd_bwd, hga_segment_workspace_size,
+                   hga_attn_fwd_bwd, hga_decode, hga_segment_fwd_bwd, hga_segment_workspace_size,
                    hga_build_summaries, hga_build_summaries_seg, hga_tier_append, hga_tier_gather,
                    hga_tier_stage_rows, hga_tier_workspace_size, hga_get_device_status,
                    hga_kernel_name,

@@ -31,9 +31,9 @@ EXPORTS = ("hga_version", "hga_status_string", "hga_build_summaries",
            "hga_timing_get", "hga_timing_reset", "hga_timing_kinds", "hga_route_noalloc",
            "hga_build_summaries_seg",
            "hga_tier_stage_rows", "hga_tier_workspace_size", "hga_tier_gather",
-           "hga_tier_append")
+           "hga_tier_append", "hga_decode")
 HGA_NOALLOC_SCRATCH_BYTES = 4 << 20
-HGA_K_COUNT = 13
+HGA_K_COUNT = 14
 
 
 class HgaError(RuntimeError):
@@ -114,6 +114,7 @@ def load() -> ctypes.CDLL:
         "hga_tier_gather": (ctypes.c_int, [CFG, P, P, I64, I64, I32, P, P, P, I64, P, P, P, SZ,
                                            P]),
         "hga_tier_append": (ctypes.c_int, [CFG, P, P, I64, P, P, I64, I64, I32, P]),
+        "hga_decode": (ctypes.c_int, [CFG, P, P, P, I64, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -239,6 +240,15 @@ def hga_route_noalloc(cfg: Config, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_b
     _check("hga_route_noalloc", load().hga_route_noalloc(
         ctypes.byref(c), _ptr(q), q_begin, s_len, ctx_cap, _ptr(bsum), _ptr(gsum),
         _ptr(sel_blk), _ptr(sel_grp), _stream(stream)))
+
+
+def hga_decode(cfg: Config, q, k, v, ctx_cap, pos, bsum, gsum, sel_blk, sel_grp, o, lse,
+               stream=None):
+    """One new token per sequence at positions pos (int64 device tensor)."""
+    c = cfg.c()
+    _check("hga_decode", load().hga_decode(
+        ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), ctx_cap, _ptr(pos), _ptr(bsum), _ptr(gsum),
+        _ptr(sel_blk), _ptr(sel_grp), _ptr(o), _ptr(lse), _stream(stream)))
 
 
 def hga_attn_fwd(cfg: Config, q, k, v, ctx_cap, q_begin, s_len, sel_grp, o, lse, stream=None):

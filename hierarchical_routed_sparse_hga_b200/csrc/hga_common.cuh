@@ -242,7 +242,7 @@ __device__ int block_enumerate_any(int n, Pred pred, Fn f, int* scratch) {
 // ---------------------------------------------------------------------------
 // block-wide top-k of n distinct-or-not uint32 keys held in shared memory:
 // sets sel[i] = 1 for the k largest keys, ties broken toward the lower index.
-// Up to 128 keys: rank counting (below).  Otherwise a radix select on 8-bit
+// Up to blockDim.x keys: rank counting (below).  Otherwise a radix select on 8-bit
 // digits (MSB first) finds the k-th largest key T; keys above T are taken,
 // and among keys equal to T the lowest indices fill the remaining slots.
 // Needs hist[256] and scratch (see block_enumerate).
@@ -255,31 +255,40 @@ __device__ void block_topk(const uint32_t* key, int n, int k, uint8_t* sel, int*
     __syncthreads();
     return;
   }
-  if (n <= 128) {
+  if (n <= nt) {
     // rank by counting: rank(i) = #{keys above key[i]} + #{equal keys before i};
     // the k smallest ranks are the k largest keys, ties to the lower index.
-    // O(n^2) comparisons with broadcast shared-memory reads (four keys per
-    // 16-byte load; `key` is 16-byte aligned), no barrier.
-    const uint4* key4 = reinterpret_cast<const uint4*>(key);
-    const int n4 = n >> 2;
-    for (int i = tid; i < n; i += nt) {
-      const uint32_t ki = key[i];
-      int rank = 0;
+    // P consecutive lanes share a key (P = the largest power of two, at most
+    // 32, with P * n <= threads), each counting over a quarter-aligned slice
+    // of the keys with broadcast 16-byte shared-memory reads (`key` is
+    // 16-byte aligned); the slices' counts are added by shuffles.  No barrier
+    // until the flags are written.
+    int P = 1;
+    while (P < 32 && 2 * P * n <= nt) P *= 2;
+    const int i = tid / P, part = tid % P;
+    const int chunk = (((n + P - 1) / P) + 3) & ~3;
+    const int j0 = part * chunk < n ? part * chunk : n;
+    const int j1 = j0 + chunk < n ? j0 + chunk : n;
+    const uint32_t ki = i < n ? key[i] : 0u;
+    int rank = 0;
+    if (i < n) {
+      const uint4* key4 = reinterpret_cast<const uint4*>(key);
+      const int q1 = j0 + ((j1 - j0) & ~3);
 #pragma unroll 4
-      for (int q = 0; q < n4; ++q) {
-        const uint4 v = key4[q];
-        const int j0 = 4 * q;
-        rank += (v.x > ki) || (v.x == ki && j0 < i);
-        rank += (v.y > ki) || (v.y == ki && j0 + 1 < i);
-        rank += (v.z > ki) || (v.z == ki && j0 + 2 < i);
-        rank += (v.w > ki) || (v.w == ki && j0 + 3 < i);
+      for (int jj = j0; jj < q1; jj += 4) {
+        const uint4 v = key4[jj >> 2];
+        rank += (v.x > ki) || (v.x == ki && jj < i);
+        rank += (v.y > ki) || (v.y == ki && jj + 1 < i);
+        rank += (v.z > ki) || (v.z == ki && jj + 2 < i);
+        rank += (v.w > ki) || (v.w == ki && jj + 3 < i);
       }
-      for (int jdx = 4 * n4; jdx < n; ++jdx) {
-        const uint32_t kj = key[jdx];
-        rank += (kj > ki) || (kj == ki && jdx < i);
+      for (int jj = q1; jj < j1; ++jj) {
+        const uint32_t kj = key[jj];
+        rank += (kj > ki) || (kj == ki && jj < i);
       }
-      sel[i] = rank < k ? 1 : 0;
     }
+    for (int o = 1; o < P; o <<= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+    if (i < n && part == 0) sel[i] = rank < k ? 1 : 0;
     __syncthreads();
     return;
   }

@@ -20,6 +20,7 @@
 #include "attn_fwd_sm100.cuh"
 #include "attn_bwd_sm100.cuh"
 #include "tier.cuh"
+#include "decode.cuh"
 #include "trace.cuh"
 
 using namespace hga;
@@ -796,7 +797,7 @@ const char* hga_kernel_name(int kind) {
       "summaries",      "route_qmean",       "route_block_score",   "route_select",
       "attn_fwd_simt",  "attn_bwd_dq_simt",  "attn_bwd_dkdv_simt",  "attn_fwd_tc",
       "attn_bwd_dq_tc", "attn_bwd_dkdv_tc",  "tier_dedup",          "tier_copy",
-      "route_fused"};
+      "route_fused",    "decode"};
   return (kind >= 0 && kind < HGA_K_COUNT) ? names[kind] : "unknown";
 }
 
@@ -853,3 +854,88 @@ void hga_timing_reset(void) {
 }
 
 }  // extern "C"
+
+namespace {
+
+template <typename T, int D, int G>
+hga_status_t launch_decode(const hga_config_t* cfg, const void* q, const void* k, const void* v,
+                           int64_t ctx_cap, const int64_t* pos, const float* bsum,
+                           const float* gsum, int32_t* sel_blk, int32_t* sel_grp, void* o,
+                           float* lse, cudaStream_t s) {
+  int dev = 0, optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return HGA_ERR_CUDA;
+  // cluster size: enough CTAs to fill the GPU about once (two per SM), more
+  // where one CTA's share of the candidate scores would not fit
+  const int64_t heads = int64_t(cfg->batch) * cfg->n_kv_heads;
+  int nc = dec::kMaxC;
+  while (nc > 1 && heads * nc > 2 * int64_t(sm_count())) nc /= 2;
+  auto plan = [&](int c, int64_t* share_cap, int* stage_units) {
+    *share_cap = (ctx_cap / kBlock + c - 1) / c;
+    const int per_cta = (kGroupsPerBlock + cfg->topk_groups + c - 1) / c;
+    const int fit = int(dec::kStageBudget / (2 * dec::unit_bytes<T, D>()));
+    *stage_units = std::max(dec::kMinStageUnits, std::min(per_cta, fit));
+    return dec::smem_bytes<T, D, G>(*share_cap, *stage_units, c);
+  };
+  int64_t share_cap = 0;
+  int stage_units = 0;
+  size_t smem = plan(nc, &share_cap, &stage_units);
+  while (smem > size_t(optin) && nc < dec::kMaxC) smem = plan(nc *= 2, &share_cap, &stage_units);
+  if (smem > size_t(optin)) return HGA_ERR_UNSUPPORTED;
+  hga_status_t e = ensure_smem(reinterpret_cast<const void*>(&dec::decode_kernel<T, D, G>), smem);
+  if (e != HGA_OK) return e;
+  const float scale_log2 = cfg->scale * 1.4426950408889634f;
+  return traced_launch(HGA_K_DECODE, s, [&] {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(unsigned(nc), cfg->n_kv_heads, cfg->batch);
+    lc.blockDim = dim3(dec::kThreads);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = unsigned(nc);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 2;
+    return cudaLaunchKernelEx(&lc, dec::decode_kernel<T, D, G>, static_cast<const T*>(q),
+        static_cast<const T*>(k), static_cast<const T*>(v), ctx_cap, pos, bsum, gsum,
+        int(cfg->n_kv_heads), int(cfg->topk_blocks), int(cfg->topk_groups), scale_log2,
+        share_cap, stage_units, sel_blk, sel_grp, static_cast<T*>(o), lse);
+  });
+}
+
+}  // namespace
+
+extern "C" hga_status_t hga_decode(const hga_config_t* cfg, const void* q, const void* k,
+                                   const void* v, int64_t ctx_cap, const int64_t* pos,
+                                   const float* bsum, const float* gsum, int32_t* sel_blk,
+                                   int32_t* sel_grp, void* o, float* lse, void* stream) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if (!q || !k || !v || !pos || !bsum || !gsum || !o || !lse) return HGA_ERR_INVALID_ARG;
+  for (const void* p : {q, k, v, static_cast<const void*>(pos), static_cast<const void*>(bsum),
+                        static_cast<const void*>(gsum), static_cast<const void*>(sel_blk),
+                        static_cast<const void*>(sel_grp), static_cast<const void*>(o),
+                        static_cast<const void*>(lse)})
+    if (p && !aligned16(p)) return HGA_ERR_INVALID_ARG;
+  if (ctx_cap <= 0 || ctx_cap % kBlock) return HGA_ERR_INVALID_ARG;
+  const int G = cfg->n_q_heads / cfg->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return HGA_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
+    switch (G) {
+      case 1: return launch_decode<T, D, 1>(cfg, q, k, v, ctx_cap, pos, bsum, gsum, sel_blk,
+                                            sel_grp, o, lse, s);
+      case 2: return launch_decode<T, D, 2>(cfg, q, k, v, ctx_cap, pos, bsum, gsum, sel_blk,
+                                            sel_grp, o, lse, s);
+      case 4: return launch_decode<T, D, 4>(cfg, q, k, v, ctx_cap, pos, bsum, gsum, sel_blk,
+                                            sel_grp, o, lse, s);
+      default: return launch_decode<T, D, 8>(cfg, q, k, v, ctx_cap, pos, bsum, gsum, sel_blk,
+                                             sel_grp, o, lse, s);
+    }
+  });
+}

@@ -162,16 +162,16 @@ __host__ __device__ inline SelectLayout select_layout(int64_t j_cap, int topk_bl
 }
 
 // Scores n rows of a summary table against q-bar (in shared memory): key[p]
-// = ordered_key(qb . rows[row_of(p)]).  A warp takes 16 rows per pass, lanes
-// across the d dimension, all 16 row loads issued before any use.
-template <int D, typename RowOf>
+// = ordered_key(qb . rows[row_of(p)]).  A warp takes kU rows per pass, lanes
+// across the d dimension, all kU row loads issued before any use.
+template <int D, typename RowOf, int kU = 16>
 __device__ __forceinline__ void score_rows(const float* __restrict__ table, const float* qb,
                                            int n, RowOf row_of, uint32_t* key) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NW = kRouteThreads / 32;
   constexpr int V4 = D / 4;  // float4 per summary row
   const float4* qb4 = reinterpret_cast<const float4*>(qb);
-  constexpr int kU = 16;
+  static_assert(kU <= 32, "one score per lane");
   constexpr int kE = (V4 + 31) / 32;  // float4 per lane per row
   for (int p0 = warp * kU; p0 < n; p0 += NW * kU) {
     float4 x[kU][kE];

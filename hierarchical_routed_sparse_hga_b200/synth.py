@@ -42,7 +42,7 @@ GROUP = 8
 QBLOCK = 64
 
 # tensor ids for the per-tensor streams
-_T_CENTROID, _T_KNOISE, _T_V, _T_TARGET, _T_QNOISE, _T_DO = range(6)
+_T_CENTROID, _T_KNOISE, _T_V, _T_TARGET, _T_QNOISE, _T_DO, _T_DEC_TARGET, _T_DEC_Q = range(8)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -218,6 +218,26 @@ def queries_head(w: Workload, b: int, hq: int, seg_begin: int) -> np.ndarray:
 def dout_head(w: Workload, b: int, hq: int, seg_begin: int) -> np.ndarray:
     rng = _rng(w, _T_DO, b, hq, seg_begin // w.seg_len)
     return to_storage(rng.standard_normal((w.seg_len, w.head_dim)), w.dtype)
+
+
+def decode_query_head(w: Workload, b: int, hq: int, pos: int) -> np.ndarray:
+    """Post-RoPE query [d] of the token at global position pos (a decode
+    step): the centroid of a planted block drawn uniformly from the complete
+    blocks before the token's own block (its own block when there are none),
+    plus 0.5 * N(0, I_d); the planted block is shared by the G heads."""
+    h = hq // w.group_heads
+    n_before = pos // BLOCK
+    r = (_rng(w, _T_DEC_TARGET, b, h, pos).integers(0, n_before) if n_before
+         else n_before)
+    noise = _rng(w, _T_DEC_Q, b, hq, pos).standard_normal(w.head_dim)
+    x = centroids(w, b, h)[r] + 0.5 * noise
+    return to_storage(_prep(x[None, :], w, pos)[0], w.dtype)
+
+
+def decode_queries(w: Workload, positions) -> np.ndarray:
+    """[B, Hq, d] decode queries, sequence b at global position positions[b]."""
+    return np.stack([np.stack([decode_query_head(w, b, hq, int(positions[b]))
+                               for hq in range(w.n_q_heads)]) for b in range(w.batch)])
 
 
 # ----------------------------------------------------------------------------

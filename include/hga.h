@@ -315,6 +315,36 @@ HGA_API hga_status_t hga_tier_append(const hga_config_t* cfg, const void* k_stag
                                      int32_t s_len, void* stream);
 
 /*
+ * Decode -- one new token per sequence [A] ("HGA can also be used for
+ * retrieval and generation"), routed and attended as in [B] with the query
+ * block reduced to that one token.  For sequence b the token sits at global
+ * position pos[b] (device array of `batch` int64; 0 <= pos[b] < ctx_cap).
+ * Per (b, KV head h), with J = pos[b] / 64 the token's own block:
+ *   qbar = mean of its query over the G heads of h;
+ *   level 1: score_c = qbar . bsum[b,h,c] for c in [0, J), keep the top
+ *            min(topk_blocks, J) (ties: lower c);
+ *   level 2: the 8 groups of each kept block, keep the top
+ *            min(topk_groups, 8*kept) (ties: lower g);
+ *   attention of each of the G heads over { 8g+i : g selected, i < 8 } U
+ *   { 64J .. pos[b] } (its own key included), scale cfg->scale.
+ * Layouts: q, o [batch, n_q_heads, head_dim] (cfg->dtype); lse
+ * [batch, n_q_heads] float32, natural log; K/V the whole-context buffers
+ * [batch, n_kv_heads, ctx_cap, head_dim] with the new token's K/V already
+ * written at row pos[b]; bsum/gsum as for hga_route, holding every complete
+ * block before the token's own block (call hga_build_summaries for a block
+ * once its 64 tokens are in K; rebuilding a range is harmless).  sel_blk
+ * [batch, n_kv_heads, topk_blocks] and sel_grp [batch, n_kv_heads,
+ * topk_groups] (int32, ascending, -1 padded) are written when not NULL.
+ * G = n_q_heads / n_kv_heads must be 1, 2, 4 or 8 (else HGA_ERR_UNSUPPORTED).
+ * A position outside [0, ctx_cap) leaves that sequence's outputs untouched and
+ * latches HGA_ERR_DEVICE_CHECK.  One launch; no workspace.
+ */
+HGA_API hga_status_t hga_decode(const hga_config_t* cfg, const void* q, const void* k,
+                                const void* v, int64_t ctx_cap, const int64_t* pos,
+                                const float* bsum, const float* gsum, int32_t* sel_blk,
+                                int32_t* sel_grp, void* o, float* lse, void* stream);
+
+/*
  * Reads and clears the calling device's latched device-side status
  * (HGA_OK, HGA_ERR_DEVICE_CHECK or HGA_ERR_TIMEOUT).  Synchronises `stream`.
  */
@@ -351,7 +381,8 @@ typedef enum {
   HGA_K_TIER_DEDUP = 10,
   HGA_K_TIER_COPY = 11,
   HGA_K_ROUTE_FUSED = 12,
-  HGA_K_COUNT = 13
+  HGA_K_DECODE = 13,
+  HGA_K_COUNT = 14
 } hga_kernel_kind_t;
 
 /* Name of a kernel kind ("attn_fwd_simt", ...). */

@@ -170,3 +170,27 @@ def compare_segment(w, gpu, q_begin, n_kv, k64, v64, backward):
         assert_close(gpu["dk"], dk, w, "dk")
         assert_close(gpu["dv"], dv, w, "dv")
     return flagged, differ
+
+
+def check_decode_selection(gpu_blk, gpu_grp, q_tok, bsum, gsum, pos, w, n_kv, what=""):
+    """check_selection for decode steps ([B, Hkv, k] selections, one token per
+    sequence at pos[b]).  Returns (flagged rows, flagged rows that differ)."""
+    sb, sg, tie = oracle.decode_route(q_tok, bsum, gsum, pos, w.topk_blocks, w.topk_groups,
+                                      n_kv)
+    gpu_blk, gpu_grp = np.asarray(gpu_blk), np.asarray(gpu_grp)
+    for name, g, r in (("sel_blk", gpu_blk, sb), ("sel_grp", gpu_grp, sg)):
+        bad = np.any(g != r, axis=-1) & ~tie
+        assert not bad.any(), f"{what}{name}: {int(bad.sum())} unflagged rows differ, " \
+                              f"first at {np.argwhere(bad)[0].tolist()}"
+    G = q_tok.shape[1] // n_kv
+    differ = 0
+    for b, h in np.argwhere(tie):
+        J = int(pos[b]) // 64
+        qbar = q_tok[b, h * G:(h + 1) * G].mean(0)
+        blocks = _valid_topk(gpu_blk[b, h], np.arange(J), bsum[b, h, :J] @ qbar,
+                             w.topk_blocks, f"{what}sel_blk{(b, h)}")
+        groups = np.array([8 * c + i for c in blocks for i in range(8)], np.int64)
+        _valid_topk(gpu_grp[b, h], groups, gsum[b, h, groups] @ qbar, w.topk_groups,
+                    f"{what}sel_grp{(b, h)}")
+        differ += int(np.any(gpu_grp[b, h] != sg[b, h]) or np.any(gpu_blk[b, h] != sb[b, h]))
+    return int(tie.sum()), differ

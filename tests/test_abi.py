@@ -162,3 +162,15 @@ def test_binding_signatures_match_the_header():
         for i, (g, w_) in enumerate(zip(got, want)):
             assert g == w_ or (w_ is ctypes.c_int and g is ctypes.c_int32), (name, i, g, w_)
         assert fn.restype == ctype_of(ret), (name, fn.restype, ret)
+
+
+def test_decode_host_argument_checks():
+    c = cfg()
+    args = (FAKE, FAKE, FAKE, 16384, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 0)
+    # G = 3 has no decode kernel; d = 96 none at all
+    assert status_of(hga.hga_decode, cfg(n_q_heads=24), *args) == 2
+    assert status_of(hga.hga_decode, cfg(head_dim=96), *args) == 2
+    # context not a multiple of 64, a missing position array, a misaligned output
+    assert status_of(hga.hga_decode, c, FAKE, FAKE, FAKE, 16380, *args[4:]) == 1
+    assert status_of(hga.hga_decode, c, FAKE, FAKE, FAKE, 16384, 0, *args[5:]) == 1
+    assert status_of(hga.hga_decode, c, *args[:9], FAKE + 8, FAKE, 0) == 1
