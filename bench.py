@@ -57,6 +57,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--no-extra", action="store_true",
+                   help="skip the 131072-token forward and the decode measurements")
     p.add_argument("--tier-sweep", action="store_true",
                    help="host-tier sweep: top-k blocks {8,16,32} x context 1K..32K, batch 8")
     args = p.parse_args()
@@ -740,6 +742,10 @@ def run_gpu(args, rank, world, local):
         e2e = {"value": round(job_throughput(tokens_per_step, args.steps, world, e_ms), 1),
                "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    extra = None
+    if world == 1 and not args.no_extra and not tiered:
+        extra = run_extras(device, max(args.steps // 2, 5), pk)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w0, budget_s=15.0)
@@ -754,6 +760,7 @@ def run_gpu(args, rank, world, local):
             "launch": {"graph": bool(args.graph), "attention": "simt" if args.simt else "auto"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(launches), "clocks": clocks, "kernels": kernels,
+            "extra": extra,
         }
         print(json.dumps(line), flush=True)
     if graph is not None:
@@ -761,6 +768,172 @@ def run_gpu(args, rank, world, local):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------
+# extra measurements on one GPU: the 131072-token forward and decode
+# ----------------------------------------------------------------------------
+
+def decode_bytes(w, positions):
+    """Algorithmic HBM bytes of one hga_decode call: per (sequence, KV head)
+    the J block summaries, the 8 k_b group summaries of the kept blocks, the
+    attended K/V rows (8 k_g routed + the own block up to the token), the G
+    query rows in and the G output rows and LSE out."""
+    d, G, el = w.head_dim, w.group_heads, (2 if w.dtype == "bf16" else 4)
+    tot = 0
+    for p in positions:
+        J = p // 64
+        kb = min(w.topk_blocks, J)
+        kg = min(w.topk_groups, 8 * kb)
+        rows = 8 * kg + (p - 64 * J + 1)
+        tot += w.n_kv_heads * (J * d * 4 + 8 * kb * d * 4 + rows * d * el * 2
+                               + 2 * G * d * el + G * 4)
+    return tot
+
+
+def run_extras(device, steps, pk):
+    """The 131072-token forward (64 segments of 2048, the long-context
+    workload) with its per-kernel table, and decode (one new token per
+    sequence, batch 8 at position 131071, four layers' caches in turn so
+    that the working set exceeds L2)."""
+    import torch
+    from hierarchical_routed_sparse_hga_b200 import (HGA_BF16, HGA_K_COUNT, Config, HgaLayer,
+                                                     hga_build_summaries, hga_kernel_name,
+                                                     hga_timing_collect, hga_timing_enable,
+                                                     hga_timing_reset, synth, timing_table)
+    out = {}
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+
+    def graph_of(fn):
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream(device)
+        cs.wait_stream(torch.cuda.current_stream(device))
+        with torch.cuda.stream(cs):
+            with torch.cuda.graph(g, stream=cs):
+                fn()
+        torch.cuda.current_stream(device).wait_stream(cs)
+        return g
+
+    # -- 131072-token forward --------------------------------------------
+    w = synth.workloads()["qwen3_fwd_128k"]
+    cfg = Config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.topk_blocks, w.topk_groups,
+                 HGA_BF16)
+    k, v, qs, _ = synth.device_inputs(w, device, backward=False)
+    layer = HgaLayer(cfg, w.ctx_len, w.seg_len, device=device, k=k, v=v)
+    segs = w.segments()
+
+    def step(record=None):
+        for i, s0 in enumerate(segs):
+            layer.segment(qs[i], s0)
+            if record is not None:
+                record.append((s0, layer.sel_grp.cpu().numpy()))
+
+    sels = []
+    step(sels)
+    step()
+    n_launch = 6 * len(segs)           # summaries, up to 3 routing kernels, forward
+    hga_timing_enable(n_launch + 16)
+    g_all = graph_of(step)
+    hga_timing_reset()
+    for _ in range(3):
+        flush.zero_()
+        g_all.replay()
+        hga_timing_collect()
+    torch.cuda.synchronize(device)
+    table = timing_table()
+    hga_timing_enable(0)
+    del g_all
+    g = graph_of(step)
+    g.replay()
+    ms = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize(device)
+        ms.append(e0.elapsed_time(e1))
+    del g
+    step_ms = statistics.mean(ms)
+    kernels = {}
+    tot = max(sum(v_[0] for v_ in table.values()), 1e-12)
+    for name, (kms, n) in table.items():
+        work, unit, bound = kernel_work(name, w, sels)
+        per_launch = work / (n / 3)
+        peak = pk["tc"] if bound == "tensor" else pk["hbm"]
+        scale = 1e12 if bound == "tensor" else 1e9
+        ach = per_launch / (kms / n / 1e3) / scale
+        kernels[name] = {"launches": n // 3, "share": round(kms / tot, 4),
+                         "avg_us": round(kms / n * 1e3, 3), "bound": bound,
+                         "achieved": round(ach, 3),
+                         "unit": "TFLOP/s" if bound == "tensor" else "GB/s",
+                         "frac": round(ach / peak, 4)}
+    route_names = [n for n in kernels if n.startswith("route")]
+    route_us = sum(table[n][0] for n in route_names) / 3 * 1e3
+    route_bytes = sum(kernel_work(n, w, sels)[0] for n in route_names)
+    out["long_context_fwd"] = {
+        "workload": w.name, "seq_len": w.ctx_len, "segments": len(segs),
+        "tokens_per_s": round(w.ctx_len / (step_ms / 1e3), 1), "ms_per_step": round(step_ms, 4),
+        "timing": "graph replay per step, CUDA events, L2 flushed between steps; kernel "
+                  "table from 3 replays with every launch bracketed",
+        "routing": {"us_per_step": round(route_us, 2),
+                    "achieved_gbs": round(route_bytes / (route_us / 1e6) / 1e9, 1),
+                    "frac_of_hbm": round(route_bytes / (route_us / 1e6) / 1e9 / pk["hbm"], 4)},
+        "kernels": kernels}
+    del layer, k, v, qs
+    torch.cuda.empty_cache()
+
+    # -- decode ------------------------------------------------------------
+    wd = synth.custom("qwen3_decode_b8_128k", batch=8, n_q_heads=32, n_kv_heads=8, head_dim=128,
+                      ctx_len=131072, seg_len=2048, topk_blocks=16, topk_groups=64,
+                      dtype="bf16", scaled=True, rope_base=1e6, seed=40)
+    n_layers = 4
+    positions = [wd.ctx_len - 1] * wd.batch
+    layers = []
+    cfg = Config(wd.batch, wd.n_q_heads, wd.n_kv_heads, wd.head_dim, wd.topk_blocks,
+                 wd.topk_groups, HGA_BF16)
+    for li in range(n_layers):
+        k, v, q_tok = synth.device_decode_inputs(dataclasses.replace(wd, seed=40 + li),
+                                                 positions, device)
+        L = HgaLayer(cfg, wd.ctx_len, wd.seg_len, device=device, k=k, v=v)
+        hga_build_summaries(cfg, L.k, wd.ctx_len, 0, wd.ctx_len, L.gsum, L.bsum)
+        layers.append((L, q_tok))
+    pos = torch.tensor(positions, dtype=torch.int64, device=device)
+    o = torch.empty((wd.batch, wd.n_q_heads, wd.head_dim), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((wd.batch, wd.n_q_heads), device=device)
+    reps = 20
+
+    def dstep():
+        for L, q_tok in layers:
+            L.decode(q_tok, pos, o, lse)
+
+    for _ in range(3):
+        dstep()
+    g = graph_of(lambda: [dstep() for _ in range(reps)])
+    g.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize(device)
+    call_us = e0.elapsed_time(e1) * 1e3 / (steps * reps * n_layers)
+    byts = decode_bytes(wd, positions)
+    ach = byts / (call_us / 1e6) / 1e9
+    out["decode"] = {
+        "workload": wd.name, "batch": wd.batch, "position": positions[0],
+        "layers_in_turn": n_layers, "us_per_layer_call": round(call_us, 3),
+        "tokens_per_s_per_layer": round(wd.batch / (call_us / 1e6), 1),
+        "timing": f"CUDA graph of {reps} x {n_layers} back-to-back calls (each layer its own "
+                  "K/V and summaries: 17 GB working set, above L2), CUDA events around the "
+                  "replays",
+        "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm"],
+                     "unit": "GB/s", "frac": round(ach / pk["hbm"], 4),
+                     "bytes_per_call": byts}}
+    del layers, g
+    torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------------------

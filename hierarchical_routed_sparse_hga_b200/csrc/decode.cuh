@@ -204,14 +204,11 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1)
                                                  sh.qb, n_loc, block_row, key1);
   __syncthreads();
   const int k_loc = kb < n_loc ? kb : n_loc;
-  block_topk(key1, n_loc, k_loc, sel1, sh.hist, sh.scratch);
-  block_enumerate_any(
-      n_loc, [&](int i) { return sel1[i] != 0; },
-      [&](int i, int r) {
-        sh.fin_key[r] = key1[i];
-        sh.fin_idx[r] = int(lo + i);
-      },
-      sh.scratch);
+  block_topk_indices(key1, n_loc, k_loc, sh.fin_idx, sel1, sh.hist, sh.scratch);
+  for (int r = tid; r < k_loc; r += kThreads) {
+    sh.fin_key[r] = key1[sh.fin_idx[r]];
+    sh.fin_idx[r] += int(lo);
+  }
   __syncthreads();
   for (int i = tid; i < nc * kb; i += kThreads) {
     const int dst = i / kb, j = i % kb;
@@ -223,10 +220,8 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1)
 
   // every CTA: the global top-k_b (ascending block index)
   const int n_m = nc * kb;
-  block_topk(sh.mkey, n_m, kb, sh.msel, sh.hist, sh.scratch);
-  block_enumerate_any(
-      n_m, [&](int i) { return sh.msel[i] != 0; }, [&](int i, int r) { sh.blocks[r] = sh.midx[i]; },
-      sh.scratch);
+  block_topk_indices(sh.mkey, n_m, kb, sh.blocks, sh.msel, sh.hist, sh.scratch);
+  for (int r = tid; r < kb; r += kThreads) sh.blocks[r] = sh.midx[sh.blocks[r]];
   __syncthreads();
   if (rank == 0 && sel_blk)
     for (int i = tid; i < topk_blocks; i += kThreads)
@@ -253,11 +248,9 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1)
     }
   cluster.sync();
   const int kg = topk_groups < n2 ? topk_groups : n2;
-  block_topk(sh.key2, n2, kg, sh.sel2, sh.hist, sh.scratch);
-  block_enumerate_any(
-      n2, [&](int pp) { return sh.sel2[pp] != 0; },
-      [&](int pp, int r) { sh.grp[r] = sh.blocks[pp >> 3] * kGroupsPerBlock + (pp & 7); },
-      sh.scratch);
+  block_topk_indices(sh.key2, n2, kg, sh.grp, sh.sel2, sh.hist, sh.scratch);
+  for (int r = tid; r < kg; r += kThreads)
+    sh.grp[r] = sh.blocks[sh.grp[r] >> 3] * kGroupsPerBlock + (sh.grp[r] & 7);
   __syncthreads();
   if (rank == 0 && sel_grp)
     for (int i = tid; i < topk_groups; i += kThreads)

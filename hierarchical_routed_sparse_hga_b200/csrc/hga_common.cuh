@@ -363,4 +363,16 @@ __device__ void block_topk(const uint32_t* key, int n, int k, uint8_t* sel, int*
   __syncthreads();
 }
 
+// block_topk followed by the ascending list of the chosen indices:
+// out[r] = the r-th smallest index among the top-k of key[0, n) (k <= n).
+// Kept out of line: a kernel that selects several times runs one copy of
+// this code, which stays in the instruction cache.
+__device__ __noinline__ void block_topk_indices(const uint32_t* key, int n, int k, int* out,
+                                                uint8_t* sel, int* hist, int* scratch) {
+  block_topk(key, n, k, sel, hist, scratch);
+  block_enumerate_any(
+      n, [&](int i) { return sel[i] != 0; }, [&](int i, int r) { out[r] = i; }, scratch);
+  __syncthreads();
+}
+
 }  // namespace hga

@@ -97,6 +97,14 @@ class HgaLayer:
                                  self.seg_len, self.bsum, self.gsum, self.sel_blk, self.sel_grp,
                                  o, lse, d_o, dq, dk, dv, self.seg_ws, stream=stream)
 
+    def decode(self, q_tok, pos, o, lse, sel_blk=None, sel_grp=None, stream=None):
+        """One new token per sequence (hga_decode): q_tok [B, Hq, d] at global
+        positions pos (int64 device tensor [B]); the token's K/V must already
+        be in self.k / self.v at pos, and every complete block before its own
+        block summarised.  Writes o [B, Hq, d] and lse [B, Hq]."""
+        _lib.hga_decode(self.cfg, q_tok, self.k, self.v, self.ctx_cap, pos, self.bsum,
+                        self.gsum, sel_blk, sel_grp, o, lse, stream)
+
     def segment(self, q, q_begin: int, d_o=None, stream=None, out=None):
         """One segment: summaries, routing, forward and (if d_o) backward
         (chained, so that the forward of each query block starts as soon as

@@ -318,3 +318,46 @@ def device_inputs(w: Workload, device, backward=True):
         if backward:
             dos.append(torch.randn((B, Hq, S, d), generator=g, device=device).to(dt))
     return k.contiguous(), v.contiguous(), qs, dos
+
+
+def device_decode_inputs(w: Workload, positions, device):
+    """K, V [B,Hkv,T,d] and the decode queries [B,Hq,d] of the tokens at
+    `positions`, drawn on `device` with the recipe above (planted block per
+    (sequence, KV head) among the complete blocks before the token's own
+    block).  Like device_inputs, for performance runs only."""
+    import torch
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed)
+    B, Hkv, Hq, T, d = w.batch, w.n_kv_heads, w.n_q_heads, w.ctx_len, w.head_dim
+    G = w.group_heads
+    scale = w.scale if w.scaled else 1.0
+
+    def rope(x, pos):
+        if w.rope_base is None:
+            return x
+        half = d // 2
+        inv = w.rope_base ** (-torch.arange(half, device=device, dtype=torch.float64) * 2.0 / d)
+        ang = pos.to(torch.float64)[..., None] * inv
+        c, s = torch.cos(ang).float(), torch.sin(ang).float()
+        x1, x2 = x[..., :half], x[..., half:]
+        return torch.cat([x1 * c - x2 * s, x2 * c + x1 * s], dim=-1)
+
+    cent = torch.randn((B, Hkv, T // BLOCK, d), generator=g, device=device)
+    k = torch.empty((B, Hkv, T, d), dtype=dt, device=device)
+    v = torch.empty((B, Hkv, T, d), dtype=dt, device=device)
+    t_idx = torch.arange(T, device=device)
+    for b in range(B):                        # one sequence at a time bounds the float32 temporaries
+        kb = cent[b].repeat_interleave(BLOCK, dim=1) + 0.5 * torch.randn(
+            (Hkv, T, d), generator=g, device=device)
+        k[b] = rope(kb * scale, t_idx[None, :].expand(Hkv, T)).to(dt)
+        v[b] = torch.randn((Hkv, T, d), generator=g, device=device).to(dt)
+    pos = torch.as_tensor(positions, device=device, dtype=torch.int64)
+    n_before = torch.clamp(pos // BLOCK, min=1)
+    r = (torch.rand((B, Hkv), generator=g, device=device) * n_before[:, None]).long()
+    r = torch.where((pos // BLOCK)[:, None] > 0, r, (pos // BLOCK)[:, None].expand(B, Hkv))
+    base = torch.gather(cent, 2, r[..., None, None].expand(B, Hkv, 1, d))[:, :, 0]
+    q = base.repeat_interleave(G, dim=1) + 0.5 * torch.randn((B, Hq, d), generator=g,
+                                                               device=device)
+    q = rope(q * scale, pos[:, None].expand(B, Hq)).to(dt)
+    return k, v, q.contiguous()
