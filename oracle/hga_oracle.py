@@ -370,3 +370,55 @@ def decode_attn(q_tok: np.ndarray, k: np.ndarray, v: np.ndarray, pos, sel_grp: n
                 o[b, hq] = (w @ vv) / w.sum()
                 lse[b, hq] = m + math.log(w.sum())
     return o, lse
+
+
+# ----------------------------------------------------------------------------
+# strictly causal routing (seventnews page, section "一个真正的警告：因果泄露":
+# because a block's routing decision uses the scores of several query
+# positions, earlier tokens can learn something about later ones; a strictly
+# causal variant is in development).  Reading C1: a query block keeps one
+# shared selection, but it is routed with the mean query of the 64 tokens
+# just before it (the previous block, global block J-1), so that every query
+# the decision uses is earlier than every token it serves.  Candidates and
+# both levels are as in route() (R3..R5).  The first block of a sequence has
+# no candidates, so it needs no earlier queries.
+# ----------------------------------------------------------------------------
+
+def query_summaries(q: np.ndarray, n_kv_heads: int) -> np.ndarray:
+    """Mean query of every 64-token block per KV head: q [B, Hq, S, d] (S a
+    multiple of 64) -> [B, Hkv, S/64, d], the mean over the block's 64 tokens
+    and the G heads of the KV head (R2)."""
+    B, Hq, S, d = q.shape
+    G = Hq // n_kv_heads
+    return q.reshape(B, n_kv_heads, G, S // QBLOCK, QBLOCK, d).mean(axis=(2, 4))
+
+
+def route_causal(q_prev_mean: np.ndarray, bsum: np.ndarray, gsum: np.ndarray, q_begin: int,
+                 n_qb: int, topk_blocks: int, topk_groups: int):
+    """Causal routing of the segment's n_qb query blocks (C1).  q_prev_mean
+    [B, Hkv, n_qb, d]: for query block j, the mean query of global block
+    q_begin/64 + j - 1 (any value where that block does not exist).  Returns
+    sel_blk, sel_grp (ascending, -1 padded) and near_tie, as route()."""
+    B, H, _, d = q_prev_mean.shape
+    sel_blk = np.full((B, H, n_qb, topk_blocks), -1, np.int32)
+    sel_grp = np.full((B, H, n_qb, topk_groups), -1, np.int32)
+    near_tie = np.zeros((B, H, n_qb), bool)
+    inv_sqrt_d = 1.0 / math.sqrt(d)
+    for b in range(B):
+        for h in range(H):
+            for j in range(n_qb):
+                own = q_begin // BLOCK + j
+                qbar = q_prev_mean[b, h, j]
+                s1 = (bsum[b, h, :own, :] @ qbar) * inv_sqrt_d
+                kb = min(topk_blocks, own)
+                blocks, s1_sorted = _topk_lower_index(s1, np.arange(own), kb)
+                blocks = np.sort(blocks)
+                groups = (blocks[:, None] * GROUPS_PER_BLOCK
+                          + np.arange(GROUPS_PER_BLOCK)[None, :]).reshape(-1)
+                s2 = (gsum[b, h, groups, :] @ qbar) * inv_sqrt_d
+                kg = min(topk_groups, len(groups))
+                chosen, s2_sorted = _topk_lower_index(s2, groups, kg)
+                sel_blk[b, h, j, :kb] = blocks
+                sel_grp[b, h, j, :kg] = np.sort(chosen)
+                near_tie[b, h, j] = _near_tie(s1_sorted, kb) or _near_tie(s2_sorted, kg)
+    return sel_blk, sel_grp, near_tie

@@ -691,3 +691,139 @@ def test_decode_pins_catch_planted_mistakes(monkeypatch, target, mutant):
         except (AssertionError, IndexError, ValueError):
             failed += 1
     assert failed >= 1, f"no pin caught the planted mistake in {target}"
+
+
+# ----------------------------------------------------------------------------
+# pins: strictly causal routing (the query block routed with the mean query
+# of the 64 tokens before it)
+# ----------------------------------------------------------------------------
+
+def causal_case(seed=21, B=2, hq=4, hkv=2, d=16, n_blocks=8, kb=2, kg=5):
+    rng = np.random.default_rng(seed)
+    T = 64 * n_blocks
+    cent = rng.standard_normal((B, hkv, n_blocks, d))
+    k = np.repeat(cent, 64, axis=2) + 0.5 * rng.standard_normal((B, hkv, T, d))
+    q_all = rng.standard_normal((B, hq, T, d))
+    return k, q_all, kb, kg, hkv
+
+
+def causal_selection(k, q_all, q_begin, S, kb, kg, hkv):
+    g, bl = summaries_upto(k, k.shape[2])
+    qs = oracle.query_summaries(q_all, hkv)                 # [B, Hkv, T/64, d]
+    J0 = q_begin // 64
+    prev = np.zeros((qs.shape[0], hkv, S // 64, qs.shape[-1]))
+    for j in range(S // 64):
+        if J0 + j >= 1:
+            prev[:, :, j] = qs[:, :, J0 + j - 1]
+    return oracle.route_causal(prev, bl, g, q_begin, S // 64, kb, kg)
+
+
+def check_query_summaries():
+    k, q_all, kb, kg, hkv = causal_case()
+    qs = oracle.query_summaries(q_all, hkv)
+    B, Hq, T, d = q_all.shape
+    G = Hq // hkv
+    for b in range(B):
+        for h in range(hkv):
+            for J in range(T // 64):
+                rows = [q_all[b, hh, t] for hh in range(h * G, (h + 1) * G)
+                        for t in range(64 * J, 64 * J + 64)]
+                assert close(qs[b, h, J], sum(rows) / len(rows))
+
+
+def test_query_summaries():
+    check_query_summaries()
+
+
+def check_causal_route_uses_no_later_token():
+    """Changing the queries of block J or of any later token leaves the
+    selections of blocks <= J as they were; changing block J-1's queries
+    changes some selection (the routing does depend on them)."""
+    k, q_all, kb, kg, hkv = causal_case()
+    q_begin, S = 128, 384
+    base = causal_selection(k, q_all, q_begin, S, kb, kg, hkv)
+    rng = np.random.default_rng(5)
+    for J in (3, 5):
+        q2 = q_all.copy()
+        q2[:, :, 64 * J:] = rng.standard_normal(q2[:, :, 64 * J:].shape) * 3
+        sb, sg, _ = causal_selection(k, q2, q_begin, S, kb, kg, hkv)
+        upto = J - q_begin // 64 + 1                        # query blocks J0 .. J
+        assert np.array_equal(sb[:, :, :upto], base[0][:, :, :upto])
+        assert np.array_equal(sg[:, :, :upto], base[1][:, :, :upto])
+    changed = 0
+    for J in range(3, 8):
+        q2 = q_all.copy()
+        q2[:, :, 64 * (J - 1):64 * J] = -q2[:, :, 64 * (J - 1):64 * J]
+        sb, sg, _ = causal_selection(k, q2, q_begin, S, kb, kg, hkv)
+        changed += int(not np.array_equal(sg, base[1]))
+    assert changed >= 3
+
+
+def test_causal_route_uses_no_later_token():
+    check_causal_route_uses_no_later_token()
+
+
+def check_causal_route_bruteforce():
+    """Literal definition: the score of block c for query block J is the mean
+    over the previous block's 64 tokens, the G heads and c's 64 keys of
+    q.k/sqrt(d); exhaustive sort by (-score, index)."""
+    k, q_all, kb, kg, hkv = causal_case(seed=22, d=8, n_blocks=6)
+    B, Hq, T, d = q_all.shape
+    G = Hq // hkv
+    q_begin, S = 64, 320
+    sb, sg, tie = causal_selection(k, q_all, q_begin, S, kb, kg, hkv)
+    for b in range(B):
+        for h in range(hkv):
+            for j in range(S // 64):
+                J = q_begin // 64 + j
+                if tie[b, h, j]:
+                    continue
+                qs = [q_all[b, hh, t] for hh in range(h * G, (h + 1) * G)
+                      for t in range(64 * (J - 1), 64 * J)]
+
+                def score(keys):
+                    return sum(float(qq @ k[b, h, t]) for qq in qs for t in keys) / (
+                        len(qs) * len(keys) * math.sqrt(d))
+                blocks = sorted(range(J), key=lambda c: (-score(range(64 * c, 64 * c + 64)), c))
+                blocks = sorted(blocks[:kb])
+                groups = [8 * c + i for c in blocks for i in range(8)]
+                groups = sorted(groups, key=lambda gg: (-score(range(8 * gg, 8 * gg + 8)), gg))
+                groups = sorted(groups[:kg])
+                assert [x for x in sb[b, h, j] if x >= 0] == blocks
+                assert [x for x in sg[b, h, j] if x >= 0] == groups
+
+
+def test_causal_route_bruteforce():
+    check_causal_route_bruteforce()
+
+
+def _mut_query_summaries_wrong_group(q, hkv):
+    return ORIG_CAUSAL["query_summaries"](np.roll(q, -(q.shape[1] // hkv), axis=1), hkv)
+
+
+def _mut_route_causal_own_block(q_prev_mean, bsum, gsum, q_begin, n_qb, kb, kg):
+    # routes block j with block j's own mean (shifted one block too late):
+    # emulated by moving every row one block back, the last from the next
+    shifted = np.concatenate([q_prev_mean[:, :, 1:], q_prev_mean[:, :, -1:]], axis=2)
+    return ORIG_CAUSAL["route_causal"](shifted, bsum, gsum, q_begin, n_qb, kb, kg)
+
+
+ORIG_CAUSAL = {"query_summaries": ho.query_summaries, "route_causal": ho.route_causal}
+CAUSAL_PINS = [check_query_summaries, check_causal_route_uses_no_later_token,
+               check_causal_route_bruteforce]
+
+
+@pytest.mark.parametrize("target,mutant", [
+    ("query_summaries", _mut_query_summaries_wrong_group),
+    ("route_causal", _mut_route_causal_own_block),
+])
+def test_causal_pins_catch_planted_mistakes(monkeypatch, target, mutant):
+    monkeypatch.setattr(ho, target, mutant)
+    monkeypatch.setattr(oracle, target, mutant)
+    failed = 0
+    for pin in CAUSAL_PINS:
+        try:
+            pin()
+        except (AssertionError, IndexError, ValueError):
+            failed += 1
+    assert failed >= 1, f"no pin caught the planted mistake in {target}"
