@@ -31,9 +31,10 @@ EXPORTS = ("hga_version", "hga_status_string", "hga_build_summaries",
            "hga_timing_get", "hga_timing_reset", "hga_timing_kinds", "hga_route_noalloc",
            "hga_build_summaries_seg",
            "hga_tier_stage_rows", "hga_tier_workspace_size", "hga_tier_gather",
-           "hga_tier_append", "hga_decode")
+           "hga_tier_append", "hga_decode", "hga_build_query_summaries",
+           "hga_route_causal")
 HGA_NOALLOC_SCRATCH_BYTES = 4 << 20
-HGA_K_COUNT = 14
+HGA_K_COUNT = 15
 
 
 class HgaError(RuntimeError):
@@ -115,6 +116,8 @@ def load() -> ctypes.CDLL:
                                            P]),
         "hga_tier_append": (ctypes.c_int, [CFG, P, P, I64, P, P, I64, I64, I32, P]),
         "hga_decode": (ctypes.c_int, [CFG, P, P, P, I64, P, P, P, P, P, P, P, P]),
+        "hga_build_query_summaries": (ctypes.c_int, [CFG, P, I64, I32, I64, P, P]),
+        "hga_route_causal": (ctypes.c_int, [CFG, P, I64, I32, I64, P, P, P, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -229,6 +232,21 @@ def hga_route(cfg: Config, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_
     ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
     _check("hga_route", load().hga_route(
         ctypes.byref(c), _ptr(q), q_begin, s_len, ctx_cap, _ptr(bsum), _ptr(gsum),
+        _ptr(sel_blk), _ptr(sel_grp), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def hga_build_query_summaries(cfg: Config, q, q_begin, s_len, ctx_cap, qsum, stream=None):
+    c = cfg.c()
+    _check("hga_build_query_summaries", load().hga_build_query_summaries(
+        ctypes.byref(c), _ptr(q), q_begin, s_len, ctx_cap, _ptr(qsum), _stream(stream)))
+
+
+def hga_route_causal(cfg: Config, q, q_begin, s_len, ctx_cap, bsum, gsum, qsum, sel_blk, sel_grp,
+                     workspace, ws_bytes=None, stream=None):
+    c = cfg.c()
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check("hga_route_causal", load().hga_route_causal(
+        ctypes.byref(c), _ptr(q), q_begin, s_len, ctx_cap, _ptr(bsum), _ptr(gsum), _ptr(qsum),
         _ptr(sel_blk), _ptr(sel_grp), _ptr(workspace), ws_bytes, _stream(stream)))
 
 

@@ -360,7 +360,7 @@ static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q
                                int32_t s_len, int64_t ctx_cap, const float* bsum,
                                const float* gsum, int32_t* sel_blk, int32_t* sel_grp,
                                void* workspace, size_t ws_bytes, int* done, uint32_t token,
-                               cudaStream_t s) {
+                               cudaStream_t s, const float* qprev = nullptr) {
   hga_status_t st = check_cfg(cfg);
   if (st != HGA_OK) return st;
   if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
@@ -385,22 +385,25 @@ static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q
         return launch_pdl(route_fused_kernel<T, D>, g1, dim3(kRouteThreads), smf, s,
                           static_cast<const T*>(q), bsum, gsum, ctx_cap, cfg->n_q_heads,
                           cfg->n_kv_heads, s_len, own0, cfg->topk_blocks, cfg->topk_groups,
-                          sel_blk, sel_grp, done, token);
+                          sel_blk, sel_grp, done, token, qprev);
       });
     }
-    dim3 g0(n_qb * G, cfg->n_kv_heads, cfg->batch);
-    hga_status_t e = traced_launch(HGA_K_QMEAN, s, [&] {
-      return launch_pdl(qmean_kernel<T, D>, g0, dim3(kQmeanThreads), 0, s, static_cast<const T*>(q),
-          cfg->n_q_heads, cfg->n_kv_heads, s_len, ws.qbar);
-    });
-    if (e != HGA_OK) return e;
+    hga_status_t e = HGA_OK;
+    if (!qprev) {
+      dim3 g0(n_qb * G, cfg->n_kv_heads, cfg->batch);
+      e = traced_launch(HGA_K_QMEAN, s, [&] {
+        return launch_pdl(qmean_kernel<T, D>, g0, dim3(kQmeanThreads), 0, s,
+            static_cast<const T*>(q), cfg->n_q_heads, cfg->n_kv_heads, s_len, ws.qbar);
+      });
+      if (e != HGA_OK) return e;
+    }
     if (j_max > 0) {
       const int n_cc = int((j_max + kScoreCands - 1) / kScoreCands);
       const int n_jc = (n_qb + kScoreQbs - 1) / kScoreQbs;
       dim3 g2(unsigned(n_cc * n_jc), cfg->n_kv_heads, cfg->batch);
       e = traced_launch(HGA_K_BLOCK_SCORE, s, [&] {
-        return launch_pdl(block_score_kernel<D>, g2, dim3(kRouteThreads), 0, s, ws.qbar, bsum,
-            ctx_cap, cfg->n_kv_heads, G, n_qb, own0, ws.scores, ws.jstride);
+        return launch_pdl(block_score_kernel<D>, g2, dim3(kRouteThreads), 0, s, ws.qbar, qprev,
+            bsum, ctx_cap, cfg->n_kv_heads, G, n_qb, own0, ws.scores, ws.jstride);
       });
       if (e != HGA_OK) return e;
     }
@@ -409,7 +412,8 @@ static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q
     e = ensure_smem(reinterpret_cast<const void*>(&select_kernel<D>), sm3);
     if (e != HGA_OK) return e;
     return traced_launch(HGA_K_SELECT, s, [&] {
-      return launch_pdl(select_kernel<D>, g1, dim3(kRouteThreads), sm3, s, ws.qbar, ws.scores, gsum,
+      return launch_pdl(select_kernel<D>, g1, dim3(kRouteThreads), sm3, s, ws.qbar, qprev,
+          ws.scores, gsum,
           ctx_cap, cfg->n_kv_heads, G, n_qb, own0, ws.jstride, cfg->topk_blocks, cfg->topk_groups,
           sel_blk, sel_grp);
     });
@@ -797,7 +801,7 @@ const char* hga_kernel_name(int kind) {
       "summaries",      "route_qmean",       "route_block_score",   "route_select",
       "attn_fwd_simt",  "attn_bwd_dq_simt",  "attn_bwd_dkdv_simt",  "attn_fwd_tc",
       "attn_bwd_dq_tc", "attn_bwd_dkdv_tc",  "tier_dedup",          "tier_copy",
-      "route_fused",    "decode"};
+      "route_fused",    "decode",            "query_summaries"};
   return (kind >= 0 && kind < HGA_K_COUNT) ? names[kind] : "unknown";
 }
 
@@ -938,4 +942,43 @@ extern "C" hga_status_t hga_decode(const hga_config_t* cfg, const void* q, const
                                              sel_grp, o, lse, s);
     }
   });
+}
+
+static hga_status_t launch_qsum(const hga_config_t* cfg, const void* q, int64_t q_begin,
+                                int32_t s_len, int64_t ctx_cap, float* qsum, cudaStream_t s) {
+  return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
+    dim3 grid(s_len / kQBlock, cfg->n_kv_heads, cfg->batch);
+    return traced_launch(HGA_K_QSUM, s, [&] {
+      return launch_pdl(qsum_kernel<T, D>, grid, dim3(kRouteThreads), 0, s,
+                        static_cast<const T*>(q), ctx_cap, cfg->n_q_heads, cfg->n_kv_heads, s_len,
+                        q_begin / kBlock, qsum);
+    });
+  });
+}
+
+extern "C" hga_status_t hga_build_query_summaries(const hga_config_t* cfg, const void* q,
+                                                  int64_t q_begin, int32_t s_len, int64_t ctx_cap,
+                                                  float* qsum, void* stream) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
+  if (!q || !qsum || !aligned16(q) || !aligned16(qsum)) return HGA_ERR_INVALID_ARG;
+  return launch_qsum(cfg, q, q_begin, s_len, ctx_cap, qsum, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" hga_status_t hga_route_causal(const hga_config_t* cfg, const void* q, int64_t q_begin,
+                                         int32_t s_len, int64_t ctx_cap, const float* bsum,
+                                         const float* gsum, float* qsum, int32_t* sel_blk,
+                                         int32_t* sel_grp, void* workspace, size_t ws_bytes,
+                                         void* stream) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
+  if (!qsum || !aligned16(qsum)) return HGA_ERR_INVALID_ARG;
+  if (!q || !bsum || !gsum || !sel_grp || !workspace) return HGA_ERR_INVALID_ARG;
+  if (ws_bytes < route_carve(cfg, s_len, q_begin, nullptr).bytes) return HGA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = launch_qsum(cfg, q, q_begin, s_len, ctx_cap, qsum, s)) != HGA_OK) return st;
+  return route_impl(cfg, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp, workspace,
+                    ws_bytes, nullptr, 0, s, qsum);
 }

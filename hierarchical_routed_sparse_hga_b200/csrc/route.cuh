@@ -82,6 +82,20 @@ __device__ __forceinline__ float qbar_elem(const float* qpart_bhj, int G, int D,
   return v;
 }
 
+// q-bar of query block j (global block own0 + j) as the routing uses it:
+// normally the sum of its G shares; in causal mode (qprev != nullptr) the
+// resident mean query of the block before it, qprev[head, own0 + j - 1, :]
+// (zero for the first block of a sequence, which has no candidates).
+__device__ __forceinline__ float route_qbar(const float* qpart, const float* qprev, int64_t head,
+                                            int n_qb, int G, int D, int j, int e, int64_t own0,
+                                            int64_t ctx_blocks) {
+  if (qprev) {
+    const int64_t J = own0 + j;
+    return J > 0 ? qprev[(head * ctx_blocks + J - 1) * D + e] : 0.f;
+  }
+  return qbar_elem(qpart + ((head * n_qb + j) * G) * D, G, D, e);
+}
+
 // grid (ceil(j_max / 32) * ceil(n_qb / 8), Hkv, B), 256 threads: a tile of
 // 32 candidate blocks x 8 query blocks, one score per thread, operands
 // staged in shared memory (candidates transposed and padded: conflict-free).
@@ -90,9 +104,9 @@ constexpr int kScoreQbs = 8;
 
 template <int D>
 __global__ void __launch_bounds__(kRouteThreads)
-    block_score_kernel(const float* __restrict__ qpart, const float* __restrict__ bsum,
-                       int64_t ctx_cap, int n_kv_heads, int G, int n_qb, int64_t own0,
-                       float* __restrict__ scores, int64_t jstride) {
+    block_score_kernel(const float* __restrict__ qpart, const float* __restrict__ qprev,
+                       const float* __restrict__ bsum, int64_t ctx_cap, int n_kv_heads, int G,
+                       int n_qb, int64_t own0, float* __restrict__ scores, int64_t jstride) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ float qb[kScoreQbs][D];
@@ -111,7 +125,8 @@ __global__ void __launch_bounds__(kRouteThreads)
 #pragma unroll
   for (int u = 0; u < kQ; ++u) {
     const int i = threadIdx.x + u * kRouteThreads, jl = i / D, e = i % D, j = j0 + jl;
-    qv[u] = j < n_qb ? qbar_elem(qpart + ((head * n_qb + j) * G) * D, G, D, e) : 0.f;
+    qv[u] = j < n_qb ? route_qbar(qpart, qprev, head, n_qb, G, D, j, e, own0, ctx_cap / kBlock)
+                     : 0.f;
   }
 #pragma unroll
   for (int u = 0; u < kB; ++u) {
@@ -264,7 +279,8 @@ __device__ __forceinline__ void select_levels(const SelectLayout& L, unsigned ch
 // grid (n_qb, Hkv, B); dynamic smem select_layout(...).total
 template <int D>
 __global__ void __launch_bounds__(kRouteThreads)
-    select_kernel(const float* __restrict__ qpart, const float* __restrict__ scores,
+    select_kernel(const float* __restrict__ qpart, const float* __restrict__ qprev,
+                  const float* __restrict__ scores,
                   const float* __restrict__ gsum, int64_t ctx_cap, int n_kv_heads, int G, int n_qb,
                   int64_t own0, int64_t jstride, int topk_blocks, int topk_groups,
                   int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp) {
@@ -281,7 +297,7 @@ __global__ void __launch_bounds__(kRouteThreads)
   const float* srow = scores + (head * n_qb + j) * jstride;
   for (int64_t i = threadIdx.x; i < J; i += kRouteThreads) key1[i] = ordered_key(srow[i]);
   for (int i = threadIdx.x; i < D; i += kRouteThreads)
-    qb[i] = qbar_elem(qpart + ((head * n_qb + j) * G) * D, G, D, i);
+    qb[i] = route_qbar(qpart, qprev, head, n_qb, G, D, j, i, own0, ctx_cap / kBlock);
   __syncthreads();
   select_levels<D>(L, sm_raw, gsum, head, ctx_cap, n_qb, j, J, topk_blocks, topk_groups, sel_blk,
                    sel_grp);
@@ -303,31 +319,15 @@ __host__ __device__ inline size_t fused_route_smem(int64_t j_cap, int topk_block
   return select_layout(j_cap, topk_blocks, D).total + size_t(fused_route_rows<D>()) * D * 4;
 }
 
-// grid (n_qb, Hkv, B)
+// Mean of the G x 64 query rows of query block j of KV head h (rows of the
+// segment's Q [B, Hq, S, d]): thread (row slot rs, 8-column chunk ch) sums
+// rows rs, rs + RS, ... (several rows' loads in flight), the RS partial rows
+// are then added in order; out[e] = mean (shared or global memory).  All
+// kRouteThreads threads; `part` is RS x D floats of shared memory.
 template <typename T, int D>
-__global__ void __launch_bounds__(kRouteThreads)
-    route_fused_kernel(const T* __restrict__ q, const float* __restrict__ bsum,
-                       const float* __restrict__ gsum, int64_t ctx_cap, int n_q_heads,
-                       int n_kv_heads, int s_len, int64_t own0, int topk_blocks, int topk_groups,
-                       int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp,
-                       int* __restrict__ done, uint32_t token) {
-  // q-bar needs only the queries, which the kernels before this one do not
-  // write: it is formed while the kernel before still runs; the summaries
-  // are read only after it has completed (the wait below).  A chained
-  // forward waits for each item's flag, so it may be scheduled at once.
-  pdl_launch_dependents();
-  extern __shared__ __align__(16) unsigned char sm_raw[];
-  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int G = n_q_heads / n_kv_heads, n_qb = s_len / kQBlock;
-  const int64_t head = int64_t(b) * n_kv_heads + h;
-  const int64_t J = own0 + j;                 // candidate blocks [0, J)
-  const SelectLayout L = select_layout(own0 + n_qb, topk_blocks, D);
-  float* qb = reinterpret_cast<float*>(sm_raw + L.qb);
-  uint32_t* key1 = reinterpret_cast<uint32_t*>(sm_raw + L.key1);
-  float* part = reinterpret_cast<float*>(sm_raw + L.total);
-
-  // q-bar: thread (row slot rs, 8-column chunk ch) sums rows rs, rs + RS, ...
-  // of the G x 64 query rows; the RS partial rows are then added in order
+__device__ __forceinline__ void block_query_mean(const T* __restrict__ q, int b, int h, int j,
+                                                 int n_q_heads, int G, int s_len, float* part,
+                                                 float* out) {
   constexpr int CH = D / 8, RS = fused_route_rows<D>();
   const int ch = threadIdx.x % CH, rs = threadIdx.x / CH;
   const int rows = G * kQBlock;
@@ -350,10 +350,55 @@ __global__ void __launch_bounds__(kRouteThreads)
   for (int e = threadIdx.x; e < D; e += kRouteThreads) {
     float sum = 0.f;
     for (int r = 0; r < RS; ++r) sum += part[r * D + e];
-    qb[e] = sum * inv;
+    out[e] = sum * inv;
   }
+}
+
+// Resident mean query of every block of the segment (for causal routing):
+// qsum[b, h, q_begin/64 + j, :] = mean of the G x 64 query rows of query
+// block j.  grid (n_qb, Hkv, B), kRouteThreads threads.
+template <typename T, int D>
+__global__ void __launch_bounds__(kRouteThreads)
+    qsum_kernel(const T* __restrict__ q, int64_t ctx_cap, int n_q_heads, int n_kv_heads,
+                int s_len, int64_t own0, float* __restrict__ qsum) {
+  pdl_launch_dependents();
+  pdl_wait();
+  __shared__ float part[fused_route_rows<D>() * D];
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int64_t head = int64_t(b) * n_kv_heads + h;
+  block_query_mean<T, D>(q, b, h, j, n_q_heads, n_q_heads / n_kv_heads, s_len, part,
+                         qsum + (head * (ctx_cap / kBlock) + own0 + j) * D);
+}
+
+// grid (n_qb, Hkv, B)
+template <typename T, int D>
+__global__ void __launch_bounds__(kRouteThreads)
+    route_fused_kernel(const T* __restrict__ q, const float* __restrict__ bsum,
+                       const float* __restrict__ gsum, int64_t ctx_cap, int n_q_heads,
+                       int n_kv_heads, int s_len, int64_t own0, int topk_blocks, int topk_groups,
+                       int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp,
+                       int* __restrict__ done, uint32_t token, const float* __restrict__ qprev) {
+  // q-bar needs only the queries, which the kernels before this one do not
+  // write: it is formed while the kernel before still runs; the summaries
+  // are read only after it has completed (the wait below).  A chained
+  // forward waits for each item's flag, so it may be scheduled at once.
+  pdl_launch_dependents();
+  extern __shared__ __align__(16) unsigned char sm_raw[];
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int G = n_q_heads / n_kv_heads, n_qb = s_len / kQBlock;
+  const int64_t head = int64_t(b) * n_kv_heads + h;
+  const int64_t J = own0 + j;                 // candidate blocks [0, J)
+  const SelectLayout L = select_layout(own0 + n_qb, topk_blocks, D);
+  float* qb = reinterpret_cast<float*>(sm_raw + L.qb);
+  uint32_t* key1 = reinterpret_cast<uint32_t*>(sm_raw + L.key1);
+  float* part = reinterpret_cast<float*>(sm_raw + L.total);
+
+  if (!qprev) block_query_mean<T, D>(q, b, h, j, n_q_heads, G, s_len, part, qb);
   // from here on everything before this kernel has completed
   pdl_wait();
+  if (qprev)
+    for (int e = threadIdx.x; e < D; e += kRouteThreads)
+      qb[e] = J > 0 ? qprev[(head * (ctx_cap / kBlock) + J - 1) * D + e] : 0.f;
   __syncthreads();
   // level-1 scores of the J candidate blocks
   score_rows<D>(bsum + head * (ctx_cap / kBlock) * D, qb, int(J),

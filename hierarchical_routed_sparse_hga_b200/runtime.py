@@ -39,6 +39,9 @@ class HgaLayer:
                                 device=self.device)
         self.bsum = torch.zeros((B, Hkv, ctx_cap // 64, d), dtype=torch.float32,
                                 device=self.device)
+        # resident mean query of every block, for causal routing
+        self.qsum = torch.zeros((B, Hkv, ctx_cap // 64, d), dtype=torch.float32,
+                                device=self.device)
         ws = max(_lib.hga_route_workspace_size(cfg, seg_len, ctx_cap - seg_len), 256)
         self.route_ws = torch.empty(ws, dtype=torch.uint8, device=self.device)
         # zeroed once: hga_attn_fwd_bwd's completion flags live in it
@@ -66,6 +69,15 @@ class HgaLayer:
     def route(self, q, q_begin: int, stream=None):
         _lib.hga_route(self.cfg, q, q_begin, self.seg_len, self.ctx_cap, self.bsum,
                        self.gsum, self.sel_blk, self.sel_grp, self.route_ws, stream=stream)
+
+    def build_query_summaries(self, q, q_begin: int, stream=None):
+        _lib.hga_build_query_summaries(self.cfg, q, q_begin, self.seg_len, self.ctx_cap,
+                                       self.qsum, stream)
+
+    def route_causal(self, q, q_begin: int, stream=None):
+        _lib.hga_route_causal(self.cfg, q, q_begin, self.seg_len, self.ctx_cap, self.bsum,
+                              self.gsum, self.qsum, self.sel_blk, self.sel_grp, self.route_ws,
+                              stream=stream)
 
     def make_outputs(self):
         """A fresh set of per-segment outputs (o, lse, dq, dk, dv), for callers
@@ -105,14 +117,22 @@ class HgaLayer:
         _lib.hga_decode(self.cfg, q_tok, self.k, self.v, self.ctx_cap, pos, self.bsum,
                         self.gsum, sel_blk, sel_grp, o, lse, stream)
 
-    def segment(self, q, q_begin: int, d_o=None, stream=None, out=None):
+    def segment(self, q, q_begin: int, d_o=None, stream=None, out=None, causal=False):
         """One segment: summaries, routing, forward and (if d_o) backward
         (chained, so that the forward of each query block starts as soon as
         its selection is written and its backward as soon as its forward is
         done).  Results go to `out` (from make_outputs) if given, else to the
-        layer's own o, lse, dq, dk, dv."""
+        layer's own o, lse, dq, dk, dv.  causal=True routes each query block
+        with the previous block's mean query (hga_route_causal; segments in
+        order), then runs the forward and backward chained."""
         self.summarize(q_begin, stream)
-        if d_o is None:
+        if causal:
+            self.route_causal(q, q_begin, stream)
+            if d_o is None:
+                self.forward(q, q_begin, stream, out)
+            else:
+                self.forward_backward(q, d_o, q_begin, stream, out)
+        elif d_o is None:
             self.route(q, q_begin, stream)
             self.forward(q, q_begin, stream, out)
         else:

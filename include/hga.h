@@ -315,6 +315,35 @@ HGA_API hga_status_t hga_tier_append(const hga_config_t* cfg, const void* k_stag
                                      int32_t s_len, void* stream);
 
 /*
+ * Strictly causal routing.  The seventnews page, section "一个真正的警告：
+ * 因果泄露" (causal leakage): a block's routing decision uses the scores of
+ * several query positions, so earlier tokens can learn something about later
+ * ones; a strictly causal variant is in development.  Here a query block keeps
+ * one shared selection but is routed with the mean query of the 64 tokens
+ * before it, so every query the decision uses is earlier than every token it
+ * serves.  Candidates and both levels are those of hga_route.
+ *
+ * qsum [batch, n_kv_heads, ctx_cap/64, head_dim] float32 holds the resident
+ * mean query of every block (mean over its 64 tokens and the G heads of the KV
+ * head), like bsum holds the mean key.  hga_build_query_summaries writes the
+ * rows of the segment's blocks q_begin/64 .. (q_begin+s_len)/64 - 1 from its
+ * Q.  hga_route_causal writes those rows too, then routes query block j
+ * (global block J = q_begin/64 + j) with row J - 1: for j = 0 that row comes
+ * from the previous segment, so route the segments of a sequence in order (or
+ * build the row of block q_begin/64 - 1 first).  The first block of a
+ * sequence has no candidates and reads no row.  Writes sel_grp and, if not
+ * NULL, sel_blk, as hga_route; workspace as hga_route_workspace_size().
+ */
+HGA_API hga_status_t hga_build_query_summaries(const hga_config_t* cfg, const void* q,
+                                               int64_t q_begin, int32_t s_len, int64_t ctx_cap,
+                                               float* qsum, void* stream);
+HGA_API hga_status_t hga_route_causal(const hga_config_t* cfg, const void* q, int64_t q_begin,
+                                      int32_t s_len, int64_t ctx_cap, const float* bsum,
+                                      const float* gsum, float* qsum, int32_t* sel_blk,
+                                      int32_t* sel_grp, void* workspace, size_t ws_bytes,
+                                      void* stream);
+
+/*
  * Decode -- one new token per sequence [A] ("HGA can also be used for
  * retrieval and generation"), routed and attended as in [B] with the query
  * block reduced to that one token.  For sequence b the token sits at global
@@ -382,7 +411,8 @@ typedef enum {
   HGA_K_TIER_COPY = 11,
   HGA_K_ROUTE_FUSED = 12,
   HGA_K_DECODE = 13,
-  HGA_K_COUNT = 14
+  HGA_K_QSUM = 14,
+  HGA_K_COUNT = 15
 } hga_kernel_kind_t;
 
 /* Name of a kernel kind ("attn_fwd_simt", ...). */

@@ -109,10 +109,11 @@ class Segmenter:
     """Runs a workload segment by segment on the GPU (HgaLayer) and, for the
     segments asked for, on the oracle with the same inputs."""
 
-    def __init__(self, w, kv_heads=None, flags=0):
+    def __init__(self, w, kv_heads=None, flags=0, causal=False):
         import torch
         from hierarchical_routed_sparse_hga_b200 import HgaLayer
         self.w = w
+        self.causal = causal
         self.heads = list(range(w.n_kv_heads)) if kv_heads is None else list(kv_heads)
         G = w.group_heads
         self.q_heads = [h * G + g for h in self.heads for g in range(G)]
@@ -127,6 +128,11 @@ class Segmenter:
             from hierarchical_routed_sparse_hga_b200 import hga_build_summaries
             hga_build_summaries(self.layer.cfg, self.layer.k, w.ctx_len, 0, first,
                                 self.layer.gsum, self.layer.bsum)
+            if causal:
+                # the mean query of the block just before the first segment
+                # (the earlier segment's queries)
+                prev = first - w.seg_len
+                self.layer.build_query_summaries(to_device(synth.queries(w, prev), w), prev)
         torch.cuda.synchronize()
 
     def run_segment(self, q_begin, backward=None):
@@ -136,14 +142,15 @@ class Segmenter:
         q_np = synth.queries(w, q_begin)
         q = to_device(q_np, w)
         d_o = to_device(synth.douts(w, q_begin), w) if backward else None
-        self.layer.segment(q, q_begin, d_o)
+        self.layer.segment(q, q_begin, d_o, causal=self.causal)
         torch.cuda.synchronize()
         L = self.layer
         hs, qs = self.heads, self.q_heads
         out = dict(q64=synth.widen(q_np[:, qs], w.dtype),
                    sel_blk=L.sel_blk[:, hs].cpu().numpy(), sel_grp=L.sel_grp[:, hs].cpu().numpy(),
                    o=to_f64(L.o[:, qs]), lse=to_f64(L.lse[:, qs]),
-                   gsum=to_f64(L.gsum[:, hs]), bsum=to_f64(L.bsum[:, hs]))
+                   gsum=to_f64(L.gsum[:, hs]), bsum=to_f64(L.bsum[:, hs]),
+                   qsum=to_f64(L.qsum[:, hs]))
         if backward:
             out.update(do64=synth.widen(synth.douts(w, q_begin)[:, qs], w.dtype),
                        dq=to_f64(L.dq[:, qs]), dk=to_f64(L.dk[:, hs]), dv=to_f64(L.dv[:, hs]))
@@ -193,4 +200,42 @@ def check_decode_selection(gpu_blk, gpu_grp, q_tok, bsum, gsum, pos, w, n_kv, wh
         _valid_topk(gpu_grp[b, h], groups, gsum[b, h, groups] @ qbar, w.topk_groups,
                     f"{what}sel_grp{(b, h)}")
         differ += int(np.any(gpu_grp[b, h] != sg[b, h]) or np.any(gpu_blk[b, h] != sb[b, h]))
+    return int(tie.sum()), differ
+
+
+def compare_segment_causal(w, gpu, q_prev_mean, q_begin, n_kv, k64, v64, backward):
+    """Causal routing against the oracle: the summaries, the segment's
+    resident block mean queries, the selections (routed with the previous
+    block's mean query, q_prev_mean [B, Hkv, n_qb, d] from the oracle) and
+    the attention on the GPU's selection."""
+    T_end = q_begin + w.seg_len
+    g_ref, b_ref = oracle.build_summaries(k64, 0, T_end)
+    assert_close(gpu["bsum"][:, :, :T_end // 64], b_ref, w, "bsum", rel=SUMMARY_REL)
+    J0 = q_begin // 64
+    qs_ref = oracle.query_summaries(gpu["q64"], n_kv)
+    assert_close(gpu["qsum"][:, :, J0:J0 + w.seg_len // 64], qs_ref, w, "qsum", rel=SUMMARY_REL)
+    sb, sg, tie = oracle.route_causal(q_prev_mean, b_ref, g_ref, q_begin, w.seg_len // 64,
+                                      w.topk_blocks, w.topk_groups)
+    for name, g, r in (("sel_blk", gpu["sel_blk"], sb), ("sel_grp", gpu["sel_grp"], sg)):
+        bad = np.any(g != r, axis=-1) & ~tie
+        assert not bad.any(), f"causal {name}: {int(bad.sum())} unflagged rows differ"
+    differ = 0
+    for b, h, j in np.argwhere(tie):
+        J = J0 + j
+        qbar = q_prev_mean[b, h, j]
+        blocks = _valid_topk(gpu["sel_blk"][b, h, j], np.arange(J), b_ref[b, h, :J] @ qbar,
+                             w.topk_blocks, f"causal sel_blk{(b, h, j)}")
+        groups = np.array([8 * c + i for c in blocks for i in range(8)], np.int64)
+        _valid_topk(gpu["sel_grp"][b, h, j], groups, g_ref[b, h, groups] @ qbar, w.topk_groups,
+                    f"causal sel_grp{(b, h, j)}")
+        differ += int(np.any(gpu["sel_grp"][b, h, j] != sg[b, h, j]))
+    o, lse = oracle.attn_fwd(gpu["q64"], k64, v64, q_begin, gpu["sel_grp"], n_kv)
+    assert_close(gpu["o"], o, w, "o")
+    assert_close(gpu["lse"], lse, w, "lse", abs_=LSE_ABS)
+    if backward:
+        dq, dk, dv = oracle.attn_bwd(gpu["q64"], k64, v64, gpu["do64"], q_begin,
+                                     gpu["sel_grp"], n_kv)
+        assert_close(gpu["dq"], dq, w, "dq")
+        assert_close(gpu["dk"], dk, w, "dk")
+        assert_close(gpu["dv"], dv, w, "dv")
     return int(tie.sum()), differ
