@@ -422,3 +422,57 @@ def route_causal(q_prev_mean: np.ndarray, bsum: np.ndarray, gsum: np.ndarray, q_
                 sel_grp[b, h, j, :kg] = np.sort(chosen)
                 near_tie[b, h, j] = _near_tie(s1_sorted, kb) or _near_tie(s2_sorted, kg)
     return sel_blk, sel_grp, near_tie
+
+
+# ----------------------------------------------------------------------------
+# the upstream pass of a segment: from the Q/K/V projection outputs to the
+# tensors and summaries the path reads (the seventnews page, section
+# "HGA的不同之处": the router scores the existing projected keys; the
+# workloads apply RoPE, base 1e6, before the summaries).  Readings:
+#   U1  the projection outputs are token-major, [B, S, H, d] per tensor;
+#   U2  RoPE is the rotate-half form: for i < d/2, with theta_i =
+#       base^(-2i/d) and angle p * theta_i at global position p,
+#       (x_i, x_{i+d/2}) -> (x_i cos - x_{i+d/2} sin, x_{i+d/2} cos + x_i sin);
+#       V is not rotated;
+#   U3  Q, K and V are stored in the path's element type (bf16: round to
+#       nearest even), and the summaries and block mean queries are taken of
+#       the stored values.
+# ----------------------------------------------------------------------------
+
+def rope(x: np.ndarray, pos0: int, base: float) -> np.ndarray:
+    """Rotate-half RoPE (U2) of x [..., S, d] at positions pos0 .. pos0+S-1."""
+    d = x.shape[-1]
+    half = d // 2
+    theta = base ** (-2.0 * np.arange(half) / d)
+    ang = (pos0 + np.arange(x.shape[-2]))[:, None] * theta[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """float64 -> nearest bfloat16 (8-bit significand, ties to even), as float64."""
+    x = np.asarray(x, np.float64)
+    m, e = np.frexp(x)                       # x = m * 2^e, 0.5 <= |m| < 1
+    scaled = np.ldexp(m, 8)                  # 8 significant bits above the point
+    return np.ldexp(np.round(scaled), e - 8)     # np.round: half to even
+
+
+def prepare_segment(q_proj, k_proj, v_proj, q_begin: int, rope_base, n_kv_heads: int,
+                    dtype: str):
+    """q_proj [B, S, Hq, d], k_proj / v_proj [B, S, Hkv, d] float64 (U1).
+    Returns q [B, Hq, S, d], k, v [B, Hkv, S, d] as stored (U2, U3), the
+    segment's gsum / bsum (R1, global indices from q_begin/8 and q_begin/64)
+    and qsum [B, Hkv, S/64, d] (the block mean queries)."""
+    q = np.transpose(q_proj, (0, 2, 1, 3))
+    k = np.transpose(k_proj, (0, 2, 1, 3))
+    v = np.transpose(v_proj, (0, 2, 1, 3))
+    if rope_base is not None:
+        q, k = rope(q, q_begin, rope_base), rope(k, q_begin, rope_base)
+    if dtype == "bf16":
+        q, k, v = round_bf16(q), round_bf16(k), round_bf16(v)
+    else:
+        q, k, v = (np.asarray(t, np.float32).astype(np.float64) for t in (q, k, v))
+    S = q.shape[2]
+    gsum, bsum = build_summaries(k, 0, S)
+    return q, k, v, gsum, bsum, query_summaries(q, n_kv_heads)

@@ -827,3 +827,105 @@ def test_causal_pins_catch_planted_mistakes(monkeypatch, target, mutant):
         except (AssertionError, IndexError, ValueError):
             failed += 1
     assert failed >= 1, f"no pin caught the planted mistake in {target}"
+
+
+# ----------------------------------------------------------------------------
+# pins: the upstream pass (RoPE, storage rounding, layout)
+# ----------------------------------------------------------------------------
+
+def check_rope_closed_forms():
+    rng = np.random.default_rng(30)
+    d, base = 16, 1e6
+    x = rng.standard_normal((2, 5, d))
+    # complex form: pair (x_i, x_{i+d/2}) as x_i + j x_{i+d/2}, times e^{j p theta_i}
+    pos0 = 1000
+    y = oracle.rope(x, pos0, base)
+    half = d // 2
+    theta = np.array([base ** (-2.0 * i / d) for i in range(half)])
+    for t in range(5):
+        z = (x[:, t, :half] + 1j * x[:, t, half:]) * np.exp(1j * (pos0 + t) * theta)
+        assert close(y[:, t, :half], z.real) and close(y[:, t, half:], z.imag)
+    # position 0 is the identity; every pair keeps its length
+    assert close(oracle.rope(x[:, :1], 0, base), x[:, :1])
+    assert close(y[..., :half] ** 2 + y[..., half:] ** 2, x[..., :half] ** 2 + x[..., half:] ** 2)
+    # q.k depends only on the distance between the two positions
+    q, k = rng.standard_normal((1, d)), rng.standard_normal((1, d))
+    a = float(oracle.rope(q, 37, base)[0] @ oracle.rope(k, 5, base)[0])
+    b = float(oracle.rope(q, 5037, base)[0] @ oracle.rope(k, 5005, base)[0])
+    assert abs(a - b) < 1e-9
+
+
+def test_rope_closed_forms():
+    check_rope_closed_forms()
+
+
+def check_round_bf16():
+    # ties go to even, and torch's float32 -> bfloat16 conversion (round to
+    # nearest even) agrees on float32 values
+    assert list(oracle.round_bf16(np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8)]))) == \
+        [1.0, 1 + 2 ** -6, -1.0]
+    rng = np.random.default_rng(31)
+    x = (rng.standard_normal(4096) * 10.0 ** rng.integers(-3, 4, 4096)).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(oracle.round_bf16(x.astype(np.float64)), ref)
+
+
+def test_round_bf16():
+    check_round_bf16()
+
+
+def check_prepare_layout():
+    """Token-major projections become head-major tensors; without RoPE and at
+    float32 the values pass through unchanged; the summaries and the block
+    mean queries are those of the stored tensors."""
+    rng = np.random.default_rng(32)
+    B, S, Hq, Hkv, d = 2, 128, 4, 2, 8
+    qp = rng.standard_normal((B, S, Hq, d)).astype(np.float32).astype(np.float64)
+    kp = rng.standard_normal((B, S, Hkv, d)).astype(np.float32).astype(np.float64)
+    vp = rng.standard_normal((B, S, Hkv, d)).astype(np.float32).astype(np.float64)
+    q, k, v, g, bl, qs = oracle.prepare_segment(qp, kp, vp, 64, None, Hkv, "f32")
+    assert np.array_equal(q[1, 3, 70], qp[1, 70, 3]) and np.array_equal(k[0, 1, 5], kp[0, 5, 1])
+    assert np.array_equal(v[1, 0, 127], vp[1, 127, 0])
+    assert close(g[0, 1, 3], kp[0, 24:32, 1].mean(0)) and close(bl[1, 0, 1], kp[1, 64:, 0].mean(0))
+    assert close(qs[0, 1, 0], qp[0, :64, 2:4].mean((0, 1)))
+    q2, k2, *_ = oracle.prepare_segment(qp, kp, vp, 64, 1e4, Hkv, "bf16")
+    assert np.array_equal(q2, oracle.round_bf16(oracle.rope(q, 64, 1e4)))
+
+
+def test_prepare_layout():
+    check_prepare_layout()
+
+
+def _mut_rope_sign(x, pos0, base):
+    # the rotation turned the other way (sine with the wrong sign)
+    d = x.shape[-1]
+    y = ORIG_PREP["rope"](x[..., ::1], -pos0, base)
+    return y if pos0 else np.concatenate([y[..., :d // 2], -y[..., d // 2:]], axis=-1)
+
+
+def _mut_rope_freq(x, pos0, base):
+    return ORIG_PREP["rope"](x, pos0, base ** 0.5)
+
+
+def _mut_round_half_up(x):
+    m, e = np.frexp(np.asarray(x, np.float64))
+    return np.ldexp(np.floor(np.ldexp(m, 8) + 0.5), e - 8)
+
+
+ORIG_PREP = {"rope": ho.rope, "round_bf16": ho.round_bf16}
+PREP_PINS = [check_rope_closed_forms, check_round_bf16, check_prepare_layout]
+
+
+@pytest.mark.parametrize("target,mutant", [
+    ("rope", _mut_rope_sign), ("rope", _mut_rope_freq), ("round_bf16", _mut_round_half_up),
+])
+def test_prepare_pins_catch_planted_mistakes(monkeypatch, target, mutant):
+    monkeypatch.setattr(ho, target, mutant)
+    monkeypatch.setattr(oracle, target, mutant)
+    failed = 0
+    for pin in PREP_PINS:
+        try:
+            pin()
+        except (AssertionError, IndexError, ValueError):
+            failed += 1
+    assert failed >= 1, f"no pin caught the planted mistake in {target}"
