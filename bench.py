@@ -350,10 +350,11 @@ class Runner:
             return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
         return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
 
-    def step(self, record_sel=None):
+    def step(self, record_sel=None, causal=False):
         L = self.layer
         for i, q_begin in enumerate(self.segs):
-            L.segment(self.q[i], q_begin, self.do[i] if self.w.backward else None)
+            L.segment(self.q[i], q_begin, self.do[i] if self.w.backward else None,
+                      causal=causal)
             if record_sel is not None:
                 record_sel.append((q_begin, L.sel_grp.cpu().numpy()))
 
@@ -744,7 +745,7 @@ def run_gpu(args, rank, world, local):
 
     extra = None
     if world == 1 and not args.no_extra and not tiered:
-        extra = run_extras(device, max(args.steps // 2, 5), pk)
+        extra = run_extras(device, max(args.steps // 2, 5), pk, run)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -791,7 +792,7 @@ def decode_bytes(w, positions):
     return tot
 
 
-def run_extras(device, steps, pk):
+def run_extras(device, steps, pk, run=None):
     """The 131072-token forward (64 segments of 2048, the long-context
     workload) with its per-kernel table, and decode (one new token per
     sequence, batch 8 at position 131071, four layers' caches in turn so
@@ -813,6 +814,99 @@ def run_extras(device, steps, pk):
                 fn()
         torch.cuda.current_stream(device).wait_stream(cs)
         return g
+
+    # -- the same fwd+bwd workload with strictly causal routing ------------
+    if run is not None and not run.w.name.startswith("qwen3_tiered"):
+        run.step(causal=True)
+        g = graph_of(lambda: run.step(causal=True))
+        g.replay()
+        ms = []
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize(device)
+            ms.append(e0.elapsed_time(e1))
+        del g
+        tokens = run.w.batch * len(run.segs) * run.w.seg_len
+        out["causal_routing"] = {
+            "workload": run.w.name, "routing": "hga_route_causal (previous block's mean query)",
+            "tokens_per_s": round(tokens / (statistics.mean(ms) / 1e3), 1),
+            "ms_per_step": round(statistics.mean(ms), 4),
+            "timing": "graph replay per step, CUDA events, L2 flushed between steps"}
+
+    # -- the same fwd+bwd workload from the projection outputs ---------------
+    if run is not None and not run.w.name.startswith("qwen3_tiered") and run.w.backward:
+        w = run.w
+        cfg = run.layer.cfg
+        k, v, qs, dos = synth.device_inputs(w, device)
+        segs = w.segments()
+        S = w.seg_len
+        # token-major [B, S, H, d] projection outputs of every segment
+        qproj = [q.transpose(1, 2).contiguous() for q in qs]
+        kproj = [k[:, :, s0:s0 + S].transpose(1, 2).contiguous() for s0 in segs]
+        vproj = [v[:, :, s0:s0 + S].transpose(1, 2).contiguous() for s0 in segs]
+        del k, v, qs
+        Lp = HgaLayer(cfg, w.ctx_len, S, device=device)
+        q_out = torch.empty((w.batch, w.n_q_heads, S, w.head_dim), dtype=torch.bfloat16,
+                            device=device)
+
+        def pstep():
+            for i, s0 in enumerate(segs):
+                Lp.segment_from_projections(qproj[i], kproj[i], vproj[i],
+                                            w.n_q_heads * w.head_dim, w.n_kv_heads * w.head_dim,
+                                            s0, w.rope_base, q_out, dos[i])
+
+        pstep()
+        hga_timing_enable(8 * len(segs) + 16)
+        g_all = graph_of(pstep)
+        hga_timing_reset()
+        for _ in range(3):
+            flush.zero_()
+            g_all.replay()
+            hga_timing_collect()
+        torch.cuda.synchronize(device)
+        ptable = timing_table()
+        hga_timing_enable(0)
+        del g_all
+        g = graph_of(pstep)
+        g.replay()
+        ms = []
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize(device)
+            ms.append(e0.elapsed_time(e1))
+        del g
+        el = 2
+        B, Hq, Hkv, d = w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim
+        # per launch: read Q/K/V projections, write Q, K, V, the summaries and block means
+        prep_bytes = (2 * B * S * (Hq + 2 * Hkv) * d * el
+                      + B * Hkv * (S // 8 + 2 * (S // 64)) * d * 4)
+        pk_ms, pk_n = ptable.get("prepare", (0.0, 0))
+        prep = None
+        if pk_n:
+            ach = prep_bytes / (pk_ms / pk_n / 1e3) / 1e9
+            prep = {"avg_us": round(pk_ms / pk_n * 1e3, 3), "bytes_per_launch": prep_bytes,
+                    "achieved": round(ach, 1), "unit": "GB/s",
+                    "frac": round(ach / pk["hbm"], 4)}
+        tokens = B * len(segs) * S
+        out["from_projections"] = {
+            "workload": w.name,
+            "step": "per segment: hga_prepare_segment (RoPE, layout, summaries, block means) -> "
+                    "hga_route_summarized -> hga_attn_fwd_bwd; inputs are the token-major "
+                    "projection outputs",
+            "tokens_per_s": round(tokens / (statistics.mean(ms) / 1e3), 1),
+            "ms_per_step": round(statistics.mean(ms), 4),
+            "prepare_kernel": prep,
+            "kernel_us_per_step": {n: round(v_[0] / 3 * 1e3, 2) for n, v_ in ptable.items()}}
+        del Lp, qproj, kproj, vproj, dos
+        torch.cuda.empty_cache()
 
     # -- 131072-token forward --------------------------------------------
     w = synth.workloads()["qwen3_fwd_128k"]

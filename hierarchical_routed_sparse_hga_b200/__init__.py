@@ -16,7 +16,7 @@ from ._lib import (EXPORTS, HGA_BF16, HGA_ERR_CUDA, HGA_ERR_DEVICE_CHECK,  # noq
                    hga_tier_stage_rows, hga_tier_workspace_size, hga_get_device_status,
                    hga_kernel_name,
                    hga_launch_count, hga_route, hga_route_causal, hga_route_noalloc,
-                   hga_build_query_summaries,
+                   hga_build_query_summaries, hga_prepare_segment, hga_route_summarized,
                    hga_route_workspace_size, hga_status_string,
                    hga_timing_collect, hga_timing_enable, hga_timing_get, hga_timing_kinds,
                    hga_timing_reset,

@@ -32,9 +32,9 @@ EXPORTS = ("hga_version", "hga_status_string", "hga_build_summaries",
            "hga_build_summaries_seg",
            "hga_tier_stage_rows", "hga_tier_workspace_size", "hga_tier_gather",
            "hga_tier_append", "hga_decode", "hga_build_query_summaries",
-           "hga_route_causal")
+           "hga_route_causal", "hga_prepare_segment", "hga_route_summarized")
 HGA_NOALLOC_SCRATCH_BYTES = 4 << 20
-HGA_K_COUNT = 15
+HGA_K_COUNT = 16
 
 
 class HgaError(RuntimeError):
@@ -118,6 +118,11 @@ def load() -> ctypes.CDLL:
         "hga_decode": (ctypes.c_int, [CFG, P, P, P, I64, P, P, P, P, P, P, P, P]),
         "hga_build_query_summaries": (ctypes.c_int, [CFG, P, I64, I32, I64, P, P]),
         "hga_route_causal": (ctypes.c_int, [CFG, P, I64, I32, I64, P, P, P, P, P, P, SZ, P]),
+        "hga_prepare_segment": (ctypes.c_int, [CFG, P, P, P, I64, I64, I64, I32, I64,
+                                               ctypes.c_float,
+                                               P, P, P, P, P, P, P]),
+        "hga_route_summarized": (ctypes.c_int, [CFG, I64, I32, I64, P, P, P, I32, P, P, P, SZ,
+                                                P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -248,6 +253,26 @@ def hga_route_causal(cfg: Config, q, q_begin, s_len, ctx_cap, bsum, gsum, qsum, 
     _check("hga_route_causal", load().hga_route_causal(
         ctypes.byref(c), _ptr(q), q_begin, s_len, ctx_cap, _ptr(bsum), _ptr(gsum), _ptr(qsum),
         _ptr(sel_blk), _ptr(sel_grp), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def hga_prepare_segment(cfg: Config, q_proj, k_proj, v_proj, q_row_stride, kv_row_stride, q_begin,
+                        s_len, ctx_cap, rope_base, q_out, k, v, gsum, bsum, qsum, stream=None):
+    c = cfg.c()
+    _check("hga_prepare_segment", load().hga_prepare_segment(
+        ctypes.byref(c), _ptr(q_proj), _ptr(k_proj), _ptr(v_proj), q_row_stride, kv_row_stride,
+        q_begin, s_len,
+        ctx_cap, float(rope_base or 0.0), _ptr(q_out), _ptr(k), _ptr(v), _ptr(gsum), _ptr(bsum),
+        _ptr(qsum), _stream(stream)))
+
+
+def hga_route_summarized(cfg: Config, q_begin, s_len, ctx_cap, bsum, gsum, qsum, causal, sel_blk,
+                         sel_grp, workspace, ws_bytes=None, stream=None):
+    c = cfg.c()
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check("hga_route_summarized", load().hga_route_summarized(
+        ctypes.byref(c), q_begin, s_len, ctx_cap, _ptr(bsum), _ptr(gsum), _ptr(qsum),
+        int(causal), _ptr(sel_blk), _ptr(sel_grp), _ptr(workspace), ws_bytes,
+        _stream(stream)))
 
 
 def hga_route_noalloc(cfg: Config, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp,

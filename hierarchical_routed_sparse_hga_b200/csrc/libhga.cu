@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <initializer_list>
 #include <map>
@@ -21,6 +22,7 @@
 #include "attn_bwd_sm100.cuh"
 #include "tier.cuh"
 #include "decode.cuh"
+#include "prepare.cuh"
 #include "trace.cuh"
 
 using namespace hga;
@@ -360,12 +362,13 @@ static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q
                                int32_t s_len, int64_t ctx_cap, const float* bsum,
                                const float* gsum, int32_t* sel_blk, int32_t* sel_grp,
                                void* workspace, size_t ws_bytes, int* done, uint32_t token,
-                               cudaStream_t s, const float* qprev = nullptr) {
+                               cudaStream_t s, const float* qprev = nullptr,
+                               int qshift = 1) {
   hga_status_t st = check_cfg(cfg);
   if (st != HGA_OK) return st;
   if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
-  if (!q || !bsum || !gsum || !sel_grp || !workspace) return HGA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(bsum) || !aligned16(gsum) || !aligned16(sel_grp) ||
+  if ((!q && !qprev) || !bsum || !gsum || !sel_grp || !workspace) return HGA_ERR_INVALID_ARG;
+  if ((q && !aligned16(q)) || !aligned16(bsum) || !aligned16(gsum) || !aligned16(sel_grp) ||
       !aligned16(workspace) || (sel_blk && !aligned16(sel_blk)))
     return HGA_ERR_INVALID_ARG;
   RouteCarve ws = route_carve(cfg, s_len, q_begin, workspace);
@@ -385,7 +388,7 @@ static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q
         return launch_pdl(route_fused_kernel<T, D>, g1, dim3(kRouteThreads), smf, s,
                           static_cast<const T*>(q), bsum, gsum, ctx_cap, cfg->n_q_heads,
                           cfg->n_kv_heads, s_len, own0, cfg->topk_blocks, cfg->topk_groups,
-                          sel_blk, sel_grp, done, token, qprev);
+                          sel_blk, sel_grp, done, token, qprev, qshift);
       });
     }
     hga_status_t e = HGA_OK;
@@ -403,7 +406,7 @@ static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q
       dim3 g2(unsigned(n_cc * n_jc), cfg->n_kv_heads, cfg->batch);
       e = traced_launch(HGA_K_BLOCK_SCORE, s, [&] {
         return launch_pdl(block_score_kernel<D>, g2, dim3(kRouteThreads), 0, s, ws.qbar, qprev,
-            bsum, ctx_cap, cfg->n_kv_heads, G, n_qb, own0, ws.scores, ws.jstride);
+            qshift, bsum, ctx_cap, cfg->n_kv_heads, G, n_qb, own0, ws.scores, ws.jstride);
       });
       if (e != HGA_OK) return e;
     }
@@ -413,7 +416,7 @@ static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q
     if (e != HGA_OK) return e;
     return traced_launch(HGA_K_SELECT, s, [&] {
       return launch_pdl(select_kernel<D>, g1, dim3(kRouteThreads), sm3, s, ws.qbar, qprev,
-          ws.scores, gsum,
+          qshift, ws.scores, gsum,
           ctx_cap, cfg->n_kv_heads, G, n_qb, own0, ws.jstride, cfg->topk_blocks, cfg->topk_groups,
           sel_blk, sel_grp);
     });
@@ -801,7 +804,7 @@ const char* hga_kernel_name(int kind) {
       "summaries",      "route_qmean",       "route_block_score",   "route_select",
       "attn_fwd_simt",  "attn_bwd_dq_simt",  "attn_bwd_dkdv_simt",  "attn_fwd_tc",
       "attn_bwd_dq_tc", "attn_bwd_dkdv_tc",  "tier_dedup",          "tier_copy",
-      "route_fused",    "decode",            "query_summaries"};
+      "route_fused",    "decode",            "query_summaries",     "prepare"};
   return (kind >= 0 && kind < HGA_K_COUNT) ? names[kind] : "unknown";
 }
 
@@ -981,4 +984,54 @@ extern "C" hga_status_t hga_route_causal(const hga_config_t* cfg, const void* q,
   if ((st = launch_qsum(cfg, q, q_begin, s_len, ctx_cap, qsum, s)) != HGA_OK) return st;
   return route_impl(cfg, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp, workspace,
                     ws_bytes, nullptr, 0, s, qsum);
+}
+
+extern "C" hga_status_t hga_prepare_segment(const hga_config_t* cfg, const void* q_proj,
+                                            const void* k_proj, const void* v_proj,
+                                            int64_t q_row_stride, int64_t kv_row_stride,
+                                            int64_t q_begin, int32_t s_len,
+                                            int64_t ctx_cap, float rope_base, void* q_out,
+                                            void* k, void* v, float* gsum, float* bsum,
+                                            float* qsum, void* stream) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
+  for (const void* p : {q_proj, k_proj, v_proj, static_cast<const void*>(q_out),
+                        static_cast<const void*>(k), static_cast<const void*>(v),
+                        static_cast<const void*>(gsum), static_cast<const void*>(bsum),
+                        static_cast<const void*>(qsum)})
+    if (!p || !aligned16(p)) return HGA_ERR_INVALID_ARG;
+  const size_t elt = cfg->dtype == HGA_BF16 ? 2 : 4;
+  if (q_row_stride < int64_t(cfg->n_q_heads) * cfg->head_dim ||
+      kv_row_stride < int64_t(cfg->n_kv_heads) * cfg->head_dim ||
+      (size_t(q_row_stride) * elt) % 16 != 0 || (size_t(kv_row_stride) * elt) % 16 != 0)
+    return HGA_ERR_INVALID_ARG;
+  if (!(rope_base >= 0.f)) return HGA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const double log2_base = rope_base > 1.f ? std::log2(double(rope_base)) : 0.0;
+  return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
+    const size_t smem = sizeof(PrepShared<D>);
+    hga_status_t e = ensure_smem(reinterpret_cast<const void*>(&prepare_kernel<T, D>), smem);
+    if (e != HGA_OK) return e;
+    dim3 grid(s_len / kQBlock, cfg->n_kv_heads, cfg->batch);
+    return traced_launch(HGA_K_PREPARE, s, [&] {
+      return launch_pdl(prepare_kernel<T, D>, grid, dim3(kPrepThreads), smem, s,
+          static_cast<const T*>(q_proj), static_cast<const T*>(k_proj),
+          static_cast<const T*>(v_proj), q_row_stride, kv_row_stride, q_begin, s_len, ctx_cap,
+          cfg->n_q_heads,
+          cfg->n_kv_heads, log2_base, static_cast<T*>(q_out), static_cast<T*>(k),
+          static_cast<T*>(v), gsum, bsum, qsum);
+    });
+  });
+}
+
+extern "C" hga_status_t hga_route_summarized(const hga_config_t* cfg, int64_t q_begin,
+                                             int32_t s_len, int64_t ctx_cap, const float* bsum,
+                                             const float* gsum, const float* qsum, int32_t causal,
+                                             int32_t* sel_blk, int32_t* sel_grp, void* workspace,
+                                             size_t ws_bytes, void* stream) {
+  if (!qsum || !aligned16(qsum) || (causal != 0 && causal != 1)) return HGA_ERR_INVALID_ARG;
+  return route_impl(cfg, nullptr, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp,
+                    workspace, ws_bytes, nullptr, 0, static_cast<cudaStream_t>(stream), qsum,
+                    causal);
 }

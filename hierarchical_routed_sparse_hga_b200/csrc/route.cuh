@@ -82,16 +82,17 @@ __device__ __forceinline__ float qbar_elem(const float* qpart_bhj, int G, int D,
   return v;
 }
 
-// q-bar of query block j (global block own0 + j) as the routing uses it:
-// normally the sum of its G shares; in causal mode (qprev != nullptr) the
-// resident mean query of the block before it, qprev[head, own0 + j - 1, :]
-// (zero for the first block of a sequence, which has no candidates).
-__device__ __forceinline__ float route_qbar(const float* qpart, const float* qprev, int64_t head,
-                                            int n_qb, int G, int D, int j, int e, int64_t own0,
-                                            int64_t ctx_blocks) {
-  if (qprev) {
-    const int64_t J = own0 + j;
-    return J > 0 ? qprev[(head * ctx_blocks + J - 1) * D + e] : 0.f;
+// q-bar of query block j (global block J = own0 + j) as the routing uses it:
+// the sum of its G shares; or, from the resident block mean queries qsum
+// (qsum != nullptr), row J - qshift: the block's own mean (qshift 0) or, for
+// causal routing, the block before it (qshift 1; zero for the first block of
+// a sequence, which has no candidates).
+__device__ __forceinline__ float route_qbar(const float* qpart, const float* qsum, int qshift,
+                                            int64_t head, int n_qb, int G, int D, int j, int e,
+                                            int64_t own0, int64_t ctx_blocks) {
+  if (qsum) {
+    const int64_t row = own0 + j - qshift;
+    return row >= 0 ? qsum[(head * ctx_blocks + row) * D + e] : 0.f;
   }
   return qbar_elem(qpart + ((head * n_qb + j) * G) * D, G, D, e);
 }
@@ -105,7 +106,7 @@ constexpr int kScoreQbs = 8;
 template <int D>
 __global__ void __launch_bounds__(kRouteThreads)
     block_score_kernel(const float* __restrict__ qpart, const float* __restrict__ qprev,
-                       const float* __restrict__ bsum, int64_t ctx_cap, int n_kv_heads, int G,
+                       int qshift, const float* __restrict__ bsum, int64_t ctx_cap, int n_kv_heads, int G,
                        int n_qb, int64_t own0, float* __restrict__ scores, int64_t jstride) {
   pdl_launch_dependents();
   pdl_wait();
@@ -125,7 +126,8 @@ __global__ void __launch_bounds__(kRouteThreads)
 #pragma unroll
   for (int u = 0; u < kQ; ++u) {
     const int i = threadIdx.x + u * kRouteThreads, jl = i / D, e = i % D, j = j0 + jl;
-    qv[u] = j < n_qb ? route_qbar(qpart, qprev, head, n_qb, G, D, j, e, own0, ctx_cap / kBlock)
+    qv[u] = j < n_qb ? route_qbar(qpart, qprev, qshift, head, n_qb, G, D, j, e, own0,
+                                      ctx_cap / kBlock)
                      : 0.f;
   }
 #pragma unroll
@@ -279,7 +281,7 @@ __device__ __forceinline__ void select_levels(const SelectLayout& L, unsigned ch
 // grid (n_qb, Hkv, B); dynamic smem select_layout(...).total
 template <int D>
 __global__ void __launch_bounds__(kRouteThreads)
-    select_kernel(const float* __restrict__ qpart, const float* __restrict__ qprev,
+    select_kernel(const float* __restrict__ qpart, const float* __restrict__ qprev, int qshift,
                   const float* __restrict__ scores,
                   const float* __restrict__ gsum, int64_t ctx_cap, int n_kv_heads, int G, int n_qb,
                   int64_t own0, int64_t jstride, int topk_blocks, int topk_groups,
@@ -297,7 +299,7 @@ __global__ void __launch_bounds__(kRouteThreads)
   const float* srow = scores + (head * n_qb + j) * jstride;
   for (int64_t i = threadIdx.x; i < J; i += kRouteThreads) key1[i] = ordered_key(srow[i]);
   for (int i = threadIdx.x; i < D; i += kRouteThreads)
-    qb[i] = route_qbar(qpart, qprev, head, n_qb, G, D, j, i, own0, ctx_cap / kBlock);
+    qb[i] = route_qbar(qpart, qprev, qshift, head, n_qb, G, D, j, i, own0, ctx_cap / kBlock);
   __syncthreads();
   select_levels<D>(L, sm_raw, gsum, head, ctx_cap, n_qb, j, J, topk_blocks, topk_groups, sel_blk,
                    sel_grp);
@@ -377,7 +379,8 @@ __global__ void __launch_bounds__(kRouteThreads)
                        const float* __restrict__ gsum, int64_t ctx_cap, int n_q_heads,
                        int n_kv_heads, int s_len, int64_t own0, int topk_blocks, int topk_groups,
                        int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp,
-                       int* __restrict__ done, uint32_t token, const float* __restrict__ qprev) {
+                       int* __restrict__ done, uint32_t token, const float* __restrict__ qprev,
+                       int qshift) {
   // q-bar needs only the queries, which the kernels before this one do not
   // write: it is formed while the kernel before still runs; the summaries
   // are read only after it has completed (the wait below).  A chained
@@ -398,7 +401,7 @@ __global__ void __launch_bounds__(kRouteThreads)
   pdl_wait();
   if (qprev)
     for (int e = threadIdx.x; e < D; e += kRouteThreads)
-      qb[e] = J > 0 ? qprev[(head * (ctx_cap / kBlock) + J - 1) * D + e] : 0.f;
+      qb[e] = J - qshift >= 0 ? qprev[(head * (ctx_cap / kBlock) + J - qshift) * D + e] : 0.f;
   __syncthreads();
   // level-1 scores of the J candidate blocks
   score_rows<D>(bsum + head * (ctx_cap / kBlock) * D, qb, int(J),

@@ -79,6 +79,33 @@ class HgaLayer:
                               self.gsum, self.qsum, self.sel_blk, self.sel_grp, self.route_ws,
                               stream=stream)
 
+    def prepare(self, q_proj, k_proj, v_proj, q_row_stride: int, kv_row_stride: int,
+                q_begin: int, rope_base, q_out, stream=None):
+        """The segment's upstream pass (hga_prepare_segment): RoPE of the
+        projections, Q into q_out, K/V into the context, summaries and block
+        mean queries into gsum, bsum, qsum."""
+        _lib.hga_prepare_segment(self.cfg, q_proj, k_proj, v_proj, q_row_stride, kv_row_stride,
+                                 q_begin, self.seg_len, self.ctx_cap, rope_base, q_out, self.k, self.v,
+                                 self.gsum, self.bsum, self.qsum, stream)
+
+    def route_summarized(self, q_begin: int, causal=False, stream=None):
+        _lib.hga_route_summarized(self.cfg, q_begin, self.seg_len, self.ctx_cap, self.bsum,
+                                  self.gsum, self.qsum, causal, self.sel_blk, self.sel_grp,
+                                  self.route_ws, stream=stream)
+
+    def segment_from_projections(self, q_proj, k_proj, v_proj, q_row_stride: int,
+                                 kv_row_stride: int, q_begin: int, rope_base, q_out, d_o=None,
+                                 causal=False, stream=None, out=None):
+        """One segment from its projection outputs: the upstream pass, routing
+        from the resident summaries, then the forward and (if d_o) backward."""
+        self.prepare(q_proj, k_proj, v_proj, q_row_stride, kv_row_stride, q_begin, rope_base,
+                     q_out, stream)
+        self.route_summarized(q_begin, causal, stream)
+        if d_o is None:
+            self.forward(q_out, q_begin, stream, out)
+        else:
+            self.forward_backward(q_out, d_o, q_begin, stream, out)
+
     def make_outputs(self):
         """A fresh set of per-segment outputs (o, lse, dq, dk, dv), for callers
         that keep one segment's results while the next one is computed."""

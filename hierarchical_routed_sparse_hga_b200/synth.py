@@ -42,7 +42,8 @@ GROUP = 8
 QBLOCK = 64
 
 # tensor ids for the per-tensor streams
-_T_CENTROID, _T_KNOISE, _T_V, _T_TARGET, _T_QNOISE, _T_DO, _T_DEC_TARGET, _T_DEC_Q = range(8)
+_T_CENTROID, _T_KNOISE, _T_V, _T_TARGET, _T_QNOISE, _T_DO, _T_DEC_TARGET, _T_DEC_Q, \
+    _T_PROJ = range(9)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -218,6 +219,33 @@ def queries_head(w: Workload, b: int, hq: int, seg_begin: int) -> np.ndarray:
 def dout_head(w: Workload, b: int, hq: int, seg_begin: int) -> np.ndarray:
     rng = _rng(w, _T_DO, b, hq, seg_begin // w.seg_len)
     return to_storage(rng.standard_normal((w.seg_len, w.head_dim)), w.dtype)
+
+
+def projections(w: Workload, seg_begin: int):
+    """Token-major projection outputs of one segment before RoPE: q_proj
+    [B, S, Hq, d], k_proj and v_proj [B, S, Hkv, d], storage dtype.  Keys and
+    queries follow the recipe above (centroids, planted target blocks, 0.5
+    noise, the 1/sqrt(d) scale of scaled workloads) without the rotation,
+    which the upstream pass applies; drawn from their own streams."""
+    S, G = w.seg_len, w.group_heads
+    B, Hq, Hkv, d = w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim
+    qp = np.empty((B, S, Hq, d))
+    kp = np.empty((B, S, Hkv, d))
+    vp = np.empty((B, S, Hkv, d))
+    scale = w.scale if w.scaled else 1.0
+    seg = seg_begin // w.seg_len
+    for b in range(B):
+        for h in range(Hkv):
+            c = centroids(w, b, h)
+            kn = _rng(w, _T_PROJ, 0, b, h, seg).standard_normal((S, d))
+            kp[b, :, h] = (np.repeat(c[seg_begin // BLOCK:(seg_begin + S) // BLOCK], BLOCK, axis=0)
+                           + 0.5 * kn) * scale
+            vp[b, :, h] = _rng(w, _T_PROJ, 1, b, h, seg).standard_normal((S, d))
+            r = targets(w, b, h, seg_begin)
+            for g in range(G):
+                qn = _rng(w, _T_PROJ, 2, b, h * G + g, seg).standard_normal((S, d))
+                qp[b, :, h * G + g] = (np.repeat(c[r], QBLOCK, axis=0) + 0.5 * qn) * scale
+    return tuple(to_storage(t, w.dtype) for t in (qp, kp, vp))
 
 
 def decode_query_head(w: Workload, b: int, hq: int, pos: int) -> np.ndarray:

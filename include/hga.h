@@ -344,6 +344,51 @@ HGA_API hga_status_t hga_route_causal(const hga_config_t* cfg, const void* q, in
                                       void* stream);
 
 /*
+ * The upstream pass of a segment, in one read of its projection outputs ([B]
+ * "HGA的不同之处": the router scores the existing projected keys; the
+ * workloads apply RoPE, base 1e6, before the summaries).  For the s_len tokens
+ * starting at global position q_begin:
+ *   q_proj [batch, s_len, n_q_heads, head_dim], k_proj and v_proj [batch,
+ *   s_len, n_kv_heads, head_dim], token-major; q_row_stride (kv_row_stride)
+ *   elements from one token's Q (K and V) row to the next: n_q_heads*head_dim
+ *   (n_kv_heads*head_dim) for separate tensors, the fused QKV width for both
+ *   when k_proj/v_proj point into the same rows as q_proj; element type
+ *   cfg->dtype, each stride times the element size a multiple of 16 bytes
+ *   (HGA_ERR_INVALID_ARG otherwise, or if a stride is below its row width);
+ *   Q and K are rotated (rotate-half RoPE: for i < d/2, theta_i =
+ *   base^(-2i/d), angle p*theta_i at the global position p; rope_base = 0
+ *   skips the rotation), V is not;
+ *   q_out [batch, n_q_heads, s_len, head_dim] receives Q; k, v (the
+ *   whole-context buffers) receive rows [q_begin, q_begin + s_len);
+ *   gsum, bsum receive the segment's group and block summaries and qsum
+ *   [batch, n_kv_heads, ctx_cap/64, head_dim] float32 its block mean queries
+ *   (mean over 64 tokens and the G heads), all of the stored (rounded) values.
+ * One launch; it replaces hga_build_summaries and, with
+ * hga_route_summarized, every read of Q and K by the routing.
+ */
+HGA_API hga_status_t hga_prepare_segment(const hga_config_t* cfg, const void* q_proj,
+                                         const void* k_proj, const void* v_proj,
+                                         int64_t q_row_stride, int64_t kv_row_stride,
+                                         int64_t q_begin, int32_t s_len,
+                                         int64_t ctx_cap, float rope_base, void* q_out, void* k,
+                                         void* v, float* gsum, float* bsum, float* qsum,
+                                         void* stream);
+
+/*
+ * hga_route (causal = 0) or hga_route_causal (causal = 1) from the resident
+ * summaries alone: query block j (global block J) is routed with row J
+ * (causal: J - 1) of qsum, which hga_prepare_segment or
+ * hga_build_query_summaries wrote; Q is not read.  Results equal those calls'
+ * when qsum holds the block means they form.  workspace as
+ * hga_route_workspace_size().
+ */
+HGA_API hga_status_t hga_route_summarized(const hga_config_t* cfg, int64_t q_begin,
+                                          int32_t s_len, int64_t ctx_cap, const float* bsum,
+                                          const float* gsum, const float* qsum, int32_t causal,
+                                          int32_t* sel_blk, int32_t* sel_grp, void* workspace,
+                                          size_t ws_bytes, void* stream);
+
+/*
  * Decode -- one new token per sequence [A] ("HGA can also be used for
  * retrieval and generation"), routed and attended as in [B] with the query
  * block reduced to that one token.  For sequence b the token sits at global
@@ -412,7 +457,8 @@ typedef enum {
   HGA_K_ROUTE_FUSED = 12,
   HGA_K_DECODE = 13,
   HGA_K_QSUM = 14,
-  HGA_K_COUNT = 15
+  HGA_K_PREPARE = 15,
+  HGA_K_COUNT = 16
 } hga_kernel_kind_t;
 
 /* Name of a kernel kind ("attn_fwd_simt", ...). */

@@ -145,7 +145,7 @@ def ctype_of(c_type):
         return ctypes.c_char_p if t == "char*" else ctypes.c_void_p
     return {"int64_t": ctypes.c_int64, "int32_t": ctypes.c_int32, "size_t": ctypes.c_size_t,
             "int": ctypes.c_int, "uint32_t": ctypes.c_uint32, "uint64_t": ctypes.c_uint64,
-            "hga_status_t": ctypes.c_int, "void": None}[t]
+            "hga_status_t": ctypes.c_int, "float": ctypes.c_float, "void": None}[t]
 
 
 def test_binding_signatures_match_the_header():
@@ -174,3 +174,29 @@ def test_decode_host_argument_checks():
     assert status_of(hga.hga_decode, c, FAKE, FAKE, FAKE, 16380, *args[4:]) == 1
     assert status_of(hga.hga_decode, c, FAKE, FAKE, FAKE, 16384, 0, *args[5:]) == 1
     assert status_of(hga.hga_decode, c, *args[:9], FAKE + 8, FAKE, 0) == 1
+
+
+def test_prepare_and_summarized_route_host_checks():
+    c = cfg()
+    a = (FAKE, FAKE, FAKE)
+    outs = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0)
+    # strides below the row widths, or not a multiple of 16 bytes
+    assert status_of(hga.hga_prepare_segment, c, *a, 32 * 128 - 8, 8 * 128, 0, 2048, 16384,
+                     1e6, *outs) == 1
+    assert status_of(hga.hga_prepare_segment, c, *a, 32 * 128, 8 * 128 - 8, 0, 2048, 16384,
+                     1e6, *outs) == 1
+    assert status_of(hga.hga_prepare_segment, c, *a, 32 * 128 + 4, 8 * 128, 0, 2048, 16384,
+                     1e6, *outs) == 1
+    # a negative RoPE base; a segment past the context
+    assert status_of(hga.hga_prepare_segment, c, *a, 4096, 1024, 0, 2048, 16384, -1.0,
+                     *outs) == 1
+    assert status_of(hga.hga_prepare_segment, c, *a, 4096, 1024, 15360, 2048, 16384, 1e6,
+                     *outs) == 1
+    # routing from summaries needs the block means, and causal is 0 or 1
+    need = hga.hga_route_workspace_size(c, 2048, 14336)
+    assert status_of(hga.hga_route_summarized, c, 14336, 2048, 16384, FAKE, FAKE, None, 0, None,
+                     FAKE, FAKE, need, 0) == 1
+    assert status_of(hga.hga_route_summarized, c, 14336, 2048, 16384, FAKE, FAKE, FAKE, 2, None,
+                     FAKE, FAKE, need, 0) == 1
+    assert status_of(hga.hga_route_causal, c, FAKE, 14336, 2048, 16384, FAKE, FAKE, FAKE, None,
+                     FAKE, FAKE, need - 256, 0) == 6
