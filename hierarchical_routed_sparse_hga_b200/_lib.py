@@ -18,7 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libhga.so")
 
 HGA_OK, HGA_ERR_INVALID_ARG, HGA_ERR_UNSUPPORTED, HGA_ERR_CUDA, HGA_ERR_TIMEOUT, \
-    HGA_ERR_DEVICE_CHECK, HGA_ERR_WORKSPACE = range(7)
+    HGA_ERR_DEVICE_CHECK, HGA_ERR_WORKSPACE, HGA_ERR_IO = range(8)
 HGA_F32, HGA_BF16 = 0, 1
 HGA_FLAG_SIMT = 1
 
@@ -32,7 +32,8 @@ EXPORTS = ("hga_version", "hga_status_string", "hga_build_summaries",
            "hga_build_summaries_seg",
            "hga_tier_stage_rows", "hga_tier_workspace_size", "hga_tier_gather",
            "hga_tier_append", "hga_decode", "hga_build_query_summaries",
-           "hga_route_causal", "hga_prepare_segment", "hga_route_summarized")
+           "hga_route_causal", "hga_prepare_segment", "hga_route_summarized",
+           "hga_tier_plan", "hga_tier_read_groups", "hga_tier_write_segment")
 HGA_NOALLOC_SCRATCH_BYTES = 4 << 20
 HGA_K_COUNT = 16
 
@@ -123,6 +124,11 @@ def load() -> ctypes.CDLL:
                                                P, P, P, P, P, P, P]),
         "hga_route_summarized": (ctypes.c_int, [CFG, I64, I32, I64, P, P, P, I32, P, P, P, SZ,
                                                 P]),
+        "hga_tier_plan": (ctypes.c_int, [CFG, I64, I32, P, I64, P, P, P, I64, P]),
+        "hga_tier_read_groups": (ctypes.c_int, [CFG, ctypes.c_int, ctypes.c_int, I64, P, P, I64,
+                                                P, P, I64, I32]),
+        "hga_tier_write_segment": (ctypes.c_int, [CFG, ctypes.c_int, ctypes.c_int, I64, I64,
+                                                  I32, P, P, I64, I32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -273,6 +279,43 @@ def hga_route_summarized(cfg: Config, q_begin, s_len, ctx_cap, bsum, gsum, qsum,
         ctypes.byref(c), q_begin, s_len, ctx_cap, _ptr(bsum), _ptr(gsum), _ptr(qsum),
         int(causal), _ptr(sel_blk), _ptr(sel_grp), _ptr(workspace), ws_bytes,
         _stream(stream)))
+
+
+def _hptr(x):
+    """Host memory (numpy array, CPU tensor or raw address) for the file tier."""
+    if x is None or isinstance(x, int):
+        return x
+    if hasattr(x, "ctypes"):
+        if not x.flags["C_CONTIGUOUS"]:
+            raise ValueError("the file tier takes contiguous host arrays")
+        return x.ctypes.data
+    if x.is_cuda or not x.is_contiguous():
+        raise ValueError("the file tier takes contiguous host tensors")
+    return x.data_ptr()
+
+
+def hga_tier_plan(cfg: Config, q_begin, s_len, sel_grp, stage_cap, sel_stage, slot_group,
+                  n_unique, slot_cap, stream=None):
+    c = cfg.c()
+    _check("hga_tier_plan", load().hga_tier_plan(
+        ctypes.byref(c), q_begin, s_len, _ptr(sel_grp), stage_cap, _ptr(sel_stage),
+        _ptr(slot_group), _ptr(n_unique), slot_cap, _stream(stream)))
+
+
+def hga_tier_read_groups(cfg: Config, fd_k, fd_v, ctx_cap, slot_group, n_unique, slot_cap,
+                         k_stage_host, v_stage_host, stage_cap, n_threads=8):
+    c = cfg.c()
+    _check("hga_tier_read_groups", load().hga_tier_read_groups(
+        ctypes.byref(c), fd_k, fd_v, ctx_cap, _hptr(slot_group), _hptr(n_unique), slot_cap,
+        _hptr(k_stage_host), _hptr(v_stage_host), stage_cap, n_threads))
+
+
+def hga_tier_write_segment(cfg: Config, fd_k, fd_v, ctx_cap, q_begin, s_len, k_seg_host,
+                           v_seg_host, seg_rows, n_threads=8):
+    c = cfg.c()
+    _check("hga_tier_write_segment", load().hga_tier_write_segment(
+        ctypes.byref(c), fd_k, fd_v, ctx_cap, q_begin, s_len, _hptr(k_seg_host),
+        _hptr(v_seg_host), seg_rows, n_threads))
 
 
 def hga_route_noalloc(cfg: Config, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp,

@@ -31,7 +31,7 @@ def nvcc() -> str:
 
 def sources():
     return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC)
-                  if f.endswith((".cu", ".cuh")))
+                  if f.endswith((".cu", ".cuh", ".h")))
 
 
 def up_to_date() -> bool:

@@ -23,6 +23,7 @@
 #include "tier.cuh"
 #include "decode.cuh"
 #include "prepare.cuh"
+#include "file_tier.h"
 #include "trace.cuh"
 
 using namespace hga;
@@ -300,6 +301,7 @@ const char* hga_status_string(hga_status_t s) {
     case HGA_ERR_TIMEOUT: return "device wait timed out";
     case HGA_ERR_DEVICE_CHECK: return "device-side index check failed";
     case HGA_ERR_WORKSPACE: return "workspace too small";
+    case HGA_ERR_IO: return "tier file read or write failed";
   }
   return "unknown status";
 }
@@ -1034,4 +1036,90 @@ extern "C" hga_status_t hga_route_summarized(const hga_config_t* cfg, int64_t q_
   return route_impl(cfg, nullptr, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp,
                     workspace, ws_bytes, nullptr, 0, static_cast<cudaStream_t>(stream), qsum,
                     causal);
+}
+
+extern "C" hga_status_t hga_tier_plan(const hga_config_t* cfg, int64_t q_begin, int32_t s_len,
+                                      const int32_t* sel_grp, int64_t stage_cap,
+                                      int32_t* sel_stage, int32_t* slot_group,
+                                      int32_t* n_unique, int64_t slot_cap, void* stream) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if (q_begin < 0 || q_begin % kBlock || s_len <= 0 || s_len % kQBlock || s_len > kMaxSegment)
+    return HGA_ERR_INVALID_ARG;
+  if (!sel_grp || !sel_stage || !slot_group || !n_unique || !aligned16(sel_grp) ||
+      !aligned16(sel_stage) || !aligned16(slot_group) || !aligned16(n_unique))
+    return HGA_ERR_INVALID_ARG;
+  if (stage_cap % kBlock || stage_cap < hga_tier_stage_rows(cfg, q_begin, s_len) ||
+      slot_cap < std::max<int64_t>(tier_slot_cap(cfg, q_begin, s_len), 1))
+    return HGA_ERR_INVALID_ARG;
+  const int n_qb = s_len / kQBlock;
+  const int64_t n_words = (q_begin / kGroup + 31) / 32;
+  const size_t sm = size_t(n_words > 0 ? n_words : 1) * 8;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
+    hga_status_t e = ensure_smem(reinterpret_cast<const void*>(&tier_dedup_kernel<D>), sm);
+    if (e != HGA_OK) return e;
+    dim3 g1(cfg->n_kv_heads, cfg->batch);
+    return traced_launch(HGA_K_TIER_DEDUP, s, [&] {
+      tier_dedup_kernel<D><<<g1, kTierThreads, sm, s>>>(sel_grp, cfg->n_kv_heads, n_qb,
+                                                        cfg->topk_groups, q_begin, stage_cap,
+                                                        s_len, sel_stage, slot_group, n_unique,
+                                                        slot_cap);
+    });
+  });
+}
+
+extern "C" hga_status_t hga_tier_read_groups(const hga_config_t* cfg, int fd_k, int fd_v,
+                                             int64_t ctx_cap, const int32_t* slot_group,
+                                             const int32_t* n_unique, int64_t slot_cap,
+                                             void* k_stage_host, void* v_stage_host,
+                                             int64_t stage_cap, int32_t n_threads) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if (fd_k < 0 || fd_v < 0 || !slot_group || !n_unique || !k_stage_host || !v_stage_host ||
+      ctx_cap <= 0 || ctx_cap % kBlock || slot_cap < 1 || stage_cap < 0 || n_threads < 1)
+    return HGA_ERR_INVALID_ARG;
+  const int64_t row = int64_t(cfg->head_dim) * (cfg->dtype == HGA_BF16 ? 2 : 4);
+  const int64_t heads = int64_t(cfg->batch) * cfg->n_kv_heads;
+  std::vector<file_tier::Run> runs;
+  for (int64_t hd = 0; hd < heads; ++hd) {
+    const int32_t U = n_unique[hd];
+    if (U < 0 || U > slot_cap || int64_t(U) * kGroup > stage_cap) return HGA_ERR_INVALID_ARG;
+    const int32_t* sg = slot_group + hd * slot_cap;
+    for (int32_t u = 0; u < U;) {
+      const int32_t g0 = sg[u];
+      if (g0 < 0 || int64_t(g0 + 1) * kGroup > ctx_cap) return HGA_ERR_INVALID_ARG;
+      int32_t n = 1;  // groups g0, g0+1, ... in slots u, u+1, ...: one transfer
+      while (u + n < U && sg[u + n] == g0 + n) ++n;
+      runs.push_back({(hd * ctx_cap + int64_t(g0) * kGroup) * row,
+                      (hd * stage_cap + int64_t(u) * kGroup) * row, int64_t(n) * kGroup * row});
+      u += n;
+    }
+  }
+  return file_tier::transfer<false>(runs, fd_k, fd_v, static_cast<char*>(k_stage_host),
+                                    static_cast<char*>(v_stage_host), n_threads)
+             ? HGA_OK
+             : HGA_ERR_IO;
+}
+
+extern "C" hga_status_t hga_tier_write_segment(const hga_config_t* cfg, int fd_k, int fd_v,
+                                               int64_t ctx_cap, int64_t q_begin, int32_t s_len,
+                                               const void* k_seg_host, const void* v_seg_host,
+                                               int64_t seg_rows, int32_t n_threads) {
+  hga_status_t st = check_cfg(cfg);
+  if (st != HGA_OK) return st;
+  if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
+  if (fd_k < 0 || fd_v < 0 || !k_seg_host || !v_seg_host || seg_rows < s_len || n_threads < 1)
+    return HGA_ERR_INVALID_ARG;
+  const int64_t row = int64_t(cfg->head_dim) * (cfg->dtype == HGA_BF16 ? 2 : 4);
+  const int64_t heads = int64_t(cfg->batch) * cfg->n_kv_heads;
+  std::vector<file_tier::Run> runs;
+  for (int64_t hd = 0; hd < heads; ++hd)
+    runs.push_back({(hd * ctx_cap + q_begin) * row, hd * seg_rows * row, int64_t(s_len) * row});
+  return file_tier::transfer<true>(runs, fd_k, fd_v,
+                                   const_cast<char*>(static_cast<const char*>(k_seg_host)),
+                                   const_cast<char*>(static_cast<const char*>(v_seg_host)),
+                                   n_threads)
+             ? HGA_OK
+             : HGA_ERR_IO;
 }

@@ -256,3 +256,69 @@ class HgaTieredLayer:
                               self.bwd_ws, stream=stream)
         if append:
             self.append_history(q_begin, stream)
+
+
+class HgaFileTieredLayer(HgaTieredLayer):
+    """The host tier with the history K/V in files (NVMe) instead of pinned
+    RAM.  Per segment the selected history groups are planned on the GPU
+    (hga_tier_plan), their list comes back to the host, the groups are read
+    from the files into pinned staging buffers laid out like the device
+    staging (hga_tier_read_groups, a pool of reader threads) and copied up
+    in one 2-D copy per tensor; the finished segment's K/V are written to the
+    files (hga_tier_write_segment).  fd_k / fd_v are open file descriptors
+    (read and write) of files of batch * n_kv_heads * ctx_cap * head_dim
+    elements; the caller owns them."""
+
+    def __init__(self, cfg: Config, ctx_cap: int, seg_len: int, fd_k: int, fd_v: int,
+                 device="cuda", n_threads: int = 8):
+        super().__init__(cfg, ctx_cap, seg_len, device=device,
+                         k_host=torch.empty(0), v_host=torch.empty(0))
+        self.fd_k, self.fd_v, self.n_threads = fd_k, fd_v, n_threads
+        B, Hkv, d = cfg.batch, cfg.n_kv_heads, cfg.head_dim
+        dt = _TORCH_DTYPE[cfg.dtype]
+        self.slot_cap = max(1, min((seg_len // 64) * cfg.topk_groups, (ctx_cap - seg_len) // 8))
+        self.slot_group = torch.empty((B, Hkv, self.slot_cap), dtype=torch.int32,
+                                      device=self.device)
+        self.slot_group_host = torch.empty_like(self.slot_group, device="cpu").pin_memory()
+        self.n_unique_host = torch.empty((B, Hkv), dtype=torch.int32).pin_memory()
+        hist_rows = self.stage_cap - seg_len
+        self.k_stage_host = torch.empty((B, Hkv, hist_rows, d), dtype=dt).pin_memory()
+        self.v_stage_host = torch.empty_like(self.k_stage_host).pin_memory()
+        self.k_seg_host = torch.empty((B, Hkv, seg_len, d), dtype=dt).pin_memory()
+        self.v_seg_host = torch.empty_like(self.k_seg_host).pin_memory()
+        self.bytes_read = 0
+
+    def gather(self, q_begin: int, stream=None):
+        if q_begin == 0:
+            return _lib.hga_tier_plan(self.cfg, q_begin, self.seg_len, self.sel_grp,
+                                      self.stage_cap, self.sel_stage, self.slot_group,
+                                      self.n_unique, self.slot_cap, stream)
+        s = torch.cuda.current_stream(self.device) if stream is None else stream
+        _lib.hga_tier_plan(self.cfg, q_begin, self.seg_len, self.sel_grp, self.stage_cap,
+                           self.sel_stage, self.slot_group, self.n_unique, self.slot_cap, s)
+        with torch.cuda.stream(s):
+            self.slot_group_host.copy_(self.slot_group, non_blocking=True)
+            self.n_unique_host.copy_(self.n_unique, non_blocking=True)
+        s.synchronize()
+        hist_rows = self.stage_cap - self.seg_len
+        _lib.hga_tier_read_groups(self.cfg, self.fd_k, self.fd_v, self.ctx_cap,
+                                  self.slot_group_host, self.n_unique_host, self.slot_cap,
+                                  self.k_stage_host, self.v_stage_host, hist_rows,
+                                  self.n_threads)
+        rows = 8 * int(self.n_unique_host.max())
+        row_bytes = self.cfg.head_dim * self.k_stage.element_size()
+        self.bytes_read += 2 * int(self.n_unique_host.sum()) * 8 * row_bytes
+        if rows:
+            with torch.cuda.stream(s):
+                self.k_stage[:, :, :rows].copy_(self.k_stage_host[:, :, :rows], non_blocking=True)
+                self.v_stage[:, :, :rows].copy_(self.v_stage_host[:, :, :rows], non_blocking=True)
+
+    def append_history(self, q_begin: int, stream=None):
+        s = torch.cuda.current_stream(self.device) if stream is None else stream
+        with torch.cuda.stream(s):
+            self.k_seg_host.copy_(self.active_k(), non_blocking=True)
+            self.v_seg_host.copy_(self.active_v(), non_blocking=True)
+        s.synchronize()
+        _lib.hga_tier_write_segment(self.cfg, self.fd_k, self.fd_v, self.ctx_cap, q_begin,
+                                    self.seg_len, self.k_seg_host, self.v_seg_host,
+                                    self.seg_len, self.n_threads)

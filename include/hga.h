@@ -80,7 +80,8 @@ typedef enum {
   HGA_ERR_CUDA = 3,
   HGA_ERR_TIMEOUT = 4,
   HGA_ERR_DEVICE_CHECK = 5,
-  HGA_ERR_WORKSPACE = 6
+  HGA_ERR_WORKSPACE = 6,
+  HGA_ERR_IO = 7
 } hga_status_t;
 
 typedef enum { HGA_F32 = 0, HGA_BF16 = 1 } hga_dtype_t;
@@ -417,6 +418,52 @@ HGA_API hga_status_t hga_decode(const hga_config_t* cfg, const void* q, const vo
                                 const void* v, int64_t ctx_cap, const int64_t* pos,
                                 const float* bsum, const float* gsum, int32_t* sel_blk,
                                 int32_t* sel_grp, void* o, float* lse, void* stream);
+
+/*
+ * Step a7, third tier: history K/V in files on NVMe ([A]: older KV is
+ * detached into RAM or NVMe; seventnews, section "意义何在": NVMe-backed
+ * tiered storage).  A K or V file holds the whole context in the layout of
+ * the device buffers, [batch, n_kv_heads, ctx_cap, head_dim] elements, so a
+ * group is one contiguous run of 8*head_dim elements.  Per segment:
+ *
+ * hga_tier_plan (device, asynchronous): the planning half of
+ *   hga_tier_gather: sel_stage receives the selection in staging indices (as
+ *   there); slot_group ([batch, n_kv_heads, slot_cap] int32) the distinct
+ *   selected history groups of each head in ascending order, n_unique
+ *   ([batch, n_kv_heads] int32) their number.  slot_cap >=
+ *   min(s_len/64 * topk_groups, q_begin/8); stage_cap as for hga_tier_gather.
+ *
+ * hga_tier_read_groups (host, synchronous): with slot_group and n_unique
+ *   copied to host memory, reads every listed group of every head from the
+ *   files fd_k / fd_v into host staging buffers laid out like the device
+ *   staging ([batch, n_kv_heads, stage_cap, head_dim]; slot u at rows
+ *   [8u, 8u+8)), one pread per run of consecutive groups, on n_threads
+ *   threads.  The caller then copies rows [0, 8*n_unique) of each head to
+ *   the device staging (one 2-D copy per tensor).  HGA_ERR_IO if a read fails
+ *   or ends early; HGA_ERR_INVALID_ARG for a group or count out of range.
+ *
+ * hga_tier_write_segment (host, synchronous): writes the segment's rows
+ *   [q_begin, q_begin + s_len) of every head from host buffers ([batch,
+ *   n_kv_heads, seg_rows, head_dim], the segment at rows [0, s_len)) into the
+ *   files, one pwrite per head and tensor on n_threads threads.
+ *
+ * The file descriptors are the caller's (opened for reading / writing; with
+ * O_DIRECT the buffers, offsets and sizes must meet the device's alignment:
+ * groups are 2 KiB at bf16, d = 128).
+ */
+HGA_API hga_status_t hga_tier_plan(const hga_config_t* cfg, int64_t q_begin, int32_t s_len,
+                                   const int32_t* sel_grp, int64_t stage_cap, int32_t* sel_stage,
+                                   int32_t* slot_group, int32_t* n_unique, int64_t slot_cap,
+                                   void* stream);
+HGA_API hga_status_t hga_tier_read_groups(const hga_config_t* cfg, int fd_k, int fd_v,
+                                          int64_t ctx_cap, const int32_t* slot_group,
+                                          const int32_t* n_unique, int64_t slot_cap,
+                                          void* k_stage_host, void* v_stage_host,
+                                          int64_t stage_cap, int32_t n_threads);
+HGA_API hga_status_t hga_tier_write_segment(const hga_config_t* cfg, int fd_k, int fd_v,
+                                            int64_t ctx_cap, int64_t q_begin, int32_t s_len,
+                                            const void* k_seg_host, const void* v_seg_host,
+                                            int64_t seg_rows, int32_t n_threads);
 
 /*
  * Reads and clears the calling device's latched device-side status
