@@ -230,7 +230,7 @@ def segment_pairs(w, sel_grp, q_begin):
     return all_pairs, act_pairs
 
 
-def kernel_work(name, w, sels, unique_groups=None):
+def kernel_work(name, w, sels, unique_groups=None, from_summaries=False):
     """Algorithmic work of ALL launches of kernel `name` over one step.
     Returns (amount, unit, bound): FLOP for contractions, bytes otherwise."""
     unique_groups = unique_groups or {}
@@ -262,10 +262,11 @@ def kernel_work(name, w, sels, unique_groups=None):
         elif name == "route_select":
             tot += B * Hkv * sum(J * 4 + 8 * k * d * 4 + d * 4 + 4 * (w.topk_blocks + w.topk_groups)
                                  for J, k in zip(Js, kb))
-        elif name == "route_fused":
-            # Q once, each block summary of the head once, the kept blocks'
-            # group summaries, the two selections written
-            tot += B * Hq * S * d * el + B * Hkv * (
+        elif name == "route_cluster":
+            # Q once (unless q-bar comes from the resident block means), each
+            # block summary of the head once, the kept blocks' group
+            # summaries, the two selections written
+            tot += (0 if from_summaries else B * Hq * S * d * el) + B * Hkv * (
                 (own0 + n_qb - 1) * d * 4
                 + sum(8 * k * d * 4 + 4 * (w.topk_blocks + w.topk_groups) for k in kb))
         elif name == "tier_copy":
@@ -976,6 +977,62 @@ def run_extras(device, steps, pk, run=None):
                     "frac_of_hbm": round(route_bytes / (route_us / 1e6) / 1e9 / pk["hbm"], 4)},
         "kernels": kernels}
     del layer, k, v, qs
+    torch.cuda.empty_cache()
+
+    # -- the file (NVMe) tier on the batched tiered workload -------------------
+    from hierarchical_routed_sparse_hga_b200 import HgaFileTieredLayer
+    wt = synth.workloads()["qwen3_tiered_b8_32k"]
+    cfg = Config(wt.batch, wt.n_q_heads, wt.n_kv_heads, wt.head_dim, wt.topk_blocks,
+                 wt.topk_groups, HGA_BF16)
+    k, v, qs, dos = synth.device_inputs(wt, device)
+    tmp = tempfile.mkdtemp(prefix="hga_tier_")
+    nbytes = k.numel() * k.element_size()
+    fds = []
+    for name in ("k.bin", "v.bin"):
+        fd = os.open(os.path.join(tmp, name), os.O_RDWR | os.O_CREAT, 0o600)
+        os.ftruncate(fd, nbytes)
+        fds.append(fd)
+    try:
+        tier = HgaFileTieredLayer(cfg, wt.ctx_len, wt.seg_len, fds[0], fds[1], device=device,
+                                  n_threads=16)
+        S = wt.seg_len
+
+        def tstep():
+            for i, s0 in enumerate(wt.segments()):
+                tier.active_k().copy_(k[:, :, s0:s0 + S])
+                tier.active_v().copy_(v[:, :, s0:s0 + S])
+                tier.segment(qs[i], s0, dos[i])
+
+        tstep()
+        tier.bytes_read = 0
+        t_steps = 2
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(t_steps):
+            tstep()
+        e1.record()
+        torch.cuda.synchronize(device)
+        t_ms = e0.elapsed_time(e1) / t_steps
+        read = tier.bytes_read / t_steps
+        out["file_tier"] = {
+            "workload": wt.name, "batch": wt.batch, "seq_len": wt.ctx_len,
+            "segments": len(wt.segments()),
+            "tokens_per_s": round(wt.batch * wt.ctx_len / (t_ms / 1e3), 1),
+            "ms_per_step": round(t_ms, 2), "file_bytes_read_per_step": int(read),
+            "file_read_gbs_over_step": round(read / (t_ms / 1e3) / 1e9, 2),
+            "timing": "CUDA events around whole steps; each segment's planned groups are read "
+                      "from the files by 16 host threads (pread) between the GPU phases; the "
+                      "files were just written, so the reads may be served by the page cache",
+        }
+        del tier
+    finally:
+        for fd in fds:
+            os.close(fd)
+        for name in ("k.bin", "v.bin"):
+            os.unlink(os.path.join(tmp, name))
+        os.rmdir(tmp)
+    del k, v, qs, dos
     torch.cuda.empty_cache()
 
     # -- decode ------------------------------------------------------------

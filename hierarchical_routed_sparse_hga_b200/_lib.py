@@ -22,7 +22,7 @@ HGA_OK, HGA_ERR_INVALID_ARG, HGA_ERR_UNSUPPORTED, HGA_ERR_CUDA, HGA_ERR_TIMEOUT,
 HGA_F32, HGA_BF16 = 0, 1
 HGA_FLAG_SIMT = 1
 
-EXPORTS = ("hga_version", "hga_status_string", "hga_build_summaries",
+EXPORTS = ("hga_version", "hga_status_string", "hga_last_cuda_error", "hga_build_summaries",
            "hga_route_workspace_size", "hga_route", "hga_attn_fwd",
            "hga_attn_bwd_workspace_size", "hga_attn_bwd", "hga_attn_fwd_bwd",
            "hga_segment_workspace_size", "hga_segment_fwd_bwd",
@@ -88,6 +88,7 @@ def load() -> ctypes.CDLL:
     sig = {
         "hga_version": (ctypes.c_char_p, []),
         "hga_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "hga_last_cuda_error": (ctypes.c_char_p, []),
         "hga_build_summaries": (ctypes.c_int, [CFG, P, I64, I64, I64, P, P, P]),
         "hga_route_workspace_size": (SZ, [CFG, I32, I64]),
         "hga_route": (ctypes.c_int, [CFG, P, I64, I32, I64, P, P, P, P, P, SZ, P]),
@@ -160,7 +161,10 @@ def _stream(stream):
 
 def _check(fn: str, status: int):
     if status != HGA_OK:
-        raise HgaError(fn, status, load().hga_status_string(status).decode())
+        text = load().hga_status_string(status).decode()
+        if status == HGA_ERR_CUDA:
+            text += f" ({load().hga_last_cuda_error().decode()})"
+        raise HgaError(fn, status, text)
 
 
 def _nbytes(t):
@@ -170,6 +174,10 @@ def _nbytes(t):
 # ----------------------------------------------------------------------------
 # entry points (same names as the C ABI)
 # ----------------------------------------------------------------------------
+
+def hga_last_cuda_error() -> str:
+    return load().hga_last_cuda_error().decode()
+
 
 def hga_version() -> str:
     return load().hga_version().decode()

@@ -162,7 +162,9 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1)
   const int n_own = int((p - own0) / kGroup) + 1;  // own-block units (the last one partial)
   const T* kh = k + head * ctx_cap * D;
   const T* vh = v + head * ctx_cap * D;
-  __syncthreads();  // barriers initialised
+  // barriers initialised, and every CTA of the cluster running before any
+  // touches a peer's shared memory
+  cluster.sync();
 
   // 0. this CTA's own-block units (u = rank + s*nc < n_own) start loading;
   //    they are the first slots, all inside the first round

@@ -22,11 +22,20 @@ namespace hga {
 
 constexpr int kPrepThreads = 256;
 
+// (cos, sin) of token t, frequency i = 8c + k (lane c of a row holds
+// frequencies 8c .. 8c+7) at cs[t][k * LANES + c]: the lanes of a warp (rows
+// t .. t+R-1, all c) read one k at a time; the row stride (LANES*8 + pad
+// entries) puts the rows on different bank halves, so a read takes the two
+// wavefronts its 256 bytes need.  The key tile and the query partials have
+// one float of padding per row for the same reason.
 template <int D>
 struct PrepShared {
-  float2 cs[kQBlock][D / 2];   // (cos, sin) per token of the block and frequency
-  float kt[kQBlock][D];        // the block's stored keys, as float
-  float qp[kPrepThreads / (D / 16)][D];  // per row slot: partial sums of the stored queries
+  static constexpr int kLanes = D / 16;
+  static constexpr int kCsStride = kLanes * 8 + (kLanes == 8 ? 8 : 4);
+  float2 cs[kQBlock][kCsStride];
+  double theta[D / 2];          // base^(-2i/d)
+  float kt[kQBlock][D + 1];     // the block's stored keys, as float
+  float qp[kPrepThreads / kLanes][D + 1];  // per row slot: partial sums of the stored queries
 };
 
 // grid (s_len/64, n_kv_heads, batch), kPrepThreads threads, dynamic shared
@@ -51,15 +60,16 @@ __global__ void __launch_bounds__(kPrepThreads)
 
   // (cos, sin) of the 64 tokens' angles, reduced modulo 2 pi in double
   if (rotate) {
+    for (int i = tid; i < HALF; i += kPrepThreads) sh.theta[i] = exp2(-(2.0 * i / D) * log2_base);
+    __syncthreads();
     constexpr double kTwoPi = 6.283185307179586476925286766559;
     for (int idx = tid; idx < kQBlock * HALF; idx += kPrepThreads) {
       const int t = idx / HALF, i = idx % HALF;
-      const double theta = exp2(-(2.0 * i / D) * log2_base);
-      const double ang = double(q_begin + int64_t(j) * kQBlock + t) * theta;
+      const double ang = double(q_begin + int64_t(j) * kQBlock + t) * sh.theta[i];
       const double red = fma(-rint(ang * (1.0 / kTwoPi)), kTwoPi, ang);
       float s, co;
       sincosf(float(red), &s, &co);
-      sh.cs[t][i] = make_float2(co, s);
+      sh.cs[t][(i % 8) * LANES + i / 8] = make_float2(co, s);
     }
   }
   pdl_wait();
@@ -95,7 +105,7 @@ __global__ void __launch_bounds__(kPrepThreads)
       if (kind <= G && rotate) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float2 cs = sh.cs[t][8 * c + i];
+          const float2 cs = sh.cs[t][i * LANES + c];
           y1[i] = x1[u][i] * cs.x - x2[u][i] * cs.y;
           y2[i] = x2[u][i] * cs.x + x1[u][i] * cs.y;
         }

@@ -35,6 +35,12 @@ inline Tracer& tracer() {
   return t;
 }
 
+// The CUDA error behind the last HGA_ERR_CUDA a launch returned (per thread).
+inline cudaError_t& last_launch_error() {
+  static thread_local cudaError_t e = cudaSuccess;
+  return e;
+}
+
 inline cudaError_t record(cudaEvent_t ev, cudaStream_t s) {
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return cudaErrorUnknown;
@@ -59,14 +65,19 @@ hga_status_t traced_launch(int kind, cudaStream_t s, F&& launch) {
   }
   if (slot && record(slot->begin, s) != cudaSuccess) return HGA_ERR_CUDA;
   if constexpr (std::is_same_v<decltype(launch()), cudaError_t>) {
-    if (launch() != cudaSuccess) {
+    const cudaError_t e = launch();
+    if (e != cudaSuccess) {
       cudaGetLastError();
+      last_launch_error() = e;
       return HGA_ERR_CUDA;
     }
   } else {
     launch();
   }
-  if (cudaGetLastError() != cudaSuccess) return HGA_ERR_CUDA;
+  if (const cudaError_t e = cudaGetLastError(); e != cudaSuccess) {
+    last_launch_error() = e;
+    return HGA_ERR_CUDA;
+  }
   if (slot && record(slot->end, s) != cudaSuccess) return HGA_ERR_CUDA;
   return HGA_OK;
 }

@@ -115,6 +115,10 @@ HGA_API const char* hga_version(void);
 /* Human-readable name of a status code. */
 HGA_API const char* hga_status_string(hga_status_t status);
 
+/* Name of the CUDA error behind the last HGA_ERR_CUDA a kernel launch of this
+ * library returned on the calling thread ("cudaSuccess" if none). */
+HGA_API const char* hga_last_cuda_error(void);
+
 /*
  * Step a1 -- summaries [B], [C].  For tokens [t_begin, t_end) of K:
  *   gsum[b,h,g] = mean of keys 8g .. 8g+7      (g = t_begin/8 .. t_end/8-1)
@@ -501,7 +505,7 @@ typedef enum {
   HGA_K_BWD_DKDV_TC = 9,
   HGA_K_TIER_DEDUP = 10,
   HGA_K_TIER_COPY = 11,
-  HGA_K_ROUTE_FUSED = 12,
+  HGA_K_ROUTE_CLUSTER = 12,
   HGA_K_DECODE = 13,
   HGA_K_QSUM = 14,
   HGA_K_PREPARE = 15,
