@@ -244,6 +244,12 @@ def kernel_work(name, w, sels, unique_groups=None, from_summaries=False):
         own0 = q_begin // 64
         Js = [own0 + j for j in range(n_qb)]
         kb = [min(w.topk_blocks, J) for J in Js]
+        # each routing kernel counts only the segments whose path it runs:
+        # one launch up to 512 candidate blocks, three kernels beyond
+        one_launch = own0 + n_qb - 1 <= 512
+        if (name == "route_fused" and not one_launch) or (
+                name in ("route_qmean", "route_block_score", "route_select") and one_launch):
+            continue
         if name.startswith("attn_fwd"):
             tot += 4 * d * pairs
         elif name.startswith("attn_bwd_dq"):
@@ -262,7 +268,7 @@ def kernel_work(name, w, sels, unique_groups=None, from_summaries=False):
         elif name == "route_select":
             tot += B * Hkv * sum(J * 4 + 8 * k * d * 4 + d * 4 + 4 * (w.topk_blocks + w.topk_groups)
                                  for J, k in zip(Js, kb))
-        elif name == "route_cluster":
+        elif name == "route_fused":
             # Q once (unless q-bar comes from the resident block means), each
             # block summary of the head once, the kept blocks' group
             # summaries, the two selections written

@@ -10,7 +10,6 @@
 #include <atomic>
 #include <initializer_list>
 #include <map>
-#include <tuple>
 #include <mutex>
 #include <utility>
 
@@ -363,101 +362,6 @@ size_t hga_route_workspace_size(const hga_config_t* cfg, int32_t s_len, int64_t 
 // The routing of hga_route.  With `done`, a fused routing launch also stores
 // `token` into done[item] once item's selections are written (chained
 // segment call); the three-launch path ignores it.
-// ---- routing launch plan (C++ helpers inside the C-linkage section) ----
-extern "C++" {
-// candidate blocks per CTA of the cluster routing
-int64_t route_cluster_share(int64_t q_begin, int32_t s_len, int C) {
-  const int64_t j_max = q_begin / kBlock + s_len / kQBlock - 1;
-  return (j_max + C - 1) / C;
-}
-
-// Launches `kernel` in clusters of (C, 1, 1) with programmatic stream
-// serialization.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_cluster_pdl(void (*kernel)(KArgs...), int C, dim3 grid, dim3 block,
-                               size_t smem, cudaStream_t s, Args&&... args) {
-  cudaLaunchConfig_t lc = {};
-  lc.gridDim = grid;
-  lc.blockDim = block;
-  lc.dynamicSmemBytes = smem;
-  lc.stream = s;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = unsigned(C);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  lc.attrs = attr;
-  lc.numAttrs = 2;
-  return cudaLaunchKernelEx(&lc, kernel, std::forward<Args>(args)...);
-}
-
-// Cluster size of the one-launch routing for this segment, or 0 when the
-// candidates do not fit (more than kClusterMax * kClusterShareRows blocks)
-// or no such cluster can be resident; then the routing runs as three
-// kernels.  At least enough CTAs for the candidates (kClusterShareRows
-// each), and up to one per SM over all (b, KV head) for parallelism.
-// Deterministic for given arguments (the occupancy answers are cached).
-template <int D>
-int route_cluster_size(const hga_config_t* cfg, int64_t q_begin, int32_t s_len) {
-  const int64_t j_max = q_begin / kBlock + s_len / kQBlock - 1;
-  const int64_t need = (j_max + kClusterShareRows - 1) / kClusterShareRows;
-  if (need > kClusterMax) return 0;
-  const int64_t heads = int64_t(cfg->batch) * cfg->n_kv_heads;
-  int64_t want = std::max<int64_t>(need, std::min<int64_t>(kClusterMax, sm_count() / heads));
-  int C = 1;
-  while (C < want) C *= 2;
-  const int n_qb = s_len / kQBlock;
-  const void* fn = reinterpret_cast<const void*>(&route_cluster_kernel<__nv_bfloat16, D>);
-  static std::mutex mu;
-  static std::map<std::tuple<int, int, size_t, int>, int> fits;  // (dev, C, smem, D) -> clusters
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  for (; C >= 1 && C >= need; C /= 2) {
-    const size_t smem = cluster_layout(int(route_cluster_share(q_begin, s_len, C)), n_qb, C,
-                                       cfg->topk_blocks, D).total;
-    std::lock_guard<std::mutex> lock(mu);
-    auto key = std::make_tuple(dev, C, smem, D);
-    auto it = fits.find(key);
-    int n = 0;
-    if (it != fits.end()) {
-      n = it->second;
-    } else {
-      // both element types have the same resources; ask once per shape
-      for (const void* f : {fn, reinterpret_cast<const void*>(&route_cluster_kernel<float, D>)}) {
-        if (C > 8 && cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-                         cudaSuccess) {
-          cudaGetLastError();
-          n = -1;
-        }
-        if (ensure_smem(f, smem) != HGA_OK) n = -1;  // only ever raises the limit
-      }
-      if (n == 0) {
-        cudaLaunchConfig_t lc = {};
-        lc.gridDim = dim3(unsigned(C), cfg->n_kv_heads, cfg->batch);
-        lc.blockDim = dim3(kRouteThreads);
-        lc.dynamicSmemBytes = smem;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = unsigned(C);
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        lc.attrs = attr;
-        lc.numAttrs = 1;
-        if (cudaOccupancyMaxActiveClusters(&n, fn, &lc) != cudaSuccess) {
-          cudaGetLastError();
-          n = 0;
-        }
-      }
-      fits[key] = n;
-    }
-    if (n > 0) return C;
-  }
-  return 0;
-}
-}  // extern "C++"
-
 static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q_begin,
                                int32_t s_len, int64_t ctx_cap, const float* bsum,
                                const float* gsum, int32_t* sel_blk, int32_t* sel_grp,
@@ -478,21 +382,19 @@ static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q
   const int64_t j_max = own0 + n_qb - 1;
   const int G = cfg->n_q_heads / cfg->n_kv_heads;
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
-    const int C = route_cluster_size<D>(cfg, q_begin, s_len);
-    if (C > 0) {
-      // the whole routing in one launch, one cluster of C CTAs per (b, KV head)
-      const ClusterLayout Lc = cluster_layout(route_cluster_share(q_begin, s_len, C), n_qb, C,
-                                              cfg->topk_blocks, D);
-      return traced_launch(HGA_K_ROUTE_CLUSTER, s, [&] {
-        return launch_cluster_pdl(route_cluster_kernel<T, D>, C,
-            dim3(unsigned(C), cfg->n_kv_heads, cfg->batch), dim3(kRouteThreads), Lc.total, s,
-            qprev ? nullptr : static_cast<const T*>(q), qprev, qshift, bsum, gsum, ctx_cap,
-            int(cfg->n_q_heads), int(cfg->n_kv_heads), int(s_len), own0,
-            route_cluster_share(q_begin, s_len, C), int(cfg->topk_blocks),
-            int(cfg->topk_groups), sel_blk, sel_grp, done, token);
+    if (j_max <= kFusedRouteMaxBlocks) {
+      // the whole routing in one launch (every CTA reads all J block summaries)
+      dim3 g1(n_qb, cfg->n_kv_heads, cfg->batch);
+      const size_t smf = fused_route_smem<D>(own0 + n_qb, cfg->topk_blocks);
+      hga_status_t e = ensure_smem(reinterpret_cast<const void*>(&route_fused_kernel<T, D>), smf);
+      if (e != HGA_OK) return e;
+      return traced_launch(HGA_K_ROUTE_FUSED, s, [&] {
+        return launch_pdl(route_fused_kernel<T, D>, g1, dim3(kRouteThreads), smf, s,
+                          static_cast<const T*>(q), bsum, gsum, ctx_cap, cfg->n_q_heads,
+                          cfg->n_kv_heads, s_len, own0, cfg->topk_blocks, cfg->topk_groups,
+                          sel_blk, sel_grp, done, token, qprev, qshift);
       });
     }
-    if (done) return HGA_ERR_INVALID_ARG;  // chaining needs the one-launch routing
     hga_status_t e = HGA_OK;
     if (!qprev) {
       dim3 g0(n_qb * G, cfg->n_kv_heads, cfg->batch);
@@ -525,11 +427,9 @@ static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q
   });
 }
 
-// whether route_impl takes the one-launch (cluster) path
-static bool route_one_launch(const hga_config_t* cfg, int64_t q_begin, int32_t s_len) {
-  return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
-           return route_cluster_size<D>(cfg, q_begin, s_len) > 0 ? HGA_OK : HGA_ERR_UNSUPPORTED;
-         }) == HGA_OK;
+// whether route_impl takes the one-launch path
+static bool route_fused(int64_t q_begin, int32_t s_len) {
+  return q_begin / kBlock + s_len / kQBlock - 1 <= kFusedRouteMaxBlocks;
 }
 
 hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, int32_t s_len,
@@ -777,7 +677,7 @@ hga_status_t hga_segment_fwd_bwd(const hga_config_t* cfg, const void* q, const v
   const size_t route_bytes = ws_bytes - bwd_bytes - bwd_flag_bytes(cfg, s_len);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint32_t token = next_call_token();
-  const bool chain = use_tensor_cores(cfg, ctx_cap, s_len) && route_one_launch(cfg, q_begin, s_len);
+  const bool chain = use_tensor_cores(cfg, ctx_cap, s_len) && route_fused(q_begin, s_len);
   st = route_impl(cfg, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp, route_ws,
                   route_bytes, chain ? route_done : nullptr, token, s);
   if (st != HGA_OK) return st;
@@ -908,7 +808,7 @@ const char* hga_kernel_name(int kind) {
       "summaries",      "route_qmean",       "route_block_score",   "route_select",
       "attn_fwd_simt",  "attn_bwd_dq_simt",  "attn_bwd_dkdv_simt",  "attn_fwd_tc",
       "attn_bwd_dq_tc", "attn_bwd_dkdv_tc",  "tier_dedup",          "tier_copy",
-      "route_cluster",  "decode",            "query_summaries",     "prepare"};
+      "route_fused",    "decode",            "query_summaries",     "prepare"};
   return (kind >= 0 && kind < HGA_K_COUNT) ? names[kind] : "unknown";
 }
 

@@ -3,9 +3,8 @@
 // are opened at 8-token-group level, the router uses no learned weights and
 // scores the existing projected keys).
 //
-// One launch (route_cluster_kernel, below) while the candidate blocks number
-// at most kClusterMax * kClusterShareRows (2048: contexts up to 131072
-// tokens); beyond that three launches, all HBM/L2-bound:
+// One launch (route_fused_kernel) while the candidate blocks number at most
+// kFusedRouteMaxBlocks; beyond that three launches, all HBM/L2-bound:
 //   qmean_kernel        per (query block j, query head): that head's share of
 //                       qbar[b,h,j], the mean of the 64 x G query rows (reads Q
 //                       once, 1024 CTAs for Qwen3 shapes, one load round);
@@ -19,10 +18,7 @@
 // the ranking.
 #pragma once
 
-#include <cooperative_groups.h>
-
 #include "hga_common.cuh"
-#include "sm100_ptx.cuh"
 
 namespace hga {
 
@@ -309,9 +305,21 @@ __global__ void __launch_bounds__(kRouteThreads)
                    sel_grp);
 }
 
-// rows summed per thread slot in block_query_mean
+// The whole routing of one (b, h, j) in one CTA, used while every CTA can
+// afford to read all J block summaries (J <= kFusedRouteMaxBlocks; they stay
+// in L2): q-bar from the G heads' 64 query rows (the loads of several rows in
+// flight per thread), the J block scores, then select_levels.  One launch
+// instead of qmean + block_score + select.  Dynamic shared memory:
+// fused_route_smem(), the select layout followed by the q-bar partial sums.
+constexpr int kFusedRouteMaxBlocks = 512;
+
 template <int D>
-__host__ __device__ constexpr int query_mean_rows() { return kRouteThreads / (D / 8); }
+__host__ __device__ constexpr int fused_route_rows() { return kRouteThreads / (D / 8); }
+
+template <int D>
+__host__ __device__ inline size_t fused_route_smem(int64_t j_cap, int topk_blocks) {
+  return select_layout(j_cap, topk_blocks, D).total + size_t(fused_route_rows<D>()) * D * 4;
+}
 
 // Mean of the G x 64 query rows of query block j of KV head h (rows of the
 // segment's Q [B, Hq, S, d]): thread (row slot rs, 8-column chunk ch) sums
@@ -322,7 +330,7 @@ template <typename T, int D>
 __device__ __forceinline__ void block_query_mean(const T* __restrict__ q, int b, int h, int j,
                                                  int n_q_heads, int G, int s_len, float* part,
                                                  float* out) {
-  constexpr int CH = D / 8, RS = query_mean_rows<D>();
+  constexpr int CH = D / 8, RS = fused_route_rows<D>();
   const int ch = threadIdx.x % CH, rs = threadIdx.x / CH;
   const int rows = G * kQBlock;
   const T* qh =
@@ -357,271 +365,56 @@ __global__ void __launch_bounds__(kRouteThreads)
                 int s_len, int64_t own0, float* __restrict__ qsum) {
   pdl_launch_dependents();
   pdl_wait();
-  __shared__ float part[query_mean_rows<D>() * D];
+  __shared__ float part[fused_route_rows<D>() * D];
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int64_t head = int64_t(b) * n_kv_heads + h;
   block_query_mean<T, D>(q, b, h, j, n_q_heads, n_q_heads / n_kv_heads, s_len, part,
                          qsum + (head * (ctx_cap / kBlock) + own0 + j) * D);
 }
 
-// ---------------------------------------------------------------------------
-// The whole routing of one (batch, KV head) in one thread-block cluster of C
-// CTAs (C in {1, 2, 4, 8, 16}; up to kClusterShareRows candidate blocks per
-// CTA).  CTA r holds candidate blocks [r*share, (r+1)*share) and owns query
-// blocks j = r, r + C, r + 2C, ...
-//   A. bulk copy of its share of the block summaries into shared memory
-//      (read once for the whole head); meanwhile q-bar of its own query
-//      blocks (from Q, then stored into every CTA) or of all of them (from
-//      the resident block mean queries); one cluster barrier;
-//   B. the scores of every query block against its share (lane = query
-//      block, rows broadcast), a local top-k_b per query block (warp rank
-//      counting over the valid candidates), the finalists stored into the
-//      owner CTA's slots in rank order (padding key 0); one cluster barrier;
-//   C. per owned query block: the top-k_b of the C*k_b finalists (slots in
-//      rank order are in ascending block order, so ties keep the lower
-//      block), the kept blocks' groups scored and the top-k_g kept; both
-//      selections written and, in a chained segment call, the item's flag
-//      released.
-// ---------------------------------------------------------------------------
-constexpr int kClusterMax = 16;
-constexpr int kClusterShareRows = 128;
-
-struct ClusterLayout {
-  size_t bs, qb, sc, fin_key, fin_idx, mkey, midx, msel, blocks, key2, sel2, grp, hist, scratch,
-      part, bar, total;
-  int qb_stride, sc_stride;
-};
-
-__host__ __device__ inline ClusterLayout cluster_layout(int share, int n_qb, int C,
-                                                        int topk_blocks, int D) {
-  ClusterLayout L;
-  const int own = (n_qb + C - 1) / C;
-  L.qb_stride = D + 4;
-  L.sc_stride = share + 1;
-  size_t o = 0;
-  L.bs = o;       o = align16(o + size_t(share) * D * 4);
-  L.qb = o;       o = align16(o + size_t(n_qb) * L.qb_stride * 4);
-  L.sc = o;       o = align16(o + size_t(n_qb) * L.sc_stride * 4);
-  L.fin_key = o;  o = align16(o + size_t(own) * C * topk_blocks * 4);
-  L.fin_idx = o;  o = align16(o + size_t(own) * C * topk_blocks * 4);
-  L.mkey = o;     o = align16(o + size_t(C) * topk_blocks * 4);
-  L.midx = o;     o = align16(o + size_t(C) * topk_blocks * 4);
-  L.msel = o;     o = align16(o + size_t(C) * topk_blocks);
-  L.blocks = o;   o = align16(o + size_t(topk_blocks) * 4);
-  L.key2 = o;     o = align16(o + size_t(8) * topk_blocks * 4);
-  L.sel2 = o;     o = align16(o + size_t(8) * topk_blocks);
-  L.grp = o;      o = align16(o + size_t(8) * topk_blocks * 4);
-  L.hist = o;     o = align16(o + 256 * 4);
-  L.scratch = o;  o = align16(o + 16 * 4);
-  L.part = o;     o = align16(o + size_t(kRouteThreads / (D / 8)) * D * 4);
-  L.bar = o;      o = align16(o + 16);
-  L.total = o;
-  return L;
-}
-
-// grid (C, n_kv_heads, batch) in clusters of (C, 1, 1).  q-bar source: the
-// segment's Q (q != nullptr), else qsum row own0 + j - qshift.
+// grid (n_qb, Hkv, B)
 template <typename T, int D>
 __global__ void __launch_bounds__(kRouteThreads)
-    route_cluster_kernel(const T* __restrict__ q, const float* __restrict__ qsum, int qshift,
-                         const float* __restrict__ bsum, const float* __restrict__ gsum,
-                         int64_t ctx_cap, int n_q_heads, int n_kv_heads, int s_len, int64_t own0,
-                         int share, int topk_blocks, int topk_groups,
-                         int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp,
-                         int* __restrict__ done, uint32_t token) {
-  namespace cg = cooperative_groups;
+    route_fused_kernel(const T* __restrict__ q, const float* __restrict__ bsum,
+                       const float* __restrict__ gsum, int64_t ctx_cap, int n_q_heads,
+                       int n_kv_heads, int s_len, int64_t own0, int topk_blocks, int topk_groups,
+                       int32_t* __restrict__ sel_blk, int32_t* __restrict__ sel_grp,
+                       int* __restrict__ done, uint32_t token, const float* __restrict__ qprev,
+                       int qshift) {
+  // q-bar needs only the queries, which the kernels before this one do not
+  // write: it is formed while the kernel before still runs; the summaries
+  // are read only after it has completed (the wait below).  A chained
+  // forward waits for each item's flag, so it may be scheduled at once.
   pdl_launch_dependents();
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = int(cluster.block_rank()), C = int(cluster.num_blocks());
   extern __shared__ __align__(16) unsigned char sm_raw[];
-  const int h = blockIdx.y, b = blockIdx.z;
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int G = n_q_heads / n_kv_heads, n_qb = s_len / kQBlock;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t head = int64_t(b) * n_kv_heads + h;
-  const ClusterLayout L = cluster_layout(share, n_qb, C, topk_blocks, D);
-  float* bs = reinterpret_cast<float*>(sm_raw + L.bs);
+  const int64_t J = own0 + j;                 // candidate blocks [0, J)
+  const SelectLayout L = select_layout(own0 + n_qb, topk_blocks, D);
   float* qb = reinterpret_cast<float*>(sm_raw + L.qb);
-  uint32_t* sc = reinterpret_cast<uint32_t*>(sm_raw + L.sc);
-  uint32_t* fin_key = reinterpret_cast<uint32_t*>(sm_raw + L.fin_key);
-  int* fin_idx = reinterpret_cast<int*>(sm_raw + L.fin_idx);
-  uint32_t* mkey = reinterpret_cast<uint32_t*>(sm_raw + L.mkey);
-  int* midx = reinterpret_cast<int*>(sm_raw + L.midx);
-  uint8_t* msel = sm_raw + L.msel;
-  int* blocks = reinterpret_cast<int*>(sm_raw + L.blocks);
-  uint32_t* key2 = reinterpret_cast<uint32_t*>(sm_raw + L.key2);
-  uint8_t* sel2 = sm_raw + L.sel2;
-  int* grp = reinterpret_cast<int*>(sm_raw + L.grp);
-  int* hist = reinterpret_cast<int*>(sm_raw + L.hist);
-  int* scratch = reinterpret_cast<int*>(sm_raw + L.scratch);
-  float* part = reinterpret_cast<float*>(sm_raw + L.part);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm_raw + L.bar);
-  __shared__ int s_abort;
-  const int64_t j_max = own0 + n_qb - 1;  // candidates of the last query block: [0, j_max)
-  const int64_t lo = j_max < int64_t(rank) * share ? j_max : int64_t(rank) * share;
-  const int n_loc = int((j_max < lo + share ? j_max : lo + share) - lo);
-  if (tid == 0) {
-    sm100::mbar_init(bar, 1);
-    s_abort = 0;
-    sm100::fence_barrier_init();
-  }
-  // every CTA of the cluster is running before any touches a peer's memory
-  cluster.sync();
+  uint32_t* key1 = reinterpret_cast<uint32_t*>(sm_raw + L.key1);
+  float* part = reinterpret_cast<float*>(sm_raw + L.total);
 
-  // A. q-bar; the block-summary share is copied in after the kernel before
-  //    has completed (it may have written the summaries)
-  if (q) {
-    for (int j = rank; j < n_qb; j += C) {
-      block_query_mean<T, D>(q, b, h, j, n_q_heads, G, s_len, part, qb + j * L.qb_stride);
-      __syncthreads();
-    }
-  }
+  if (!qprev) block_query_mean<T, D>(q, b, h, j, n_q_heads, G, s_len, part, qb);
+  // from here on everything before this kernel has completed
   pdl_wait();
-  if (tid == 0 && n_loc > 0) {
-    const uint32_t bytes = uint32_t(n_loc) * D * 4;
-    sm100::mbar_arrive_expect_tx(bar, bytes);
-    const char* src = reinterpret_cast<const char*>(bsum + (head * (ctx_cap / kBlock) + lo) * D);
-    for (uint32_t off = 0; off < bytes; off += 32768u)
-      sm100::bulk_load(reinterpret_cast<char*>(bs) + off, src + off,
-                       bytes - off < 32768u ? bytes - off : 32768u, bar);
-  }
-  if (q) {
-    // own q-bar rows into every peer
-    for (int j = rank; j < n_qb; j += C)
-      for (int i = tid; i < (C - 1) * D; i += kRouteThreads) {
-        const int dst = (rank + 1 + i / D) % C, e = i % D;
-        cluster.map_shared_rank(qb, dst)[j * L.qb_stride + e] = qb[j * L.qb_stride + e];
-      }
-  } else {
-    for (int i = tid; i < n_qb * D; i += kRouteThreads) {
-      const int j = i / D, e = i % D;
-      const int64_t row = own0 + j - qshift;
-      qb[j * L.qb_stride + e] = row >= 0 ? qsum[(head * (ctx_cap / kBlock) + row) * D + e] : 0.f;
-    }
-  }
-  bool fail = false;
-  if (n_loc > 0) fail = !sm100::mbar_wait(bar, 0, &s_abort);
-  const bool ok = !__syncthreads_or(fail);
-  cluster.sync();
-
-  // B. scores of every query block against the share: lane = query block
-  //    (two rounds past 32), each warp a slice of the rows, 8 rows at a time
-  if (ok) {
-    const int rows_per_warp = (n_loc + 7) / 8;
-    const int r0 = warp * rows_per_warp;
-    const int r1 = r0 + rows_per_warp < n_loc ? r0 + rows_per_warp : n_loc;
-    for (int jb = 0; jb < n_qb; jb += 32) {
-      const int j = jb + lane;
-      const float4* qj = reinterpret_cast<const float4*>(qb + (j < n_qb ? j : 0) * L.qb_stride);
-      for (int i0 = r0; i0 < r1; i0 += 8) {
-        float acc[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) acc[u] = 0.f;
-#pragma unroll 4
-        for (int e4 = 0; e4 < D / 4; ++e4) {
-          const float4 x = qj[e4];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u < r1 ? i0 + u : i0;
-            const float4 y = reinterpret_cast<const float4*>(bs + size_t(i) * D)[e4];
-            acc[u] = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, acc[u]))));
-          }
-        }
-        if (j < n_qb)
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            if (i0 + u < r1) sc[j * L.sc_stride + i0 + u] = ordered_key(acc[u]);
-      }
-    }
-  }
+  if (qprev)
+    for (int e = threadIdx.x; e < D; e += kRouteThreads)
+      qb[e] = J - qshift >= 0 ? qprev[(head * (ctx_cap / kBlock) + J - qshift) * D + e] : 0.f;
   __syncthreads();
-  // local top-k_b of each query block over its valid candidates (c < own0 + j),
-  // one warp per query block; finalists in ascending index into the owner
-  if (ok) {
-    for (int j = warp; j < n_qb; j += kRouteThreads / 32) {
-      const int64_t J = own0 + j;
-      const int kb = int(J < topk_blocks ? J : topk_blocks);
-      int n_val = int(J - lo);
-      n_val = n_val < 0 ? 0 : (n_val > n_loc ? n_loc : n_val);
-      const int k_loc = kb < n_val ? kb : n_val;
-      const uint32_t* row = sc + j * L.sc_stride;
-      const int owner = j % C, jl = j / C;
-      uint32_t* okey = cluster.map_shared_rank(fin_key, owner) + (jl * C + rank) * topk_blocks;
-      int* oidx = cluster.map_shared_rank(fin_idx, owner) + (jl * C + rank) * topk_blocks;
-      int written = 0;
-      for (int m0 = 0; m0 < n_val; m0 += 32) {
-        const int i = m0 + lane;
-        bool pick = false;
-        if (i < n_val && k_loc > 0) {
-          const uint32_t ki = row[i];
-          int r = 0;
-          for (int i2 = 0; i2 < n_val; ++i2) {
-            const uint32_t k2 = row[i2];
-            r += (k2 > ki) || (k2 == ki && i2 < i);
-          }
-          pick = r < k_loc;
-        }
-        const unsigned ball = __ballot_sync(0xffffffffu, pick);
-        if (pick) {
-          const int pos = written + __popc(ball & ((1u << lane) - 1u));
-          okey[pos] = row[i];
-          oidx[pos] = int(lo + i);
-        }
-        written += __popc(ball);
-      }
-      for (int p = k_loc + lane; p < kb; p += 32) {
-        okey[p] = 0u;
-        oidx[p] = -1;
-      }
-    }
-  }
-  cluster.sync();
-
-  // C. the owned query blocks: merge, level 2, write
-  if (ok) {
-    for (int j = rank; j < n_qb; j += C) {
-      const int jl = j / C;
-      const int64_t J = own0 + j;
-      const int kb = int(J < topk_blocks ? J : topk_blocks);
-      const int n_m = C * kb;
-      for (int i = tid; i < n_m; i += kRouteThreads) {
-        const int r = i / kb, p = i % kb;
-        mkey[i] = fin_key[(jl * C + r) * topk_blocks + p];
-        midx[i] = fin_idx[(jl * C + r) * topk_blocks + p];
-      }
-      __syncthreads();
-      block_topk_indices(mkey, n_m, kb, blocks, msel, hist, scratch);
-      for (int r = tid; r < kb; r += kRouteThreads) blocks[r] = midx[blocks[r]];
-      __syncthreads();
-      if (sel_blk)
-        for (int i = tid; i < topk_blocks; i += kRouteThreads)
-          sel_blk[(head * n_qb + j) * topk_blocks + i] = i < kb ? blocks[i] : -1;
-      const int n2 = 8 * kb;
-      score_rows<D>(gsum + head * (ctx_cap / kGroup) * D, qb + j * L.qb_stride, n2,
-                    [&](int p) {
-                      // a block index below 0 only comes from a non-finite summary;
-                      // it is kept in bounds (the attention rejects the result)
-                      const int blk = blocks[p >> 3];
-                      return int64_t(blk < 0 ? 0 : blk) * kGroupsPerBlock + (p & 7);
-                    },
-                    key2);
-      __syncthreads();
-      const int kg = n2 < topk_groups ? n2 : topk_groups;
-      block_topk_indices(key2, n2, kg, grp, sel2, hist, scratch);
-      int32_t* out = sel_grp + (head * n_qb + j) * topk_groups;
-      for (int i = tid; i < topk_groups; i += kRouteThreads)
-        out[i] = i < kg ? blocks[grp[i] >> 3] * kGroupsPerBlock + (grp[i] & 7) : -1;
-      if (done) {
-        // chained segment call: this item's selections are written
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) flag_release(done + j + n_qb * (h + n_kv_heads * b), token);
-      }
-      __syncthreads();
-    }
-  } else if (tid == 0) {
-    // a copy did not land in time (HGA_ERR_TIMEOUT is latched): give it a
-    // bounded time more before the CTA leaves; no selection is written
-    sm100::mbar_wait(bar, 0, &s_abort, 200000000LL);
+  // level-1 scores of the J candidate blocks
+  score_rows<D>(bsum + head * (ctx_cap / kBlock) * D, qb, int(J),
+                [](int p) { return int64_t(p); }, key1);
+  __syncthreads();
+  select_levels<D>(L, sm_raw, gsum, head, ctx_cap, n_qb, j, J, topk_blocks, topk_groups, sel_blk,
+                   sel_grp);
+  if (done) {
+    // chained segment call: this item's selections are written
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0)
+      flag_release(done + blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z), token);
   }
 }
 

@@ -505,7 +505,7 @@ typedef enum {
   HGA_K_BWD_DKDV_TC = 9,
   HGA_K_TIER_DEDUP = 10,
   HGA_K_TIER_COPY = 11,
-  HGA_K_ROUTE_CLUSTER = 12,
+  HGA_K_ROUTE_FUSED = 12,
   HGA_K_DECODE = 13,
   HGA_K_QSUM = 14,
   HGA_K_PREPARE = 15,

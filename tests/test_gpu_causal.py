@@ -51,9 +51,9 @@ def test_causal_qwen3_fwdbwd_16k_all_segments():
     run_causal(WL["qwen3_fwdbwd_16k"])
 
 
-def test_causal_cluster_routing_at_131k():
-    # the one-launch routing at its largest (2047 candidate blocks): the
-    # last segment of the 131072-token context, two KV heads checked
+def test_causal_routing_at_131k():
+    # the last segment of the 131072-token context (2047 candidate blocks),
+    # two KV heads checked
     w = dataclasses.replace(WL["qwen3_fwdbwd_16k"], name="qwen3_fwd_131k_last",
                             ctx_len=131072, first_seg=63, backward=False)
     run_causal(w, kv_heads=[1, 4])
@@ -66,10 +66,10 @@ def test_causal_history_before_first_segment():
 
 
 def test_causal_long_context_three_kernel_routing():
-    # past 2048 candidate blocks (the three-kernel routing), last segment of
-    # a 133120-token context, two KV heads checked
-    w = dataclasses.replace(WL["qwen3_fwdbwd_16k"], name="qwen3_fwdbwd_133k_last",
-                            ctx_len=133120, first_seg=64)
+    # past 512 candidate blocks (the three-kernel routing), last segment of
+    # a 36864-token context, two KV heads checked
+    w = dataclasses.replace(WL["qwen3_fwdbwd_16k"], name="qwen3_fwdbwd_36k_last",
+                            ctx_len=36864, first_seg=17)
     run_causal(w, kv_heads=[2, 7])
 
 

@@ -112,19 +112,18 @@ def test_chained_segment_call_equals_separate_calls():
 
 
 def test_chained_segment_call_long_context_routing():
-    # past 2048 candidate blocks (contexts above 131072 tokens) the routing
-    # runs as three kernels and the chained call waits for the whole routing
-    # grid instead of per-item flags; the selections and outputs still equal
-    # the separate calls'
+    # past 512 candidate blocks the routing runs as three kernels and the
+    # chained call waits for the whole routing grid instead of per-item
+    # flags; the selections and outputs still equal the separate calls'
     import dataclasses
 
     import torch
-    w = dataclasses.replace(WL["qwen3_fwdbwd_16k"], name="qwen3_fwdbwd_133k_last",
-                            ctx_len=133120, first_seg=64)
+    w = dataclasses.replace(WL["qwen3_fwdbwd_16k"], name="qwen3_fwdbwd_36k_last",
+                            ctx_len=36864, first_seg=17)
     seg = Segmenter(w)
     L = seg.layer
     q_begin = w.ctx_len - w.seg_len
-    assert q_begin // 64 + w.seg_len // 64 - 1 > 2048
+    assert q_begin // 64 > 512
     q = to_device(synth.queries(w, q_begin), w)
     d_o = to_device(synth.douts(w, q_begin), w)
     L.summarize(q_begin)

@@ -7,10 +7,10 @@ device.  hga_route_noalloc serves them by taking the router's scratch (the
 mean queries and the block scores) from an array built into the library
 instead of a caller-provided workspace.
 
-The context here is long enough (more than 2048 candidate blocks) that the
+The context here is long enough (more than 512 candidate blocks) that the
 routing runs as its three-kernel form, which is the form that writes and
 reads that scratch.  The test calls the entry point through the C ABI twice
-in a row: first at the end of a 135168-token context, then on an earlier
+in a row: first at the end of a 40960-token context, then on an earlier
 segment with fewer candidates, so the second call's score rows are shorter
 than the first call's and sit over its leftover contents.  Each result must
 equal the workspace-taking hga_route's exactly (selections are integer
@@ -34,7 +34,7 @@ def test_route_noalloc_matches_route_on_two_calls_in_a_row():
                                                      hga_build_summaries, hga_route,
                                                      hga_route_noalloc)
 
-    w = synth.custom(n_q_heads=32, n_kv_heads=8, head_dim=128, ctx_len=135168, seg_len=2048,
+    w = synth.custom(n_q_heads=32, n_kv_heads=8, head_dim=128, ctx_len=40960, seg_len=2048,
                      topk_blocks=16, topk_groups=64, dtype="bf16", scaled=True,
                      rope_base=1e6, seed=21)
     dev = torch.device("cuda", 0)
@@ -49,8 +49,8 @@ def test_route_noalloc_matches_route_on_two_calls_in_a_row():
     hga_build_summaries(cfg, layer.k, w.ctx_len, 0, w.ctx_len, layer.gsum, layer.bsum)
 
     n_qb = w.seg_len // 64
-    for q_begin in (133120, 131072):      # two calls in a row, the second with shorter rows
-        assert q_begin // 64 + 31 > 2048  # past the one-launch routing's limit
+    for q_begin in (38912, 34816):        # two calls in a row, the second with shorter rows
+        assert q_begin // 64 > 512        # past the single-kernel routing's limit
         q = bf16(synth.queries(w, q_begin))
         ref_blk = torch.full((1, 8, n_qb, 16), -9, dtype=torch.int32, device=dev)
         ref_grp = torch.full((1, 8, n_qb, 64), -9, dtype=torch.int32, device=dev)
