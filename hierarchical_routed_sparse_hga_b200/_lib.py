@@ -91,7 +91,7 @@ def load() -> ctypes.CDLL:
         "hga_last_cuda_error": (ctypes.c_char_p, []),
         "hga_build_summaries": (ctypes.c_int, [CFG, P, I64, I64, I64, P, P, P]),
         "hga_route_workspace_size": (SZ, [CFG, I32, I64]),
-        "hga_route": (ctypes.c_int, [CFG, P, I64, I32, I64, P, P, P, P, P, SZ, P]),
+        "hga_route": (ctypes.c_int, [CFG, P, I64, I32, I64, P, P, P, P, P, P, SZ, P]),
         "hga_attn_fwd": (ctypes.c_int, [CFG, P, P, P, I64, I64, I32, P, P, P, P]),
         "hga_attn_bwd_workspace_size": (SZ, [CFG, I32]),
         "hga_attn_bwd": (ctypes.c_int, [CFG, P, P, P, I64, I64, I32, P, P, P, P, P, P, P,
@@ -246,12 +246,15 @@ def hga_route_workspace_size(cfg: Config, s_len, q_begin) -> int:
 
 
 def hga_route(cfg: Config, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp,
-              workspace, ws_bytes=None, stream=None):
+              workspace, ws_bytes=None, stream=None, scores_out=None):
+    """scores_out (optional, [B, Hkv, s_len/64, 4] float32) is the C call's
+    argument after sel_grp; a keyword here."""
     c = cfg.c()
     ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
     _check("hga_route", load().hga_route(
         ctypes.byref(c), _ptr(q), q_begin, s_len, ctx_cap, _ptr(bsum), _ptr(gsum),
-        _ptr(sel_blk), _ptr(sel_grp), _ptr(workspace), ws_bytes, _stream(stream)))
+        _ptr(sel_blk), _ptr(sel_grp), _ptr(scores_out), _ptr(workspace), ws_bytes,
+        _stream(stream)))
 
 
 def hga_build_query_summaries(cfg: Config, q, q_begin, s_len, ctx_cap, qsum, stream=None):

@@ -363,13 +363,48 @@ __device__ void block_topk(const uint32_t* key, int n, int k, uint8_t* sel, int*
   __syncthreads();
 }
 
+// The float score behind an ordered key (inverse of ordered_key).
+__device__ __forceinline__ float key_score(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// After block_topk: out[0] = the k-th largest score (the smallest chosen
+// key), out[1] = the (k+1)-th (the largest key not chosen), both times
+// `scale`; -inf where there is none (k = 0, or every key chosen; padding key
+// 0 counts as none).  Every thread calls it; thread 0 writes out.
+__device__ void kth_scores(const uint32_t* key, const uint8_t* sel, int n, float scale,
+                           float* out) {
+  __shared__ uint32_t s_lo, s_hi;
+  if (threadIdx.x == 0) {
+    s_lo = 0xffffffffu;
+    s_hi = 0u;
+  }
+  __syncthreads();
+  uint32_t lo = 0xffffffffu, hi = 0u;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const uint32_t k = key[i];
+    if (sel[i]) lo = k < lo ? k : lo;
+    else hi = k > hi ? k : hi;
+  }
+  if (lo != 0xffffffffu) atomicMin(&s_lo, lo);
+  if (hi != 0u) atomicMax(&s_hi, hi);
+  __syncthreads();
+  if (threadIdx.x == 0 && out) {
+    out[0] = s_lo == 0xffffffffu || s_lo == 0u ? -INFINITY : key_score(s_lo) * scale;
+    out[1] = s_hi == 0u ? -INFINITY : key_score(s_hi) * scale;
+  }
+  __syncthreads();
+}
+
 // block_topk followed by the ascending list of the chosen indices:
 // out[r] = the r-th smallest index among the top-k of key[0, n) (k <= n).
 // Kept out of line: a kernel that selects several times runs one copy of
 // this code, which stays in the instruction cache.
 __device__ __noinline__ void block_topk_indices(const uint32_t* key, int n, int k, int* out,
-                                                uint8_t* sel, int* hist, int* scratch) {
+                                                uint8_t* sel, int* hist, int* scratch,
+                                                float scale = 0.f, float* scores = nullptr) {
   block_topk(key, n, k, sel, hist, scratch);
+  if (scores) kth_scores(key, sel, n, scale, scores);
   block_enumerate_any(
       n, [&](int i) { return sel[i] != 0; }, [&](int i, int r) { out[r] = i; }, scratch);
   __syncthreads();

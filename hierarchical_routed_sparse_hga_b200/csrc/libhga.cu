@@ -238,23 +238,30 @@ hga_status_t launch_bwd_tc(const hga_config_t* cfg, const void* q, const void* k
 }
 
 struct RouteCarve {
-  float* qbar;
-  float* scores;
-  int64_t jstride;
+  float* qbar;          // [B, Hkv, S/64, d]
+  uint32_t* fin_key;    // [B, Hkv, S/64, n_chunks, topk_blocks + 1]
+  int32_t* fin_idx;     // same
+  int n_chunks;
   size_t bytes;
 };
 
+// The routing workspace of the three-launch path: the query blocks' q-bar,
+// then the candidate chunks' finalists (keys, then block indices), each
+// section 256-byte aligned.
 RouteCarve route_carve(const hga_config_t* c, int32_t s_len, int64_t q_begin, void* base) {
   const int64_t n_qb = s_len / kQBlock;
   const int64_t heads = int64_t(c->batch) * c->n_kv_heads;
+  const int64_t j_max = q_begin / kBlock + n_qb - 1;
   RouteCarve r;
-  r.jstride = ((q_begin / kBlock + n_qb) + 3) & ~int64_t(3);
-  const int64_t G = c->n_q_heads / c->n_kv_heads;
-  const size_t qbar_bytes = align256(size_t(heads * n_qb * G * c->head_dim) * 4);
-  const size_t score_bytes = align256(size_t(heads * n_qb * r.jstride) * 4);
+  r.n_chunks = int(j_max > 0 ? (j_max + kChunkCands - 1) / kChunkCands : 1);
+  const size_t qbar_bytes = align256(size_t(heads * n_qb * c->head_dim) * 4);
+  const size_t fin_bytes =
+      align256(size_t(heads * n_qb) * r.n_chunks * (c->topk_blocks + 1) * 4);
+  char* p = static_cast<char*>(base);
   r.qbar = static_cast<float*>(base);
-  r.scores = base ? reinterpret_cast<float*>(static_cast<char*>(base) + qbar_bytes) : nullptr;
-  r.bytes = qbar_bytes + score_bytes;
+  r.fin_key = base ? reinterpret_cast<uint32_t*>(p + qbar_bytes) : nullptr;
+  r.fin_idx = base ? reinterpret_cast<int32_t*>(p + qbar_bytes + fin_bytes) : nullptr;
+  r.bytes = qbar_bytes + 2 * fin_bytes;
   return r;
 }
 
@@ -367,20 +374,20 @@ static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q
                                const float* gsum, int32_t* sel_blk, int32_t* sel_grp,
                                void* workspace, size_t ws_bytes, int* done, uint32_t token,
                                cudaStream_t s, const float* qprev = nullptr,
-                               int qshift = 1) {
+                               int qshift = 1, float* scores_out = nullptr) {
   hga_status_t st = check_cfg(cfg);
   if (st != HGA_OK) return st;
   if ((st = check_segment(ctx_cap, q_begin, s_len)) != HGA_OK) return st;
   if ((!q && !qprev) || !bsum || !gsum || !sel_grp || !workspace) return HGA_ERR_INVALID_ARG;
   if ((q && !aligned16(q)) || !aligned16(bsum) || !aligned16(gsum) || !aligned16(sel_grp) ||
-      !aligned16(workspace) || (sel_blk && !aligned16(sel_blk)))
+      !aligned16(workspace) || (sel_blk && !aligned16(sel_blk)) ||
+      (scores_out && !aligned16(scores_out)))
     return HGA_ERR_INVALID_ARG;
   RouteCarve ws = route_carve(cfg, s_len, q_begin, workspace);
   if (ws_bytes < ws.bytes) return HGA_ERR_WORKSPACE;
   const int n_qb = s_len / kQBlock;
   const int64_t own0 = q_begin / kBlock;
   const int64_t j_max = own0 + n_qb - 1;
-  const int G = cfg->n_q_heads / cfg->n_kv_heads;
   return dispatch(cfg, [&]<typename T, int D>() -> hga_status_t {
     if (j_max <= kFusedRouteMaxBlocks) {
       // the whole routing in one launch (every CTA reads all J block summaries)
@@ -392,37 +399,49 @@ static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q
         return launch_pdl(route_fused_kernel<T, D>, g1, dim3(kRouteThreads), smf, s,
                           static_cast<const T*>(q), bsum, gsum, ctx_cap, cfg->n_q_heads,
                           cfg->n_kv_heads, s_len, own0, cfg->topk_blocks, cfg->topk_groups,
-                          sel_blk, sel_grp, done, token, qprev, qshift);
+                          sel_blk, sel_grp, done, token, qprev, qshift, cfg->scale,
+                          scores_out);
       });
     }
+    // three launches: q-bar (unless it comes from the resident block means),
+    // the chunks' scores and finalists, the merge and level 2
     hga_status_t e = HGA_OK;
     if (!qprev) {
-      dim3 g0(n_qb * G, cfg->n_kv_heads, cfg->batch);
+      dim3 g0(n_qb, cfg->n_kv_heads, cfg->batch);
       e = traced_launch(HGA_K_QMEAN, s, [&] {
-        return launch_pdl(qmean_kernel<T, D>, g0, dim3(kQmeanThreads), 0, s,
+        return launch_pdl(qbar_kernel<T, D>, g0, dim3(kRouteThreads), 0, s,
             static_cast<const T*>(q), cfg->n_q_heads, cfg->n_kv_heads, s_len, ws.qbar);
       });
       if (e != HGA_OK) return e;
     }
+    const float* qsrc = qprev ? qprev : ws.qbar;
+    const int shift = qprev ? qshift : 0;
+    const float* qpart = qprev ? nullptr : ws.qbar;
     if (j_max > 0) {
-      const int n_cc = int((j_max + kScoreCands - 1) / kScoreCands);
-      const int n_jc = (n_qb + kScoreQbs - 1) / kScoreQbs;
-      dim3 g2(unsigned(n_cc * n_jc), cfg->n_kv_heads, cfg->batch);
+      // the query blocks split over CTAs of at most 32 each (splitting
+      // further measured slower: the CTAs are not short of SMs)
+      const int n_split = (n_qb + 31) / 32;
+      const int nq_max = (n_qb + n_split - 1) / n_split;
+      const size_t sm2 = chunk_layout(nq_max, D).total;
+      e = ensure_smem(reinterpret_cast<const void*>(&block_topk_kernel<D>), sm2);
+      if (e != HGA_OK) return e;
+      dim3 g2(unsigned(ws.n_chunks), cfg->n_kv_heads, cfg->batch * n_split);
       e = traced_launch(HGA_K_BLOCK_SCORE, s, [&] {
-        return launch_pdl(block_score_kernel<D>, g2, dim3(kRouteThreads), 0, s, ws.qbar, qprev,
-            qshift, bsum, ctx_cap, cfg->n_kv_heads, G, n_qb, own0, ws.scores, ws.jstride);
+        return launch_pdl(block_topk_kernel<D>, g2, dim3(kRouteThreads), sm2, s, qpart,
+            qprev ? qsrc : nullptr, shift, bsum, ctx_cap, cfg->n_kv_heads, n_qb, own0,
+            cfg->topk_blocks, n_split, nq_max, ws.fin_key, ws.fin_idx);
       });
       if (e != HGA_OK) return e;
     }
     dim3 g1(n_qb, cfg->n_kv_heads, cfg->batch);
-    const size_t sm3 = select_layout(own0 + n_qb, cfg->topk_blocks, D).total;
+    const size_t sm3 = merge_layout(ws.n_chunks, cfg->topk_blocks, D).total;
     e = ensure_smem(reinterpret_cast<const void*>(&select_kernel<D>), sm3);
     if (e != HGA_OK) return e;
     return traced_launch(HGA_K_SELECT, s, [&] {
-      return launch_pdl(select_kernel<D>, g1, dim3(kRouteThreads), sm3, s, ws.qbar, qprev,
-          qshift, ws.scores, gsum,
-          ctx_cap, cfg->n_kv_heads, G, n_qb, own0, ws.jstride, cfg->topk_blocks, cfg->topk_groups,
-          sel_blk, sel_grp);
+      return launch_pdl(select_kernel<D>, g1, dim3(kRouteThreads), sm3, s, qpart,
+          qprev ? qsrc : nullptr, shift, ws.fin_key, ws.fin_idx, ws.n_chunks, gsum, ctx_cap,
+          cfg->n_kv_heads, n_qb, own0, cfg->topk_blocks, cfg->topk_groups, sel_blk, sel_grp,
+          cfg->scale, scores_out);
     });
   });
 }
@@ -434,9 +453,11 @@ static bool route_fused(int64_t q_begin, int32_t s_len) {
 
 hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, int32_t s_len,
                        int64_t ctx_cap, const float* bsum, const float* gsum, int32_t* sel_blk,
-                       int32_t* sel_grp, void* workspace, size_t ws_bytes, void* stream) {
+                       int32_t* sel_grp, float* scores_out, void* workspace, size_t ws_bytes,
+                       void* stream) {
   return route_impl(cfg, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp, workspace,
-                    ws_bytes, nullptr, 0, static_cast<cudaStream_t>(stream));
+                    ws_bytes, nullptr, 0, static_cast<cudaStream_t>(stream), nullptr, 1,
+                    scores_out);
 }
 
 hga_status_t hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k, const void* v,
@@ -484,8 +505,8 @@ hga_status_t hga_route_noalloc(const hga_config_t* cfg, const void* q, int64_t q
     return HGA_ERR_WORKSPACE;
   void* scratch = noalloc_scratch();
   if (!scratch) return HGA_ERR_CUDA;
-  return hga_route(cfg, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp, scratch,
-                   HGA_NOALLOC_SCRATCH_BYTES, stream);
+  return hga_route(cfg, q, q_begin, s_len, ctx_cap, bsum, gsum, sel_blk, sel_grp, nullptr,
+                   scratch, HGA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 // backward workspace, 256-byte aligned sections: D = rowsum(dO * O)

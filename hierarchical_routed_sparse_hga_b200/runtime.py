@@ -66,9 +66,10 @@ class HgaLayer:
         _lib.hga_build_summaries(self.cfg, self.k, self.ctx_cap, q_begin,
                                  q_begin + self.seg_len, self.gsum, self.bsum, stream)
 
-    def route(self, q, q_begin: int, stream=None):
+    def route(self, q, q_begin: int, stream=None, scores_out=None):
         _lib.hga_route(self.cfg, q, q_begin, self.seg_len, self.ctx_cap, self.bsum,
-                       self.gsum, self.sel_blk, self.sel_grp, self.route_ws, stream=stream)
+                       self.gsum, self.sel_blk, self.sel_grp, self.route_ws, stream=stream,
+                       scores_out=scores_out)
 
     def build_query_summaries(self, q, q_begin: int, stream=None):
         _lib.hga_build_query_summaries(self.cfg, q, q_begin, self.seg_len, self.ctx_cap,

@@ -156,14 +156,18 @@ HGA_API size_t hga_route_workspace_size(const hga_config_t* cfg, int32_t s_len, 
  *            keep the top min(topk_groups, 8*kept) (ties: lower g).
  * Scores are ranked without the positive factor 1/sqrt(d) (order unchanged).
  * Writes sel_grp and, if sel_blk is not NULL, sel_blk (ascending, -1 padded).
+ * If scores_out ([batch, n_kv_heads, s_len/64, 4] float32) is not NULL it
+ * receives, per (b, h, j), the k-th and (k+1)-th largest scores of level 1
+ * and of level 2, scaled by cfg->scale (-inf where there is none): a caller
+ * can flag near ties from them, e.g. |s_k - s_k+1| <= 1e-3 max(|s_k|, |s_k+1|).
  * bsum/gsum must hold every block/group before the segment's last block
  * (call hga_build_summaries for the segment first).
  * workspace: at least hga_route_workspace_size() bytes of device memory.
  */
 HGA_API hga_status_t hga_route(const hga_config_t* cfg, const void* q, int64_t q_begin, int32_t s_len,
                        int64_t ctx_cap, const float* bsum, const float* gsum,
-                       int32_t* sel_blk, int32_t* sel_grp, void* workspace, size_t ws_bytes,
-                       void* stream);
+                       int32_t* sel_blk, int32_t* sel_grp, float* scores_out, void* workspace,
+                       size_t ws_bytes, void* stream);
 
 /*
  * Step a4 -- exact-token attention forward [A], [B].  Query t of head h'
@@ -183,14 +187,15 @@ HGA_API hga_status_t hga_attn_fwd(const hga_config_t* cfg, const void* q, const 
  * every byte of device memory and hands its extensions no allocator, or code
  * that must not allocate after start-up because cudaMalloc can synchronise
  * the device and has unbounded latency.  Such callers still pass every input
- * and output buffer; only the router's scratch (mean queries and block scores)
+ * and output buffer; only the router's scratch (the mean queries and the
+ * candidate chunks' finalists)
  * comes from a fixed array inside the library.
  *
  * The array is HGA_NOALLOC_SCRATCH_BYTES (4 MiB) of device memory that every
  * GPU which loads the library holds until the process exits.  A call whose
  * hga_route_workspace_size() exceeds it returns HGA_ERR_WORKSPACE and
  * launches nothing (for the Qwen3-8B shape -- 32 query / 8 KV heads, d = 128,
- * 2048-token segments, batch 1 -- contexts up to 229,376 tokens fit).
+ * 2048-token segments, batch 1 -- contexts up to 950,272 tokens fit).
  *
  * The first call on each device looks up the array's device address (with
  * that device current) and caches it; make that first call before any stream

@@ -91,10 +91,11 @@ def test_host_argument_checks():
 
 def test_workspace_sizes():
     c = cfg()
-    # per-head shares of qbar: 8 KV heads x 32 blocks x 4 query heads x 128 floats,
-    # + block scores 8 x 32 x 256 floats (each part 256-B aligned)
-    assert hga.hga_route_workspace_size(c, 2048, 14336) == (8 * 32 * 4 * 128 * 4
-                                                           + 8 * 32 * 256 * 4)
+    # q-bar: 8 KV heads x 32 query blocks x 128 floats; then, for the 2
+    # candidate chunks of 128 blocks (255 candidates), the finalists' keys and
+    # block indices: 8 x 32 x 2 x (16 + 1) each (each part 256-B aligned)
+    assert hga.hga_route_workspace_size(c, 2048, 14336) == (8 * 32 * 128 * 4
+                                                           + 2 * 8 * 32 * 2 * 17 * 4)
     # D = rowsum(dO * O) per query row, the dK/dV kernel's work counter, two
     # arrays of per-item flags (8 KV heads x 32 query blocks) for the fused
     # call, and the inverted selection (8 KV heads x 32 key blocks x 32 query blocks)

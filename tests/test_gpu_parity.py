@@ -170,6 +170,61 @@ def test_largest_segment_and_topk():
     run_and_compare(w, segments=[8192], kv_heads=[3])
 
 
+@pytest.mark.parametrize("ctx", [16384, 36864])
+def test_route_scores_out(ctx):
+    # hga_route's scores_out: the k-th and (k+1)-th largest scores of both
+    # levels, against float64 scores from the oracle's summaries (level 2
+    # where the GPU kept the oracle's blocks); one launch at 16384 tokens,
+    # three past 512 candidate blocks at 36864
+    import dataclasses
+    import math
+
+    import torch
+
+    import oracle
+    from hga_testlib import to_device
+    w = dataclasses.replace(WL["qwen3_fwd_16k"], ctx_len=ctx, first_seg=ctx // 2048 - 1)
+    seg = Segmenter(w)
+    L = seg.layer
+    q_begin = ctx - 2048
+    q_np = synth.queries(w, q_begin)
+    L.summarize(q_begin)
+    so = torch.full((1, 8, 32, 4), float("nan"), device="cuda")
+    L.route(to_device(q_np, w), q_begin, scores_out=so)
+    torch.cuda.synchronize()
+    so = so.cpu().numpy()
+    q64 = synth.widen(q_np, w.dtype)
+    g, b = oracle.build_summaries(seg.k64, 0, ctx)
+    sb, _, _ = oracle.route(q64, b, g, q_begin, 16, 64, 8)
+    gpu_blk = L.sel_blk.cpu().numpy()
+    inv = 1.0 / math.sqrt(128)
+    n2 = 0
+    for h in range(8):
+        for j in range(32):
+            J = q_begin // 64 + j
+            qbar = q64[0, 4 * h:4 * h + 4, 64 * j:64 * j + 64].reshape(-1, 128).mean(0)
+            s1 = np.sort(b[0, h, :J] @ qbar * inv)[::-1]
+            want = [s1[15], s1[16] if J > 16 else -np.inf]
+            assert np.allclose(so[0, h, j, :2], want, rtol=1e-4, atol=1e-6), (h, j)
+            if np.array_equal(gpu_blk[0, h, j], sb[0, h, j]):
+                grp = np.array([8 * c + i for c in sb[0, h, j] for i in range(8)])
+                s2 = np.sort(g[0, h, grp] @ qbar * inv)[::-1]
+                assert np.allclose(so[0, h, j, 2:], [s2[63], s2[64]], rtol=1e-4, atol=1e-6)
+                n2 += 1
+    assert n2 >= 200
+
+
+def test_long_context_routing_odd_query_blocks():
+    # the three-kernel routing (past 512 candidate blocks) with 63 query
+    # blocks per segment (split 32 + 31 over the block-score CTAs) and ragged
+    # k: the last segment of 36288 tokens, both KV heads checked
+    w = synth.custom(n_q_heads=8, n_kv_heads=2, head_dim=128, ctx_len=36288, seg_len=4032,
+                     topk_blocks=5, topk_groups=13, dtype="bf16", scaled=True, rope_base=1e6,
+                     seed=17, first_seg=8)
+    assert 32256 // 64 + 62 > 512
+    run_and_compare(w)
+
+
 @pytest.mark.parametrize("kw", [
     # ragged: k_g not a multiple of 8, more k_b than candidates early on
     dict(n_q_heads=4, n_kv_heads=1, head_dim=64, ctx_len=576, seg_len=192, topk_blocks=5,
@@ -237,6 +292,45 @@ def test_corrupt_selection_is_skipped_and_latched():
     ref_sel[0, 0, 1, 0] = -1
     o, lse = oracle.attn_fwd(out["q64"], seg.k64, seg.v64, 384, ref_sel, 1)
     assert_close(L.o.double().cpu().numpy(), o, w, "o")
+    assert_close(L.lse.double().cpu().numpy(), lse, w, "lse", abs_=1e-4)
+
+
+def test_corrupt_selection_tensor_core_path():
+    # bf16, d = 128, G = 4: the tensor-core forward, dQ and dK/dV kernels skip
+    # bad entries (beyond the own block; negative but not -1) and latch
+    # HGA_ERR_DEVICE_CHECK; outputs and gradients equal the oracle's with
+    # those entries dropped
+    import torch
+    import oracle
+    from hierarchical_routed_sparse_hga_b200 import (HGA_ERR_DEVICE_CHECK, HGA_OK, hga_attn_bwd,
+                                                     hga_attn_fwd, hga_get_device_status)
+    from hga_testlib import assert_close, to_device
+    w = synth.custom(n_q_heads=8, n_kv_heads=2, head_dim=128, ctx_len=1024, seg_len=256,
+                     topk_blocks=3, topk_groups=12, dtype="bf16", scaled=True, rope_base=1e6,
+                     first_seg=3, seed=4)
+    seg = Segmenter(w)
+    out = seg.run_segment(768)
+    assert hga_get_device_status() == HGA_OK
+    L = seg.layer
+    bad = L.sel_grp.clone()
+    bad[0, 0, 0, 1] = 10_000          # beyond the query block's own block
+    bad[0, 1, 2, 0] = -7              # negative, not the -1 padding
+    bad[0, 1, 3, 5] = 8 * (768 // 64 + 3) + 2   # a group of the query block's own block
+    q = to_device(synth.queries(w, 768), w)
+    d_o = to_device(synth.douts(w, 768), w)
+    hga_attn_fwd(L.cfg, q, L.k, L.v, w.ctx_len, 768, w.seg_len, bad, L.o, L.lse)
+    assert hga_get_device_status() == HGA_ERR_DEVICE_CHECK
+    hga_attn_bwd(L.cfg, q, L.k, L.v, w.ctx_len, 768, w.seg_len, bad, L.o, L.lse, d_o, L.dq, L.dk,
+                 L.dv, L.bwd_ws)
+    assert hga_get_device_status() == HGA_ERR_DEVICE_CHECK
+    assert hga_get_device_status() == HGA_OK          # reading clears it
+    ref_sel = bad.cpu().numpy().copy()
+    for idx in ((0, 0, 0, 1), (0, 1, 2, 0), (0, 1, 3, 5)):
+        ref_sel[idx] = -1
+    o, lse = oracle.attn_fwd(out["q64"], seg.k64, seg.v64, 768, ref_sel, 2)
+    dq, dk, dv = oracle.attn_bwd(out["q64"], seg.k64, seg.v64, out["do64"], 768, ref_sel, 2)
+    for name, ref in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv)):
+        assert_close(getattr(L, name).double().cpu().numpy(), ref, w, name)
     assert_close(L.lse.double().cpu().numpy(), lse, w, "lse", abs_=1e-4)
 
 

@@ -4,17 +4,17 @@ Some callers have no way to call cudaMalloc -- a plugin inside a host runtime
 that owns all device memory and gives its extensions no allocator, or code
 that must not allocate once running because cudaMalloc can synchronise the
 device.  hga_route_noalloc serves them by taking the router's scratch (the
-mean queries and the block scores) from an array built into the library
-instead of a caller-provided workspace.
+mean queries and the candidate chunks' finalists) from an array built into
+the library instead of a caller-provided workspace.
 
 The context here is long enough (more than 512 candidate blocks) that the
 routing runs as its three-kernel form, which is the form that writes and
 reads that scratch.  The test calls the entry point through the C ABI twice
 in a row: first at the end of a 40960-token context, then on an earlier
-segment with fewer candidates, so the second call's score rows are shorter
-than the first call's and sit over its leftover contents.  Each result must
-equal the workspace-taking hga_route's exactly (selections are integer
-indices).
+segment with fewer candidates, so the second call's finalist rows are
+shorter than the first call's and sit over its leftover contents.  Each
+result must equal the workspace-taking hga_route's exactly (selections are
+integer indices).
 
 The file name sorts last so that a run which stops at the first failure has
 already run every other test.
@@ -75,5 +75,5 @@ def test_route_noalloc_rejects_work_beyond_its_scratch():
     cfg = Config(1, 32, 8, 128, 16, 64)
     fake = 0x10000  # never dereferenced: the size check fails before any launch
     with pytest.raises(HgaError) as e:
-        hga_route_noalloc(cfg, fake, 227392, 2048, 229440, fake, fake, None, fake, 0)
+        hga_route_noalloc(cfg, fake, 1015808, 2048, 1017856, fake, fake, None, fake, 0)
     assert e.value.status == HGA_ERR_WORKSPACE
