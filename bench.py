@@ -248,8 +248,9 @@ def kernel_work(name, w, sels, unique_groups=None, from_summaries=False):
         # one launch up to 512 candidate blocks, three kernels beyond
         one_launch = own0 + n_qb - 1 <= 512
         if (name == "route_fused" and not one_launch) or (
-                name in ("route_qmean", "route_block_score", "route_select") and one_launch):
+                name in ("route_qbar", "route_block_topk", "route_select") and one_launch):
             continue
+        n_chunks = -(-(own0 + n_qb - 1) // 128)       # candidate chunks of 128 blocks
         if name.startswith("attn_fwd"):
             tot += 4 * d * pairs
         elif name.startswith("attn_bwd_dq"):
@@ -261,13 +262,19 @@ def kernel_work(name, w, sels, unique_groups=None, from_summaries=False):
             tot += 4 * d * act
         elif name == "summaries":
             tot += B * Hkv * (S * d * el + (S // 8 + S // 64) * d * 4)
-        elif name == "route_qmean":
+        elif name == "route_qbar":
+            # Q once, q-bar written
             tot += B * (Hq * S * d * el + Hkv * n_qb * d * 4)
-        elif name == "route_block_score":
-            tot += B * Hkv * ((own0 + n_qb - 1) * d * 4 + n_qb * d * 4 + sum(Js) * 4)
+        elif name == "route_block_topk":
+            # each block summary of the head once, q-bar, the finalists
+            # (key and index, k_b + 1 per chunk and query block) written
+            tot += B * Hkv * ((own0 + n_qb - 1) * d * 4 + n_qb * d * 4
+                              + n_chunks * n_qb * (w.topk_blocks + 1) * 8)
         elif name == "route_select":
-            tot += B * Hkv * sum(J * 4 + 8 * k * d * 4 + d * 4 + 4 * (w.topk_blocks + w.topk_groups)
-                                 for J, k in zip(Js, kb))
+            # the finalists and q-bar read, the kept blocks' group summaries,
+            # the two selections written
+            tot += B * Hkv * sum(n_chunks * (w.topk_blocks + 1) * 8 + d * 4 + 8 * k * d * 4
+                                 + 4 * (w.topk_blocks + w.topk_groups) for k in kb)
         elif name == "route_fused":
             # Q once (unless q-bar comes from the resident block means), each
             # block summary of the head once, the kept blocks' group

@@ -472,13 +472,16 @@ struct KvShared {
   uint64_t sdp_full[2];
   uint64_t pds_full[2];
   uint64_t mma_done;
+  uint64_t issued_all;  // the producer has requested every item of the unit
+  uint64_t plan_full;   // the next unit's plan is in (phase n: the plan of unit n)
   uint32_t tmem_base;
   int abort;
-  int n_items;
-  int unit;
-  int pre_issued;  // items whose Q/dO the unit's set-up already requested
-  int masks[64];
-  int js[64];
+  // plans of two units (slot = unit index & 1): the unit, its item count,
+  // the attending query blocks in increasing order and their group masks
+  int unit[2];
+  int n_items[2];
+  int masks[2][64];
+  int js[2][64];
 };
 
 template <int MT>
@@ -520,7 +523,68 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
       }
     }
   };
+  // K and V of key block gblk of (b, h)
+  auto load_kv = [&](int b, int h, int64_t gblk) {
+    const int32_t krow = int32_t((int64_t(b) * n_kv_heads + h) * ctx_cap + gblk * kBlock);
+    mbar_arrive_expect_tx(&sh.kv_full, 32768);
+    for (int gi = 0; gi < 8; ++gi)
+      for (int hf = 0; hf < 2; ++hf) {
+        tma_load_2d(smem + L::kK + hf * 8192 + gi * 1024, &tm_k, &sh.kv_full, hf * 64,
+                    krow + gi * kGroup);
+        tma_load_2d(smem + L::kV + hf * 8192 + gi * 1024, &tm_v, &sh.kv_full, hf * 64,
+                    krow + gi * kGroup);
+      }
+  };
   volatile int* abort = &sh.abort;
+  // The plan of the next unit (one warp, all lanes): claim it from the
+  // counter, then find the later query blocks of the segment that selected
+  // groups of its key block (only query blocks after kb can).  Their dQ CTAs
+  // wrote the inverted selection, tagged with the call's token, before
+  // releasing their D flags; the entry and (fused) the flag are read in one
+  // round, and an entry that is not yet this call's is read again once the
+  // flag is in.  The own block is always the first item.
+  auto plan = [&](int slot) {
+    int w = 0;
+    if (lane == 0) w = *abort ? n_units : atomicAdd(unit_counter, 1);
+    w = __shfl_sync(kFullMask, w, 0);
+    int n = 0;
+    if (w < n_units) {
+      const int kb = w / n_bh, bh = w % n_bh;
+      const int* inv_row = inv + (int64_t(bh) * n_qb + kb) * n_qb;
+      const uint32_t tk = token & 0xffffffu;
+      for (int c0 = kb; c0 < n_qb; c0 += 32) {
+        const int jj = c0 + lane;
+        int mask = 0;
+        if (jj < n_qb) {
+          uint32_t v = jj > kb ? uint32_t(__ldcg(inv_row + jj)) : 0u;
+          const bool ready = !d_done || flag_wait(d_done + bh * n_qb + jj, token, abort);
+          if (jj == kb) {
+            mask = 0xff;
+          } else if (ready) {
+            if ((v >> 8) != tk) v = uint32_t(__ldcg(inv_row + jj));
+            if ((v >> 8) != tk)
+              latch_status(HGA_ERR_DEVICE_CHECK);
+            else
+              mask = int(v & 0xffu);
+          }
+        }
+        const bool on = mask != 0;
+        const unsigned ball = __ballot_sync(kFullMask, on);
+        if (on) {
+          sh.js[slot][n + __popc(ball & ((1u << lane) - 1u))] = jj;
+          sh.masks[slot][jj] = mask;
+        }
+        n += __popc(ball);
+      }
+    }
+    if (lane == 0) {
+      sh.unit[slot] = w;
+      sh.n_items[slot] = n * MT;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh.plan_full);
+    __syncwarp();
+  };
   pdl_launch_dependents();
 
   if (tid == 0) {
@@ -532,6 +596,8 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
       mbar_init(&sh.pds_full[u], 128);
     }
     mbar_init(&sh.mma_done, 2);  // one commit from each issuer per unit
+    mbar_init(&sh.issued_all, 1);
+    mbar_init(&sh.plan_full, 1);
     sh.abort = 0;
     fence_barrier_init();
   }
@@ -560,89 +626,47 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
   // that the most query blocks can select come first; each CTA takes the
   // next unit from the counter until none is left.  Item indices run on
   // across units (it_base), so every barrier's phase sequence continues.
+  // Warp 2 plans unit n + 1 while unit n runs (once unit n's last item has
+  // been requested, so that a CTA does not hold a unit long before it can
+  // start it), and the producer requests the next unit's K/V and first items
+  // as soon as unit n's MMAs are done, under unit n's epilogue.
+  if (warp == 2) plan(0);
+  __syncthreads();
   int it_base = 0;
-  for (int un = 0;; ++un) {
-    if (tid == 0) sh.unit = *abort ? n_units : atomicAdd(unit_counter, 1);
-    for (int i = tid; i < 64; i += blockDim.x) sh.masks[i] = 0;
-    __syncthreads();
-    const int w = sh.unit;
+  // producer (warp 0): what it has already requested of the next unit
+  bool ahead_kv = false;
+  int ahead_items = 0;
+  int un = 0;
+  for (;; ++un) {
+    const int slot = un & 1;
+    const int w = sh.unit[slot];
     if (w >= n_units) break;
     const int kb = w / n_bh, bh = w % n_bh, b = bh / n_kv_heads, h = bh % n_kv_heads;
     const int64_t gblk = q_begin / kBlock + kb;  // global index of this key block
-    if (tid == 0) {
-      // this block's keys and values first: they do not depend on the selection
-      // (the previous unit's MMAs have all completed: see the end of the loop)
-      sh.masks[kb] = 0xff;
-      const int32_t krow = int32_t((int64_t(b) * n_kv_heads + h) * ctx_cap + gblk * kBlock);
-      mbar_arrive_expect_tx(&sh.kv_full, 32768);
-      for (int gi = 0; gi < 8; ++gi)
-        for (int hf = 0; hf < 2; ++hf) {
-          tma_load_2d(smem + L::kK + hf * 8192 + gi * 1024, &tm_k, &sh.kv_full, hf * 64,
-                      krow + gi * kGroup);
-          tma_load_2d(smem + L::kV + hf * 8192 + gi * 1024, &tm_v, &sh.kv_full, hf * 64,
-                      krow + gi * kGroup);
-        }
-      // and the first items, the own block's M tiles (always the first in
-      // the visiting order), before the selection is read
-      int pre = 0;
-      for (int it = 0; it < MT; ++it) {
-        const int gi = it_base + it, u = gi & 1;
-        if (gi >= 2 && !mbar_wait(&sh.qd_empty[u], ((gi >> 1) - 1) & 1, abort)) break;
-        load_qd(u, b, h, kb, it);
-        ++pre;
-      }
-      sh.pre_issued = pre;
-    }
-    // which later query blocks of the segment selected groups of this block
-    // (only query blocks after kb can): their dQ CTAs wrote it, tagged with
-    // the call's token, before releasing their D flags.  Fused: wait for
-    // those flags (and the own block's) first.
-    {
-      const int* inv_row = inv + (int64_t(bh) * n_qb + kb) * n_qb;
-      const uint32_t tk = token & 0xffffffu;
-      for (int jj = kb + 1 + tid; jj < n_qb; jj += blockDim.x) {
-        if (d_done && !flag_wait(d_done + bh * n_qb + jj, token, abort)) continue;
-        const uint32_t v = uint32_t(inv_row[jj]);
-        if ((v >> 8) != tk) {
-          latch_status(HGA_ERR_DEVICE_CHECK);
-          continue;
-        }
-        if (v & 0xffu) sh.masks[jj] = int(v & 0xffu);
-      }
-      if (d_done && tid == blockDim.x - 1) flag_wait(d_done + bh * n_qb + kb, token, abort);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      int n = 0;
-      for (int c0 = 0; c0 < n_qb; c0 += 32) {
-        const int jj = c0 + lane;
-        const bool on = jj < n_qb && jj >= kb && sh.masks[jj] != 0;
-        const unsigned ball = __ballot_sync(0xffffffffu, on);
-        if (on) sh.js[n + __popc(ball & ((1u << lane) - 1u))] = jj;
-        n += __popc(ball);
-      }
-      if (lane == 0) sh.n_items = n * MT;  // >= MT: the own block is always in
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const int n_items = sh.n_items;
+    const int n_items = sh.n_items[slot];
+    const int* js = sh.js[slot];
+    const int* masks = sh.masks[slot];
 
     if (warp == 0) {
       // ---------------- TMA producer (whole warp; one elected lane issues) --
-      int issued = sh.pre_issued;
-      const bool pre_ok = issued == MT;  // else the set-up was aborted
-      for (int it = issued; pre_ok && it < n_items; ++it) {
+      // this block's keys and values, unless requested during the last unit
+      if (!ahead_kv && elect_one()) load_kv(b, h, gblk);
+      __syncwarp();
+      int issued = ahead_items;
+      for (int it = issued; it < n_items; ++it) {
         const int gi = it_base + it, u = gi & 1;
         const bool free_ok =
             gi < 2 || mbar_wait(&sh.qd_empty[u], ((gi >> 1) - 1) & 1, abort);
         if (!__all_sync(kFullMask, free_ok)) break;
-        const int jj = sh.js[it / MT], m = it % MT;
+        const int jj = js[it / MT], m = it % MT;
         if (elect_one()) load_qd(u, b, h, jj, m);
         __syncwarp();
         issued = it + 1;
       }
-      // drain: wait (bounded, independent of abort) for the copies in flight
+      if (elect_one()) mbar_arrive(&sh.issued_all);
+      __syncwarp();
+      // drain: wait (bounded, independent of abort) for this unit's copies,
+      // before the next unit's requests arm the same barriers again
       if (lane == 0) {
         int never = 0;
         mbar_wait(&sh.kv_full, un & 1, &never);
@@ -651,6 +675,35 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
           mbar_wait(&sh.qd_full[gi & 1], (gi >> 1) & 1, &never);
         }
       }
+      __syncwarp();
+      // the next unit: once its plan is in and every MMA of this unit has
+      // completed (the K/V tiles and both Q/dO buffers are free), its K/V
+      // and its first two items (item i of it reuses the buffer of this
+      // unit's item n_items - 2 + i, whose copy has landed: the drain)
+      ahead_kv = false;
+      ahead_items = 0;
+      const bool next_ok =
+          issued == n_items &&
+          __all_sync(kFullMask, mbar_wait(&sh.plan_full, (un + 1) & 1, abort) &&
+                                    mbar_wait(&sh.mma_done, un & 1, abort) && !*abort);
+      const int w2 = sh.unit[slot ^ 1];
+      if (next_ok && w2 < n_units) {
+        const int kb2 = w2 / n_bh, bh2 = w2 % n_bh;
+        const int b2 = bh2 / n_kv_heads, h2 = bh2 % n_kv_heads;
+        const int n2 = min(2, sh.n_items[slot ^ 1]);
+        if (elect_one()) {
+          load_kv(b2, h2, q_begin / kBlock + kb2);
+          for (int it = 0; it < n2; ++it)
+            load_qd((it_base + n_items + it) & 1, b2, h2, sh.js[slot ^ 1][it / MT], it % MT);
+        }
+        __syncwarp();
+        ahead_kv = true;
+        ahead_items = n2;
+      }
+    } else if (warp == 2) {
+      // ---------------- planner: the next unit, once this one is requested --
+      mbar_wait(&sh.issued_all, un & 1, abort);
+      plan(slot ^ 1);
     } else if (warp == 1 || warp == 3) {
       // ---------------- MMA issuers (whole warp each, one lane issues) ------
       // Warp 1 issues S/dP(i) into TMEM buffer i & 1 once Q/dO of item i
@@ -724,9 +777,9 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
       // this group's items: those whose running index has parity u
       for (int it = (u - it_base) & 1; it < n_items && ok; it += 2) {
         const int gi = it_base + it;
-        const int jj = sh.js[it / MT], m = it % MT;
+        const int jj = js[it / MT], m = it % MT;
         const bool own = jj == kb;
-        const uint32_t mask = sh.masks[jj];
+        const uint32_t mask = masks[jj];
         const int hq = h * G + 2 * m + g;
         const int64_t rix = (int64_t(b) * n_q_heads + hq) * s_len + int64_t(jj) * kQBlock + r;
         const float lse2 = lse[rix] * 1.4426950408889634f;
@@ -802,6 +855,16 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     if (*abort) break;
+  }
+  // copies the producer requested for a unit that will not run (the loop
+  // ended on an abort): wait for them (bounded, independent of abort)
+  if (warp == 0 && lane == 0 && ahead_kv) {
+    int never = 0;
+    mbar_wait(&sh.kv_full, (un + 1) & 1, &never);
+    for (int it = 0; it < ahead_items; ++it) {
+      const int gi = it_base + it;
+      mbar_wait(&sh.qd_full[gi & 1], (gi >> 1) & 1, &never);
+    }
   }
 
   tc_fence_before();

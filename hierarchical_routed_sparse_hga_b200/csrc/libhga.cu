@@ -408,7 +408,7 @@ static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q
     hga_status_t e = HGA_OK;
     if (!qprev) {
       dim3 g0(n_qb, cfg->n_kv_heads, cfg->batch);
-      e = traced_launch(HGA_K_QMEAN, s, [&] {
+      e = traced_launch(HGA_K_QBAR, s, [&] {
         return launch_pdl(qbar_kernel<T, D>, g0, dim3(kRouteThreads), 0, s,
             static_cast<const T*>(q), cfg->n_q_heads, cfg->n_kv_heads, s_len, ws.qbar);
       });
@@ -426,7 +426,7 @@ static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q
       e = ensure_smem(reinterpret_cast<const void*>(&block_topk_kernel<D>), sm2);
       if (e != HGA_OK) return e;
       dim3 g2(unsigned(ws.n_chunks), cfg->n_kv_heads, cfg->batch * n_split);
-      e = traced_launch(HGA_K_BLOCK_SCORE, s, [&] {
+      e = traced_launch(HGA_K_BLOCK_TOPK, s, [&] {
         return launch_pdl(block_topk_kernel<D>, g2, dim3(kRouteThreads), sm2, s, qpart,
             qprev ? qsrc : nullptr, shift, bsum, ctx_cap, cfg->n_kv_heads, n_qb, own0,
             cfg->topk_blocks, n_split, nq_max, ws.fin_key, ws.fin_idx);
@@ -826,7 +826,7 @@ hga_status_t hga_get_device_status(void* stream) {
 
 const char* hga_kernel_name(int kind) {
   static const char* names[HGA_K_COUNT] = {
-      "summaries",      "route_qmean",       "route_block_score",   "route_select",
+      "summaries",      "route_qbar",        "route_block_topk",    "route_select",
       "attn_fwd_simt",  "attn_bwd_dq_simt",  "attn_bwd_dkdv_simt",  "attn_fwd_tc",
       "attn_bwd_dq_tc", "attn_bwd_dkdv_tc",  "tier_dedup",          "tier_copy",
       "route_fused",    "decode",            "query_summaries",     "prepare"};

@@ -49,7 +49,6 @@ __global__ void __launch_bounds__(kPrepThreads)
                    int64_t ctx_cap, int n_q_heads, int n_kv_heads, double log2_base,
                    T* __restrict__ q_out, T* __restrict__ k, T* __restrict__ v,
                    float* __restrict__ gsum, float* __restrict__ bsum, float* __restrict__ qsum) {
-  pdl_launch_dependents();
   extern __shared__ __align__(16) unsigned char sm_raw[];
   PrepShared<D>& sh = *reinterpret_cast<PrepShared<D>*>(sm_raw);
   constexpr int HALF = D / 2, LANES = D / 16, SLOTS = kPrepThreads / LANES;
@@ -170,6 +169,13 @@ __global__ void __launch_bounds__(kPrepThreads)
     for (int r = 0; r < SLOTS; ++r) qs += sh.qp[r][e];
     qsum[(head * (ctx_cap / kBlock) + blk) * D + e] = qs / float(G * kQBlock);
   }
+  // The next kernel may start only once every CTA's stores are visible:
+  // the routing and summary kernels read Q and K before their own wait for
+  // this grid, so the trigger comes after the CTA's last store (the barrier)
+  // and a device-scope fence.
+  __syncthreads();
+  __threadfence();
+  pdl_launch_dependents();
 }
 
 }  // namespace hga

@@ -27,7 +27,6 @@
 namespace hga {
 
 constexpr int kRouteThreads = 256;
-constexpr int kScoreChunk = 16;  // candidate blocks per block_score CTA
 
 // qbar of (b, h, j) = sum over the G shares (G <= 8), added in order
 // g = 0 .. G-1; all G loads are issued before the adds
@@ -187,7 +186,7 @@ __device__ __forceinline__ void select_levels(const SelectLayout& L, unsigned ch
 // afford to read all J block summaries (J <= kFusedRouteMaxBlocks; they stay
 // in L2): q-bar from the G heads' 64 query rows (the loads of several rows in
 // flight per thread), the J block scores, then select_levels.  One launch
-// instead of qmean + block_score + select.  Dynamic shared memory:
+// instead of qbar + block_topk + select.  Dynamic shared memory:
 // fused_route_smem(), the select layout followed by the q-bar partial sums.
 constexpr int kFusedRouteMaxBlocks = 512;
 
@@ -204,7 +203,11 @@ __host__ __device__ inline size_t fused_route_smem(int64_t j_cap, int topk_block
 // rows rs, rs + RS, ... (several rows' loads in flight), the RS partial rows
 // are then added in order; out[e] = mean (shared or global memory).  All
 // kRouteThreads threads; `part` is RS x D floats of shared memory.
-template <typename T, int D>
+// With kWaitBeforeWrite, the grid-dependency wait comes between reading Q
+// and writing `out`: Q is read while the kernel before still runs (none of
+// the library's kernels that trigger their dependents early writes Q), and
+// `out` is written only once that kernel has completed.
+template <typename T, int D, bool kWaitBeforeWrite = false>
 __device__ __forceinline__ void block_query_mean(const T* __restrict__ q, int b, int h, int j,
                                                  int n_q_heads, int G, int s_len, float* part,
                                                  float* out) {
@@ -225,6 +228,7 @@ __device__ __forceinline__ void block_query_mean(const T* __restrict__ q, int b,
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) part[rs * D + ch * 8 + e] = acc[e];
+  if constexpr (kWaitBeforeWrite) pdl_wait();
   __syncthreads();
   const float inv = 1.f / float(rows);
   for (int e = threadIdx.x; e < D; e += kRouteThreads) {
@@ -308,12 +312,11 @@ __global__ void __launch_bounds__(kRouteThreads)
     qbar_kernel(const T* __restrict__ q, int n_q_heads, int n_kv_heads, int s_len,
                 float* __restrict__ qbar) {
   pdl_launch_dependents();
-  pdl_wait();
   __shared__ float part[fused_route_rows<D>() * D];
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int n_qb = s_len / kQBlock;
-  block_query_mean<T, D>(q, b, h, j, n_q_heads, n_q_heads / n_kv_heads, s_len, part,
-                         qbar + ((int64_t(b) * n_kv_heads + h) * n_qb + j) * D);
+  block_query_mean<T, D, true>(q, b, h, j, n_q_heads, n_q_heads / n_kv_heads, s_len, part,
+                               qbar + ((int64_t(b) * n_kv_heads + h) * n_qb + j) * D);
 }
 
 struct ChunkLayout {

@@ -499,8 +499,8 @@ HGA_API hga_status_t hga_get_device_status(void* stream);
 /* Kernel kinds reported by the timing facility. */
 typedef enum {
   HGA_K_SUMMARIES = 0,
-  HGA_K_QMEAN = 1,
-  HGA_K_BLOCK_SCORE = 2,
+  HGA_K_QBAR = 1,
+  HGA_K_BLOCK_TOPK = 2,
   HGA_K_SELECT = 3,
   HGA_K_FWD_SIMT = 4,
   HGA_K_BWD_DQ_SIMT = 5,
