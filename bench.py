@@ -293,11 +293,34 @@ def kernel_work(name, w, sels, unique_groups=None, from_summaries=False):
     return tot, "B", "hbm"
 
 
-def source_hash():
+# the source files each kernel's device code comes from, besides the shared
+# device headers and the C header they include
+KERNEL_SOURCE = {
+    "summaries": ("summaries.cuh",), "route_fused": ("route.cuh",),
+    "route_qbar": ("route.cuh",), "route_block_topk": ("route.cuh",),
+    "route_select": ("route.cuh",), "query_summaries": ("route.cuh",),
+    "attn_fwd_tc": ("attn_fwd_sm100.cuh",), "attn_bwd_dq_tc": ("attn_bwd_sm100.cuh",),
+    "attn_bwd_dkdv_tc": ("attn_bwd_sm100.cuh",), "attn_fwd_simt": ("attn_simt.cuh",),
+    "attn_bwd_dq_simt": ("attn_simt.cuh",), "attn_bwd_dkdv_simt": ("attn_simt.cuh",),
+    "tier_dedup": ("tier.cuh",), "tier_copy": ("tier.cuh",),
+    "decode": ("decode.cuh", "route.cuh"), "prepare": ("prepare.cuh",),
+}
+SHARED_SOURCES = ("hga_common.cuh", "sm100_ptx.cuh")
+
+
+def source_hash(kernel=None):
+    """Hash of the sources a kernel is compiled from (all of csrc/ when the
+    kernel is not listed), so that a stored ncu figure is used only while
+    they are unchanged."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hierarchical_routed_sparse_hga_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        h.update(open(os.path.join(csrc, f), "rb").read())
+    if kernel in KERNEL_SOURCE:
+        paths = [os.path.join(csrc, f) for f in SHARED_SOURCES + KERNEL_SOURCE[kernel]]
+        paths.append(os.path.join(ROOT, "include", "hga.h"))
+    else:
+        paths = [os.path.join(csrc, f) for f in sorted(os.listdir(csrc))]
+    for f in paths:
+        h.update(open(f, "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -309,7 +332,7 @@ def measured_traffic(kernel, workload):
         return None
     d = json.load(open(path))
     e = d.get(workload, {}).get(kernel)
-    if not e or e.get("source_hash") != source_hash():
+    if not e or e.get("source_hash") != source_hash(kernel):
         return None
     return e.get("bytes_per_launch")
 
