@@ -69,14 +69,36 @@ def test_measured_traffic_only_for_the_current_sources(tmp_path, monkeypatch):
     bench = load_bench()
     prof = tmp_path / "profiles"
     prof.mkdir()
-    entry = {"bytes_per_launch": 1234, "source_hash": bench.source_hash()}
+    entry = {"bytes_per_launch": 1234, "source_hash": bench.source_hash("k")}
     (prof / "dram_traffic.json").write_text(json.dumps({"wl": {"k": entry}}))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "source_hash", lambda: entry["source_hash"])
+    monkeypatch.setattr(bench, "source_hash", lambda kernel=None: entry["source_hash"])
     assert bench.measured_traffic("k", "wl") == 1234
     assert bench.measured_traffic("other", "wl") is None
-    monkeypatch.setattr(bench, "source_hash", lambda: "changed")
+    monkeypatch.setattr(bench, "source_hash", lambda kernel=None: "changed")
     assert bench.measured_traffic("k", "wl") is None
+
+
+def test_source_hash_follows_each_kernels_own_files(tmp_path, monkeypatch):
+    # a kernel's stored figures go stale when its own file, a shared device
+    # header or the C header changes, and not when another kernel's does
+    bench = load_bench()
+    csrc = tmp_path / "hierarchical_routed_sparse_hga_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "include").mkdir()
+    names = set(bench.SHARED_SOURCES) | {f for fs in bench.KERNEL_SOURCE.values() for f in fs}
+    for f in names:
+        (csrc / f).write_text(f)
+    (tmp_path / "include" / "hga.h").write_text("h")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    before = {k: bench.source_hash(k) for k in ("attn_bwd_dq_tc", "route_fused", "decode")}
+    (csrc / "route.cuh").write_text("route changed")
+    after = {k: bench.source_hash(k) for k in before}
+    assert after["attn_bwd_dq_tc"] == before["attn_bwd_dq_tc"]
+    assert after["route_fused"] != before["route_fused"]
+    assert after["decode"] != before["decode"]          # decode includes the routing code
+    (csrc / "hga_common.cuh").write_text("common changed")
+    assert bench.source_hash("attn_bwd_dq_tc") != before["attn_bwd_dq_tc"]
 
 
 def test_both_arms_describe_the_same_workload():
