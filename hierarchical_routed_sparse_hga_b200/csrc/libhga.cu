@@ -427,7 +427,7 @@ static hga_status_t route_impl(const hga_config_t* cfg, const void* q, int64_t q
       if (e != HGA_OK) return e;
       dim3 g2(unsigned(ws.n_chunks), cfg->n_kv_heads, cfg->batch * n_split);
       e = traced_launch(HGA_K_BLOCK_TOPK, s, [&] {
-        return launch_pdl(block_topk_kernel<D>, g2, dim3(kRouteThreads), sm2, s, qpart,
+        return launch_pdl(block_topk_kernel<D>, g2, dim3(kChunkThreads), sm2, s, qpart,
             qprev ? qsrc : nullptr, shift, bsum, ctx_cap, cfg->n_kv_heads, n_qb, own0,
             cfg->topk_blocks, n_split, nq_max, ws.fin_key, ws.fin_idx);
       });

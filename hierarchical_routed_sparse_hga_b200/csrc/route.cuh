@@ -319,6 +319,10 @@ __global__ void __launch_bounds__(kRouteThreads)
                                qbar + ((int64_t(b) * n_kv_heads + h) * n_qb + j) * D);
 }
 
+// threads of a block_topk_kernel CTA: 16 warps, each scoring 8 of the
+// chunk's rows and ranking 2 of the 32 query blocks
+constexpr int kChunkThreads = 512;
+
 struct ChunkLayout {
   size_t bs, qb, sc, cand, total;
   int qb_stride, sc_stride;
@@ -332,12 +336,16 @@ __host__ __device__ inline ChunkLayout chunk_layout(int n_qb, int D) {
   L.bs = o;  o = align16(o + size_t(kChunkCands) * D * 4);
   L.qb = o;  o = align16(o + size_t(n_qb) * L.qb_stride * 4);
   L.sc = o;  o = align16(o + size_t(n_qb) * L.sc_stride * 4);
-  L.cand = o; o = align16(o + size_t(kRouteThreads / 32) * kChunkCands * 8);
   L.total = o;
+  // each warp's candidate list (keys and indices) over the block summaries,
+  // which are dead once the scores are in
+  L.cand = L.bs;
+  static_assert(size_t(kChunkThreads / 32) * kChunkCands * 8 <= size_t(kChunkCands) * 64 * 4,
+                "candidate lists fit in the block-summary tile");
   return L;
 }
 
-// grid (n_chunks, Hkv, B * n_split), kRouteThreads threads, dynamic shared
+// grid (n_chunks, Hkv, B * n_split), kChunkThreads threads, dynamic shared
 // memory chunk_layout(nq_max, D).total; split z % n_split takes query blocks
 // [split * nq_max, min(n_qb, (split + 1) * nq_max)).  Chunk c holds candidate blocks
 // [c*kChunkCands, ...) of the segment's largest candidate set [0, j_max).
@@ -348,7 +356,7 @@ __host__ __device__ inline ChunkLayout chunk_layout(int n_qb, int D) {
 // finite score; index -1).  The extra one makes the global (k+1)-th score
 // available to the merge.
 template <int D>
-__global__ void __launch_bounds__(kRouteThreads)
+__global__ void __launch_bounds__(kChunkThreads)
     block_topk_kernel(const float* __restrict__ qpart, const float* __restrict__ qprev,
                       int qshift, const float* __restrict__ bsum, int64_t ctx_cap,
                       int n_kv_heads, int n_qb, int64_t own0, int topk_blocks, int n_split,
@@ -373,27 +381,27 @@ __global__ void __launch_bounds__(kRouteThreads)
 
   // the chunk's block summaries (16-byte loads, 16 per thread in flight)
   {
-    constexpr int kV = kChunkCands * D / 4 / kRouteThreads;
+    constexpr int kV = kChunkCands * D / 4 / kChunkThreads;
     const float4* src = reinterpret_cast<const float4*>(bsum + (head * ctx_blocks + lo) * D);
     float4* dst = reinterpret_cast<float4*>(bs);
     const int n4 = n_loc * D / 4;
     float4 x[kV];
 #pragma unroll
     for (int u = 0; u < kV; ++u) {
-      const int i = tid + u * kRouteThreads;
+      const int i = tid + u * kChunkThreads;
       x[u] = i < n4 ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int u = 0; u < kV; ++u) dst[tid + u * kRouteThreads] = x[u];
+    for (int u = 0; u < kV; ++u) dst[tid + u * kChunkThreads] = x[u];
   }
   // every query block's q-bar row (the segment's rows of qpart, or rows
   // own0 + j - qshift of the resident block means), all loads in flight
   {
-    constexpr int kQV = 32 * D / 4 / kRouteThreads;  // up to 32 query blocks per CTA
+    constexpr int kQV = 32 * D / 4 / kChunkThreads;  // up to 32 query blocks per CTA
     float4 x[kQV];
 #pragma unroll
     for (int u = 0; u < kQV; ++u) {
-      const int i = tid + u * kRouteThreads, jj = i / (D / 4), e4 = i % (D / 4);
+      const int i = tid + u * kChunkThreads, jj = i / (D / 4), e4 = i % (D / 4);
       const float* src = nullptr;
       if (jj < nq) {
         if (qprev) {
@@ -407,16 +415,18 @@ __global__ void __launch_bounds__(kRouteThreads)
     }
 #pragma unroll
     for (int u = 0; u < kQV; ++u) {
-      const int i = tid + u * kRouteThreads, jj = i / (D / 4), e4 = i % (D / 4);
+      const int i = tid + u * kChunkThreads, jj = i / (D / 4), e4 = i % (D / 4);
       if (jj < nq) reinterpret_cast<float4*>(qb + jj * L.qb_stride)[e4] = x[u];
     }
   }
   __syncthreads();
 
   // scores: lane = query block (a second round past 32), each warp a slice
-  // of the chunk's rows, 8 rows at a time, the rows read as broadcasts
+  // of the chunk's rows (8 of 128), 8 rows at a time, the rows read as
+  // broadcasts
   {
-    const int rows_per_warp = (n_loc + 7) / 8;
+    constexpr int kWarps = kChunkThreads / 32;
+    const int rows_per_warp = (n_loc + kWarps - 1) / kWarps;
     const int r0 = warp * rows_per_warp;
     const int r1 = r0 + rows_per_warp < n_loc ? r0 + rows_per_warp : n_loc;
     for (int jb = 0; jb < nq; jb += 32) {
@@ -448,7 +458,7 @@ __global__ void __launch_bounds__(kRouteThreads)
   // local top-k_b of each query block over its valid candidates, one warp
   // per query block (rank counting; ties to the lower index), compacted in
   // ascending index by ballots
-  for (int jl = warp; jl < nq; jl += kRouteThreads / 32) {
+  for (int jl = warp; jl < nq; jl += kChunkThreads / 32) {
     const int jj = q0 + jl;   // query block within the segment
     const int64_t J = own0 + jj;
     const int kb = int(J < topk_blocks ? J : topk_blocks) + 1;   // + the (k+1)-th
