@@ -97,6 +97,16 @@ def test_decode_custom_shapes(kw):
     run_decode(w, positions)
 
 
+def test_decode_block_boundary_positions():
+    # the token alone in its block: the very first token (no candidates, it
+    # attends to itself only), the first token of block 1 (one candidate),
+    # and two later block starts
+    w = synth.custom(batch=4, n_q_heads=4, n_kv_heads=2, head_dim=128, ctx_len=1024,
+                     seg_len=64, topk_blocks=4, topk_groups=16, dtype="bf16", scaled=True,
+                     rope_base=1e6, seed=14)
+    run_decode(w, [0, 64, 64 * 7, 1024 - 64])
+
+
 def test_decode_is_deterministic():
     w = synth.custom(batch=2, n_q_heads=32, n_kv_heads=8, head_dim=128, ctx_len=4096,
                      seg_len=2048, topk_blocks=16, topk_groups=64, dtype="bf16", scaled=True,
