@@ -219,12 +219,19 @@ __device__ __forceinline__ void block_query_mean(const T* __restrict__ q, int b,
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll 8
-  for (int rr = rs; rr < rows; rr += RS) {
-    float f[8];
-    load8(qh + (int64_t(rr >> 6) * s_len + (rr & 63)) * D, f);
+  // rows whose loads are in flight together (raw, 4 or 8 registers each):
+  // at d = 128 and G <= 4 every row of the thread in one round
+  constexpr int kRound = sizeof(T) == 2 ? 16 : 8;
+  for (int rr0 = rs; rr0 < rows; rr0 += kRound * RS) {
+    Raw8<T> x[kRound];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += f[e];
+    for (int u = 0; u < kRound; ++u) {
+      const int rr = rr0 + u * RS;
+      if (rr < rows) x[u].load(qh + (int64_t(rr >> 6) * s_len + (rr & 63)) * D);
+    }
+#pragma unroll
+    for (int u = 0; u < kRound; ++u)
+      if (rr0 + u * RS < rows) x[u].add_to(acc);
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) part[rs * D + ch * 8 + e] = acc[e];
