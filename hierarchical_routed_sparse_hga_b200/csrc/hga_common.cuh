@@ -101,6 +101,14 @@ struct Raw8<__nv_bfloat16> {
       acc[2 * i + 1] += __uint_as_float(w[i] & 0xffff0000u);
     }
   }
+  __device__ __forceinline__ void get(float* f) const {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
 };
 template <>
 struct Raw8<float> {
@@ -112,6 +120,10 @@ struct Raw8<float> {
   __device__ __forceinline__ void add_to(float* acc) const {
     acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
     acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+  }
+  __device__ __forceinline__ void get(float* f) const {
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
   }
 };
 

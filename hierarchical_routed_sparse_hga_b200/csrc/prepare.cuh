@@ -57,6 +57,34 @@ __global__ void __launch_bounds__(kPrepThreads)
   const int tid = threadIdx.x, c = tid % LANES, slot = tid / LANES;
   const bool rotate = log2_base > 0.0;
 
+  // rows: G x 64 query rows, then 64 key rows, then 64 value rows; a round
+  // takes kBatch rows per row slot, their loads in flight together (raw
+  // 8-element words until used)
+  const int n_rows = (G + 2) * kQBlock;
+  constexpr int kBatch = sizeof(T) == 2 ? 6 : 3;
+  auto row_src = [&](int r) {
+    const int kind = r / kQBlock;  // 0..G-1: query head; G: key; G+1: value
+    const int64_t tok = int64_t(b) * s_len + int64_t(j) * kQBlock + r % kQBlock;
+    return kind < G ? q_proj + tok * q_row_stride + int64_t(h * G + kind) * D
+                    : (kind == G ? k_proj : v_proj) + tok * kv_row_stride + int64_t(h) * D;
+  };
+  Raw8<T> x1[kBatch], x2[kBatch];
+  auto load_round = [&](int r0) {
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int r = r0 + u * SLOTS;
+      if (r < n_rows) {
+        const T* src = row_src(r);
+        x1[u].load(src + 8 * c);
+        x2[u].load(src + HALF + 8 * c);
+      }
+    }
+  };
+  // the projections are inputs no kernel of the library writes: the first
+  // round's loads go out before the table is built and before the wait for
+  // the previous kernel (which only this kernel's stores must follow)
+  load_round(slot);
+
   // (cos, sin) of the 64 tokens' angles, reduced modulo 2 pi in double
   if (rotate) {
     for (int i = tid; i < HALF; i += kPrepThreads) sh.theta[i] = exp2(-(2.0 * i / D) * log2_base);
@@ -74,26 +102,11 @@ __global__ void __launch_bounds__(kPrepThreads)
   pdl_wait();
   __syncthreads();
 
-  // rows: G x 64 query rows, then 64 key rows, then 64 value rows
-  const int n_rows = (G + 2) * kQBlock;
   float qacc[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) qacc[e] = 0.f;
-  constexpr int kBatch = 4;  // rows whose loads are in flight together
   for (int r0 = slot; r0 < n_rows; r0 += kBatch * SLOTS) {
-    float x1[kBatch][8], x2[kBatch][8];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int r = r0 + u * SLOTS;
-      if (r >= n_rows) continue;
-      const int kind = r / kQBlock;  // 0..G-1: query head; G: key; G+1: value
-      const int t = r % kQBlock;
-      const int64_t tok = int64_t(b) * s_len + int64_t(j) * kQBlock + t;
-      const T* src = kind < G ? q_proj + tok * q_row_stride + int64_t(h * G + kind) * D
-                              : (kind == G ? k_proj : v_proj) + tok * kv_row_stride + int64_t(h) * D;
-      load8(src + 8 * c, x1[u]);
-      load8(src + HALF + 8 * c, x2[u]);
-    }
+    if (r0 != slot) load_round(r0);
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int r = r0 + u * SLOTS;
@@ -101,18 +114,15 @@ __global__ void __launch_bounds__(kPrepThreads)
       const int kind = r / kQBlock;
       const int t = r % kQBlock;
       float y1[8], y2[8];
+      x1[u].get(y1);
+      x2[u].get(y2);
       if (kind <= G && rotate) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float2 cs = sh.cs[t][i * LANES + c];
-          y1[i] = x1[u][i] * cs.x - x2[u][i] * cs.y;
-          y2[i] = x2[u][i] * cs.x + x1[u][i] * cs.y;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          y1[i] = x1[u][i];
-          y2[i] = x2[u][i];
+          const float a = y1[i], bb = y2[i];
+          y1[i] = a * cs.x - bb * cs.y;
+          y2[i] = bb * cs.x + a * cs.y;
         }
       }
       // the stored values (rounded to T) are what the summaries see
