@@ -145,6 +145,19 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
         tma_load_2d(dst, &tm_q, &sh.q_full, hf * 64, row);
       }
     }
+    // and tile 0, the causal own block, which does not depend on it either
+    if (!(flags & kTestDropFirstTile)) {
+      mbar_arrive_expect_tx(&sh.kv_full[0], L::kStageBytes);
+      const int64_t own_row0 =
+          (int64_t(b) * n_kv_heads + h) * ctx_cap + own_blk * kBlock;
+      uint8_t* kdst = smem + L::kKV;
+#pragma unroll
+      for (int gi = 0; gi < 8; ++gi) {
+        const int32_t row = int32_t(own_row0 + gi * kGroup);
+        tma_load_3d(kdst + gi * 2048, &tm_k, &sh.kv_full[0], 0, row, 0);
+        tma_load_3d(kdst + gi * 2048 + 16384, &tm_v, &sh.kv_full[0], 0, row, 0);
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, L::kTmemCols);
@@ -172,17 +185,14 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
     // 3-D box (64 columns x 8 rows x 2 halves) per group and tensor (Q was
     // issued during set-up)
     const int64_t kv_row0 = (int64_t(b) * n_kv_heads + h) * ctx_cap;
-    int issued = 0;
-    for (int t = 0; t < n_tiles; ++t) {
+    // tile 0 (the own block) was requested during set-up; with the test
+    // hook it is never armed, so its consumers must time out
+    int issued = (flags & kTestDropFirstTile) ? 0 : 1;
+    for (int t = 1; t < n_tiles; ++t) {
       const int st = t % kStages;
       const bool free_ok =
           t < kStages || mbar_wait(&sh.kv_empty[st], ((t / kStages) - 1) & 1, abort);
       if (!__all_sync(kFullMask, free_ok)) break;
-      if ((flags & kTestDropFirstTile) && t == 0) {
-        // test hook: tile 0 is never armed, so its consumers must time out
-        if (__any_sync(kFullMask, *abort != 0)) break;
-        continue;
-      }
       if (elect_one()) {
         mbar_arrive_expect_tx(&sh.kv_full[st], L::kStageBytes);
         uint8_t* kdst = smem + L::kKV + st * L::kStageBytes;
@@ -286,7 +296,7 @@ __global__ void __launch_bounds__(Layout<MT>::kThreads, 1)
       tmem_ld32(tmem + lane_addr + L::colS(m, buf), s);
       tmem_ld32(tmem + lane_addr + L::colS(m, buf) + 32, s + 32);
       tmem_wait_ld();
-      const bool own = t == n_tiles - 1;
+      const bool own = t == 0;
       const uint32_t mask = sh.tile_mask[t];
       if (own || mask != 0xffu) {
 #pragma unroll

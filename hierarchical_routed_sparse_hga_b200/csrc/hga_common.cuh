@@ -153,12 +153,13 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float* f) {
 
 // ---------------------------------------------------------------------------
 // Key-tile schedule of one query block, built by one full warp into shared
-// memory: the valid selected groups in their (ascending) order, 8 per tile,
-// the last routed tile padded with copies of the first valid group (masked
-// out by tile_mask), then the causal own block as the last tile.  An index
-// that is neither -1 nor an earlier group latches HGA_ERR_DEVICE_CHECK and is
-// skipped.  All of the row's loads are issued before the first is used
-// (topk_groups <= 256: 8 per lane).
+// memory: the causal own block first (tile 0: it needs no selection, so its
+// K/V can be requested before the selection is read), then the valid
+// selected groups in their (ascending) order, 8 per tile, the last routed
+// tile padded with the own block's first group (masked out by tile_mask).
+// An index that is neither -1 nor an earlier group latches
+// HGA_ERR_DEVICE_CHECK and is skipped.  All of the row's loads are issued
+// before the first is used (topk_groups <= 256: 8 per lane).
 // ---------------------------------------------------------------------------
 template <typename SH>
 __device__ __forceinline__ void build_tile_schedule(SH& sh, const int32_t* srow, int topk_groups,
@@ -170,6 +171,8 @@ __device__ __forceinline__ void build_tile_schedule(SH& sh, const int32_t* srow,
     const int idx = i * 32 + lane;
     gv[i] = idx < topk_groups ? srow[idx] : -1;
   }
+  const int own0 = int(own_blk * kGroupsPerBlock);
+  int* routed = sh.grp + kGroupsPerBlock;
   int n_valid = 0;
 #pragma unroll
   for (int i = 0; i < kRounds; ++i) {
@@ -180,19 +183,19 @@ __device__ __forceinline__ void build_tile_schedule(SH& sh, const int32_t* srow,
       if (!ok) latch_status(HGA_ERR_DEVICE_CHECK);
     }
     const unsigned ball = __ballot_sync(0xffffffffu, ok);
-    if (ok) sh.grp[n_valid + __popc(ball & ((1u << lane) - 1u))] = g;
+    if (ok) routed[n_valid + __popc(ball & ((1u << lane) - 1u))] = g;
     n_valid += __popc(ball);
   }
   __syncwarp();
   const int n_rt = (n_valid + 7) / 8;
-  for (int i = n_valid + lane; i < n_rt * 8; i += 32) sh.grp[i] = sh.grp[0];
+  for (int i = n_valid + lane; i < n_rt * 8; i += 32) routed[i] = own0;
   for (int t = lane; t < n_rt; t += 32) {
     const int left = n_valid - 8 * t;
-    sh.tile_mask[t] = left >= 8 ? 0xffu : uint8_t((1u << left) - 1u);
+    sh.tile_mask[1 + t] = left >= 8 ? 0xffu : uint8_t((1u << left) - 1u);
   }
-  for (int i = lane; i < 8; i += 32) sh.grp[n_rt * 8 + i] = int(own_blk * kGroupsPerBlock + i);
+  for (int i = lane; i < kGroupsPerBlock; i += 32) sh.grp[i] = own0 + i;
   if (lane == 0) {
-    sh.tile_mask[n_rt] = 0xffu;
+    sh.tile_mask[0] = 0xffu;
     sh.n_tiles = n_rt + 1;
   }
 }
