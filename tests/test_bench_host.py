@@ -7,6 +7,7 @@
   active-segment restriction that the dK/dV work uses.
 * The DRAM traffic it reports comes from a committed ncu summary only while
   that summary was taken on the current kernel sources.
+* Routing work is credited only to the kernels whose path a segment takes.
 * Both arms describe the same workload in their JSON line.
 """
 import importlib.util
@@ -110,3 +111,27 @@ def test_both_arms_describe_the_same_workload():
     assert (cfg["seq_len"], cfg["seg_len"], cfg["n_q_heads"], cfg["n_kv_heads"],
             cfg["head_dim"]) == (16384, 2048, 32, 8, 128)
     assert cfg["backward"] is True and cfg["parallelism"] == "replicas1"
+
+
+def test_routing_work_goes_to_the_kernels_that_run():
+    # one launch of the fused routing kernel up to 512 candidate blocks, the
+    # three long-context kernels beyond; each is credited only with the
+    # segments whose path it runs, under the library's own kernel names
+    bench = load_bench()
+    from hierarchical_routed_sparse_hga_b200 import HGA_K_COUNT, hga_kernel_name
+    from hierarchical_routed_sparse_hga_b200 import synth
+    names = {hga_kernel_name(k) for k in range(HGA_K_COUNT)}
+    three = ("route_qbar", "route_block_topk", "route_select")
+    assert set(three) | {"route_fused"} <= names
+    w = synth.custom(n_q_heads=32, n_kv_heads=8, head_dim=128, ctx_len=65536, seg_len=2048,
+                     topk_blocks=16, topk_groups=64, dtype="bf16", backward=False)
+    sel = np.zeros((1, 8, 32, 64), np.int32)
+    short = [(14336, sel)]                    # last candidate block 255
+    long = [(63488, sel)]                     # last candidate block 1023
+    for k in three:
+        assert bench.kernel_work(k, w, short)[0] == 0
+        assert bench.kernel_work(k, w, long)[0] > 0
+    assert bench.kernel_work("route_fused", w, short)[0] > 0
+    assert bench.kernel_work("route_fused", w, long)[0] == 0
+    # q-bar reads every query row once: Hq x S x d bf16 plus the means written
+    assert bench.kernel_work("route_qbar", w, long)[0] == 32 * 2048 * 128 * 2 + 8 * 32 * 128 * 4
