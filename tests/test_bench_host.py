@@ -135,3 +135,15 @@ def test_routing_work_goes_to_the_kernels_that_run():
     assert bench.kernel_work("route_fused", w, long)[0] == 0
     # q-bar reads every query row once: Hq x S x d bf16 plus the means written
     assert bench.kernel_work("route_qbar", w, long)[0] == 32 * 2048 * 128 * 2 + 8 * 32 * 128 * 4
+
+
+def test_profile_cases_reject_an_unknown_case():
+    # the profiling driver lists its cases and refuses any other name before
+    # touching a GPU
+    from hierarchical_routed_sparse_hga_b200 import profile_cases
+    assert set(profile_cases.CASES) == {"bench16k", "long128k", "decode", "prepare", "tier",
+                                        "simt"}
+    with pytest.raises(SystemExit):
+        profile_cases.run("no_such_case", None)
+    with pytest.raises(SystemExit):
+        profile_cases.main([])
