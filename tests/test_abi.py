@@ -201,3 +201,16 @@ def test_prepare_and_summarized_route_host_checks():
                      FAKE, FAKE, need, 0) == 1
     assert status_of(hga.hga_route_causal, c, FAKE, 14336, 2048, 16384, FAKE, FAKE, FAKE, None,
                      FAKE, FAKE, need - 256, 0) == 6
+
+
+def test_noalloc_limit_on_the_host():
+    # the no-workspace routing takes its scratch from a fixed 4 MiB array: for
+    # the Qwen3-8B shape at batch 1 and 2048-token segments the largest
+    # context it accepts is 950,272 tokens; past it the call returns
+    # HGA_ERR_WORKSPACE before touching the GPU
+    c = cfg()
+    limit = 4 << 20
+    assert hga.hga_route_workspace_size(c, 2048, 950272 - 2048) <= limit
+    assert hga.hga_route_workspace_size(c, 2048, 950272) > limit
+    assert status_of(hga.hga_route_noalloc, c, FAKE, 950272, 2048, 952320, FAKE, FAKE, None,
+                     FAKE, 0) == 6
