@@ -469,8 +469,11 @@ struct KvLayout {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t colS(int u) { return u * 128; }
   static constexpr uint32_t colDP(int u) { return u * 128 + 64; }
-  static constexpr uint32_t kColDV = 256;
-  static constexpr uint32_t kColDK = 320;
+  // dV^T and dK^T of a unit in one of two sets (unit n uses set n & 1), so
+  // that a unit's epilogue can read its set while the next unit's MMAs
+  // accumulate into the other
+  static constexpr uint32_t colDV(int set) { return 256 + set * 128; }
+  static constexpr uint32_t colDK(int set) { return 320 + set * 128; }
 };
 
 struct KvShared {
@@ -638,9 +641,34 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
   // been requested, so that a CTA does not hold a unit long before it can
   // start it), and the producer requests the next unit's K/V and first items
   // as soon as unit n's MMAs are done, under unit n's epilogue.
+  // dV and dK of unit w from tensor-memory set `set` (warp group 0: TMEM
+  // lanes 0..127 are the 128 head dims), once every MMA of that unit has
+  // completed (its mma_done phase, parity `par`)
+  auto epilogue = [&](int set, int w, int par) {
+    if (!mbar_wait(&sh.mma_done, par, abort)) return;
+    tc_fence_after();
+    const int wq = warp & 3, dcol = wq * 32 + lane;
+    const uint32_t lane_addr = uint32_t(wq * 32) << 16;
+    const int ekb = w / n_bh, ebh = w % n_bh;
+    const int eb = ebh / n_kv_heads, eh = ebh % n_kv_heads;
+    const int64_t base = ((int64_t(eb) * n_kv_heads + eh) * s_len + int64_t(ekb) * kBlock) * kD;
+    for (int c = 0; c < 64; c += 32) {
+      float vv[32], kk[32];
+      tmem_ld32(tmem + lane_addr + L::colDV(set) + c, vv);
+      tmem_ld32(tmem + lane_addr + L::colDK(set) + c, kk);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int64_t at = base + int64_t(c + i) * kD + dcol;
+        dv[at] = __float2bfloat16_rn(vv[i]);
+        dk[at] = __float2bfloat16_rn(kk[i] * scale);
+      }
+    }
+  };
   if (warp == 2) plan(0);
   __syncthreads();
   int it_base = 0;
+  int prev_w = -1;  // the unit whose epilogue is still to run (warp group 0)
   // producer (warp 0): what it has already requested of the next unit
   bool ahead_kv = false;
   int ahead_items = 0;
@@ -754,9 +782,9 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
             for (int s8 = 0; s8 < 8; ++s8) {
               const uint32_t ro = s8 * 2048;
               const uint32_t acc = (it > 0 || s8 > 0) ? 1u : 0u;
-              mma_bf16(tmem + L::kColDV, smem_desc_sw128(qd + 32768 + ro, 16384, 1024),
+              mma_bf16(tmem + L::colDV(un & 1), smem_desc_sw128(qd + 32768 + ro, 16384, 1024),
                        smem_desc_sw128(pd + ro, 8192, 1024), idesc_t, acc);
-              mma_bf16(tmem + L::kColDK, smem_desc_sw128(qd + ro, 16384, 1024),
+              mma_bf16(tmem + L::colDK(un & 1), smem_desc_sw128(qd + ro, 16384, 1024),
                        smem_desc_sw128(pd + 16384 + ro, 8192, 1024), idesc_t, acc);
             }
             mma_commit(&sh.qd_empty[u]);
@@ -782,6 +810,9 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
       bool ok = true;
       uint8_t* prow = smem + L::kPD + u * L::kPDBytes + row * 128;
       uint8_t* drow = prow + 16384;
+      // warp group 0 first stores the previous unit's dV and dK (its set is
+      // not touched by this unit's MMAs)
+      if (u == 0 && prev_w >= 0 && !*abort) epilogue((un - 1) & 1, prev_w, (un - 1) & 1);
       // this group's items: those whose running index has parity u
       for (int it = (u - it_base) & 1; it < n_items && ok; it += 2) {
         const int gi = it_base + it;
@@ -834,36 +865,17 @@ __global__ void __launch_bounds__(KvLayout::kThreads, 1)
         tc_fence_before();
         mbar_arrive(&sh.pds_full[u]);
       }
-      // epilogue: warp group 0 owns TMEM lanes 0..127 = the 128 head dims
-      if (u == 0) {
-        if (ok) ok = mbar_wait(&sh.mma_done, un & 1, abort);
-        if (ok) {
-          tc_fence_after();
-          const int dcol = row;
-          const int64_t base =
-              ((int64_t(b) * n_kv_heads + h) * s_len + int64_t(kb) * kBlock) * kD;
-          for (int c = 0; c < 64; c += 32) {
-            float vv[32], kk[32];
-            tmem_ld32(tmem + lane_addr + L::kColDV + c, vv);
-            tmem_ld32(tmem + lane_addr + L::kColDK + c, kk);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int64_t at = base + int64_t(c + i) * kD + dcol;
-              dv[at] = __float2bfloat16_rn(vv[i]);
-              dk[at] = __float2bfloat16_rn(kk[i] * scale);
-            }
-          }
-        }
-      }
     }
     it_base += n_items;
+    prev_w = w;
     // end of the unit: every role is done with its barriers, tiles and TMEM
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (*abort) break;
   }
+  // the last unit's dV and dK (the loop ended at a unit that does not exist)
+  if (warp >= 4 && warp < 8 && prev_w >= 0 && !*abort) epilogue((un - 1) & 1, prev_w, (un - 1) & 1);
   // copies the producer requested for a unit that will not run (the loop
   // ended on an abort): wait for them (bounded, independent of abort)
   if (warp == 0 && lane == 0 && ahead_kv) {
